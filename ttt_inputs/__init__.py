@@ -1,0 +1,144 @@
+"""Seeded synthetic inputs for the multi-pass TTT trunk+branch attention.
+
+This module is the only code shared by the fp64 oracle (``oracle/``) and the
+CUDA path (``attention_pass_rope_b200``).  It draws random numbers and packs
+them into tensors; it holds none of the attention arithmetic (no RoPE, no
+softmax, no masking).
+
+Recipe (the same for every workload):
+
+* one ``torch.Generator`` on the CPU, seeded with ``seed``;
+* for packed variable-length (THD) workloads the sequence lengths are drawn
+  first, ``torch.randint(lo, hi + 1, (nseq,))``;
+* then, in this order, Q ``[P, T, H, D]``, K ``[P, T, Hkv, D]``,
+  V ``[P, T, Hkv, D]`` and the output gradient dO ``[P, T, H, D]``, each
+  fp32 N(0, 1) times ``scale`` and rounded to bf16 (round to nearest even,
+  torch's cast).
+
+Dense ``[B, S, ...]`` batches are stored pass-major as ``[P, B*S, ...]``: the
+token axis of a dense batch is the concatenation of its B sequences, so a
+dense batch is the THD layout with ``cu_seqlens = [0, S, 2S, ..., B*S]``.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """Shape of one attention call.
+
+    ``lengths`` lists the sequence lengths; a dense batch has ``B`` equal
+    lengths ``S``.  ``dense`` selects the public lse layout ``[P, B, H, S]``
+    (dense) or ``[P, H, T]`` (THD).
+    """
+
+    name: str
+    P: int
+    H: int
+    Hkv: int
+    D: int
+    theta: float
+    lengths: tuple
+    dense: bool
+    scale: float = 1.0
+    seed: int = 0
+    len_range: tuple = ()   # (lo, hi) when the lengths were drawn from the generator
+
+    @property
+    def T(self) -> int:
+        return int(sum(self.lengths))
+
+    @property
+    def nseq(self) -> int:
+        return len(self.lengths)
+
+    @property
+    def max_seqlen(self) -> int:
+        return int(max(self.lengths))
+
+    @property
+    def cu_seqlens(self) -> list:
+        out = [0]
+        for n in self.lengths:
+            out.append(out[-1] + int(n))
+        return out
+
+    @property
+    def trunk_pairs(self) -> int:
+        """Visible (query, trunk key) pairs summed over sequences, per head and pass."""
+        return int(sum(n * (n + 1) // 2 for n in self.lengths))
+
+    def flops_fwd_bwd(self, per_pair: int = 14) -> float:
+        """Algorithmic flops: ``per_pair * D`` per visible trunk pair, head and pass,
+        plus the branch keys (4*D fwd + 10*D bwd per branch key and query)."""
+        trunk = per_pair * self.D * self.trunk_pairs * self.H * self.P
+        branch_keys = self.T * self.H * sum(p - 1 for p in range(1, self.P + 1))
+        return float(trunk + per_pair * self.D * branch_keys)
+
+    def flops_fwd(self) -> float:
+        return self.flops_fwd_bwd(per_pair=4)
+
+
+def dense(name, B, S, P, H, Hkv, D, theta, scale=1.0, seed=0) -> Workload:
+    return Workload(name, P, H, Hkv, D, float(theta), tuple([S] * B), True, scale, seed)
+
+
+def thd(name, lengths, P, H, Hkv, D, theta, scale=1.0, seed=0) -> Workload:
+    return Workload(name, P, H, Hkv, D, float(theta), tuple(int(x) for x in lengths), False, scale, seed)
+
+
+def thd_random_lengths(name, nseq, lo, hi, P, H, Hkv, D, theta, scale=1.0, seed=0) -> Workload:
+    g = torch.Generator().manual_seed(seed)
+    lengths = torch.randint(lo, hi + 1, (nseq,), generator=g).tolist()
+    w = thd(name, lengths, P, H, Hkv, D, theta, scale, seed)
+    return dataclasses.replace(w, len_range=(lo, hi))
+
+
+# The five workloads the method is measured on (sizes from the benchmark spec).
+def workloads() -> dict:
+    return {
+        "tiny": dense("tiny", B=1, S=128, P=3, H=4, Hkv=2, D=64, theta=1e4),
+        "qwen3_8b_4k": dense("qwen3_8b_4k", B=2, S=4096, P=3, H=32, Hkv=8, D=128, theta=1e6),
+        "deep_ttt_8k": dense("deep_ttt_8k", B=1, S=8192, P=7, H=32, Hkv=8, D=128, theta=1e6),
+        "thd_packed": thd_random_lengths("thd_packed", nseq=16, lo=256, hi=4096, P=3, H=32, Hkv=8,
+                                         D=128, theta=1e6),
+        "long_32k": dense("long_32k", B=1, S=32768, P=5, H=32, Hkv=8, D=128, theta=1e6, scale=0.5),
+    }
+
+
+@dataclasses.dataclass
+class Inputs:
+    """bf16 tensors on the CPU, pass-major, token axis packed."""
+
+    q: torch.Tensor   # [P, T, H, D]
+    k: torch.Tensor   # [P, T, Hkv, D]
+    v: torch.Tensor   # [P, T, Hkv, D]
+    do: torch.Tensor  # [P, T, H, D]
+
+
+def make_inputs(w: Workload, with_grad: bool = True, seed: Optional[int] = None) -> Inputs:
+    """Draw the inputs of ``w`` in the documented order (see module docstring)."""
+    g = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    if w.len_range and (seed is None or seed == w.seed):
+        # the lengths were the first draw of this generator: replay it
+        lo, hi = w.len_range
+        drawn = torch.randint(lo, hi + 1, (w.nseq,), generator=g).tolist()
+        assert tuple(drawn) == w.lengths
+
+    def draw(*shape):
+        x = torch.randn(*shape, generator=g, dtype=torch.float32)
+        if w.scale != 1.0:
+            x.mul_(w.scale)
+        return x.to(torch.bfloat16)
+
+    T = w.T
+    q = draw(w.P, T, w.H, w.D)
+    k = draw(w.P, T, w.Hkv, w.D)
+    v = draw(w.P, T, w.Hkv, w.D)
+    do = draw(w.P, T, w.H, w.D) if with_grad else None
+    return Inputs(q, k, v, do)
