@@ -1,0 +1,100 @@
+"""ctypes view of libttt_attn.so (declarations in include/ttt_attn.h)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttt_attn.so")
+
+TTT_OK = 0
+TTT_ERR_INVALID_ARG = 1
+TTT_ERR_UNSUPPORTED = 2
+TTT_ERR_WORKSPACE = 3
+TTT_ERR_CUDA = 4
+TTT_ERR_DEVICE_TIMEOUT = 5
+
+TTT_LAYOUT_BSHD = 0
+TTT_LAYOUT_THD = 1
+
+KERNELS = ("rope_fwd", "trunk_fwd", "branch_merge_fwd", "rope_bwd", "bwd_preprocess", "trunk_bwd", "branch_bwd")
+KERNEL_COUNT = 8
+
+
+class TTTEvents(ctypes.Structure):
+    _fields_ = [("start", ctypes.c_void_p * KERNEL_COUNT), ("stop", ctypes.c_void_p * KERNEL_COUNT)]
+
+
+class TTTDesc(ctypes.Structure):
+    _fields_ = [
+        ("layout", ctypes.c_int),
+        ("P", ctypes.c_int),
+        ("B", ctypes.c_int),
+        ("S", ctypes.c_int),
+        ("H", ctypes.c_int),
+        ("Hkv", ctypes.c_int),
+        ("D", ctypes.c_int),
+        ("rope_theta", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("nseq", ctypes.c_int),
+        ("total_tokens", ctypes.c_int),
+        ("max_seqlen", ctypes.c_int),
+        ("events", ctypes.c_void_p),
+    ]
+
+
+class TTTError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library; raises if it has not been built (there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m attention_pass_rope_b200.build` "
+            "(the TTT attention has no other implementation)")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    vp, sz, u32, u64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_uint64
+    D = P(TTTDesc)
+    L.ttt_attn_workspace_size.argtypes = [D, ctypes.c_int]
+    L.ttt_attn_workspace_size.restype = sz
+    L.ttt_attn_workspace_layout.argtypes = [D, ctypes.c_int, P(sz)]
+    L.ttt_attn_workspace_layout.restype = ctypes.c_int
+    L.ttt_attn_fwd.argtypes = [D, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.ttt_attn_fwd.restype = ctypes.c_int
+    L.ttt_attn_bwd.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.ttt_attn_bwd.restype = ctypes.c_int
+    L.ttt_attn_device_status.argtypes = [vp, vp, P(u32)]
+    L.ttt_attn_device_status.restype = ctypes.c_int
+    L.ttt_attn_watchdog_selftest.argtypes = [vp, sz, u64, vp]
+    L.ttt_attn_watchdog_selftest.restype = ctypes.c_int
+    L.ttt_attn_set_wait_budget_ns.argtypes = [u64]
+    L.ttt_attn_set_wait_budget_ns.restype = None
+    L.ttt_status_string.argtypes = [ctypes.c_int]
+    L.ttt_status_string.restype = ctypes.c_char_p
+    L.ttt_attn_version.argtypes = []
+    L.ttt_attn_version.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().ttt_status_string(status).decode()
+    except Exception:  # pragma: no cover - only used for messages
+        return "unknown"
+
+
+def check(status: int, what: str) -> None:
+    if status != TTT_OK:
+        raise TTTError(status, what)

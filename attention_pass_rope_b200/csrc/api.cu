@@ -1,0 +1,307 @@
+// C ABI of libttt_attn.so (declared in include/ttt_attn.h): argument validation,
+// workspace layout, TMA descriptors and the launch sequence of the forward and
+// backward passes on the caller's stream.  No allocation, no per-call state.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "../../include/ttt_attn.h"
+#include "ttt_internal.h"
+
+namespace ttt {
+namespace {
+
+std::atomic<uint64_t> g_wait_budget_ns{2000000000ull};
+
+constexpr size_t kAlign = 1024;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Plan {
+  Geometry g;
+  size_t off[8];
+  int noff;
+  size_t total;
+};
+
+bool ptr_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Validate the descriptor and derive the geometry and workspace layout.
+ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
+  if (!d) return TTT_ERR_INVALID_ARG;
+  Plan pl{};
+  Geometry& g = pl.g;
+  if (d->layout != TTT_LAYOUT_BSHD && d->layout != TTT_LAYOUT_THD) return TTT_ERR_INVALID_ARG;
+  if (d->P < 1 || d->H < 1 || d->Hkv < 1 || d->D < 1) return TTT_ERR_INVALID_ARG;
+  if (d->H % d->Hkv != 0) return TTT_ERR_INVALID_ARG;
+  if (d->P > 16) return TTT_ERR_UNSUPPORTED;
+  if (d->D != 64 && d->D != 128) return TTT_ERR_UNSUPPORTED;  // rotary needs an even D; kernels take 64/128
+  if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return TTT_ERR_INVALID_ARG;
+  if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return TTT_ERR_INVALID_ARG;
+  g.P = d->P;
+  g.H = d->H;
+  g.Hkv = d->Hkv;
+  g.D = d->D;
+  g.theta = d->rope_theta;
+  g.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt(static_cast<float>(d->D));
+  if (d->layout == TTT_LAYOUT_BSHD) {
+    if (d->B < 0 || d->S < 0) return TTT_ERR_INVALID_ARG;
+    const long long T = static_cast<long long>(d->B) * d->S;
+    if (T > (1LL << 30)) return TTT_ERR_UNSUPPORTED;
+    g.si.cu_seqlens = nullptr;
+    g.si.nseq = d->B;
+    g.si.S = d->S;
+    g.si.T = static_cast<int>(T);
+    g.si.max_len = d->S;
+  } else {
+    if (d->nseq < 0 || d->total_tokens < 0 || d->max_seqlen < 0) return TTT_ERR_INVALID_ARG;
+    if (d->total_tokens > 0 && (!d->cu_seqlens || d->nseq < 1 || d->max_seqlen < 1)) return TTT_ERR_INVALID_ARG;
+    if (d->max_seqlen > d->total_tokens) return TTT_ERR_INVALID_ARG;
+    if (d->total_tokens > (1 << 30)) return TTT_ERR_UNSUPPORTED;
+    g.si.cu_seqlens = d->cu_seqlens;
+    g.si.nseq = d->nseq;
+    g.si.S = 0;
+    g.si.T = d->total_tokens;
+    g.si.max_len = d->max_seqlen;
+  }
+  // index arithmetic in the kernels: P*H*T*D elements must fit comfortably in int64,
+  // per-pass offsets in int32 where they are formed that way
+  const long long rows = static_cast<long long>(g.P) * g.H * g.si.T;
+  if (rows * g.D > (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+
+  const size_t T = static_cast<size_t>(g.si.T);
+  const size_t P = g.P, H = g.H, Hkv = g.Hkv, D = g.D;
+  size_t o = 0;
+  pl.off[0] = 0;
+  o = align_up(256);
+  pl.off[1] = o;  // q~
+  o = align_up(o + P * H * T * D * 2);
+  pl.off[2] = o;  // k~
+  o = align_up(o + P * Hkv * T * D * 2);
+  if (!for_backward) {
+    pl.off[3] = o;  // O_t
+    o = align_up(o + P * H * T * D * 4);
+    pl.off[4] = o;  // lse_t
+    o = align_up(o + P * H * T * 4);
+    pl.noff = 5;
+  } else {
+    pl.off[3] = o;  // delta
+    o = align_up(o + P * H * T * 4);
+    pl.off[4] = o;  // dq~ accumulator
+    o = align_up(o + P * H * T * D * 4);
+    pl.off[5] = o;  // dk~_1 accumulator
+    o = align_up(o + Hkv * T * D * 4);
+    pl.noff = 6;
+  }
+  pl.total = o;
+  *out = pl;
+  return TTT_OK;
+}
+
+// ---- TMA descriptors (driver entry point fetched through the runtime)
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D bf16 tensor map, 128-byte swizzle, box {64, b1, b2}; dims/strides innermost first.
+bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
+              uint64_t s2_bytes, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  const cuuint32_t box[3] = {64, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct EventScope {
+  const ttt_attn_events* ev;
+  int k;
+  cudaStream_t s;
+  EventScope(const ttt_attn_events* e, int kk, cudaStream_t st) : ev(e), k(kk), s(st) {
+    if (ev && ev->start[k]) cudaEventRecord(static_cast<cudaEvent_t>(ev->start[k]), s);
+  }
+  ~EventScope() {
+    if (ev && ev->stop[k]) cudaEventRecord(static_cast<cudaEvent_t>(ev->stop[k]), s);
+  }
+};
+
+#define TTT_CHECK_CUDA(expr)                 \
+  do {                                       \
+    if ((expr) != cudaSuccess) return TTT_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+}  // namespace ttt
+
+using namespace ttt;
+
+extern "C" {
+
+size_t ttt_attn_workspace_size(const ttt_attn_desc* desc, int for_backward) {
+  Plan pl;
+  if (make_plan(desc, for_backward, &pl) != TTT_OK) return 0;
+  return pl.total;
+}
+
+int ttt_attn_workspace_layout(const ttt_attn_desc* desc, int for_backward, size_t* offsets) {
+  Plan pl;
+  if (!offsets || make_plan(desc, for_backward, &pl) != TTT_OK) return 0;
+  for (int i = 0; i < pl.noff; ++i) offsets[i] = pl.off[i];
+  return pl.noff;
+}
+
+ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, void* o, float* lse,
+                        void* workspace, size_t workspace_bytes, void* stream_) {
+  Plan pl;
+  ttt_status st = make_plan(desc, 0, &pl);
+  if (st != TTT_OK) return st;
+  const Geometry& g = pl.g;
+  if (g.si.T == 0) return TTT_OK;
+  if (!q || !k || !v || !o || !lse) return TTT_ERR_INVALID_ARG;
+  if (!ptr_aligned(q, 16) || !ptr_aligned(k, 16) || !ptr_aligned(v, 16) || !ptr_aligned(o, 16) ||
+      !ptr_aligned(lse, 4))
+    return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + pl.off[0]);
+  void* qr = ws + pl.off[1];
+  void* kr = ws + pl.off[2];
+  float* o_t = reinterpret_cast<float*>(ws + pl.off[3]);
+  float* lse_t = reinterpret_cast<float*>(ws + pl.off[4]);
+  const uint64_t T = g.si.T, D = g.D;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, qr, D, T, static_cast<uint64_t>(g.P) * g.H, D * 2, T * D * 2, 128, 1) ||
+      !make_map(&mk, kr, D, T, g.Hkv, D * 2, T * D * 2, 128, 1) ||
+      !make_map(&mv, v, D, g.Hkv, T, D * 2, g.Hkv * D * 2, 1, 128))
+    return TTT_ERR_CUDA;
+
+  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  {
+    EventScope es(desc->events, TTT_KERNEL_ROPE_FWD, stream);
+    TTT_CHECK_CUDA(launch_rope_fwd(g, q, k, qr, kr, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
+    TrunkFwdArgs a{g, o_t, lse_t, status, g_wait_budget_ns.load()};
+    TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_BRANCH_MERGE_FWD, stream);
+    TTT_CHECK_CUDA(launch_branch_merge_fwd(g, qr, kr, v, o_t, lse_t, o, lse, stream));
+  }
+  return TTT_OK;
+}
+
+ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                        size_t workspace_bytes, void* stream_) {
+  Plan pl;
+  ttt_status st = make_plan(desc, 1, &pl);
+  if (st != TTT_OK) return st;
+  const Geometry& g = pl.g;
+  if (g.si.T == 0) return TTT_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return TTT_ERR_INVALID_ARG;
+  if (!ptr_aligned(q, 16) || !ptr_aligned(k, 16) || !ptr_aligned(v, 16) || !ptr_aligned(o, 16) ||
+      !ptr_aligned(dout, 16) || !ptr_aligned(dq, 16) || !ptr_aligned(dk, 16) || !ptr_aligned(dv, 16) ||
+      !ptr_aligned(lse, 4))
+    return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + pl.off[0]);
+  void* qr = ws + pl.off[1];
+  void* kr = ws + pl.off[2];
+  float* delta = reinterpret_cast<float*>(ws + pl.off[3]);
+  float* dq_acc = reinterpret_cast<float*>(ws + pl.off[4]);
+  float* dk1_acc = reinterpret_cast<float*>(ws + pl.off[5]);
+  const uint64_t T = g.si.T, D = g.D;
+
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, qr, D, T, static_cast<uint64_t>(g.P) * g.H, D * 2, T * D * 2, 64, 1) ||
+      !make_map(&mk, kr, D, T, g.Hkv, D * 2, T * D * 2, 128, 1) ||
+      !make_map(&mv, v, D, g.Hkv, T, D * 2, g.Hkv * D * 2, 1, 128) ||
+      !make_map(&mdo, dout, D, g.H, static_cast<uint64_t>(g.P) * T, D * 2, g.H * D * 2, 1, 64))
+    return TTT_ERR_CUDA;
+
+  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  {
+    EventScope es(desc->events, TTT_KERNEL_ROPE_BWD, stream);
+    TTT_CHECK_CUDA(launch_rope_fwd(g, q, k, qr, kr, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, delta, stream));
+    TTT_CHECK_CUDA(cudaMemsetAsync(dq_acc, 0, static_cast<size_t>(g.P) * g.H * T * D * 4, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);
+    TrunkBwdArgs a{g, lse, delta, dq_acc, dk1_acc, dv, status, g_wait_budget_ns.load()};
+    TTT_CHECK_CUDA(launch_trunk_bwd(a, mq, mk, mv, mdo, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_BRANCH_BWD, stream);
+    TTT_CHECK_CUDA(launch_branch_bwd(g, qr, kr, v, dout, lse, delta, dq_acc, dk1_acc, dq, dk, dv, stream));
+  }
+  return TTT_OK;
+}
+
+ttt_status ttt_attn_device_status(void* workspace, void* stream_, uint32_t* detail) {
+  if (!workspace) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  if (detail) *detail = word;
+  if (word == 0) return TTT_OK;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  return TTT_ERR_DEVICE_TIMEOUT;
+}
+
+ttt_status ttt_attn_watchdog_selftest(void* workspace, size_t workspace_bytes, uint64_t budget_ns, void* stream_) {
+  if (!workspace || workspace_bytes < 256 || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  TTT_CHECK_CUDA(launch_watchdog_selftest(status, budget_ns, stream));
+  return TTT_OK;
+}
+
+void ttt_attn_set_wait_budget_ns(uint64_t budget_ns) {
+  g_wait_budget_ns.store(budget_ns == 0 ? 1 : budget_ns);
+}
+
+const char* ttt_status_string(ttt_status s) {
+  switch (s) {
+    case TTT_OK: return "ok";
+    case TTT_ERR_INVALID_ARG: return "invalid argument";
+    case TTT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TTT_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case TTT_ERR_CUDA: return "CUDA error";
+    case TTT_ERR_DEVICE_TIMEOUT: return "bounded in-kernel wait ran out";
+  }
+  return "unknown status";
+}
+
+const char* ttt_attn_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,440 @@
+// a6: trunk backward on the 5th-generation tensor cores.
+//
+// Gradient of the trunk half of the two-part attention ("DFlash/DSpark and EAGLE-3
+// TTT draft co-training ...", NeMo-RL issue 3698, "What I'm working on", item 1),
+// recomputing the probabilities from the MERGED log-sum-exp, so that the branch
+// keys' share of each row's softmax is accounted for exactly:
+//   P = exp(s - lse),  dP = dO V^T,  dS = P (dP - delta),  delta = rowsum(dO * O)
+//   dV_1 += P^T dO,  dk~_1 += dS^T q~,  dq~ += dS k~_1      (sigma applied later)
+//
+// One CTA owns one 128-key tile of one KV head and walks every (pass, group head)
+// query head and every 64-row query tile at or after the tile's diagonal, keeping
+// dK and dV of its keys in TMEM for the whole walk (no atomics on dK/dV).
+// Transposed products keep the key dimension on the TMEM lanes:
+//   S^T  = K~ Q~^T        (M=128 keys, N=64 queries)      SS
+//   dP^T = V dO^T         (M=128 keys, N=64)              SS
+//   dV  += P^T dO         (M=128, N=D, K=64 queries)      TS  (P^T in TMEM, bf16)
+//   dK  += dS^T Q~        (M=128, N=D, K=64)              SS  (dS^T in smem, bf16)
+//   dQ^T = K~^T dS^T      (M=128 rows of d, N=64, K=128)  SS  (both MN-major)
+// dQ^T goes TMEM -> registers -> smem (fp32, row-major [q][d]) and is added to the
+// fp32 dq~ accumulator with one bulk reduce-add per tile.
+//
+// CTA = 16 warps: warp 0 TMA producer (+ lse/delta rows), warp 1 TMEM allocator and
+// MMA issuer, warps 4-7 and 8-11 the two halves (query columns 0-31 / 32-63) of the
+// probability / dS step, warps 12-15 the dQ writer.  S^T/dP^T of tile n+1 are
+// issued before the dV/dK/dQ products of tile n so that the CUDA-core work of one
+// tile overlaps the tensor-core work of the previous one; P^T and dS^T are double
+// buffered for that reason.
+#include "common.cuh"
+
+namespace ttt {
+
+namespace {
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BK = 128;  // keys per CTA
+  static constexpr int BQ = 64;   // queries per step
+  static constexpr int ST = 2;    // Q~/dO ring stages
+  static constexpr int KCH = D / 64;
+  static constexpr int KCHUNK = 128 * 128;   // 128 rows x 64 bf16
+  static constexpr int QCHUNK = 64 * 128;    // 64 rows x 64 bf16
+  static constexpr int KTILE = 2 * KCHUNK;   // K~ always 2 chunks (D=64: chunk 1 is zero padding)
+  static constexpr int VTILE = KCH * KCHUNK;
+  static constexpr int QTILE = KCH * QCHUNK;
+  static constexpr int DSTILE = 128 * 128;   // 128 keys x 64 queries bf16
+  static constexpr int DQSTAGE = BQ * D * 4;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KTILE;
+  static constexpr int OFF_Q = OFF_V + (VTILE < KCHUNK ? KCHUNK : VTILE);
+  static constexpr int OFF_DO = OFF_Q + ST * QTILE;
+  static constexpr int OFF_DS = OFF_DO + ST * QTILE;
+  static constexpr int OFF_DQ = OFF_DS + 2 * DSTILE;
+  static constexpr int OFF_LD = OFF_DQ + DQSTAGE;          // [ST][2][64] floats: lse*log2e, delta
+  static constexpr int OFF_BAR = OFF_LD + ST * 2 * BQ * 4;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_USED = OFF_BAR + BAR_BYTES;
+  static constexpr int SMEM = (SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED) + 1024;
+  static constexpr int COL_DV = 0;
+  static constexpr int COL_DK = D;
+  static constexpr int COL_S = 2 * D;
+  static constexpr int COL_DP = 2 * D + 64;
+  static constexpr int COL_DQ = 2 * D + 128;
+  static constexpr int COL_PT = 2 * D + 192;  // two buffers of 32 columns
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 512;
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct IterInfo {
+  int p, h, q0;
+};
+
+__device__ __forceinline__ IterInfo decode_iter(int it, int nqt, int jq0, int gsz, int kvh) {
+  const int qh = it / nqt;
+  IterInfo r;
+  r.p = qh / gsz;
+  r.h = kvh * gsz + qh % gsz;
+  r.q0 = (jq0 + it % nqt) * 64;
+  return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+    trunk_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+                     const TrunkBwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+
+  const Geometry& g = a.g;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (key tile jk, sequence n, KV head), smallest jk (most work) first
+  const int per_jk = g.si.nseq * g.Hkv;
+  const int jk = static_cast<int>(blockIdx.x) / per_jk;
+  const int n = (static_cast<int>(blockIdx.x) % per_jk) / g.Hkv;
+  const int kvh = static_cast<int>(blockIdx.x) % g.Hkv;
+  int seq_start, len;
+  seq_bounds(g.si, n, seq_start, len);
+  const int k0 = jk * C::BK;
+  if (k0 >= len) return;
+  const int gsz = g.H / g.Hkv;
+  const int G = g.P * gsz;
+  const int jq0 = k0 / C::BQ;
+  const int nqt = (len + C::BQ - 1) / C::BQ - jq0;
+  const int NIT = G * nqt;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_bar = bars + 0;
+  uint64_t* qdo_full = bars + 1;            // [ST]
+  uint64_t* qdo_empty = bars + 1 + C::ST;   // [ST]
+  uint64_t* sdp_full = bars + 1 + 2 * C::ST;
+  uint64_t* ds_ready = sdp_full + 1;
+  uint64_t* mma_done = ds_ready + 1;        // [2]
+  uint64_t* dq_full = mma_done + 2;
+  uint64_t* dq_free = dq_full + 1;
+  uint64_t* final_bar = dq_free + 1;
+  uint64_t* drain = final_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sDO = smem + C::OFF_DO;
+  uint8_t* sDS = smem + C::OFF_DS;
+  float* sDQ = reinterpret_cast<float*>(smem + C::OFF_DQ);
+  float* sLD = reinterpret_cast<float*>(smem + C::OFF_LD);
+
+  if (D == 64) {
+    // zero padding rows d = 64..127 of K~ (the dQ^T product runs with M = 128)
+    uint4* z = reinterpret_cast<uint4*>(sK + C::KCHUNK);
+    for (int i = threadIdx.x; i < C::KCHUNK / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(kv_bar, 1);
+    for (int s = 0; s < C::ST; ++s) {
+      mbar_init(qdo_full + s, 2);
+      mbar_init(qdo_empty + s, 1);
+    }
+    mbar_init(sdp_full, 1);
+    mbar_init(ds_ready, 256);
+    mbar_init(mma_done + 0, 1);
+    mbar_init(mma_done + 1, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(final_bar, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, a.status, a.budget_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      tma_prefetch_desc(&map_do);
+      mbar_arrive_expect_tx(kv_bar, 2 * C::KCH * C::KCHUNK);
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_3d(sK + c * C::KCHUNK, &map_k, kv_bar, c * 64, seq_start + k0, kvh);
+        tma_load_3d(sV + c * C::KCHUNK, &map_v, kv_bar, c * 64, kvh, seq_start + k0);
+      }
+    }
+    for (int it = 0; it < NIT; ++it) {
+      const int s = it % C::ST;
+      bool ok = true;
+      if (lane == 0 && it >= C::ST) ok = wait_bounded(qdo_empty + s, ((it / C::ST) - 1) & 1, wd, kSiteBwdQdoEmpty);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(qdo_full + s, 2 * C::QTILE);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d(sQ + s * C::QTILE + c * C::QCHUNK, &map_q, qdo_full + s, c * 64, seq_start + ii.q0,
+                      ii.p * g.H + ii.h);
+          tma_load_3d(sDO + s * C::QTILE + c * C::QCHUNK, &map_do, qdo_full + s, c * 64, ii.h,
+                      ii.p * g.si.T + seq_start + ii.q0);
+        }
+      }
+      float* ld = sLD + s * 2 * C::BQ;
+      for (int r = lane; r < C::BQ; r += 32) {
+        const int qpos = ii.q0 + r;
+        float l2 = 0.f, dl = 0.f;
+        if (qpos < len) {
+          const int64_t idx = lse_index(g.si, g.H, ii.p, ii.h, n, seq_start + qpos, qpos);
+          l2 = a.lse[idx] * kLog2e;
+          dl = a.delta[idx];
+        }
+        ld[r] = l2;
+        ld[C::BQ + r] = dl;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qdo_full + s);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idSP = idesc_bf16_f32(128, C::BQ, false, false);
+      constexpr uint32_t idDV = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idDQ = idesc_bf16_f32(128, C::BQ, true, true);
+      const uint32_t kA = smem_u32(sK), vA = smem_u32(sV), qA = smem_u32(sQ), doA = smem_u32(sDO),
+                     dsA = smem_u32(sDS);
+      auto issue_sdp = [&](int it) {
+        const int s = it % C::ST;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ok_ = (kk >> 2) * C::KCHUNK + (kk & 3) * 32;
+          const uint32_t oq_ = (kk >> 2) * C::QCHUNK + (kk & 3) * 32;
+          umma_ss(tmem + C::COL_S, sdesc_sw128(kA + ok_, 16, 1024),
+                  sdesc_sw128(qA + s * C::QTILE + oq_, 16, 1024), idSP, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ok_ = (kk >> 2) * C::KCHUNK + (kk & 3) * 32;
+          const uint32_t oq_ = (kk >> 2) * C::QCHUNK + (kk & 3) * 32;
+          umma_ss(tmem + C::COL_DP, sdesc_sw128(vA + ok_, 16, 1024),
+                  sdesc_sw128(doA + s * C::QTILE + oq_, 16, 1024), idSP, kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = wait_bounded(kv_bar, 0, wd, kSiteBwdKv) && wait_bounded(qdo_full, 0, wd, kSiteBwdQdoFull);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0);
+        umma_commit(sdp_full);
+      }
+      for (int it = 0; ok && it < NIT; ++it) {
+        const int s = it % C::ST;
+        const int b = it & 1;
+        if (!wait_bounded(ds_ready, it & 1, wd, kSiteBwdDsReady)) break;
+        tc_fence_after();
+        if (it + 1 < NIT) {
+          if (!wait_bounded(qdo_full + (it + 1) % C::ST, ((it + 1) / C::ST) & 1, wd, kSiteBwdQdoFull)) break;
+          tc_fence_after();
+          issue_sdp(it + 1);
+          umma_commit(sdp_full);
+        }
+        // dV += P^T dO   (P^T: TMEM, 64 queries = 32 packed columns)
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          umma_ts(tmem + C::COL_DV, tmem + C::COL_PT + 32 * b + kk * 8,
+                  sdesc_sw128(doA + s * C::QTILE + kk * 2048, C::QCHUNK, 1024), idDV,
+                  (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q~
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          umma_ss(tmem + C::COL_DK, sdesc_sw128(dsA + b * C::DSTILE + kk * 32, 16, 1024),
+                  sdesc_sw128(qA + s * C::QTILE + kk * 2048, C::QCHUNK, 1024), idDV,
+                  (it > 0 || kk > 0) ? 1u : 0u);
+        if (it > 0) {
+          if (!wait_bounded(dq_free, (it - 1) & 1, wd, kSiteBwdDqFree)) break;
+          tc_fence_after();
+        }
+        // dQ^T = K~^T dS^T
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          umma_ss(tmem + C::COL_DQ, sdesc_sw128(kA + kk * 2048, C::KCHUNK, 1024),
+                  sdesc_sw128(dsA + b * C::DSTILE + kk * 2048, C::KCHUNK, 1024), idDQ, kk > 0 ? 1u : 0u);
+        umma_commit(mma_done + b);
+        umma_commit(qdo_empty + s);
+        umma_commit(dq_full);
+      }
+      umma_commit(final_bar);
+      umma_commit(drain);
+      wait_drain(drain, 0, wd, kSiteBwdDrain);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ P / dS
+    const int hf = (warp - 4) >> 2;  // query columns [32*hf, 32*hf+32)
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;    // key row
+    const int kpos = k0 + r;
+    const bool kvalid = kpos < len;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float sl2 = g.scale * kLog2e;
+    bool ok = true;
+    for (int it = 0; it < NIT; ++it) {
+      const int s = it % C::ST;
+      const int b = it & 1;
+      const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
+      if (!wait_bounded(sdp_full, it & 1, wd, kSiteBwdSdpFull) ||
+          !wait_bounded(qdo_full + s, (it / C::ST) & 1, wd, kSiteBwdQdoFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[32], dp[32];
+      tmem_ld32(lane_base + C::COL_S + 32 * hf, sv);
+      tmem_ld32(lane_base + C::COL_DP + 32 * hf, dp);
+      tmem_ld_wait();
+      reg_fence32(sv);
+      reg_fence32(dp);
+      if (it >= 2 && !wait_bounded(mma_done + b, ((it >> 1) - 1) & 1, wd, kSiteBwdMmaDone)) {
+        ok = false;
+        break;
+      }
+      const float* ld = sLD + s * 2 * C::BQ + 32 * hf;
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        float pv[2], dsv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = 2 * e + u;
+          const int qpos = ii.q0 + 32 * hf + c;
+          const bool vis = kvalid && qpos < len && kpos <= qpos;
+          const float pr = vis ? exp2_approx(fmaf(__uint_as_float(sv[c]), sl2, -ld[c])) : 0.f;
+          pv[u] = pr;
+          dsv[u] = pr * (__uint_as_float(dp[c]) - ld[C::BQ + c]);
+        }
+        pk[e] = pack_bf16x2(pv[0], pv[1]);
+        dk[e] = pack_bf16x2(dsv[0], dsv[1]);
+      }
+      tmem_st16(lane_base + C::COL_PT + 32 * b + 16 * hf, pk);
+      // dS^T row r, 128-byte swizzle: 16-byte chunk c of the row sits at c ^ (r & 7)
+      uint8_t* row = sDS + b * C::DSTILE + r * 128;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int cc = 4 * hf + i;
+        *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(dk[4 * i], dk[4 * i + 1], dk[4 * i + 2], dk[4 * i + 3]);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(ds_ready);
+    }
+    // ---- epilogue: dV (half 0) and dK~ (half 1) of this CTA's keys
+    if (ok && wait_bounded(final_bar, 0, wd, kSiteBwdFinal)) {
+      tc_fence_after();
+      const int64_t tau = seq_start + kpos;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + (hf == 0 ? C::COL_DV : C::COL_DK) + 32 * c, v);
+        tmem_ld_wait();
+        reg_fence32(v);
+        if (!kvalid) continue;
+        if (hf == 0) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dv) + (tau * g.Hkv + kvh) * D + 32 * c;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w = make_uint4(pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                                 pack_bf16x2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
+                                 pack_bf16x2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
+                                 pack_bf16x2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+            *reinterpret_cast<uint4*>(dst + e) = w;
+          }
+        } else {
+          float* dst = a.dk1_acc + (static_cast<int64_t>(kvh) * g.si.T + tau) * D + 32 * c;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) =
+                make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                            __uint_as_float(v[e + 3]));
+        }
+      }
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ dQ writer
+    const int wq = warp & 3;
+    const int d = wq * 32 + lane;  // TMEM lane = head dimension
+    const int tid = threadIdx.x - 384;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    for (int it = 0; it < NIT; ++it) {
+      const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
+      if (!wait_bounded(dq_full, it & 1, wd, kSiteBwdDqFull)) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(lane_base + C::COL_DQ, v0);
+      tmem_ld32(lane_base + C::COL_DQ + 32, v1);
+      tmem_ld_wait();
+      reg_fence32(v0);
+      reg_fence32(v1);
+      tc_fence_before();
+      mbar_arrive(dq_free);
+      if (tid == 0) bulk_wait_read0();  // the staging buffer has been read by the last reduce
+      named_bar_sync(1, 128);
+      if (d < D) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) sDQ[q * D + d] = __uint_as_float(v0[q]);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) sDQ[(32 + q) * D + d] = __uint_as_float(v1[q]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (tid == 0) {
+        const int nrows = min(C::BQ, len - ii.q0);
+        if (nrows > 0) {
+          float* dst = a.dq_acc + ((static_cast<int64_t>(ii.p) * g.H + ii.h) * g.si.T + seq_start + ii.q0) * D;
+          bulk_reduce_add_f32(dst, sDQ, static_cast<uint32_t>(nrows * D * 4));
+          bulk_commit();
+        }
+      }
+    }
+    if (tid == 0) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+template <int D>
+cudaError_t launch(const TrunkBwdArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const CUtensorMap& mdo, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(trunk_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int njk = (a.g.si.max_len + C::BK - 1) / C::BK;
+  const long long blocks = static_cast<long long>(njk) * a.g.si.nseq * a.g.Hkv;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  trunk_bwd_kernel<D><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
+                             const CUtensorMap& map_v, const CUtensorMap& map_do, cudaStream_t stream) {
+  return a.g.D == 128 ? launch<128>(a, map_q, map_k, map_v, map_do, stream)
+                      : launch<64>(a, map_q, map_k, map_v, map_do, stream);
+}
+
+}  // namespace ttt

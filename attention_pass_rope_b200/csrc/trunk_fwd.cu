@@ -1,0 +1,342 @@
+// a2: trunk causal attention forward on the 5th-generation tensor cores.
+//
+// "DFlash/DSpark and EAGLE-3 TTT draft co-training ..." (NeMo-RL issue 3698),
+// "What I'm working on", item 1: the trunk half of the two-part trunk+branch
+// attention.  Every pass p and every query head of a GQA group attends to the SAME
+// pass-1 keys with the SAME index-causal predicate (key t <= query i), so one CTA
+// stacks two (pass, head) query tiles of one KV head and streams each K/V tile once
+// for both.
+//
+// CTA = 12 warps:
+//   warp 0      TMA producer: two Q tiles once, then K/V tiles into a 2-stage ring
+//   warp 1      TMEM allocator and MMA issuer (one thread): S = Q K^T (SS form),
+//               O += P V (TS form, P read from TMEM)
+//   warps 4-7   softmax for query tile 0 (one TMEM lane = one query row per thread)
+//   warps 8-11  softmax for query tile 1
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
+// P_t (bf16, two per column) overwrites the first 64 columns of S_t.
+// The online softmax keeps a running max per row and rescales O (in TMEM) only when
+// the max grows by more than 2^8; the final normalisation uses the same max, so the
+// result is exact up to rounding.
+// Output: O_t (normalised, fp32, head-major) and lse_t (natural log) per row.
+#include "common.cuh"
+
+namespace ttt {
+
+namespace {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;  // query rows per tile
+  static constexpr int BN = 128;  // keys per KV tile
+  static constexpr int NQ = 2;    // query tiles per CTA
+  static constexpr int ST = 2;    // K/V ring stages
+  static constexpr int KCH = D / 64;
+  static constexpr int CHUNK = 128 * 128;         // one 64-column chunk of a 128-row tile
+  static constexpr int TILE = KCH * CHUNK;        // 128 rows x D bf16
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQ * TILE;
+  static constexpr int OFF_V = OFF_K + ST * TILE;
+  static constexpr int OFF_BAR = OFF_V + ST * TILE;
+  static constexpr int BAR_BYTES = 256;
+  // D = 64 needs only 96 KB; ask for more so that one CTA holds the SM (and its TMEM).
+  static constexpr int SMEM_USED = OFF_BAR + BAR_BYTES;
+  static constexpr int SMEM = (SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED) + 1024;
+  static constexpr int COL_S0 = 0;
+  static constexpr int COL_O0 = 256;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 384;
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+    trunk_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                     const __grid_constant__ CUtensorMap map_v, const TrunkFwdArgs a) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+
+  const Geometry& g = a.g;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (query block jq, sequence n, KV head, pair of (pass, head) tiles),
+  // largest jq first (longest causal rows first).
+  const int gsz = g.H / g.Hkv;
+  const int G = g.P * gsz;  // query heads per KV head
+  const int npairs = (G + 1) >> 1;
+  const int njq = (g.si.max_len + C::BM - 1) / C::BM;
+  const int per_jq = g.si.nseq * g.Hkv * npairs;
+  const int jq = njq - 1 - static_cast<int>(blockIdx.x) / per_jq;
+  int rem = static_cast<int>(blockIdx.x) % per_jq;
+  const int n = rem / (g.Hkv * npairs);
+  rem %= g.Hkv * npairs;
+  const int kvh = rem / npairs;
+  const int pair = rem % npairs;
+  int seq_start, len;
+  seq_bounds(g.si, n, seq_start, len);
+  if (jq * C::BM >= len) return;  // the whole CTA leaves before touching TMEM
+  const int nq_tiles = (2 * pair + 1 < G) ? 2 : 1;
+  const int nkv = jq + 1;
+  const int q0 = jq * C::BM;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;            // [ST]
+  uint64_t* kv_empty = bars + 1 + C::ST;   // [ST]
+  uint64_t* s_full = bars + 1 + 2 * C::ST; // [NQ]
+  uint64_t* p_full = s_full + C::NQ;       // [NQ]
+  uint64_t* o_final = p_full + C::NQ;      // [NQ]
+  uint64_t* drain = o_final + C::NQ;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < C::ST; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int t = 0; t < C::NQ; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(p_full + t, 128);
+      mbar_init(o_final + t, 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, a.status, a.budget_ns};
+
+  int p_of[2], h_of[2];
+  for (int t = 0; t < 2; ++t) {
+    const int qh = min(2 * pair + t, G - 1);
+    p_of[t] = qh / gsz;
+    h_of[t] = kvh * gsz + qh % gsz;
+  }
+
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      mbar_arrive_expect_tx(q_full, nq_tiles * C::TILE);
+      for (int t = 0; t < nq_tiles; ++t)
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &map_q, q_full, c * 64, seq_start + q0,
+                      p_of[t] * g.H + h_of[t]);
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % C::ST;
+        if (j >= C::ST && !wait_bounded(kv_empty + s, ((j / C::ST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
+        mbar_arrive_expect_tx(kv_full + s, 2 * C::TILE);
+        const int krow = seq_start + j * C::BN;
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d(sK + s * C::TILE + c * C::CHUNK, &map_k, kv_full + s, c * 64, krow, kvh);
+          tma_load_3d(sV + s * C::TILE + c * C::CHUNK, &map_v, kv_full + s, c * 64, kvh, krow);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, false, false);
+      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
+      const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK), vb = smem_u32(sV);
+      auto issue_s = [&](int t, int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_ss(tmem + C::COL_S0 + 128 * t, sdesc_sw128(qa + t * C::TILE + off, 16, 1024),
+                  sdesc_sw128(kb + s * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          umma_ts(tmem + C::COL_O0 + D * t, tmem + C::COL_S0 + 128 * t + kk * 8,
+                  sdesc_sw128(vb + s * C::TILE + kk * 2048, C::CHUNK, 1024), idO, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = wait_bounded(q_full, 0, wd, kSiteFwdQ);
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % C::ST;
+        if (!wait_bounded(kv_full + s, (j / C::ST) & 1, wd, kSiteFwdKvFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int t = 0; t < nq_tiles; ++t) {
+          if (j > 0) {
+            if (!wait_bounded(p_full + t, (j - 1) & 1, wd, kSiteFwdPFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(t, (j - 1) % C::ST, j - 1 > 0);
+          }
+          issue_s(t, s);
+          umma_commit(s_full + t);
+        }
+        if (!ok) break;
+        if (j > 0) umma_commit(kv_empty + (j - 1) % C::ST);
+      }
+      if (ok) {
+        for (int t = 0; t < nq_tiles; ++t) {
+          if (!wait_bounded(p_full + t, (nkv - 1) & 1, wd, kSiteFwdPFull)) break;
+          tc_fence_after();
+          issue_pv(t, (nkv - 1) % C::ST, nkv - 1 > 0);
+          umma_commit(o_final + t);
+        }
+      }
+      // nothing may still be running on the tensor cores when TMEM is released
+      umma_commit(drain);
+      wait_drain(drain, 0, wd, kSiteFwdDrain);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 4 + 4 * nq_tiles) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int qpos = q0 + row;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t colS = C::COL_S0 + 128 * t;
+    const uint32_t colO = C::COL_O0 + D * t;
+    const float sl2 = g.scale * kLog2e;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      if (!wait_bounded(s_full + t, j & 1, wd, kSiteFwdSFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + colS + 32 * c, sr[c]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
+      const int k0 = j * C::BN;
+      if (k0 + C::BN - 1 > qpos) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (k0 + 32 * c + e > qpos) sr[c][e] = __float_as_uint(-INFINITY);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const bool rescale = m_new > m_run + kRescaleThreshold;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = exp2_approx(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = exp2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_run));
+          const float p1 = exp2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_run));
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(lane_base + colS + 16 * c, pk);
+      }
+      l_run += rs;
+      if (rescale && j > 0) {
+        // O of this row was complete up to tile j-1 when s_full fired (in-order MMAs)
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + colO + 32 * c, o);
+          tmem_ld_wait();
+          reg_fence32(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(lane_base + colO + 32 * c, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full + t);
+    }
+    if (ok && wait_bounded(o_final + t, 0, wd, kSiteFwdOFinal)) {
+      tc_fence_after();
+      const bool valid = qpos < len;
+      const float inv_l = 1.f / l_run;
+      const int64_t rowid = static_cast<int64_t>(p_of[t] * g.H + h_of[t]) * g.si.T + seq_start + qpos;
+      float* dst = a.o_t + rowid * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + colO + 32 * c, o);
+        tmem_ld_wait();
+        reg_fence32(o);
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float4 v4 = make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
+                                    __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+            *reinterpret_cast<float4*>(dst + 32 * c + e) = v4;
+          }
+        }
+      }
+      if (valid) a.lse_t[rowid] = (m_run + __log2f(l_run)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+template <int D>
+cudaError_t launch(const TrunkFwdArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(trunk_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int G = a.g.P * (a.g.H / a.g.Hkv);
+  const int npairs = (G + 1) / 2;
+  const int njq = (a.g.si.max_len + C::BM - 1) / C::BM;
+  const long long blocks = static_cast<long long>(njq) * a.g.si.nseq * a.g.Hkv * npairs;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  trunk_fwd_kernel<D><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
+                             const CUtensorMap& map_v, cudaStream_t stream) {
+  return a.g.D == 128 ? launch<128>(a, map_q, map_k, map_v, stream) : launch<64>(a, map_q, map_k, map_v, stream);
+}
+
+}  // namespace ttt

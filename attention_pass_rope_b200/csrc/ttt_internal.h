@@ -1,0 +1,102 @@
+// Internal declarations shared by the host launcher (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ttt {
+
+// Status word values (first 32-bit word of the workspace).
+constexpr uint32_t kStatusTimeoutBase = 0x7100'0000u;  // | site code
+
+// Wait-site codes recorded on timeout (low bits of the status word).
+enum WaitSite : uint32_t {
+  kSiteSelftest = 1,
+  kSiteFwdQ = 0x10,
+  kSiteFwdKvFull = 0x11,
+  kSiteFwdKvEmpty = 0x12,
+  kSiteFwdSFull = 0x13,
+  kSiteFwdPFull = 0x14,
+  kSiteFwdOFinal = 0x15,
+  kSiteFwdDrain = 0x16,
+  kSiteBwdQdoFull = 0x20,
+  kSiteBwdQdoEmpty = 0x21,
+  kSiteBwdKv = 0x22,
+  kSiteBwdSdpFull = 0x23,
+  kSiteBwdDsReady = 0x24,
+  kSiteBwdMmaDone = 0x25,
+  kSiteBwdDqFull = 0x26,
+  kSiteBwdDqFree = 0x27,
+  kSiteBwdFinal = 0x28,
+  kSiteBwdDrain = 0x29,
+};
+
+// Where the sequences are: dense batches (cu_seqlens == nullptr) hold nseq = B
+// sequences of length S back to back; packed batches read cu_seqlens.
+struct SeqInfo {
+  const int32_t* cu_seqlens;  // device, nullptr for dense
+  int nseq;                   // B (dense) or number of sequences
+  int S;                      // dense sequence length (0 for packed)
+  int T;                      // total tokens (B*S or cu_seqlens[nseq])
+  int max_len;                // longest sequence
+};
+
+struct Geometry {
+  SeqInfo si;
+  int P, H, Hkv, D;
+  float theta;
+  float scale;  // softmax scale sigma
+};
+
+// ----------------------------------------------------------------- launchers
+// All launchers enqueue on `stream` and return the launch error.
+
+// a1: q~ = R(i+p) q (head-major [P][H][T][D]), k~ = R(i+p) k ([P][Hkv][T][D]), bf16.
+cudaError_t launch_rope_fwd(const Geometry& g, const void* q, const void* k, void* qr, void* kr,
+                            cudaStream_t stream);
+
+struct TrunkFwdArgs {
+  Geometry g;
+  float* o_t;      // fp32 [P][H][T][D]
+  float* lse_t;    // fp32 [P][H][T]
+  uint32_t* status;
+  uint64_t budget_ns;
+};
+// a2: trunk causal attention on tcgen05; maps: q~ (3D {D, T, P*H}), k~_1 (3D {D, T, Hkv}),
+// V_1 (3D {D, Hkv, T}), all 64-element (128-byte) swizzled boxes.
+cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
+                             const CUtensorMap& map_v, cudaStream_t stream);
+
+// a3+a4: branch keys (warp dot products) and the joint-LSE merge.
+cudaError_t launch_branch_merge_fwd(const Geometry& g, const void* qr, const void* kr, const void* v,
+                                    const float* o_t, const float* lse_t, void* o, float* lse,
+                                    cudaStream_t stream);
+
+// a5: delta = rowsum(dO * O) in the public lse layout.
+cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, float* delta,
+                                  cudaStream_t stream);
+
+struct TrunkBwdArgs {
+  Geometry g;
+  const float* lse;    // public layout
+  const float* delta;  // public lse layout
+  float* dq_acc;       // fp32 [P][H][T][D], zeroed before the launch
+  float* dk1_acc;      // fp32 [Hkv][T][D]  (unscaled sum of dS^T q~)
+  void* dv;            // bf16 public dv; pass 0 written here
+  uint32_t* status;
+  uint64_t budget_ns;
+};
+// a6: trunk backward on tcgen05; maps: q~ (box 64 rows), k~_1 (box 128 rows),
+// V_1 (box 128 rows), dO (3D {D, H, P*T}, box 64 rows).
+cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
+                             const CUtensorMap& map_v, const CUtensorMap& map_do, cudaStream_t stream);
+
+// a7+a8: branch backward, dq finalize (inverse RoPE), dk of every pass.
+cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr, const void* v,
+                              const void* dout, const float* lse, const float* delta, const float* dq_acc,
+                              const float* dk1_acc, void* dq, void* dk, void* dv, cudaStream_t stream);
+
+cudaError_t launch_watchdog_selftest(uint32_t* status, uint64_t budget_ns, cudaStream_t stream);
+
+}  // namespace ttt

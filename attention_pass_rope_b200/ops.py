@@ -1,0 +1,199 @@
+"""PyTorch-facing calls of the TTT trunk+branch attention.
+
+Argument marshalling only: tensors are checked for dtype/shape/device/contiguity,
+outputs and the workspace are allocated with torch, and the C ABI of
+libttt_attn.so is called on the current CUDA stream.  Every arithmetic step runs in
+the library's kernels; there is no other implementation to fall back to.
+
+Shapes (pass-major, trunk = index 0 along P):
+  dense:  q [P, B, S, H, D], k/v [P, B, S, Hkv, D]    -> o like q, lse [P, B, H, S]
+  packed: q [P, T, H, D],    k/v [P, T, Hkv, D] with cu_seqlens (int32, cuda)
+                                                      -> o like q, lse [P, H, T]
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+
+@dataclasses.dataclass
+class Layout:
+    P: int
+    H: int
+    Hkv: int
+    D: int
+    dense: bool
+    B: int = 0
+    S: int = 0
+    T: int = 0
+    nseq: int = 0
+    max_seqlen: int = 0
+    cu_seqlens: Optional[torch.Tensor] = None
+
+    @property
+    def lse_shape(self):
+        return (self.P, self.B, self.H, self.S) if self.dense else (self.P, self.H, self.T)
+
+
+def _layout(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens, max_seqlen) -> Layout:
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("q, k, v must be bfloat16")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    if cu_seqlens is None:
+        if q.dim() != 5:
+            raise ValueError("dense q must be [P, B, S, H, D]")
+        P, B, S, H, D = q.shape
+        Hkv = k.shape[3]
+        if k.shape != (P, B, S, Hkv, D) or v.shape != k.shape:
+            raise ValueError("k, v must be [P, B, S, Hkv, D]")
+        return Layout(P, H, Hkv, D, True, B=B, S=S, T=B * S, nseq=B, max_seqlen=S)
+    if q.dim() != 4:
+        raise ValueError("packed q must be [P, T, H, D]")
+    P, T, H, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (P, T, Hkv, D) or v.shape != k.shape:
+        raise ValueError("k, v must be [P, T, Hkv, D]")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+    if max_seqlen is None:
+        raise ValueError("max_seqlen is required with cu_seqlens")
+    return Layout(P, H, Hkv, D, False, T=T, nseq=cu_seqlens.numel() - 1, max_seqlen=int(max_seqlen),
+                  cu_seqlens=cu_seqlens.contiguous())
+
+
+def make_desc(lay: Layout, theta: float, scale: Optional[float], events=None) -> _lib.TTTDesc:
+    d = _lib.TTTDesc()
+    d.layout = _lib.TTT_LAYOUT_BSHD if lay.dense else _lib.TTT_LAYOUT_THD
+    d.P, d.H, d.Hkv, d.D = lay.P, lay.H, lay.Hkv, lay.D
+    d.B, d.S = lay.B, lay.S
+    d.rope_theta = float(theta)
+    d.softmax_scale = 0.0 if scale is None else float(scale)
+    if not lay.dense:
+        d.cu_seqlens = lay.cu_seqlens.data_ptr()
+        d.nseq, d.total_tokens, d.max_seqlen = lay.nseq, lay.T, lay.max_seqlen
+    d.events = ctypes.addressof(events) if events is not None else None
+    return d
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def workspace_bytes(lay: Layout, theta: float, scale=None, for_backward=False) -> int:
+    d = make_desc(lay, theta, scale)
+    n = _lib.lib().ttt_attn_workspace_size(ctypes.byref(d), int(for_backward))
+    if n == 0 and lay.T > 0:
+        raise _lib.TTTError(_lib.TTT_ERR_INVALID_ARG, "ttt_attn_workspace_size")
+    return int(n)
+
+
+def workspace_layout(lay: Layout, theta: float, scale=None, for_backward=False) -> list:
+    d = make_desc(lay, theta, scale)
+    offs = (ctypes.c_size_t * 8)()
+    n = _lib.lib().ttt_attn_workspace_layout(ctypes.byref(d), int(for_backward), offs)
+    return [int(offs[i]) for i in range(n)]
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def ttt_attn_fwd(q, k, v, *, theta: float, scale: Optional[float] = None, cu_seqlens=None, max_seqlen=None,
+                 workspace: Optional[torch.Tensor] = None, out=None, events=None):
+    """Forward: returns (o, lse).  ``out=(o, lse)`` writes into given tensors."""
+    lay = _layout(q, k, v, cu_seqlens, max_seqlen)
+    _contig(q, k, v)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(lay.lse_shape, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    desc = make_desc(lay, theta, scale, events)
+    L = _lib.lib()
+    need = L.ttt_attn_workspace_size(ctypes.byref(desc), 0)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = L.ttt_attn_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _stream())
+    _lib.check(st, "ttt_attn_fwd")
+    return o, lse
+
+
+def ttt_attn_bwd(q, k, v, o, lse, dout, *, theta: float, scale: Optional[float] = None, cu_seqlens=None,
+                 max_seqlen=None, workspace: Optional[torch.Tensor] = None, out=None, events=None):
+    """Backward: returns (dq, dk, dv) with respect to the pre-RoPE q, k, v."""
+    lay = _layout(q, k, v, cu_seqlens, max_seqlen)
+    _contig(q, k, v, o, lse, dout)
+    if dout.dtype != torch.bfloat16 or o.dtype != torch.bfloat16 or lse.dtype != torch.float32:
+        raise TypeError("o, dout must be bfloat16 and lse float32")
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    desc = make_desc(lay, theta, scale, events)
+    L = _lib.lib()
+    need = L.ttt_attn_workspace_size(ctypes.byref(desc), 1)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = L.ttt_attn_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                        _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                        _stream())
+    _lib.check(st, "ttt_attn_bwd")
+    return dq, dk, dv
+
+
+def device_status(workspace: torch.Tensor) -> tuple:
+    """(status, raw word) of the bounded in-kernel waits of the last call (synchronises)."""
+    word = ctypes.c_uint32(0)
+    st = _lib.lib().ttt_attn_device_status(_ptr(workspace), _stream(), ctypes.byref(word))
+    return st, word.value
+
+
+def watchdog_selftest(workspace: torch.Tensor, budget_ns: int) -> int:
+    st = _lib.lib().ttt_attn_watchdog_selftest(_ptr(workspace), workspace.numel(), int(budget_ns), _stream())
+    _lib.check(st, "ttt_attn_watchdog_selftest")
+    return st
+
+
+def set_wait_budget_ns(budget_ns: int) -> None:
+    _lib.lib().ttt_attn_set_wait_budget_ns(int(budget_ns))
+
+
+class _TTTAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, theta, scale, cu_seqlens, max_seqlen):
+        o, lse = ttt_attn_fwd(q, k, v, theta=theta, scale=scale, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)
+        ctx.save_for_backward(q, k, v, o, lse, cu_seqlens)
+        ctx.theta, ctx.scale, ctx.max_seqlen = theta, scale, max_seqlen
+        ctx.has_cu = cu_seqlens is not None
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse, cu = ctx.saved_tensors
+        dq, dk, dv = ttt_attn_bwd(q, k, v, o, lse, do.contiguous(), theta=ctx.theta, scale=ctx.scale,
+                                  cu_seqlens=cu if ctx.has_cu else None, max_seqlen=ctx.max_seqlen)
+        return dq, dk, dv, None, None, None, None
+
+
+def ttt_attention(q, k, v, *, theta: float, scale: Optional[float] = None, cu_seqlens=None, max_seqlen=None):
+    """Differentiable TTT trunk+branch attention (autograd over the C ABI)."""
+    return _TTTAttention.apply(q, k, v, theta, scale, cu_seqlens, max_seqlen)

@@ -1,0 +1,379 @@
+"""Throughput of the TTT trunk+branch attention, forward + backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one forward and one backward (every kernel of the path) over one batch
+of the workload, inputs resident in HBM; the algorithmic work is 14*D flops per
+visible (query, trunk key) pair per query head and pass plus the branch keys.
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own copy of the
+workload (independent batches, no collective): weak scaling.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (one sequence and one KV head group), scaled to the metric's unit.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import ttt_inputs  # noqa: E402
+
+METRIC = "TTT attention fwd+bwd TFLOP/s and tokens/s at 1 B200; % of bf16 tensor peak"
+DEFAULT_WORKLOAD = "qwen3_8b_4k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- ours
+
+def run_ours(args, rank, world, local):
+    from attention_pass_rope_b200 import _lib, ops
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    w = ttt_inputs.workloads()[args.workload]
+    # every rank draws its own batch (weak scaling); the sizes are the workload's
+    inp = ttt_inputs.make_inputs(w, seed=w.seed + rank)
+
+    def dev(t):
+        t = t.to(device)
+        if w.dense:
+            t = t.view(t.shape[0], len(w.lengths), w.lengths[0], *t.shape[2:])
+        return t.contiguous()
+
+    q, k, v, do = dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.do)
+    cu = None if w.dense else torch.tensor(w.cu_seqlens, dtype=torch.int32, device=device)
+    kw = dict(theta=w.theta, cu_seqlens=cu, max_seqlen=None if w.dense else w.max_seqlen)
+    lay = ops._layout(q, k, v, cu, kw["max_seqlen"])
+    ws = ops.alloc_workspace(max(ops.workspace_bytes(lay, w.theta), ops.workspace_bytes(lay, w.theta, for_backward=True)),
+                             device)
+    o = torch.empty_like(q)
+    lse = torch.empty(lay.lse_shape, dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    # per-kernel CUDA events, recorded by the library on the launching stream
+    K = args.steps
+    evs = [_lib.TTTEvents() for _ in range(K)]
+    ev_objs = []
+    for e in evs:
+        objs = []
+        for kk in range(len(_lib.KERNELS)):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e.start[kk] = a.cuda_event
+            e.stop[kk] = b.cuda_event
+            objs.append((a, b))
+        ev_objs.append(objs)
+
+    def step(events=None):
+        ops.ttt_attn_fwd(q, k, v, workspace=ws, out=(o, lse), events=events, **kw)
+        ops.ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, out=(dq, dk, dv), events=events, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, word = ops.device_status(ws)
+    if st != _lib.TTT_OK:
+        raise RuntimeError(f"device status after warm-up: {st} {word:#x}")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K):
+        step(evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    per_kernel = {}
+    for kk, name in enumerate(_lib.KERNELS):
+        per_kernel[name] = sum(ev_objs[i][kk][0].elapsed_time(ev_objs[i][kk][1]) for i in range(K)) / K
+    st, word = ops.device_status(ws)
+    if st != _lib.TTT_OK:
+        raise RuntimeError(f"device status after timing: {st} {word:#x}")
+
+    # end to end: pinned host inputs -> device, fwd+bwd, results back to pinned host memory
+    host_in = [t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.do)]
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    dev_in = [q, k, v, do]
+
+    def e2e_step():
+        for hsrc, dst in zip(host_in, dev_in):
+            dst.view(-1).copy_(hsrc.view(-1), non_blocking=True)
+        step()
+        for src, hdst in zip((o, lse, dq, dk, dv), host_out):
+            hdst.copy_(src, non_blocking=True)
+
+    E = max(1, min(K, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(E):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms], device=device)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), float(tt[1])
+
+    ms_step = ms / K
+    flops = w.flops_fwd_bwd()
+    tflops = flops * world / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops_sustained"]
+    # dominant kernel: the trunk backward (tensor bound); its algorithmic flops per launch
+    # are 10*D per visible trunk pair per query head and pass
+    bwd_flops = 10 * w.D * w.trunk_pairs * w.H * w.P
+    bwd_ms = per_kernel["trunk_bwd"]
+    achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    traffic = read_traffic("trunk_bwd", args.workload)
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={len(w.lengths)} S={w.lengths[0]} P={w.P} H={w.H}/{w.Hkv} D={w.D} "
+                               f"theta={w.theta:g}" if w.dense else
+                   f"{w.name}: THD nseq={w.nseq} T={w.T} P={w.P} H={w.H}/{w.Hkv} D={w.D} theta={w.theta:g}",
+                   "tokens_per_step": w.T, "flops_per_step": flops, "parallelism": f"replicas{world}",
+                   "l2": "inputs per step (q,k,v,dO: %.0f MB) exceed L2 (126 MB)" % (h2d / 1e6)},
+        "tokens_per_s": round(w.T * world / (ms_step * 1e-3), 1),
+        "pct_of_peak": round(100.0 * tflops / world / peak, 2),
+        "kernel_ms": {k_: round(v_, 4) for k_, v_ in per_kernel.items()},
+        "roofline": {"kernel": "trunk_bwd", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
+                     "traffic": traffic},
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 7 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def read_traffic(kernel, workload):
+    """dram bytes per launch from the committed ncu summary, if one matches the kernel."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            return json.load(f).get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------------------- oracle
+
+def oracle_sample(w, n_groups=1):
+    """The bounded sample: sequence 0, KV heads 0..n_groups-1 (all their query heads
+    and passes), fwd + bwd.  Returns (seconds, flops of the sample)."""
+    import numpy as np
+    from oracle import ttt_oracle as orc
+
+    inp = ttt_inputs.make_inputs(w)
+    a, b = w.cu_seqlens[0], w.cu_seqlens[1]
+    g = w.H // w.Hkv
+    kvs = list(range(n_groups))
+    heads = [h for kv in kvs for h in range(kv * g, (kv + 1) * g)]
+    q = inp.q[:, a:b].double().numpy()
+    k = inp.k[:, a:b].double().numpy()
+    v = inp.v[:, a:b].double().numpy()
+    do = inp.do[:, a:b].double().numpy()
+    t0 = time.perf_counter()
+    O, lse = orc.forward_twopart(q, k, v, w.theta, heads=heads)
+    orc.backward_twopart(q, k, v, do, lse, w.theta, kv_heads=kvs)
+    dt = time.perf_counter() - t0
+    L = b - a
+    sub = ttt_inputs.thd("sample", [L], w.P, len(heads), n_groups, w.D, w.theta)
+    return dt, sub.flops_fwd_bwd(), np
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 0) for i in threadpool_info()), default=None)
+    except Exception:
+        return None
+
+
+def cpu_baseline(w, budget_s=30.0):
+    dt, fl, _ = oracle_sample(w)
+    cores = blas_threads() or len(os.sched_getaffinity(0))
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, fwd+bwd of sequence 0 and KV head 0 ({w.H // w.Hkv} query heads x "
+                      f"{w.P} passes x {w.lengths[0]} positions) = 1/{w.nseq * w.Hkv} of the workload, {dt:.1f} s",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = ttt_inputs.workloads()[args.workload]
+    for _ in range(args.warmup and 1):
+        pass  # the oracle has no warm-up state; one untimed sample below warms the BLAS pool
+    oracle_sample(ttt_inputs.thd("warm", [256], w.P, w.H // w.Hkv, 1, w.D, w.theta))
+    times, fl = [], None
+    for _ in range(args.steps):
+        dt, fl, _ = oracle_sample(w)
+        times.append(dt)
+    dt = sum(times) / len(times)
+    value = fl / dt / 1e12
+    cores = blas_threads() or len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "parallelism": "cpu oracle, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"sequence 0, KV head 0 of {args.workload} per step"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ttt_inputs.workloads()))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=30.0)
+    args = ap.parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

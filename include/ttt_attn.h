@@ -1,0 +1,157 @@
+/*
+ * ttt_attn.h — C ABI of libttt_attn.so: forward and backward of the multi-pass
+ * EAGLE-3 test-time-training (TTT) trunk+branch attention on NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  Sources: "DFlash/DSpark and EAGLE-3 TTT draft co-training for
+ * speculative decoding (Megatron backend)" (NeMo-RL issue 3698), section "What I'm
+ * working on", items 1 and 4; "bounded multi-pass EAGLE-3 TTT provider" (NeMo-RL
+ * PR 3725), Summary and self-review.
+ *
+ *   For pass p = 1..P, query head h, sequence position i (0-based within its
+ *   sequence), with kv(h) = h / (H / Hkv) and sigma the softmax scale:
+ *     q~_p[i] = R(i+p-1) Q_p[i],  k~_p[i] = R(i+p-1) K_p[i]      (rotate-half RoPE)
+ *     trunk keys:  k~_1[t], V_1[t]  for t = 0..i                   (causal)
+ *     branch keys: k~_j[i], V_j[i]  for j = 2..p                   (staircase)
+ *     s = sigma * q~_p[i] . k ;  lse_t, O_t over the trunk keys, lse_b, O_b over
+ *     the branch keys (empty for p = 1: lse_b = -inf);
+ *     lse = logaddexp(lse_t, lse_b),  O = e^(lse_t-lse) O_t + e^(lse_b-lse) O_b.
+ *   This equals one softmax over the (i+1)+(p-1) visible keys.  The rotated q~ and
+ *   k~ are computed in fp32 and rounded to bf16 before the dot products.
+ *   R(m) pairs dimension d with d + D/2 and rotates by m * theta^(-2d/D).
+ *
+ * Layouts (all pass-major, the trunk is index 0 along P, row-major, contiguous):
+ *   dense (TTT_LAYOUT_BSHD):  q, o, dout, dq  [P][B][S][H][D]    bf16
+ *                             k, v, dk, dv    [P][B][S][Hkv][D]  bf16
+ *                             lse             [P][B][H][S]       fp32 (natural log)
+ *   packed (TTT_LAYOUT_THD):  q, o, dout, dq  [P][T][H][D], k, v, dk, dv [P][T][Hkv][D],
+ *                             lse [P][H][T]; sequences given by cu_seqlens (int32,
+ *                             device memory, nseq+1 entries, cu_seqlens[0] = 0,
+ *                             non-decreasing, cu_seqlens[nseq] = T); positions restart
+ *                             at 0 at every sequence start and no attention crosses
+ *                             a sequence boundary.
+ *   Supported: D in {64, 128}; H a multiple of Hkv; 1 <= P <= 16.
+ *
+ * Ownership.  Every pointer is device memory owned by the caller, including the
+ * workspace, whose size ttt_attn_workspace_size() returns.  The library allocates
+ * nothing and keeps no state between calls.  Outputs must not alias inputs.
+ *
+ * Asynchrony and errors.  Calls enqueue work on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and return without synchronising.  Argument errors
+ * are reported before anything is enqueued.  TTT_ERR_CUDA reports a launch error.
+ * Every wait inside the kernels is bounded; a wait that runs out records its site
+ * in the workspace status word and the kernel exits cleanly;
+ * ttt_attn_device_status() synchronises the stream and reports it as
+ * TTT_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef TTT_ATTN_H_
+#define TTT_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = 1,    /* null pointer, bad size, inconsistent shape */
+  TTT_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. D = 96) */
+  TTT_ERR_WORKSPACE = 3,      /* workspace missing, too small or misaligned */
+  TTT_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+  TTT_ERR_DEVICE_TIMEOUT = 5  /* a bounded in-kernel wait ran out */
+} ttt_status;
+
+typedef enum { TTT_LAYOUT_BSHD = 0, TTT_LAYOUT_THD = 1 } ttt_layout;
+
+/* Optional per-kernel timing: when the descriptor points at one of these, each
+ * kernel k of a call is bracketed by cudaEventRecord(start[k]) / (stop[k]) on the
+ * call's stream (entries left NULL are skipped).  Indices: TTT_KERNEL_*. */
+enum {
+  TTT_KERNEL_ROPE_FWD = 0,
+  TTT_KERNEL_TRUNK_FWD = 1,
+  TTT_KERNEL_BRANCH_MERGE_FWD = 2,
+  TTT_KERNEL_ROPE_BWD = 3,
+  TTT_KERNEL_BWD_PREPROCESS = 4,
+  TTT_KERNEL_TRUNK_BWD = 5,
+  TTT_KERNEL_BRANCH_BWD = 6,
+  TTT_KERNEL_COUNT = 8
+};
+typedef struct {
+  void* start[TTT_KERNEL_COUNT]; /* cudaEvent_t */
+  void* stop[TTT_KERNEL_COUNT];  /* cudaEvent_t */
+} ttt_attn_events;
+
+typedef struct {
+  int layout;          /* ttt_layout */
+  int P;               /* TTT passes (1 = plain causal attention) */
+  int B, S;            /* dense: batch and sequence length (ignored for THD) */
+  int H, Hkv, D;       /* query heads, KV heads, head dimension */
+  float rope_theta;    /* RoPE base, > 0 */
+  float softmax_scale; /* 0 selects 1/sqrt(D) */
+  const int32_t* cu_seqlens; /* THD only: device int32[nseq+1] */
+  int nseq;            /* THD only: number of sequences */
+  int total_tokens;    /* THD only: T = cu_seqlens[nseq] */
+  int max_seqlen;      /* THD only: upper bound on every sequence length */
+  const ttt_attn_events* events; /* optional, NULL for none */
+} ttt_attn_desc;
+
+/* Bytes of workspace that ttt_attn_fwd (for_backward = 0) or ttt_attn_bwd
+ * (for_backward = 1) needs for `desc`; 0 if the descriptor is invalid.  The
+ * workspace must be 256-byte aligned. */
+size_t ttt_attn_workspace_size(const ttt_attn_desc* desc, int for_backward);
+
+/* Forward.  q, k, v: bf16 pre-RoPE inputs (layouts above).  o: bf16 output, same
+ * layout as q.  lse: fp32 merged log-sum-exp (natural log of the sum of
+ * exp(sigma * q~.k) over the visible keys).  The workspace holds, after the call,
+ * the rotated q~ / k~ and the trunk partials (see ttt_attn_workspace_layout). */
+ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, void* o,
+                        float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of the forward above, recomputing the probabilities from the merged
+ * lse.  dout: bf16 gradient of o.  dq, dk, dv: bf16 gradients with respect to the
+ * PRE-RoPE q, k and v (the RoPE rotation is transposed; its bf16 rounding is
+ * treated as the identity).  o and lse must be the forward's outputs for the same
+ * inputs.  dk/dv of the trunk pass collect every pass and query head of the
+ * group; those of branch pass j collect passes p >= j at the same position. */
+ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream` and returns TTT_OK if no bounded wait of the calls made
+ * with this workspace ran out since the last check, TTT_ERR_DEVICE_TIMEOUT (and
+ * the raw status word in *detail if non-NULL) otherwise, or TTT_ERR_CUDA.  The
+ * status word is cleared. */
+ttt_status ttt_attn_device_status(void* workspace, void* stream, uint32_t* detail);
+
+/* Workspace sub-buffers (byte offsets from the workspace base), for inspection of
+ * the intermediate results by tests:
+ *   fwd: [0] status word, [1] q~ bf16 [P][H][Tt][D], [2] k~ bf16 [P][Hkv][Tt][D],
+ *        [3] O_t fp32 [P][H][Tt][D] (trunk-only normalised output),
+ *        [4] lse_t fp32 [P][H][Tt] (trunk-only log-sum-exp);
+ *   bwd: [0] status, [1] q~, [2] k~, [3] delta fp32 (lse layout),
+ *        [4] dq~ accumulator fp32 [P][H][Tt][D], [5] dk~_1 accumulator fp32 [Hkv][Tt][D].
+ * Tt = B*S (dense) or T (packed).  Returns the number of entries written to
+ * offsets (at most 8), or 0 for an invalid descriptor. */
+int ttt_attn_workspace_layout(const ttt_attn_desc* desc, int for_backward, size_t* offsets);
+
+/* Self-test of the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing will ever complete, with a limit of budget_ns nanoseconds.
+ * The kernel gives up, records the timeout in the workspace status word and
+ * exits; read it back with ttt_attn_device_status().  No other work is done. */
+ttt_status ttt_attn_watchdog_selftest(void* workspace, size_t workspace_bytes, uint64_t budget_ns, void* stream);
+
+/* Limit, in nanoseconds, for every in-kernel wait of later calls (default 2e9).
+ * Process-wide setting. */
+void ttt_attn_set_wait_budget_ns(uint64_t budget_ns);
+
+const char* ttt_status_string(ttt_status status);
+
+/* Library version, e.g. "0.1.0". */
+const char* ttt_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_ATTN_H_ */

@@ -1,0 +1,100 @@
+"""Helpers for comparing the CUDA path with the fp64 oracle (test code only)."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import ttt_inputs
+from oracle import ttt_oracle as orc
+
+# Tolerances from the method's accuracy statement: bf16 inputs, fp32 accumulation.
+O_MAX_ABS = 2e-2
+LSE_MAX_ABS = 1e-3
+GRAD_REL_L2 = 1e-2
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
+    a = a.ravel()
+    b = b.ravel()
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def gpu_shapes(w: ttt_inputs.Workload, inp: ttt_inputs.Inputs, device="cuda"):
+    """Move inputs to the device in the public layout of the workload."""
+    def dev(t):
+        if t is None:
+            return None
+        t = t.to(device)
+        if w.dense:
+            B, S = len(w.lengths), w.lengths[0]
+            t = t.view(t.shape[0], B, S, *t.shape[2:])
+        return t.contiguous()
+    cu = None
+    if not w.dense:
+        cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device=device)
+    return dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.do), cu
+
+
+def flat(t: torch.Tensor, w) -> torch.Tensor:
+    """[P, B, S, ...] -> [P, T, ...] (dense); packed tensors unchanged."""
+    if w.dense:
+        return t.reshape(t.shape[0], -1, *t.shape[3:])
+    return t
+
+
+def run_gpu(w, inp, with_grad=True):
+    from attention_pass_rope_b200 import ttt_attn_bwd, ttt_attn_fwd
+    q, k, v, do, cu = gpu_shapes(w, inp)
+    kw = dict(theta=w.theta, cu_seqlens=cu, max_seqlen=None if w.dense else w.max_seqlen)
+    o, lse = ttt_attn_fwd(q, k, v, **kw)
+    out = {"o": flat(o, w), "lse": lse}
+    if with_grad:
+        dq, dk, dv = ttt_attn_bwd(q, k, v, o, lse, do, **kw)
+        out.update(dq=flat(dq, w), dk=flat(dk, w), dv=flat(dv, w))
+    torch.cuda.synchronize()
+    return out
+
+
+def oracle_np(inp):
+    return tuple(to64(t) if t is not None else None for t in (inp.q, inp.k, inp.v, inp.do))
+
+
+def compare_full(w, inp, gpu, with_grad=True, kv_heads=None, seqs=None):
+    """Oracle on (a subset of) the workload, element-wise comparison.  Returns metrics."""
+    q, k, v, do = oracle_np(inp)
+    cu = w.cu_seqlens
+    heads = None
+    if kv_heads is not None:
+        g = w.H // w.Hkv
+        heads = [h for kv in kv_heads for h in range(kv * g, (kv + 1) * g)]
+    O, lse = orc.forward_packed(q, k, v, cu, w.theta, w.dense, heads=heads, seqs=seqs)
+    m = {}
+    Og = to64(gpu["o"])
+    lg = to64(gpu["lse"])
+    sel = ~np.isnan(O)
+    m["o_max_abs"] = float(np.max(np.abs(Og[sel] - O[sel])))
+    sl = ~np.isnan(lse)
+    m["lse_max_abs"] = float(np.max(np.abs(lg[sl] - lse[sl])))
+    assert np.all(np.isfinite(Og)) and np.all(np.isfinite(lg))
+    if with_grad:
+        # rows outside the sampled subset are NaN in the oracle lse and never read
+        dq, dk, dv = orc.backward_packed(q, k, v, do, lse, cu, w.theta, w.dense, kv_heads=kv_heads, seqs=seqs)
+        for name, ref in (("dq", dq), ("dk", dk), ("dv", dv)):
+            got = to64(gpu[name])
+            s = ~np.isnan(ref)
+            assert np.all(np.isfinite(got))
+            m[name + "_rel_l2"] = rel_l2(got[s], ref[s])
+    return m
+
+
+def assert_within(m):
+    assert m["o_max_abs"] <= O_MAX_ABS, m
+    assert m["lse_max_abs"] <= LSE_MAX_ABS, m
+    for k in ("dq_rel_l2", "dk_rel_l2", "dv_rel_l2"):
+        if k in m:
+            assert m[k] <= GRAD_REL_L2, m

@@ -1,0 +1,132 @@
+"""C ABI checks that need no GPU: the library loads, exports every function the
+header declares, sizes workspaces and rejects bad arguments before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_pass_rope_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ttt_attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "ttt_attn_fwd" in names and "ttt_attn_bwd" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def desc(**kw):
+    d = _lib.TTTDesc()
+    d.layout, d.P, d.B, d.S, d.H, d.Hkv, d.D = 0, 3, 2, 4096, 32, 8, 128
+    d.rope_theta, d.softmax_scale = 1e6, 0.0
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_workspace_size_dense(L):
+    d = desc()
+    fwd = L.ttt_attn_workspace_size(ctypes.byref(d), 0)
+    bwd = L.ttt_attn_workspace_size(ctypes.byref(d), 1)
+    P, T, H, Hkv, D = 3, 8192, 32, 8, 128
+    assert fwd >= P * T * H * D * 2 + P * T * Hkv * D * 2 + P * T * H * D * 4 + P * H * T * 4
+    assert bwd >= P * T * H * D * 2 + P * T * Hkv * D * 2 + P * H * T * 4 + P * T * H * D * 4 + Hkv * T * D * 4
+    offs = (ctypes.c_size_t * 8)()
+    n = L.ttt_attn_workspace_layout(ctypes.byref(d), 0, offs)
+    assert n == 5
+    assert all(offs[i] % 1024 == 0 for i in range(1, n))
+    assert list(offs[:n]) == sorted(offs[:n])
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("D", 96, _lib.TTT_ERR_UNSUPPORTED),
+    ("D", 0, _lib.TTT_ERR_INVALID_ARG),
+    ("H", 30, _lib.TTT_ERR_INVALID_ARG),      # not a multiple of Hkv
+    ("P", 0, _lib.TTT_ERR_INVALID_ARG),
+    ("P", 17, _lib.TTT_ERR_UNSUPPORTED),
+    ("rope_theta", 0.0, _lib.TTT_ERR_INVALID_ARG),
+    ("rope_theta", -1.0, _lib.TTT_ERR_INVALID_ARG),
+    ("softmax_scale", -0.5, _lib.TTT_ERR_INVALID_ARG),
+    ("layout", 7, _lib.TTT_ERR_INVALID_ARG),
+    ("B", -1, _lib.TTT_ERR_INVALID_ARG),
+])
+def test_invalid_descriptor(L, field, value, status):
+    d = desc(**{field: value})
+    assert L.ttt_attn_workspace_size(ctypes.byref(d), 0) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    st = L.ttt_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, fake, 1 << 40, None)
+    assert st == status
+
+
+def test_null_descriptor(L):
+    assert L.ttt_attn_fwd(None, None, None, None, None, None, None, 0, None) == _lib.TTT_ERR_INVALID_ARG
+    assert L.ttt_attn_workspace_size(None, 0) == 0
+
+
+def test_null_tensor_pointers(L):
+    d = desc()
+    fake = ctypes.c_void_p(1 << 20)
+    st = L.ttt_attn_fwd(ctypes.byref(d), None, fake, fake, fake, fake, fake, 1 << 40, None)
+    assert st == _lib.TTT_ERR_INVALID_ARG
+    st = L.ttt_attn_bwd(ctypes.byref(d), fake, fake, fake, fake, fake, None, fake, fake, fake, fake, 1 << 40, None)
+    assert st == _lib.TTT_ERR_INVALID_ARG
+
+
+def test_misaligned_tensor(L):
+    d = desc()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    st = L.ttt_attn_fwd(ctypes.byref(d), odd, fake, fake, fake, fake, fake, 1 << 40, None)
+    assert st == _lib.TTT_ERR_INVALID_ARG
+
+
+def test_workspace_errors(L):
+    d = desc()
+    fake = ctypes.c_void_p(1 << 20)
+    need = L.ttt_attn_workspace_size(ctypes.byref(d), 0)
+    st = L.ttt_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, fake, need - 1, None)
+    assert st == _lib.TTT_ERR_WORKSPACE
+    st = L.ttt_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, None, need, None)
+    assert st == _lib.TTT_ERR_WORKSPACE
+    st = L.ttt_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, ctypes.c_void_p((1 << 20) + 64), need, None)
+    assert st == _lib.TTT_ERR_WORKSPACE
+
+
+def test_packed_layout_validation(L):
+    d = desc(layout=1, nseq=2, total_tokens=100, max_seqlen=60)
+    assert L.ttt_attn_workspace_size(ctypes.byref(d), 0) == 0       # cu_seqlens missing
+    d.cu_seqlens = 1 << 20
+    assert L.ttt_attn_workspace_size(ctypes.byref(d), 0) > 0
+    d.max_seqlen = 101                                               # longer than the batch
+    assert L.ttt_attn_workspace_size(ctypes.byref(d), 0) == 0
+
+
+def test_empty_batch_is_a_no_op(L):
+    d = desc(B=0)
+    assert L.ttt_attn_fwd(ctypes.byref(d), None, None, None, None, None, None, 0, None) == _lib.TTT_OK
+    d = desc(layout=1, nseq=0, total_tokens=0, max_seqlen=0)
+    assert L.ttt_attn_bwd(ctypes.byref(d), None, None, None, None, None, None, None, None, None, None, 0,
+                          None) == _lib.TTT_OK
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.ttt_status_string(s)
+    assert L.ttt_attn_version().decode().count(".") == 2
