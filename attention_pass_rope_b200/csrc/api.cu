@@ -84,8 +84,8 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
     o = align_up(o + P * H * T * 4);
     pl.noff = 5;
   } else {
-    pl.off[3] = o;  // delta
-    o = align_up(o + P * H * T * 4);
+    pl.off[3] = o;  // tile-aligned row statistics (lse*log2e, delta)
+    o = align_up(o + P * H * static_cast<size_t>(ld_slots(g.si)) * 128 * 4);
     pl.off[4] = o;  // dq~ accumulator
     o = align_up(o + P * H * T * D * 4);
     pl.off[5] = o;  // dk~_1 accumulator
@@ -228,7 +228,7 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + pl.off[0]);
   void* qr = ws + pl.off[1];
   void* kr = ws + pl.off[2];
-  float* delta = reinterpret_cast<float*>(ws + pl.off[3]);
+  float* ld = reinterpret_cast<float*>(ws + pl.off[3]);
   float* dq_acc = reinterpret_cast<float*>(ws + pl.off[4]);
   float* dk1_acc = reinterpret_cast<float*>(ws + pl.off[5]);
   const uint64_t T = g.si.T, D = g.D;
@@ -247,17 +247,17 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
-    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, delta, stream));
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, stream));
     TTT_CHECK_CUDA(cudaMemsetAsync(dq_acc, 0, static_cast<size_t>(g.P) * g.H * T * D * 4, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);
-    TrunkBwdArgs a{g, lse, delta, dq_acc, dk1_acc, dv, status, g_wait_budget_ns.load()};
+    TrunkBwdArgs a{g, ld, dq_acc, dk1_acc, dv, status, g_wait_budget_ns.load()};
     TTT_CHECK_CUDA(launch_trunk_bwd(a, mq, mk, mv, mdo, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BRANCH_BWD, stream);
-    TTT_CHECK_CUDA(launch_branch_bwd(g, qr, kr, v, dout, lse, delta, dq_acc, dk1_acc, dq, dk, dv, stream));
+    TTT_CHECK_CUDA(launch_branch_bwd(g, qr, kr, v, dout, lse, ld, dq_acc, dk1_acc, dq, dk, dv, stream));
   }
   return TTT_OK;
 }

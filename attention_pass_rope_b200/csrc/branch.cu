@@ -185,12 +185,13 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 }
 
 // ---------------------------------------------------------------------------
-// a5: delta = rowsum(dO * O), written in the public lse layout.
+// a5: delta = rowsum(dO * O).  Written, with lse * log2(e), into the tile-aligned
+// row-statistics array that the trunk backward fetches one 512-byte slot at a time.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     bwd_preprocess_kernel(Geometry g, const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                          float* __restrict__ delta) {
+                          const float* __restrict__ lse, float* __restrict__ ld) {
   const int lane = threadIdx.x & 31;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   const int T = g.si.T;
@@ -207,7 +208,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   if (lane == 0) {
     int n, pos;
     token_position(g.si, tau, n, pos);
-    delta[lse_index(g.si, g.H, p, h, n, tau, pos)] = s;
+    const int slot = ld_slot(tau - pos, n, pos);
+    float* row = ld + ((static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + slot) * 128;
+    row[pos & 63] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)] * 1.4426950408889634f;
+    row[64 + (pos & 63)] = s;
   }
 }
 
@@ -226,7 +230,7 @@ template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     branch_bwd_kernel(Geometry g, const __nv_bfloat16* __restrict__ qr, const __nv_bfloat16* __restrict__ kr,
                       const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
-                      const float* __restrict__ lse, const float* __restrict__ delta,
+                      const float* __restrict__ lse, const float* __restrict__ ld,
                       const float* __restrict__ dq_acc, const float* __restrict__ dk1_acc,
                       __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
   extern __shared__ float acc_smem[];
@@ -266,7 +270,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         load_bf16_row<D>(dout + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D, lane, dO);
         const int64_t li = lse_index(g.si, g.H, p, h, n, tau, pos);
         const float lse_v = lse[li];
-        const float dl = delta[li];
+        const float dl = ld[((static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + ld_slot(tau - pos, n, pos)) * 128 +
+                            64 + (pos & 63)];
         for (int j = 1; j <= p; ++j) {
           float kj[2][D / 64], vj[2][D / 64];
           load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
@@ -365,21 +370,21 @@ cudaError_t launch_branch_merge_fwd(const Geometry& g, const void* qr, const voi
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, float* delta,
+cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
                                   cudaStream_t stream) {
   const int64_t warps = static_cast<int64_t>(g.P) * g.si.T * g.H;
   if (warps == 0) return cudaSuccess;
   auto* ob = static_cast<const __nv_bfloat16*>(o);
   auto* db = static_cast<const __nv_bfloat16*>(dout);
   if (g.D == 128)
-    bwd_preprocess_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, delta);
+    bwd_preprocess_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
   else
-    bwd_preprocess_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, delta);
+    bwd_preprocess_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
   return cudaGetLastError();
 }
 
 cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr, const void* v, const void* dout,
-                              const float* lse, const float* delta, const float* dq_acc, const float* dk1_acc,
+                              const float* lse, const float* ld, const float* dq_acc, const float* dk1_acc,
                               void* dq, void* dk, void* dv, cudaStream_t stream) {
   const int64_t warps = static_cast<int64_t>(g.si.T) * g.Hkv;
   if (warps == 0) return cudaSuccess;
@@ -396,12 +401,12 @@ cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr,
   if (g.D == 128) {
     e = cudaFuncSetAttribute(branch_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    branch_bwd_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, delta,
+    branch_bwd_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, ld,
                                                                                       dq_acc, dk1_acc, dqb, dkb, dvb);
   } else {
     e = cudaFuncSetAttribute(branch_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    branch_bwd_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, delta,
+    branch_bwd_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, ld,
                                                                                      dq_acc, dk1_acc, dqb, dkb, dvb);
   }
   return cudaGetLastError();

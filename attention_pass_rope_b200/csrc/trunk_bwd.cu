@@ -35,7 +35,7 @@ template <int D>
 struct BwdCfg {
   static constexpr int BK = 128;  // keys per CTA
   static constexpr int BQ = 64;   // queries per step
-  static constexpr int ST = 2;    // Q~/dO ring stages
+  static constexpr int ST = 3;    // Q~/dO ring stages
   static constexpr int KCH = D / 64;
   static constexpr int KCHUNK = 128 * 128;   // 128 rows x 64 bf16
   static constexpr int QCHUNK = 64 * 128;    // 64 rows x 64 bf16
@@ -43,7 +43,7 @@ struct BwdCfg {
   static constexpr int VTILE = KCH * KCHUNK;
   static constexpr int QTILE = KCH * QCHUNK;
   static constexpr int DSTILE = 128 * 128;   // 128 keys x 64 queries bf16
-  static constexpr int DQSTAGE = BQ * D * 4;
+  static constexpr int DQSTAGE = 32 * D * 4;    // half a query tile of dQ, fp32
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KTILE;
   static constexpr int OFF_Q = OFF_V + (VTILE < KCHUNK ? KCHUNK : VTILE);
@@ -139,15 +139,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_bar, 1);
     for (int s = 0; s < C::ST; ++s) {
-      mbar_init(qdo_full + s, 2);
+      mbar_init(qdo_full + s, 1);
       mbar_init(qdo_empty + s, 1);
     }
     mbar_init(sdp_full, 1);
-    mbar_init(ds_ready, 256);
+    mbar_init(ds_ready, 8);   // one arrival per P/dS warp
     mbar_init(mma_done + 0, 1);
     mbar_init(mma_done + 1, 1);
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
+    mbar_init(dq_free, 4);    // one arrival per dQ-writer warp
     mbar_init(final_bar, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -173,36 +173,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         tma_load_3d(sV + c * C::KCHUNK, &map_v, kv_bar, c * 64, kvh, seq_start + k0);
       }
     }
-    for (int it = 0; it < NIT; ++it) {
-      const int s = it % C::ST;
-      bool ok = true;
-      if (lane == 0 && it >= C::ST) ok = wait_bounded(qdo_empty + s, ((it / C::ST) - 1) & 1, wd, kSiteBwdQdoEmpty);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(qdo_full + s, 2 * C::QTILE);
+    if (lane == 0) {
+      const int nslots = ld_slots(g.si);
+      for (int it = 0; it < NIT; ++it) {
+        const int s = it % C::ST;
+        if (it >= C::ST && !wait_bounded(qdo_empty + s, ((it / C::ST) - 1) & 1, wd, kSiteBwdQdoEmpty)) break;
+        const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
+        mbar_arrive_expect_tx(qdo_full + s, 2 * C::QTILE + 2 * C::BQ * 4);
         for (int c = 0; c < C::KCH; ++c) {
           tma_load_3d(sQ + s * C::QTILE + c * C::QCHUNK, &map_q, qdo_full + s, c * 64, seq_start + ii.q0,
                       ii.p * g.H + ii.h);
           tma_load_3d(sDO + s * C::QTILE + c * C::QCHUNK, &map_do, qdo_full + s, c * 64, ii.h,
                       ii.p * g.si.T + seq_start + ii.q0);
         }
+        const float* src =
+            a.ld + ((static_cast<int64_t>(ii.p) * g.H + ii.h) * nslots + ld_slot(seq_start, n, ii.q0)) * 128;
+        bulk_load(sLD + s * 2 * C::BQ, src, 2 * C::BQ * 4, qdo_full + s);
       }
-      float* ld = sLD + s * 2 * C::BQ;
-      for (int r = lane; r < C::BQ; r += 32) {
-        const int qpos = ii.q0 + r;
-        float l2 = 0.f, dl = 0.f;
-        if (qpos < len) {
-          const int64_t idx = lse_index(g.si, g.H, ii.p, ii.h, n, seq_start + qpos, qpos);
-          l2 = a.lse[idx] * kLog2e;
-          dl = a.delta[idx];
-        }
-        ld[r] = l2;
-        ld[C::BQ + r] = dl;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(qdo_full + s);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -307,22 +294,40 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         ok = false;
         break;
       }
-      const float* ld = sLD + s * 2 * C::BQ + 32 * hf;
+      const float* ldp = sLD + s * 2 * C::BQ + 32 * hf;
+      // interior tile: every (key, query) pair of this half is visible
+      const int qlo = ii.q0 + 32 * hf;
+      const bool interior = (qlo >= k0 + C::BK - 1) && (qlo + 32 <= len) && (k0 + C::BK <= len);
+      // P and dS overwrite S^T and dP^T in place, 8 columns at a time
+#pragma unroll
+      for (int c0 = 0; c0 < 32; c0 += 8) {
+        const float4 l0 = *reinterpret_cast<const float4*>(ldp + c0);
+        const float4 l1 = *reinterpret_cast<const float4*>(ldp + c0 + 4);
+        const float4 d0 = *reinterpret_cast<const float4*>(ldp + C::BQ + c0);
+        const float4 d1 = *reinterpret_cast<const float4*>(ldp + C::BQ + c0 + 4);
+        const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+        const float dv8[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int c = c0 + u;
+          float pr = exp2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lv[u]));
+          float ds = pr * (__uint_as_float(dp[c]) - dv8[u]);
+          if (!interior) {
+            // padding rows of the statistics are never written: select, do not multiply
+            const int qpos = qlo + c;
+            const bool vis = kvalid && qpos < len && kpos <= qpos;
+            pr = vis ? pr : 0.f;
+            ds = vis ? ds : 0.f;
+          }
+          sv[c] = __float_as_uint(pr);
+          dp[c] = __float_as_uint(ds);
+        }
+      }
       uint32_t pk[16], dk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        float pv[2], dsv[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = 2 * e + u;
-          const int qpos = ii.q0 + 32 * hf + c;
-          const bool vis = kvalid && qpos < len && kpos <= qpos;
-          const float pr = vis ? exp2_approx(fmaf(__uint_as_float(sv[c]), sl2, -ld[c])) : 0.f;
-          pv[u] = pr;
-          dsv[u] = pr * (__uint_as_float(dp[c]) - ld[C::BQ + c]);
-        }
-        pk[e] = pack_bf16x2(pv[0], pv[1]);
-        dk[e] = pack_bf16x2(dsv[0], dsv[1]);
+        pk[e] = pack_bf16x2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1]));
+        dk[e] = pack_bf16x2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1]));
       }
       tmem_st16(lane_base + C::COL_PT + 32 * b + 16 * hf, pk);
       // dS^T row r, 128-byte swizzle: 16-byte chunk c of the row sits at c ^ (r & 7)
@@ -336,7 +341,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(ds_ready);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_ready);
     }
     // ---- epilogue: dV (half 0) and dK~ (half 1) of this CTA's keys
     if (ok && wait_bounded(final_bar, 0, wd, kSiteBwdFinal)) {
@@ -386,23 +392,27 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       reg_fence32(v0);
       reg_fence32(v1);
       tc_fence_before();
-      mbar_arrive(dq_free);
-      if (tid == 0) bulk_wait_read0();  // the staging buffer has been read by the last reduce
-      named_bar_sync(1, 128);
-      if (d < D) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+      // two halves of 32 query rows through a 16 KB staging buffer
 #pragma unroll
-        for (int q = 0; q < 32; ++q) sDQ[q * D + d] = __uint_as_float(v0[q]);
+      for (int hq = 0; hq < 2; ++hq) {
+        if (tid == 0) bulk_wait_read0();  // the staging buffer has been read by the last reduce
+        named_bar_sync(1, 128);
+        if (d < D) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) sDQ[(32 + q) * D + d] = __uint_as_float(v1[q]);
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (tid == 0) {
-        const int nrows = min(C::BQ, len - ii.q0);
-        if (nrows > 0) {
-          float* dst = a.dq_acc + ((static_cast<int64_t>(ii.p) * g.H + ii.h) * g.si.T + seq_start + ii.q0) * D;
-          bulk_reduce_add_f32(dst, sDQ, static_cast<uint32_t>(nrows * D * 4));
-          bulk_commit();
+          for (int q = 0; q < 32; ++q) sDQ[q * D + d] = __uint_as_float(hq == 0 ? v0[q] : v1[q]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (tid == 0) {
+          const int r0 = ii.q0 + 32 * hq;
+          const int nrows = min(32, len - r0);
+          if (nrows > 0) {
+            float* dst = a.dq_acc + ((static_cast<int64_t>(ii.p) * g.H + ii.h) * g.si.T + seq_start + r0) * D;
+            bulk_reduce_add_f32(dst, sDQ, static_cast<uint32_t>(nrows * D * 4));
+            bulk_commit();
+          }
         }
       }
     }

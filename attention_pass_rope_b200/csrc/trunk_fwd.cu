@@ -30,14 +30,15 @@ struct FwdCfg {
   static constexpr int BM = 128;  // query rows per tile
   static constexpr int BN = 128;  // keys per KV tile
   static constexpr int NQ = 2;    // query tiles per CTA
-  static constexpr int ST = 2;    // K/V ring stages
+  static constexpr int KST = 3;   // K ring stages
+  static constexpr int VST = 2;   // V ring stages (V_j is read one iteration after K_j)
   static constexpr int KCH = D / 64;
   static constexpr int CHUNK = 128 * 128;         // one 64-column chunk of a 128-row tile
   static constexpr int TILE = KCH * CHUNK;        // 128 rows x D bf16
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * TILE;
-  static constexpr int OFF_V = OFF_K + ST * TILE;
-  static constexpr int OFF_BAR = OFF_V + ST * TILE;
+  static constexpr int OFF_V = OFF_K + KST * TILE;
+  static constexpr int OFF_BAR = OFF_V + VST * TILE;
   static constexpr int BAR_BYTES = 256;
   // D = 64 needs only 96 KB; ask for more so that one CTA holds the SM (and its TMEM).
   static constexpr int SMEM_USED = OFF_BAR + BAR_BYTES;
@@ -86,9 +87,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;            // [ST]
-  uint64_t* kv_empty = bars + 1 + C::ST;   // [ST]
-  uint64_t* s_full = bars + 1 + 2 * C::ST; // [NQ]
+  uint64_t* k_full = bars + 1;             // [KST]
+  uint64_t* k_empty = k_full + C::KST;     // [KST]
+  uint64_t* v_full = k_empty + C::KST;     // [VST]
+  uint64_t* v_empty = v_full + C::VST;     // [VST]
+  uint64_t* s_full = v_empty + C::VST;     // [NQ]
   uint64_t* p_full = s_full + C::NQ;       // [NQ]
   uint64_t* o_final = p_full + C::NQ;      // [NQ]
   uint64_t* drain = o_final + C::NQ;
@@ -97,13 +100,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < C::ST; ++s) {
-      mbar_init(kv_full + s, 1);
-      mbar_init(kv_empty + s, 1);
+    for (int s = 0; s < C::KST; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < C::VST; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
     }
     for (int t = 0; t < C::NQ; ++t) {
       mbar_init(s_full + t, 1);
-      mbar_init(p_full + t, 128);
+      mbar_init(p_full + t, 4);  // one arrival per softmax warp
       mbar_init(o_final + t, 1);
     }
     mbar_init(drain, 1);
@@ -140,14 +147,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &map_q, q_full, c * 64, seq_start + q0,
                       p_of[t] * g.H + h_of[t]);
       for (int j = 0; j < nkv; ++j) {
-        const int s = j % C::ST;
-        if (j >= C::ST && !wait_bounded(kv_empty + s, ((j / C::ST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
-        mbar_arrive_expect_tx(kv_full + s, 2 * C::TILE);
         const int krow = seq_start + j * C::BN;
-        for (int c = 0; c < C::KCH; ++c) {
-          tma_load_3d(sK + s * C::TILE + c * C::CHUNK, &map_k, kv_full + s, c * 64, krow, kvh);
-          tma_load_3d(sV + s * C::TILE + c * C::CHUNK, &map_v, kv_full + s, c * 64, kvh, krow);
-        }
+        const int ks = j % C::KST;
+        if (j >= C::KST && !wait_bounded(k_empty + ks, ((j / C::KST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
+        mbar_arrive_expect_tx(k_full + ks, C::TILE);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sK + ks * C::TILE + c * C::CHUNK, &map_k, k_full + ks, c * 64, krow, kvh);
+        const int vs = j % C::VST;
+        if (j >= C::VST && !wait_bounded(v_empty + vs, ((j / C::VST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
+        mbar_arrive_expect_tx(v_full + vs, C::TILE);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sV + vs * C::TILE + c * C::CHUNK, &map_v, v_full + vs, c * 64, kvh, krow);
       }
     }
     __syncwarp();
@@ -173,34 +183,35 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
       };
       bool ok = wait_bounded(q_full, 0, wd, kSiteFwdQ);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % C::ST;
-        if (!wait_bounded(kv_full + s, (j / C::ST) & 1, wd, kSiteFwdKvFull)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      // Order per KV tile j: for each query tile t, O_t += P_t(j-1) V_{j-1}, then
+      // S_t(j) = Q_t K_j^T.  The in-order tensor pipe finishes reading P_t(j-1) (which
+      // overlays S_t) before S_t(j) overwrites it.
+      for (int j = 0; ok && j <= nkv; ++j) {
         for (int t = 0; t < nq_tiles; ++t) {
           if (j > 0) {
             if (!wait_bounded(p_full + t, (j - 1) & 1, wd, kSiteFwdPFull)) {
               ok = false;
               break;
             }
+            if (t == 0 && !wait_bounded(v_full + (j - 1) % C::VST, ((j - 1) / C::VST) & 1, wd, kSiteFwdKvFull)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
-            issue_pv(t, (j - 1) % C::ST, j - 1 > 0);
+            issue_pv(t, (j - 1) % C::VST, j - 1 > 0);
+            if (j == nkv) umma_commit(o_final + t);
+            if (t == nq_tiles - 1) umma_commit(v_empty + (j - 1) % C::VST);
           }
-          issue_s(t, s);
-          umma_commit(s_full + t);
-        }
-        if (!ok) break;
-        if (j > 0) umma_commit(kv_empty + (j - 1) % C::ST);
-      }
-      if (ok) {
-        for (int t = 0; t < nq_tiles; ++t) {
-          if (!wait_bounded(p_full + t, (nkv - 1) & 1, wd, kSiteFwdPFull)) break;
-          tc_fence_after();
-          issue_pv(t, (nkv - 1) % C::ST, nkv - 1 > 0);
-          umma_commit(o_final + t);
+          if (j < nkv) {
+            if (t == 0 && !wait_bounded(k_full + j % C::KST, (j / C::KST) & 1, wd, kSiteFwdKvFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(t, j % C::KST);
+            umma_commit(s_full + t);
+            if (t == nq_tiles - 1) umma_commit(k_empty + j % C::KST);
+          }
         }
       }
       // nothing may still be running on the tensor cores when TMEM is released
@@ -241,12 +252,24 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int e = 0; e < 32; ++e)
             if (k0 + 32 * c + e > qpos) sr[c][e] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // row max: 8 independent chains, then a tree
+      float mxv[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int u = 0; u < 8; ++u) mxv[u] = fmaxf(__uint_as_float(sr[0][u]), __uint_as_float(sr[0][u + 8]));
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-      const float m_new = fmaxf(m_run, mx * sl2);
+      for (int u = 0; u < 8; ++u) {
+        mxv[u] = fmaxf(mxv[u], fmaxf(__uint_as_float(sr[0][u + 16]), __uint_as_float(sr[0][u + 24])));
+#pragma unroll
+        for (int c = 1; c < 4; ++c)
+          mxv[u] = fmaxf(fmaxf(mxv[u], __uint_as_float(sr[c][u])),
+                         fmaxf(fmaxf(__uint_as_float(sr[c][u + 8]), __uint_as_float(sr[c][u + 16])),
+                               __uint_as_float(sr[c][u + 24])));
+      }
+#pragma unroll
+      for (int u = 4; u > 0; u >>= 1)
+#pragma unroll
+        for (int v = 0; v < u; ++v) mxv[v] = fmaxf(mxv[v], mxv[v + u]);
+      const float m_new = fmaxf(m_run, mxv[0] * sl2);
       const bool rescale = m_new > m_run + kRescaleThreshold;
       float alpha = 1.f;
       if (rescale) {
@@ -254,7 +277,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         l_run *= alpha;
         m_run = m_new;
       }
-      float rs = 0.f;
+      float rsv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -262,12 +285,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int e = 0; e < 16; ++e) {
           const float p0 = exp2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_run));
           const float p1 = exp2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_run));
-          rs += p0 + p1;
+          rsv[(2 * e) & 7] += p0;
+          rsv[(2 * e + 1) & 7] += p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(lane_base + colS + 16 * c, pk);
       }
-      l_run += rs;
+#pragma unroll
+      for (int u = 4; u > 0; u >>= 1)
+#pragma unroll
+        for (int v = 0; v < u; ++v) rsv[v] += rsv[v + u];
+      l_run += rsv[0];
       if (rescale && j > 0) {
         // O of this row was complete up to tile j-1 when s_full fired (in-order MMAs)
 #pragma unroll 1
@@ -283,7 +311,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full + t);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + t);
     }
     if (ok && wait_bounded(o_final + t, 0, wd, kSiteFwdOFinal)) {
       tc_fence_after();

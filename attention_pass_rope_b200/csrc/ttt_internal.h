@@ -73,14 +73,20 @@ cudaError_t launch_branch_merge_fwd(const Geometry& g, const void* qr, const voi
                                     const float* o_t, const float* lse_t, void* o, float* lse,
                                     cudaStream_t stream);
 
-// a5: delta = rowsum(dO * O) in the public lse layout.
-cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, float* delta,
+// Row statistics of the backward, tile-aligned: for query head (p, h) and the 64-row
+// query tile j of sequence n, slot = start_n / 64 + n + j holds 64 values of
+// lse * log2(e) followed by 64 values of delta (512 bytes, one bulk copy).  Slots of
+// consecutive sequences never overlap: start_n/64 + n + ceil(len_n/64) <=
+// start_{n+1}/64 + n + 1.  Padding entries are never written.
+__host__ __device__ inline int ld_slots(const SeqInfo& si) { return si.T / 64 + si.nseq + 1; }
+
+// a5: delta = rowsum(dO * O); writes the tile-aligned (lse*log2e, delta) rows.
+cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
                                   cudaStream_t stream);
 
 struct TrunkBwdArgs {
   Geometry g;
-  const float* lse;    // public layout
-  const float* delta;  // public lse layout
+  const float* ld;     // tile-aligned (lse*log2e, delta) rows, see ld_slots
   float* dq_acc;       // fp32 [P][H][T][D], zeroed before the launch
   float* dk1_acc;      // fp32 [Hkv][T][D]  (unscaled sum of dS^T q~)
   void* dv;            // bf16 public dv; pass 0 written here
@@ -94,7 +100,7 @@ cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, co
 
 // a7+a8: branch backward, dq finalize (inverse RoPE), dk of every pass.
 cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr, const void* v,
-                              const void* dout, const float* lse, const float* delta, const float* dq_acc,
+                              const void* dout, const float* lse, const float* ld, const float* dq_acc,
                               const float* dk1_acc, void* dq, void* dk, void* dv, cudaStream_t stream);
 
 cudaError_t launch_watchdog_selftest(uint32_t* status, uint64_t budget_ns, cudaStream_t stream);

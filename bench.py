@@ -118,7 +118,7 @@ def run_ours(args, rank, world, local):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
-    w = ttt_inputs.workloads()[args.workload]
+    w = workload(args)
     # every rank draws its own batch (weak scaling); the sizes are the workload's
     inp = ttt_inputs.make_inputs(w, seed=w.seed + rank)
 
@@ -146,6 +146,8 @@ def run_ours(args, rank, world, local):
         objs = []
         for kk in range(len(_lib.KERNELS)):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()  # torch creates the CUDA event on first use; the library re-records it
+            b.record()
             e.start[kk] = a.cuda_event
             e.stop[kk] = b.cuda_event
             objs.append((a, b))
@@ -267,6 +269,15 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def workload(args):
+    w = ttt_inputs.workloads()[args.workload]
+    if args.batch and w.dense:
+        # a smaller batch of the same sequences (profiling captures)
+        w = ttt_inputs.dense(f"{w.name}_b{args.batch}", args.batch, w.lengths[0], w.P, w.H, w.Hkv, w.D, w.theta,
+                             w.scale, w.seed)
+    return w
+
+
 def read_traffic(kernel, workload):
     """dram bytes per launch from the committed ncu summary, if one matches the kernel."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
@@ -325,7 +336,7 @@ def cpu_baseline(w, budget_s=30.0):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = ttt_inputs.workloads()[args.workload]
+    w = workload(args)
     for _ in range(args.warmup and 1):
         pass  # the oracle has no warm-up state; one untimed sample below warms the BLAS pool
     oracle_sample(ttt_inputs.thd("warm", [256], w.P, w.H // w.Hkv, 1, w.D, w.theta))
@@ -361,12 +372,13 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ttt_inputs.workloads()))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=30.0)
+    ap.add_argument("--batch", type=int, default=0, help="override B of a dense workload (profiling)")
     args = ap.parse_args()
     rank, world, local = dist_env()
     if args.impl == "reference":
