@@ -13,6 +13,33 @@
 namespace ttt {
 
 // ---------------------------------------------------------------------------
+// Kernel timeline trace (profiling builds only: -DTTT_KERNEL_TRACE).  CTA 0 of a
+// launch records %clock64 at numbered points, per loop iteration; the trace build
+// exports ttt_trace_read_<kernel>() to copy the table out.  In normal builds every
+// trace point compiles to nothing.
+// ---------------------------------------------------------------------------
+#ifdef TTT_KERNEL_TRACE
+constexpr int kTraceSlots = 24;
+constexpr int kTraceIters = 1024;
+static __device__ long long g_trace[kTraceSlots][kTraceIters];
+__device__ __forceinline__ void trace_point(int slot, int j) {
+  if (blockIdx.x == 0 && j < kTraceIters) {
+    long long t;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+    g_trace[slot][j] = t;
+  }
+}
+#define TTT_TRACE(slot, j) ::ttt::trace_point((slot), (j))
+#define TTT_TRACE_READER(name)                                                                       \
+  extern "C" int name(void* host) {                                                                  \
+    return static_cast<int>(cudaMemcpyFromSymbol(host, ::ttt::g_trace, sizeof(::ttt::g_trace)));     \
+  }
+#else
+#define TTT_TRACE(slot, j) ((void)0)
+#define TTT_TRACE_READER(name)
+#endif
+
+// ---------------------------------------------------------------------------
 // generic
 // ---------------------------------------------------------------------------
 
@@ -110,6 +137,13 @@ static __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, co
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Watchdog& wd, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   return wait_slow(bar, parity, wd, site);
+}
+
+// Warp-uniform bounded wait: every lane waits (and acquires); the result is agreed
+// across the warp so that control flow stays uniform.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const Watchdog& wd, uint32_t site) {
+  const bool ok = wait_bounded(bar, parity, wd, site);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Bounded wait that ignores the abort flag: used on the exit path to let operations
@@ -219,6 +253,38 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Warp-wide forms: the whole warp executes them with identical (warp-uniform)
+// operands and one elected lane issues, so that descriptors stay in the uniform
+// datapath and the issuing warp spends few instructions per MMA.
+__device__ __forceinline__ void umma_ss_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
       : "memory");
 }
 

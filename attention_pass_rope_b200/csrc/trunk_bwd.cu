@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       for (int it = 0; it < NIT; ++it) {
         const int s = it % C::ST;
         if (it >= C::ST && !wait_bounded(qdo_empty + s, ((it / C::ST) - 1) & 1, wd, kSiteBwdQdoEmpty)) break;
+        TTT_TRACE(16, it);
         const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
         mbar_arrive_expect_tx(qdo_full + s, 2 * C::QTILE + 2 * C::BQ * 4);
         for (int c = 0; c < C::KCH; ++c) {
@@ -194,73 +195,85 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {
       constexpr uint32_t idSP = idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idDV = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t idDQ = idesc_bf16_f32(128, C::BQ, true, true);
-      const uint32_t kA = smem_u32(sK), vA = smem_u32(sV), qA = smem_u32(sQ), doA = smem_u32(sDO),
-                     dsA = smem_u32(sDS);
+      // Descriptors are built once; a k-step only adds a constant to the start-address
+      // field (bits 0-13 hold address >> 4, and every operand lies below 256 KB).
+      const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);          // K~ as K-major A
+      const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), C::KCHUNK, 1024);  // K~ as MN-major A
+      const uint64_t dV_k = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dQ_k = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), C::QCHUNK, 1024);
+      const uint64_t dO_k = sdesc_sw128(smem_u32(sDO), 16, 1024);
+      const uint64_t dO_mn = sdesc_sw128(smem_u32(sDO), C::QCHUNK, 1024);
+      const uint64_t dS_k = sdesc_sw128(smem_u32(sDS), 16, 1024);
+      const uint64_t dS_mn = sdesc_sw128(smem_u32(sDS), C::KCHUNK, 1024);
       auto issue_sdp = [&](int it) {
-        const int s = it % C::ST;
+        const uint32_t so = static_cast<uint32_t>(((it % C::ST) * C::QTILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ok_ = (kk >> 2) * C::KCHUNK + (kk & 3) * 32;
-          const uint32_t oq_ = (kk >> 2) * C::QCHUNK + (kk & 3) * 32;
-          umma_ss(tmem + C::COL_S, sdesc_sw128(kA + ok_, 16, 1024),
-                  sdesc_sw128(qA + s * C::QTILE + oq_, 16, 1024), idSP, kk > 0 ? 1u : 0u);
+          const uint32_t ok_ = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t oq_ = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          umma_ss_warp(tmem + C::COL_S, dK_k + ok_, dQ_k + so + oq_, idSP, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ok_ = (kk >> 2) * C::KCHUNK + (kk & 3) * 32;
-          const uint32_t oq_ = (kk >> 2) * C::QCHUNK + (kk & 3) * 32;
-          umma_ss(tmem + C::COL_DP, sdesc_sw128(vA + ok_, 16, 1024),
-                  sdesc_sw128(doA + s * C::QTILE + oq_, 16, 1024), idSP, kk > 0 ? 1u : 0u);
+          const uint32_t ok_ = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t oq_ = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          umma_ss_warp(tmem + C::COL_DP, dV_k + ok_, dO_k + so + oq_, idSP, kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = wait_bounded(kv_bar, 0, wd, kSiteBwdKv) && wait_bounded(qdo_full, 0, wd, kSiteBwdQdoFull);
+      bool ok = wait_warp(kv_bar, 0, wd, kSiteBwdKv) && wait_warp(qdo_full, 0, wd, kSiteBwdQdoFull);
       if (ok) {
         tc_fence_after();
         issue_sdp(0);
-        umma_commit(sdp_full);
+        umma_commit_warp(sdp_full);
       }
       for (int it = 0; ok && it < NIT; ++it) {
         const int s = it % C::ST;
         const int b = it & 1;
-        if (!wait_bounded(ds_ready, it & 1, wd, kSiteBwdDsReady)) break;
+        if (!wait_warp(ds_ready, it & 1, wd, kSiteBwdDsReady)) break;
+        TTT_TRACE(0, it);
         tc_fence_after();
         if (it + 1 < NIT) {
-          if (!wait_bounded(qdo_full + (it + 1) % C::ST, ((it + 1) / C::ST) & 1, wd, kSiteBwdQdoFull)) break;
+          if (!wait_warp(qdo_full + (it + 1) % C::ST, ((it + 1) / C::ST) & 1, wd, kSiteBwdQdoFull)) break;
           tc_fence_after();
           issue_sdp(it + 1);
-          umma_commit(sdp_full);
+          umma_commit_warp(sdp_full);
         }
+        TTT_TRACE(1, it);
+        const uint32_t so = static_cast<uint32_t>((s * C::QTILE) >> 4);
+        const uint32_t bo = static_cast<uint32_t>((b * C::DSTILE) >> 4);
         // dV += P^T dO   (P^T: TMEM, 64 queries = 32 packed columns)
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_ts(tmem + C::COL_DV, tmem + C::COL_PT + 32 * b + kk * 8,
-                  sdesc_sw128(doA + s * C::QTILE + kk * 2048, C::QCHUNK, 1024), idDV,
+          umma_ts_warp(tmem + C::COL_DV, tmem + C::COL_PT + 32 * b + kk * 8, dO_mn + so + ((kk * 2048) >> 4), idDV,
                   (it > 0 || kk > 0) ? 1u : 0u);
         // dK += dS^T Q~
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_ss(tmem + C::COL_DK, sdesc_sw128(dsA + b * C::DSTILE + kk * 32, 16, 1024),
-                  sdesc_sw128(qA + s * C::QTILE + kk * 2048, C::QCHUNK, 1024), idDV,
+          umma_ss_warp(tmem + C::COL_DK, dS_k + bo + ((kk * 32) >> 4), dQ_mn + so + ((kk * 2048) >> 4), idDV,
                   (it > 0 || kk > 0) ? 1u : 0u);
+        TTT_TRACE(2, it);
         if (it > 0) {
-          if (!wait_bounded(dq_free, (it - 1) & 1, wd, kSiteBwdDqFree)) break;
+          if (!wait_warp(dq_free, (it - 1) & 1, wd, kSiteBwdDqFree)) break;
           tc_fence_after();
         }
+        TTT_TRACE(3, it);
         // dQ^T = K~^T dS^T
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_ss(tmem + C::COL_DQ, sdesc_sw128(kA + kk * 2048, C::KCHUNK, 1024),
-                  sdesc_sw128(dsA + b * C::DSTILE + kk * 2048, C::KCHUNK, 1024), idDQ, kk > 0 ? 1u : 0u);
-        umma_commit(mma_done + b);
-        umma_commit(qdo_empty + s);
-        umma_commit(dq_full);
+          umma_ss_warp(tmem + C::COL_DQ, dK_mn + ((kk * 2048) >> 4), dS_mn + bo + ((kk * 2048) >> 4), idDQ,
+                  kk > 0 ? 1u : 0u);
+        umma_commit_warp(mma_done + b);
+        umma_commit_warp(qdo_empty + s);
+        umma_commit_warp(dq_full);
+        TTT_TRACE(4, it);
       }
-      umma_commit(final_bar);
-      umma_commit(drain);
+      umma_commit_warp(final_bar);
+      umma_commit_warp(drain);
       wait_drain(drain, 0, wd, kSiteBwdDrain);
     }
     __syncwarp();
@@ -283,6 +296,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         ok = false;
         break;
       }
+      if (lane == 0 && warp == 4) TTT_TRACE(5, it);
       tc_fence_after();
       uint32_t sv[32], dp[32];
       tmem_ld32(lane_base + C::COL_S + 32 * hf, sv);
@@ -294,6 +308,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         ok = false;
         break;
       }
+      if (lane == 0 && warp == 4) TTT_TRACE(7, it);
       const float* ldp = sLD + s * 2 * C::BQ + 32 * hf;
       // interior tile: every (key, query) pair of this half is visible
       const int qlo = ii.q0 + 32 * hf;
@@ -329,6 +344,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         pk[e] = pack_bf16x2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1]));
         dk[e] = pack_bf16x2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1]));
       }
+      if (lane == 0 && warp == 4) TTT_TRACE(8, it);
       tmem_st16(lane_base + C::COL_PT + 32 * b + 16 * hf, pk);
       // dS^T row r, 128-byte swizzle: 16-byte chunk c of the row sits at c ^ (r & 7)
       uint8_t* row = sDS + b * C::DSTILE + r * 128;
@@ -343,6 +359,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_ready);
+      if (lane == 0 && warp == 4) TTT_TRACE(9, it);
     }
     // ---- epilogue: dV (half 0) and dK~ (half 1) of this CTA's keys
     if (ok && wait_bounded(final_bar, 0, wd, kSiteBwdFinal)) {
@@ -384,6 +401,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     for (int it = 0; it < NIT; ++it) {
       const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
       if (!wait_bounded(dq_full, it & 1, wd, kSiteBwdDqFull)) break;
+      if (tid == 0) TTT_TRACE(10, it);
       tc_fence_after();
       uint32_t v0[32], v1[32];
       tmem_ld32(lane_base + C::COL_DQ, v0);
@@ -448,3 +466,5 @@ cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, co
 }
 
 }  // namespace ttt
+
+TTT_TRACE_READER(ttt_trace_read_bwd)

@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const int krow = seq_start + j * C::BN;
         const int ks = j % C::KST;
         if (j >= C::KST && !wait_bounded(k_empty + ks, ((j / C::KST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
+        TTT_TRACE(14, j);
         mbar_arrive_expect_tx(k_full + ks, C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sK + ks * C::TILE + c * C::CHUNK, &map_k, k_full + ks, c * 64, krow, kvh);
@@ -163,59 +164,69 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {
       constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
-      const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK), vb = smem_u32(sV);
+      // Descriptors are built once; a k-step only adds a constant to the start-address
+      // field (bits 0-13 hold address >> 4, and every operand lies below 256 KB).
+      const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(sV), C::CHUNK, 1024);
       auto issue_s = [&](int t, int s) {
+        const uint64_t qd = dq0 + static_cast<uint32_t>((t * C::TILE) >> 4);
+        const uint64_t kd = dk0 + static_cast<uint32_t>((s * C::TILE) >> 4);
+        const uint32_t d_tmem = tmem + C::COL_S0 + 128 * t;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tmem + C::COL_S0 + 128 * t, sdesc_sw128(qa + t * C::TILE + off, 16, 1024),
-                  sdesc_sw128(kb + s * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4;
+          umma_ss_warp(d_tmem, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int s, bool acc) {
+        const uint64_t vd = dv0 + static_cast<uint32_t>((s * C::TILE) >> 4);
+        const uint32_t d_tmem = tmem + C::COL_O0 + D * t;
+        const uint32_t a_tmem = tmem + C::COL_S0 + 128 * t;
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tmem + C::COL_O0 + D * t, tmem + C::COL_S0 + 128 * t + kk * 8,
-                  sdesc_sw128(vb + s * C::TILE + kk * 2048, C::CHUNK, 1024), idO, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          umma_ts_warp(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), idO, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_bounded(q_full, 0, wd, kSiteFwdQ);
+      bool ok = wait_warp(q_full, 0, wd, kSiteFwdQ);
       // Order per KV tile j: for each query tile t, O_t += P_t(j-1) V_{j-1}, then
       // S_t(j) = Q_t K_j^T.  The in-order tensor pipe finishes reading P_t(j-1) (which
       // overlays S_t) before S_t(j) overwrites it.
       for (int j = 0; ok && j <= nkv; ++j) {
         for (int t = 0; t < nq_tiles; ++t) {
           if (j > 0) {
-            if (!wait_bounded(p_full + t, (j - 1) & 1, wd, kSiteFwdPFull)) {
+            if (!wait_warp(p_full + t, (j - 1) & 1, wd, kSiteFwdPFull)) {
               ok = false;
               break;
             }
-            if (t == 0 && !wait_bounded(v_full + (j - 1) % C::VST, ((j - 1) / C::VST) & 1, wd, kSiteFwdKvFull)) {
+            TTT_TRACE(0 + t, j);
+            if (t == 0 && !wait_warp(v_full + (j - 1) % C::VST, ((j - 1) / C::VST) & 1, wd, kSiteFwdKvFull)) {
               ok = false;
               break;
             }
             tc_fence_after();
             issue_pv(t, (j - 1) % C::VST, j - 1 > 0);
-            if (j == nkv) umma_commit(o_final + t);
-            if (t == nq_tiles - 1) umma_commit(v_empty + (j - 1) % C::VST);
+            if (j == nkv) umma_commit_warp(o_final + t);
+            if (t == nq_tiles - 1) umma_commit_warp(v_empty + (j - 1) % C::VST);
           }
           if (j < nkv) {
-            if (t == 0 && !wait_bounded(k_full + j % C::KST, (j / C::KST) & 1, wd, kSiteFwdKvFull)) {
+            if (t == 0 && !wait_warp(k_full + j % C::KST, (j / C::KST) & 1, wd, kSiteFwdKvFull)) {
               ok = false;
               break;
             }
+            if (t == 0) TTT_TRACE(15, j);
             tc_fence_after();
             issue_s(t, j % C::KST);
-            umma_commit(s_full + t);
-            if (t == nq_tiles - 1) umma_commit(k_empty + j % C::KST);
+            umma_commit_warp(s_full + t);
+            TTT_TRACE(2 + t, j);
+            if (t == nq_tiles - 1) umma_commit_warp(k_empty + j % C::KST);
           }
         }
       }
       // nothing may still be running on the tensor cores when TMEM is released
-      umma_commit(drain);
+      umma_commit_warp(drain);
       wait_drain(drain, 0, wd, kSiteFwdDrain);
     }
     __syncwarp();
@@ -237,6 +248,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         ok = false;
         break;
       }
+      if (lane == 0 && wq == 0) TTT_TRACE(4 + t, j);
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
@@ -270,6 +282,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int v = 0; v < u; ++v) mxv[v] = fmaxf(mxv[v], mxv[v + u]);
       const float m_new = fmaxf(m_run, mxv[0] * sl2);
+      if (lane == 0 && wq == 0) TTT_TRACE(8 + t, j);
       const bool rescale = m_new > m_run + kRescaleThreshold;
       float alpha = 1.f;
       if (rescale) {
@@ -278,6 +291,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         m_run = m_new;
       }
       float rsv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // P = 2^(s*scale*log2e - m), bf16 pairs into the first 64 columns of S_t
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -296,6 +310,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int v = 0; v < u; ++v) rsv[v] += rsv[v + u];
       l_run += rsv[0];
+      if (lane == 0 && wq == 0) TTT_TRACE(10 + t, j);
       if (rescale && j > 0) {
         // O of this row was complete up to tile j-1 when s_full fired (in-order MMAs)
 #pragma unroll 1
@@ -313,6 +328,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + t);
+      if (lane == 0 && wq == 0) TTT_TRACE(12 + t, j);
     }
     if (ok && wait_bounded(o_final + t, 0, wd, kSiteFwdOFinal)) {
       tc_fence_after();
@@ -369,3 +385,5 @@ cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, co
 }
 
 }  // namespace ttt
+
+TTT_TRACE_READER(ttt_trace_read_fwd)
