@@ -118,6 +118,24 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
                         const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/* Forward for callers that cannot allocate device memory.  The pages describe no
+ * such entry point; it is a deployment aid.  A caller such as a plugin in a host
+ * framework that owns every device allocation, or a latency-critical loop where
+ * cudaMalloc (which can synchronise the device) is not acceptable, has no way to
+ * provide the workspace ttt_attn_fwd needs.  This call computes exactly what
+ * ttt_attn_fwd computes (same arguments, same outputs) with its scratch in a fixed
+ * 32 MiB array inside the library's own device memory, held by every GPU that
+ * loads the library until the process exits.  It allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library call).  Returns TTT_ERR_WORKSPACE, before
+ * enqueuing anything, when ttt_attn_workspace_size(desc, 0) exceeds 32 MiB.  The
+ * first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture.  All
+ * calls on a device share the array and it keeps the last call's contents (the
+ * call clears what must start at zero); calls whose GPU work overlaps (unordered
+ * streams) race on it, so order them on one stream. */
+ttt_status ttt_attn_fwd_noalloc(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, void* o,
+                                float* lse, void* stream);
+
 /* Synchronises `stream` and returns TTT_OK if no bounded wait of the calls made
  * with this workspace ran out since the last check, TTT_ERR_DEVICE_TIMEOUT (and
  * the raw status word in *detail if non-NULL) otherwise, or TTT_ERR_CUDA.  The
