@@ -17,7 +17,7 @@ TTT_ERR_DEVICE_TIMEOUT = 5
 TTT_LAYOUT_BSHD = 0
 TTT_LAYOUT_THD = 1
 
-KERNELS = ("rope_fwd", "trunk_fwd", "branch_merge_fwd", "rope_bwd", "bwd_preprocess", "trunk_bwd", "branch_bwd")
+KERNELS = ("rope_fwd", "trunk_fwd", "unused_2", "rope_bwd", "bwd_preprocess", "trunk_bwd", "branch_bwd")
 KERNEL_COUNT = 8
 
 

@@ -78,11 +78,7 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
   pl.off[2] = o;  // k~
   o = align_up(o + P * Hkv * T * D * 2);
   if (!for_backward) {
-    pl.off[3] = o;  // O_t
-    o = align_up(o + P * H * T * D * 4);
-    pl.off[4] = o;  // lse_t
-    o = align_up(o + P * H * T * 4);
-    pl.noff = 5;
+    pl.noff = 3;
   } else {
     pl.off[3] = o;  // tile-aligned row statistics (lse*log2e, delta)
     o = align_up(o + P * H * static_cast<size_t>(ld_slots(g.si)) * 128 * 4);
@@ -182,8 +178,6 @@ ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k,
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + pl.off[0]);
   void* qr = ws + pl.off[1];
   void* kr = ws + pl.off[2];
-  float* o_t = reinterpret_cast<float*>(ws + pl.off[3]);
-  float* lse_t = reinterpret_cast<float*>(ws + pl.off[4]);
   const uint64_t T = g.si.T, D = g.D;
 
   CUtensorMap mq, mk, mv;
@@ -199,12 +193,8 @@ ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k,
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
-    TrunkFwdArgs a{g, o_t, lse_t, status, g_wait_budget_ns.load()};
+    TrunkFwdArgs a{g, kr, v, o, lse, status, g_wait_budget_ns.load()};
     TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
-  }
-  {
-    EventScope es(desc->events, TTT_KERNEL_BRANCH_MERGE_FWD, stream);
-    TTT_CHECK_CUDA(launch_branch_merge_fwd(g, qr, kr, v, o_t, lse_t, o, lse, stream));
   }
   return TTT_OK;
 }

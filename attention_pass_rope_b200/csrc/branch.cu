@@ -114,77 +114,6 @@ __device__ __forceinline__ void rotate_back(float (&x)[2][D / 64], const float (
 }
 
 // ---------------------------------------------------------------------------
-// a3 + a4: branch softmax over keys of passes 2..p at the same position, merged
-// with the trunk partial: lse = logaddexp(lse_t, lse_b),
-// O = e^(lse_t - lse) O_t + e^(lse_b - lse) O_b.
-// ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
-    branch_merge_fwd_kernel(Geometry g, const __nv_bfloat16* __restrict__ qr, const __nv_bfloat16* __restrict__ kr,
-                            const __nv_bfloat16* __restrict__ v, const float* __restrict__ o_t,
-                            const float* __restrict__ lse_t, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
-  const int lane = threadIdx.x & 31;
-  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
-  const int T = g.si.T;
-  if (w >= static_cast<int64_t>(g.P) * T * g.Hkv) return;
-  const int p = static_cast<int>(w / (static_cast<int64_t>(T) * g.Hkv));
-  const int rem = static_cast<int>(w % (static_cast<int64_t>(T) * g.Hkv));
-  const int tau = rem / g.Hkv;
-  const int kvh = rem % g.Hkv;
-  int n, pos;
-  token_position(g.si, tau, n, pos);
-  const int gsz = g.H / g.Hkv;
-  for (int hi = 0; hi < gsz; ++hi) {
-    const int h = kvh * gsz + hi;
-    const int64_t trow = (static_cast<int64_t>(p) * g.H + h) * T + tau;
-    float ot[2][D / 64];
-    load_f32_row<D>(o_t + trow * D, lane, ot);
-    const float lt = lse_t[trow];
-    float out[2][D / 64];
-    float lse_m = lt;
-    if (p == 0) {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int e = 0; e < D / 64; ++e) out[hh][e] = ot[hh][e];
-    } else {
-      float q[2][D / 64];
-      load_bf16_row<D>(qr + trow * D, lane, q);
-      // online softmax over the p branch keys (passes 1..p, 0-based)
-      float m = -INFINITY, l = 0.f;
-      float ob[2][D / 64] = {};
-      for (int j = 1; j <= p; ++j) {
-        float kj[2][D / 64], vj[2][D / 64];
-        load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
-        load_bf16_row<D>(v + ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D, lane, vj);
-        const float s = dot_row<D>(q, kj) * g.scale;
-        const float m_new = fmaxf(m, s);
-        const float alpha = __expf(m - m_new);
-        const float pj = __expf(s - m_new);
-        l = l * alpha + pj;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int e = 0; e < D / 64; ++e) ob[hh][e] = fmaf(ob[hh][e], alpha, pj * vj[hh][e]);
-        m = m_new;
-      }
-      const float lb = m + __logf(l);
-      // exact merge: lse = logaddexp(lt, lb)
-      const float mx = fmaxf(lt, lb);
-      lse_m = mx + log1pf(__expf(-fabsf(lt - lb)));
-      const float wt = __expf(lt - lse_m);
-      const float wb = __expf(m - lse_m);  // e^(lb - lse) / l, applied to the unnormalised ob
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int e = 0; e < D / 64; ++e) out[hh][e] = fmaf(wt, ot[hh][e], wb * ob[hh][e]);
-    }
-    store_bf16_row<D>(o + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D, lane, out);
-    if (lane == 0) lse[lse_index(g.si, g.H, p, h, n, tau, pos)] = lse_m;
-  }
-}
-
-// ---------------------------------------------------------------------------
 // a5: delta = rowsum(dO * O).  Written, with lse * log2(e), into the tile-aligned
 // row-statistics array that the trunk backward fetches one 512-byte slot at a time.
 // ---------------------------------------------------------------------------
@@ -354,21 +283,6 @@ inline unsigned blocks_for(int64_t warps) {
 }
 
 }  // namespace
-
-cudaError_t launch_branch_merge_fwd(const Geometry& g, const void* qr, const void* kr, const void* v,
-                                    const float* o_t, const float* lse_t, void* o, float* lse, cudaStream_t stream) {
-  const int64_t warps = static_cast<int64_t>(g.P) * g.si.T * g.Hkv;
-  if (warps == 0) return cudaSuccess;
-  auto* qb = static_cast<const __nv_bfloat16*>(qr);
-  auto* kb = static_cast<const __nv_bfloat16*>(kr);
-  auto* vb = static_cast<const __nv_bfloat16*>(v);
-  auto* ob = static_cast<__nv_bfloat16*>(o);
-  if (g.D == 128)
-    branch_merge_fwd_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, qb, kb, vb, o_t, lse_t, ob, lse);
-  else
-    branch_merge_fwd_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, qb, kb, vb, o_t, lse_t, ob, lse);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
                                   cudaStream_t stream) {

@@ -52,6 +52,7 @@ struct FwdCfg {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kMaxBranch = 15;             // P <= 16 passes: at most 15 branch keys per query
 
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
@@ -332,10 +333,50 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
     if (ok && wait_bounded(o_final + t, 0, wd, kSiteFwdOFinal)) {
       tc_fence_after();
+      // ---- epilogue: branch keys (a3) and the exact joint-LSE merge (a4).
+      // Query (pass p, position qpos) also sees k~_j[tau], V_j[tau] of the branch passes
+      // j = 1..p (0-based) at its own position; scores on the CUDA cores.  The trunk
+      // partial is (m_run, l_run, unnormalised O in TMEM), all in log2 units.
       const bool valid = qpos < len;
-      const float inv_l = 1.f / l_run;
-      const int64_t rowid = static_cast<int64_t>(p_of[t] * g.H + h_of[t]) * g.si.T + seq_start + qpos;
-      float* dst = a.o_t + rowid * D;
+      const int p = p_of[t], h = h_of[t];
+      const int tau = seq_start + qpos;
+      const int T = g.si.T;
+      float bs[kMaxBranch];
+      float m = m_run;
+#pragma unroll
+      for (int j = 1; j <= kMaxBranch; ++j) {
+        bs[j - 1] = -INFINITY;
+        if (j <= p && valid) {
+          const uint4* kj = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) +
+                                                           ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D);
+          const uint8_t* qrow = sQ + t * C::TILE + row * 128;
+          float acc = 0.f;
+#pragma unroll 4
+          for (int c8 = 0; c8 < D / 8; ++c8) {
+            const uint4 qv = *reinterpret_cast<const uint4*>(qrow + (c8 >> 3) * C::CHUNK + (((c8 & 7) ^ (row & 7)) << 4));
+            const uint4 kv = __ldg(kj + c8);
+            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qv);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kv);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 a2 = __bfloat1622float2(q2[u]);
+              const float2 b2 = __bfloat1622float2(k2[u]);
+              acc = fmaf(a2.x, b2.x, fmaf(a2.y, b2.y, acc));
+            }
+          }
+          bs[j - 1] = acc * sl2;
+          m = fmaxf(m, bs[j - 1]);
+        }
+      }
+      const float scale_t = exp2_approx(m_run - m);
+      float l = l_run * scale_t;
+#pragma unroll
+      for (int j = 0; j < kMaxBranch; ++j) {
+        bs[j] = exp2_approx(bs[j] - m);  // branch weights (0 for absent passes)
+        l += bs[j];
+      }
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -343,15 +384,38 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         tmem_ld_wait();
         reg_fence32(o);
         if (valid) {
+          float acc[32];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float4 v4 = make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
-                                    __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
-            *reinterpret_cast<float4*>(dst + 32 * c + e) = v4;
+          for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * scale_t;
+#pragma unroll
+          for (int j = 1; j <= kMaxBranch; ++j) {
+            if (j <= p) {
+              const uint4* vj = reinterpret_cast<const uint4*>(
+                  static_cast<const __nv_bfloat16*>(a.v) + ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D +
+                  32 * c);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const uint4 vv = __ldg(vj + q4);
+                const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const float2 f2 = __bfloat1622float2(v2[u]);
+                  acc[8 * q4 + 2 * u] = fmaf(bs[j - 1], f2.x, acc[8 * q4 + 2 * u]);
+                  acc[8 * q4 + 2 * u + 1] = fmaf(bs[j - 1], f2.y, acc[8 * q4 + 2 * u + 1]);
+                }
+              }
+            }
           }
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[q4] = make_uint4(pack_bf16x2(acc[8 * q4] * inv_l, acc[8 * q4 + 1] * inv_l),
+                                 pack_bf16x2(acc[8 * q4 + 2] * inv_l, acc[8 * q4 + 3] * inv_l),
+                                 pack_bf16x2(acc[8 * q4 + 4] * inv_l, acc[8 * q4 + 5] * inv_l),
+                                 pack_bf16x2(acc[8 * q4 + 6] * inv_l, acc[8 * q4 + 7] * inv_l));
         }
       }
-      if (valid) a.lse_t[rowid] = (m_run + __log2f(l_run)) * kLn2;
+      if (valid) a.lse[lse_index(g.si, g.H, p, h, n, tau, qpos)] = (m + __log2f(l)) * kLn2;
     }
   }
 

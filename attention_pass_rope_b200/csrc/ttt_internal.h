@@ -58,20 +58,18 @@ cudaError_t launch_rope_fwd(const Geometry& g, const void* q, const void* k, voi
 
 struct TrunkFwdArgs {
   Geometry g;
-  float* o_t;      // fp32 [P][H][T][D]
-  float* lse_t;    // fp32 [P][H][T]
+  const void* kr;  // bf16 k~ head-major [P][Hkv][T][D] (branch keys, passes >= 1)
+  const void* v;   // bf16 V, public layout [P][T][Hkv][D] (branch values)
+  void* o;         // bf16 output, public layout [P][T][H][D]
+  float* lse;      // fp32 merged lse, public layout
   uint32_t* status;
   uint64_t budget_ns;
 };
-// a2: trunk causal attention on tcgen05; maps: q~ (3D {D, T, P*H}), k~_1 (3D {D, T, Hkv}),
+// a2+a3+a4: trunk causal attention on tcgen05 with the branch keys and the exact
+// joint-LSE merge in its epilogue.  Maps: q~ (3D {D, T, P*H}), k~_1 (3D {D, T, Hkv}),
 // V_1 (3D {D, Hkv, T}), all 64-element (128-byte) swizzled boxes.
 cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
                              const CUtensorMap& map_v, cudaStream_t stream);
-
-// a3+a4: branch keys (warp dot products) and the joint-LSE merge.
-cudaError_t launch_branch_merge_fwd(const Geometry& g, const void* qr, const void* kr, const void* v,
-                                    const float* o_t, const float* lse_t, void* o, float* lse,
-                                    cudaStream_t stream);
 
 // Row statistics of the backward, tile-aligned: for query head (p, h) and the 64-row
 // query tile j of sequence n, slot = start_n / 64 + n + j holds 64 values of

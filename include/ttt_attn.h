@@ -70,7 +70,7 @@ typedef enum { TTT_LAYOUT_BSHD = 0, TTT_LAYOUT_THD = 1 } ttt_layout;
 enum {
   TTT_KERNEL_ROPE_FWD = 0,
   TTT_KERNEL_TRUNK_FWD = 1,
-  TTT_KERNEL_BRANCH_MERGE_FWD = 2,
+  TTT_KERNEL_UNUSED_2 = 2, /* the branch keys and the merge run in the trunk forward's epilogue */
   TTT_KERNEL_ROPE_BWD = 3,
   TTT_KERNEL_BWD_PREPROCESS = 4,
   TTT_KERNEL_TRUNK_BWD = 5,
@@ -104,7 +104,7 @@ size_t ttt_attn_workspace_size(const ttt_attn_desc* desc, int for_backward);
 /* Forward.  q, k, v: bf16 pre-RoPE inputs (layouts above).  o: bf16 output, same
  * layout as q.  lse: fp32 merged log-sum-exp (natural log of the sum of
  * exp(sigma * q~.k) over the visible keys).  The workspace holds, after the call,
- * the rotated q~ / k~ and the trunk partials (see ttt_attn_workspace_layout). */
+ * the rotated q~ / k~ (see ttt_attn_workspace_layout). */
 ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, void* o,
                         float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
@@ -144,9 +144,7 @@ ttt_status ttt_attn_device_status(void* workspace, void* stream, uint32_t* detai
 
 /* Workspace sub-buffers (byte offsets from the workspace base), for inspection of
  * the intermediate results by tests:
- *   fwd: [0] status word, [1] q~ bf16 [P][H][Tt][D], [2] k~ bf16 [P][Hkv][Tt][D],
- *        [3] O_t fp32 [P][H][Tt][D] (trunk-only normalised output),
- *        [4] lse_t fp32 [P][H][Tt] (trunk-only log-sum-exp);
+ *   fwd: [0] status word, [1] q~ bf16 [P][H][Tt][D], [2] k~ bf16 [P][Hkv][Tt][D];
  *   bwd: [0] status, [1] q~, [2] k~, [3] row statistics fp32: for query head (p, h)
  *        and the 64-row query tile j of sequence n, 128 floats at slot
  *        start_n/64 + n + j of row p*H + h (lse * log2(e) of the 64 rows, then their

@@ -56,9 +56,9 @@ def test_4k_config_sampled_group():
 
 
 @needs_cuda
-def test_intermediates_tiny():
-    """Workspace contents after the forward: rotated q~/k~ (bf16) and the trunk-only
-    O_t / lse_t, against the oracle's rotation and its two-part pieces."""
+def test_rotated_inputs_tiny():
+    """Workspace contents after the forward: the rotated q~ / k~ (bf16), head-major,
+    against the oracle's fp64 rotation rounded to bf16."""
     from attention_pass_rope_b200 import ops
     w = ttt_inputs.workloads()["tiny"]
     inp = ttt_inputs.make_inputs(w, with_grad=False)
@@ -68,6 +68,7 @@ def test_intermediates_tiny():
     ops.ttt_attn_fwd(q, k, v, theta=w.theta, workspace=ws)
     torch.cuda.synchronize()
     offs = ops.workspace_layout(lay, w.theta)
+    assert len(offs) == 3
     P, T, H, Hkv, D = w.P, w.T, w.H, w.Hkv, w.D
 
     def view(i, n, dtype):
@@ -75,8 +76,6 @@ def test_intermediates_tiny():
 
     qr = view(1, P * H * T * D, torch.bfloat16).view(P, H, T, D).permute(0, 2, 1, 3)
     kr = view(2, P * Hkv * T * D, torch.bfloat16).view(P, Hkv, T, D).permute(0, 2, 1, 3)
-    o_t = view(3, P * H * T * D, torch.float32).view(P, H, T, D).permute(0, 2, 1, 3)
-    lse_t = view(4, P * H * T, torch.float32).view(P, H, T)
     qn, kn, vn, _ = parity.oracle_np(inp)
     qr_ref, kr_ref = orc.rotate_inputs(qn, kn, w.theta, rope_round="bf16")
     # fp32 rotation vs fp64 rotation, both rounded to bf16: a rare one-ulp flip
@@ -84,9 +83,6 @@ def test_intermediates_tiny():
     assert np.mean(dq_ > 0) < 2e-3 and np.max(dq_) <= 2.0 ** -7 * np.max(np.abs(qr_ref))
     dk_ = np.abs(parity.to64(kr) - kr_ref)
     assert np.mean(dk_ > 0) < 2e-3
-    _, _, parts = orc.forward_twopart(qn, kn, vn, w.theta, return_parts=True)
-    assert np.max(np.abs(parity.to64(o_t) - parts["O_t"])) < 1e-2
-    assert np.max(np.abs(parity.to64(lse_t) - parts["lse_t"])) < 1e-3
 
 
 @needs_cuda
