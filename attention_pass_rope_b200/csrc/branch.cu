@@ -11,6 +11,8 @@
 // These are memory-bound kernels with <= P-1 keys per query: one warp per
 // (position, KV head) row group, each lane holding D/32 elements of a row, dot
 // products finished with warp shuffles.  No tensor cores.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace ttt {
@@ -116,31 +118,62 @@ __device__ __forceinline__ void rotate_back(float (&x)[2][D / 64], const float (
 // ---------------------------------------------------------------------------
 // a5: delta = rowsum(dO * O).  Written, with lse * log2(e), into the tile-aligned
 // row-statistics array that the trunk backward fetches one 512-byte slot at a time.
+// Memory bound (reads O and dO once): D/8 lanes per row, one 16-byte load of each
+// per lane, kUnroll rows per lane group in flight.
 // ---------------------------------------------------------------------------
+constexpr int kUnroll = 4;
+
 template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     bwd_preprocess_kernel(Geometry g, const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                           const float* __restrict__ lse, float* __restrict__ ld) {
+  constexpr int LPR = D / 8;    // lanes per row
+  constexpr int RPW = 32 / LPR;  // rows per warp and step
   const int lane = threadIdx.x & 31;
-  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int sub = lane / LPR, c = lane % LPR;
   const int T = g.si.T;
-  if (w >= static_cast<int64_t>(g.P) * T * g.H) return;
-  const int p = static_cast<int>(w / (static_cast<int64_t>(T) * g.H));
-  const int rem = static_cast<int>(w % (static_cast<int64_t>(T) * g.H));
-  const int tau = rem / g.H;
-  const int h = rem % g.H;
-  const int64_t off = ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D;
-  float a[2][D / 64], b[2][D / 64];
-  load_bf16_row<D>(o + off, lane, a);
-  load_bf16_row<D>(dout + off, lane, b);
-  const float s = dot_row<D>(a, b);
-  if (lane == 0) {
-    int n, pos;
-    token_position(g.si, tau, n, pos);
-    const int slot = ld_slot(tau - pos, n, pos);
-    float* row = ld + ((static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + slot) * 128;
-    row[pos & 63] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)] * 1.4426950408889634f;
-    row[64 + (pos & 63)] = s;
+  const int64_t nrows = static_cast<int64_t>(g.P) * T * g.H;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
+  const int nslots = ld_slots(g.si);
+  for (int64_t r0 = (static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5)) * RPW * kUnroll;
+       r0 < nrows; r0 += nwarps * RPW * kUnroll) {
+    uint4 a[kUnroll], b[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t row = r0 + u * RPW + sub;
+      if (row < nrows) {
+        a[u] = __ldg(reinterpret_cast<const uint4*>(o + row * D) + c);
+        b[u] = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + c);
+      } else {
+        a[u] = make_uint4(0, 0, 0, 0);
+        b[u] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+      const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+        acc = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, acc));
+      }
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const int64_t row = r0 + u * RPW + sub;
+      if (c == 0 && row < nrows) {
+        const int h = static_cast<int>(row % g.H);
+        const int64_t pt = row / g.H;
+        const int tau = static_cast<int>(pt % T);
+        const int p = static_cast<int>(pt / T);
+        int n, pos;
+        token_position(g.si, tau, n, pos);
+        float* slot = ld + ((static_cast<int64_t>(p) * g.H + h) * nslots + ld_slot(tau - pos, n, pos)) * 128;
+        slot[pos & 63] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)] * 1.4426950408889634f;
+        slot[64 + (pos & 63)] = acc;
+      }
+    }
   }
 }
 
@@ -286,14 +319,17 @@ inline unsigned blocks_for(int64_t warps) {
 
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
                                   cudaStream_t stream) {
-  const int64_t warps = static_cast<int64_t>(g.P) * g.si.T * g.H;
-  if (warps == 0) return cudaSuccess;
+  const int64_t rows = static_cast<int64_t>(g.P) * g.si.T * g.H;
+  if (rows == 0) return cudaSuccess;
+  const int rpw = 32 / (g.D / 8);
+  const int64_t warps = (rows + rpw * kUnroll - 1) / (rpw * kUnroll);
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(blocks_for(warps), 148 * 32));
   auto* ob = static_cast<const __nv_bfloat16*>(o);
   auto* db = static_cast<const __nv_bfloat16*>(dout);
   if (g.D == 128)
-    bwd_preprocess_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
+    bwd_preprocess_kernel<128><<<blocks, kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
   else
-    bwd_preprocess_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
+    bwd_preprocess_kernel<64><<<blocks, kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
   return cudaGetLastError();
 }
 
