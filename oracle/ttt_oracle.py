@@ -414,3 +414,98 @@ def backward_packed(q, k, v, do, lse, cu_seqlens, theta, dense, scale=None, rope
                              rope_round, kv_heads=kv_heads)
         dq[:, a:b], dk[:, a:b], dv[:, a:b] = g
     return dq, dk, dv
+
+
+# --------------------------------------------------------------------------
+# single rows straight from the definition (for samples of full-size workloads)
+# --------------------------------------------------------------------------
+
+
+def _rot_rows(x_rows, positions, theta, rope_round):
+    """Rotate rows x_rows[n, D] at positions[n] (one position per row)."""
+    out = np.empty_like(x_rows, dtype=np.float64)
+    for n, m in enumerate(positions):
+        out[n] = rope_rotate(x_rows[n][None, None, :].astype(np.float64), [int(m)], theta)[0, 0]
+    if rope_round == "bf16":
+        out = bf16_round(out)
+    return out
+
+
+def rotate_trunk_keys(k, kv, theta, rope_round="bf16"):
+    """Rotated trunk keys k~_1[0..L-1] of KV head kv (key t at position t)."""
+    L = k.shape[1]
+    return _rot_rows(k[0, :, kv], np.arange(L), theta, rope_round)
+
+
+def _visible(q, k, v, theta, sc, rope_round, p0, i, h, g, kt=None):
+    """Rotated query row, visible keys and values of query (pass p0, position i, head h).
+    ``kt``: rotated trunk keys of the KV head (rotate_trunk_keys), computed if absent."""
+    kv = h // g
+    qr = _rot_rows(q[p0, i, h][None, :], [i + p0], theta, rope_round)[0]
+    if kt is None:
+        kt = _rot_rows(k[0, : i + 1, kv], np.arange(i + 1), theta, rope_round)   # trunk keys 0..i
+    keys = [kt[: i + 1]]
+    vals = [v[0, : i + 1, kv].astype(np.float64)]
+    if p0 > 0:                                                                     # branch keys j = 1..p0
+        kb = np.stack([k[j, i, kv] for j in range(1, p0 + 1)])
+        keys.append(_rot_rows(kb, [i + j for j in range(1, p0 + 1)], theta, rope_round))
+        vals.append(np.stack([v[j, i, kv] for j in range(1, p0 + 1)]).astype(np.float64))
+    return qr, np.concatenate(keys), np.concatenate(vals)
+
+
+def row_forward(q, k, v, theta, p0, i, h, scale=None, rope_round="bf16", kt=None):
+    """O[p0, i, h, :] and lse[p0, h, i] of one sequence by the plain definition."""
+    H, D = q.shape[2], q.shape[3]
+    g = H // k.shape[2]
+    sc = _scale(D, scale)
+    qr, K, V = _visible(q, k, v, theta, sc, rope_round, p0, i, h, g, kt)
+    s = sc * (K @ qr)
+    m = s.max()
+    e = np.exp(s - m)
+    return (e / e.sum()) @ V, m + np.log(e.sum())
+
+
+def _row_grads(q, k, v, do, theta, sc, rope_round, p0, i, h, g, kt=None):
+    """Softmax and its gradient pieces for one query row: (qr, K, V, P, dS)."""
+    qr, K, V = _visible(q, k, v, theta, sc, rope_round, p0, i, h, g, kt)
+    s = sc * (K @ qr)
+    P = np.exp(s - s.max())
+    P /= P.sum()
+    dP = V @ do[p0, i, h].astype(np.float64)
+    dS = P * (dP - np.dot(P, dP))
+    return qr, K, V, P, dS
+
+
+def row_dq(q, k, v, do, theta, p0, i, h, scale=None, rope_round="bf16", kt=None):
+    """dQ[p0, i, h, :] (w.r.t. the pre-RoPE query) of one sequence."""
+    H, D = q.shape[2], q.shape[3]
+    g = H // k.shape[2]
+    sc = _scale(D, scale)
+    _, K, _, _, dS = _row_grads(q, k, v, do, theta, sc, rope_round, p0, i, h, g, kt)
+    dqr = sc * (dS @ K)
+    return rope_rotate(dqr[None, None, :], [i + p0], theta, inverse=True)[0, 0]
+
+
+def row_dkv(q, k, v, do, theta, j0, t, kv, scale=None, rope_round="bf16"):
+    """dK[j0, t, kv, :] (pre-RoPE) and dV[j0, t, kv, :] of one sequence: the sum over
+    every query row that sees key (pass j0, position t) of KV head kv."""
+    P_, L, H, D = q.shape
+    g = H // k.shape[2]
+    sc = _scale(D, scale)
+    dkr = np.zeros(D)
+    dv = np.zeros(D)
+    kt = rotate_trunk_keys(k, kv, theta, rope_round)
+    for h in range(kv * g, (kv + 1) * g):
+        if j0 == 0:
+            rows = [(p0, i) for p0 in range(P_) for i in range(t, L)]   # trunk key t: every query i >= t
+            col = lambda p0, i: t                                        # index among the visible keys
+        else:
+            rows = [(p0, t) for p0 in range(j0, P_)]                      # branch key: queries at position t
+            col = lambda p0, i: (i + 1) + (j0 - 1)
+        for p0, i in rows:
+            qr, K, V, Pr, dS = _row_grads(q, k, v, do, theta, sc, rope_round, p0, i, h, g, kt)
+            c = col(p0, i)
+            dkr += sc * dS[c] * qr
+            dv += Pr[c] * do[p0, i, h].astype(np.float64)
+    dk = rope_rotate(dkr[None, None, :], [t + j0], theta, inverse=True)[0, 0]
+    return dk, dv

@@ -114,3 +114,67 @@ def test_no_device_timeouts_after_calls():
     assert ops.device_status(ws)[0] == _lib.TTT_OK
     ops.ttt_attn_bwd(q, k, v, o, lse, do, theta=w.theta, workspace=ws)
     assert ops.device_status(ws)[0] == _lib.TTT_OK
+
+
+# ----------------------------------------------------------------------------- full size
+
+@needs_cuda
+def test_deep_ttt_8k_sampled_group():
+    """B=1, S=8192, P=7, 32/8 heads, D=128: full tensors of KV head 3 (its 4 query heads
+    and all 7 passes) against the oracle."""
+    _check(ttt_inputs.workloads()["deep_ttt_8k"], kv_heads=[3])
+
+
+@needs_cuda
+def test_thd_packed_sampled_sequences():
+    """16 packed sequences (T = 38 264): full tensors of sequences 5 (649 tokens) and
+    4 (3696 tokens), KV head 2."""
+    _check(ttt_inputs.workloads()["thd_packed"], kv_heads=[2], seqs=[4, 5])
+
+
+@needs_cuda
+def test_long_32k_sampled_rows():
+    """B=1, S=32768, P=5, 32/8 heads, D=128, inputs scaled by 0.5: single rows computed
+    one by one by the oracle -- outputs and dQ of query rows across the sequence, dK/dV
+    of trunk keys near the end (seen by few queries) and of branch keys anywhere."""
+    w = ttt_inputs.workloads()["long_32k"]
+    inp = ttt_inputs.make_inputs(w)
+    gpu = parity.run_gpu(w, inp, with_grad=True)
+    # float32 copies hold the bf16 values exactly; the oracle widens the rows it uses
+    q, k, v, do = (t.float().numpy() for t in (inp.q, inp.k, inp.v, inp.do))
+    g = w.H // w.Hkv
+    kts = {}
+    o_err, l_err, dq_ref, dq_got = 0.0, 0.0, [], []
+    for (p0, i, h) in [(0, 0, 0), (4, 0, 31), (1, 127, 5), (2, 128, 9), (3, 4097, 14), (0, 20000, 22),
+                       (4, 32767, 7), (2, 32766, 30)]:
+        kv = h // g
+        if kv not in kts:
+            kts[kv] = orc.rotate_trunk_keys(k, kv, w.theta)
+        o_r, l_r = orc.row_forward(q, k, v, w.theta, p0, i, h, kt=kts[kv])
+        o_err = max(o_err, float(np.max(np.abs(parity.to64(gpu["o"][p0, i, h]) - o_r))))
+        l_err = max(l_err, abs(float(gpu["lse"][p0, 0, h, i]) - l_r))
+        dq_ref.append(orc.row_dq(q, k, v, do, w.theta, p0, i, h, kt=kts[kv]))
+        dq_got.append(parity.to64(gpu["dq"][p0, i, h]))
+    dk_ref, dk_got, dv_ref, dv_got = [], [], [], []
+    for (j0, t, kv) in [(0, 32767, 0), (0, 32760, 5), (1, 0, 2), (2, 9000, 7), (4, 32767, 1), (3, 15, 4)]:
+        dk_r, dv_r = orc.row_dkv(q, k, v, do, w.theta, j0, t, kv)
+        dk_ref.append(dk_r)
+        dv_ref.append(dv_r)
+        dk_got.append(parity.to64(gpu["dk"][j0, t, kv]))
+        dv_got.append(parity.to64(gpu["dv"][j0, t, kv]))
+    m = {"o_max_abs": o_err, "lse_max_abs": l_err,
+         "dq_rel_l2": parity.rel_l2(np.array(dq_got), np.array(dq_ref)),
+         "dk_rel_l2": parity.rel_l2(np.array(dk_got), np.array(dk_ref)),
+         "dv_rel_l2": parity.rel_l2(np.array(dv_got), np.array(dv_ref))}
+    print("long_32k", m)
+    parity.assert_within(m)
+
+
+@needs_cuda
+def test_long_32k_outputs_finite():
+    """Whole-tensor property at the largest size: every output and lse entry is finite."""
+    w = ttt_inputs.workloads()["long_32k"]
+    inp = ttt_inputs.make_inputs(w, with_grad=False)
+    gpu = parity.run_gpu(w, inp, with_grad=False)
+    assert torch.isfinite(gpu["o"].float()).all()
+    assert torch.isfinite(gpu["lse"]).all()

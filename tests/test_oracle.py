@@ -256,3 +256,21 @@ def test_packed_layouts():
     assert lse2.shape == (P, 2, H, 4)
     Os, ls = orc.forward_twopart(q[:, 4:8], k[:, 4:8], v[:, 4:8], 1e4)
     np.testing.assert_array_equal(lse2[:, 1], ls)
+
+
+def test_single_row_functions_match_full_oracle():
+    """The per-row forms (used on samples of full-size workloads) agree with the
+    two-part oracle element by element."""
+    P, L, H, Hkv, D = 3, 9, 4, 2, 8
+    q, k, v, do = rnd(P, L, H, D), rnd(P, L, Hkv, D), rnd(P, L, Hkv, D), rnd(P, L, H, D)
+    O, lse = orc.forward_twopart(q, k, v, 1e4)
+    dq, dk, dv = orc.backward_twopart(q, k, v, do, lse, 1e4)
+    for (p0, i, h) in [(0, 0, 0), (1, 4, 3), (2, 8, 1), (2, 0, 2)]:
+        o_r, l_r = orc.row_forward(q, k, v, 1e4, p0, i, h)
+        np.testing.assert_allclose(o_r, O[p0, i, h], atol=1e-13)
+        assert abs(l_r - lse[p0, h, i]) < 1e-13
+        np.testing.assert_allclose(orc.row_dq(q, k, v, do, 1e4, p0, i, h), dq[p0, i, h], atol=1e-12)
+    for (j0, t, kv) in [(0, 0, 0), (0, 7, 1), (1, 3, 0), (2, 8, 1)]:
+        dk_r, dv_r = orc.row_dkv(q, k, v, do, 1e4, j0, t, kv)
+        np.testing.assert_allclose(dk_r, dk[j0, t, kv], atol=1e-12)
+        np.testing.assert_allclose(dv_r, dv[j0, t, kv], atol=1e-12)
