@@ -231,7 +231,7 @@ def run_ours(args, rank, world, local):
     bwd_flops = 10 * w.D * w.trunk_pairs * w.H * w.P
     bwd_ms = per_kernel["trunk_bwd"]
     achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
-    traffic = read_traffic("trunk_bwd", args.workload)
+    traffic = read_traffic("trunk_bwd", w.name)
     line = {
         "metric": METRIC,
         "value": round(tflops, 2),
@@ -281,14 +281,20 @@ def workload(args):
 
 
 def read_traffic(kernel, workload):
-    """dram bytes per launch from the committed ncu summary, if one matches the kernel."""
+    """DRAM bytes per launch from the committed ncu record of the kernel, or None when
+    there is none or the kernel's source changed since the counters were taken."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
-            return json.load(f).get("dram_bytes_per_launch")
-    except (OSError, ValueError):
+            d = json.load(f)
+        with open(os.path.join(ROOT, d["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != d["source_sha256"]:
+                return None
+        return d.get("dram_bytes_per_launch")
+    except (OSError, ValueError, KeyError):
         return None
 
 
