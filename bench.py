@@ -54,7 +54,7 @@ def dist_env():
 class ClockSampler:
     """nvidia-smi clock/throttle samples every 200 ms while running."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -77,7 +77,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, name):
+        setattr(self, name, time.time())
 
     def stop(self):
         if self.proc is None:
@@ -91,7 +94,11 @@ class ClockSampler:
             self.t.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0 = getattr(self, "t_begin", 0.0)
+        t1 = getattr(self, "t_end", float("inf"))
+        for ts, ln in self.lines:
+            if not (t0 <= ts <= t1 + 0.25):
+                continue  # only samples taken while the timed steps ran
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -171,11 +178,13 @@ def run_ours(args, rank, world, local):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark("t_begin")
     t0.record()
     for i in range(K):
         step(evs[i])
     t1.record()
     torch.cuda.synchronize()
+    sampler.mark("t_end")
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
@@ -380,7 +389,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ttt_inputs.workloads()))
