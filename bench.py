@@ -44,6 +44,18 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (the job is as slow as its slowest rank)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(flops_per_rank_step, world, ms_per_step):
+    """Aggregate throughput: the work of all ranks over the (max-over-ranks) step time."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -226,13 +238,11 @@ def run_ours(args, rank, world, local):
     e2e_ms = e0.elapsed_time(e1) / E
 
     if world > 1:
-        tt = torch.tensor([ms, e2e_ms], device=device)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms = float(tt[0]), float(tt[1])
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms], device)
 
     ms_step = ms / K
     flops = w.flops_fwd_bwd()
-    tflops = flops * world / (ms_step * 1e-3) / 1e12
+    tflops = whole_job_tflops(flops, world, ms_step)
     peaks, peak_src = load_peaks()
     peak = peaks["bf16_tflops_sustained"]
     # dominant kernel: the trunk backward (tensor bound); its algorithmic flops per launch
