@@ -80,7 +80,7 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
   if (!for_backward) {
     pl.noff = 3;
   } else {
-    pl.off[3] = o;  // tile-aligned row statistics (lse*log2e, delta)
+    pl.off[3] = o;  // tile-aligned row statistics (-lse*log2e, delta)
     o = align_up(o + P * H * static_cast<size_t>(ld_slots(g.si)) * 128 * 4);
     pl.off[4] = o;  // dq~ accumulator
     o = align_up(o + P * H * T * D * 4);

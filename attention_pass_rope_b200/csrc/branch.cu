@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         int n, pos;
         token_position(g.si, tau, n, pos);
         float* slot = ld + ((static_cast<int64_t>(p) * g.H + h) * nslots + ld_slot(tau - pos, n, pos)) * 128;
-        slot[pos & 63] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)] * 1.4426950408889634f;
+        slot[pos & 63] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)] * -1.4426950408889634f;
         slot[64 + (pos & 63)] = acc;
       }
     }

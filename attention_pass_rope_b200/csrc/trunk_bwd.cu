@@ -20,11 +20,12 @@
 // fp32 dq~ accumulator with one bulk reduce-add per tile.
 //
 // CTA = 16 warps: warp 0 TMA producer (+ lse/delta rows), warp 1 TMEM allocator and
-// MMA issuer, warps 4-7 and 8-11 the two halves (query columns 0-31 / 32-63) of the
-// probability / dS step, warps 12-15 the dQ writer.  S^T/dP^T of tile n+1 are
-// issued before the dV/dK/dQ products of tile n so that the CUDA-core work of one
-// tile overlaps the tensor-core work of the previous one; P^T and dS^T are double
-// buffered for that reason.
+// S^T/dP^T issuer, warp 2 dV/dK/dQ^T issuer, warps 4-7 and 8-11 the two halves (query
+// columns 0-31 / 32-63) of the probability / dS step, warps 12-15 the dQ writer.
+// S^T/dP^T of step n+1 are issued as soon as the P/dS warps have read step n's into
+// registers, so they are complete before those warps finish step n, and the
+// dV/dK/dQ^T products of step n run under the CUDA-core work of step n+1.  P^T and
+// dS^T are double buffered for that reason; S^T/dP^T are single buffered.
 #include "common.cuh"
 
 namespace ttt {
@@ -50,11 +51,12 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + ST * QTILE;
   static constexpr int OFF_DS = OFF_DO + ST * QTILE;
   static constexpr int OFF_DQ = OFF_DS + 2 * DSTILE;
-  static constexpr int OFF_LD = OFF_DQ + DQSTAGE;          // [ST][2][64] floats: lse*log2e, delta
+  static constexpr int OFF_LD = OFF_DQ + 2 * DQSTAGE;      // [ST][2][64] floats: lse*log2e, delta
   static constexpr int OFF_BAR = OFF_LD + ST * 2 * BQ * 4;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_USED = OFF_BAR + BAR_BYTES;
   static constexpr int SMEM = (SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED) + 1024;
+  static_assert(SMEM <= 227 * 1024, "dynamic shared memory above the per-block limit");
   static constexpr int COL_DV = 0;
   static constexpr int COL_DK = D;
   static constexpr int COL_S = 2 * D;
@@ -71,12 +73,16 @@ struct IterInfo {
   int p, h, q0;
 };
 
-__device__ __forceinline__ IterInfo decode_iter(int it, int nqt, int jq0, int gsz, int kvh) {
-  const int qh = it / nqt;
+// Walk order: query tiles from the last one down to the diagonal (outer), the G =
+// P * (H / Hkv) query heads of this KV head (inner).  CTAs of the same KV head that
+// run at the same time then read the same q~/dO tiles and reduce into the same dq~
+// rows within a short window, so both stay in L2.
+__device__ __forceinline__ IterInfo decode_iter(int it, int nqt, int jq0, int G, int gsz, int kvh) {
+  const int qh = it % G;
   IterInfo r;
   r.p = qh / gsz;
   r.h = kvh * gsz + qh % gsz;
-  r.q0 = (jq0 + it % nqt) * 64;
+  r.q0 = (jq0 + nqt - 1 - it / G) * 64;
   return r;
 }
 
@@ -113,8 +119,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   uint64_t* qdo_full = bars + 1;            // [ST]
   uint64_t* qdo_empty = bars + 1 + C::ST;   // [ST]
   uint64_t* sdp_full = bars + 1 + 2 * C::ST;
-  uint64_t* ds_ready = sdp_full + 1;
-  uint64_t* mma_done = ds_ready + 1;        // [2]
+  uint64_t* sdp_free = sdp_full + 1;
+  uint64_t* ds_ready = sdp_free + 1;        // [2], by step parity
+  uint64_t* mma_done = ds_ready + 2;        // [2]
   uint64_t* dq_full = mma_done + 2;
   uint64_t* dq_free = dq_full + 1;
   uint64_t* final_bar = dq_free + 1;
@@ -143,13 +150,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(qdo_empty + s, 1);
     }
     mbar_init(sdp_full, 1);
-    mbar_init(ds_ready, 8);   // one arrival per P/dS warp
+    mbar_init(sdp_free, 8);   // one arrival per P/dS warp
+    mbar_init(ds_ready + 0, 8);   // one arrival per P/dS warp
+    mbar_init(ds_ready + 1, 8);
     mbar_init(mma_done + 0, 1);
     mbar_init(mma_done + 1, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);    // one arrival per dQ-writer warp
-    mbar_init(final_bar, 1);
-    mbar_init(drain, 1);
+    mbar_init(final_bar, 2);  // one commit per MMA-issuing warp
+    mbar_init(drain, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -179,7 +188,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int s = it % C::ST;
         if (it >= C::ST && !wait_bounded(qdo_empty + s, ((it / C::ST) - 1) & 1, wd, kSiteBwdQdoEmpty)) break;
         TTT_TRACE(16, it);
-        const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
+        const IterInfo ii = decode_iter(it, nqt, jq0, G, gsz, kvh);
         mbar_arrive_expect_tx(qdo_full + s, 2 * C::QTILE + 2 * C::BQ * 4);
         for (int c = 0; c < C::KCH; ++c) {
           tma_load_3d(sQ + s * C::QTILE + c * C::QCHUNK, &map_q, qdo_full + s, c * 64, seq_start + ii.q0,
@@ -193,8 +202,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues S^T/dP^T, warp 2 the dV/dK/dQ^T products.  An issuing thread blocks
+    // until the tensor pipe accepts its instruction, and a barrier check queued behind
+    // it costs a few hundred cycles even when the barrier has completed; with two
+    // issuers one warp's checks are covered by the other's products.  The two streams
+    // share no TMEM columns, and each commit tracks only its own warp's products
+    // (every cross-stream dependency is ordered through the P/dS barriers).
     {
       constexpr uint32_t idSP = idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idDV = idesc_bf16_f32(128, D, false, true);
@@ -225,53 +240,58 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           umma_ss_warp(tmem + C::COL_DP, dV_k + ok_, dO_k + so + oq_, idSP, kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = wait_warp(kv_bar, 0, wd, kSiteBwdKv) && wait_warp(qdo_full, 0, wd, kSiteBwdQdoFull);
-      if (ok) {
-        tc_fence_after();
-        issue_sdp(0);
-        umma_commit_warp(sdp_full);
-      }
-      for (int it = 0; ok && it < NIT; ++it) {
-        const int s = it % C::ST;
-        const int b = it & 1;
-        if (!wait_warp(ds_ready, it & 1, wd, kSiteBwdDsReady)) break;
-        TTT_TRACE(0, it);
-        tc_fence_after();
-        if (it + 1 < NIT) {
-          if (!wait_warp(qdo_full + (it + 1) % C::ST, ((it + 1) / C::ST) & 1, wd, kSiteBwdQdoFull)) break;
+      bool ok = true;
+      if (warp == 1) {
+        // S^T/dP^T(n+2) once the P/dS warps hold S^T/dP^T(n+1) in registers: it is
+        // complete before they finish step n+1
+        ok = wait_warp(kv_bar, 0, wd, kSiteBwdKv);
+        for (int it = 0; ok && it < NIT; ++it) {
+          if (it > 0 && !wait_warp(sdp_free, (it - 1) & 1, wd, kSiteBwdSdpFree)) break;
+          if (!wait_warp(qdo_full + it % C::ST, (it / C::ST) & 1, wd, kSiteBwdQdoFull)) break;
+          TTT_TRACE(12, it);
           tc_fence_after();
-          issue_sdp(it + 1);
+          issue_sdp(it);
           umma_commit_warp(sdp_full);
+          TTT_TRACE(1, it);
         }
-        TTT_TRACE(1, it);
-        const uint32_t so = static_cast<uint32_t>((s * C::QTILE) >> 4);
-        const uint32_t bo = static_cast<uint32_t>((b * C::DSTILE) >> 4);
-        // dV += P^T dO   (P^T: TMEM, 64 queries = 32 packed columns)
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_ts_warp(tmem + C::COL_DV, tmem + C::COL_PT + 32 * b + kk * 8, dO_mn + so + ((kk * 2048) >> 4), idDV,
-                  (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q~
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_ss_warp(tmem + C::COL_DK, dS_k + bo + ((kk * 32) >> 4), dQ_mn + so + ((kk * 2048) >> 4), idDV,
-                  (it > 0 || kk > 0) ? 1u : 0u);
-        TTT_TRACE(2, it);
-        if (it > 0) {
-          if (!wait_warp(dq_free, (it - 1) & 1, wd, kSiteBwdDqFree)) break;
+      } else {
+        ok = wait_warp(kv_bar, 0, wd, kSiteBwdKv);
+        for (int it = 0; ok && it < NIT; ++it) {
+          const int s = it % C::ST;
+          const int b = it & 1;
+          if (!wait_warp(ds_ready + b, (it >> 1) & 1, wd, kSiteBwdDsReady)) break;
+          TTT_TRACE(0, it);
           tc_fence_after();
-        }
-        TTT_TRACE(3, it);
-        // dQ^T = K~^T dS^T
+          const uint32_t so = static_cast<uint32_t>((s * C::QTILE) >> 4);
+          const uint32_t bo = static_cast<uint32_t>((b * C::DSTILE) >> 4);
+          // dV += P^T dO   (P^T: TMEM, 64 queries = 32 packed columns)
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_ss_warp(tmem + C::COL_DQ, dK_mn + ((kk * 2048) >> 4), dS_mn + bo + ((kk * 2048) >> 4), idDQ,
-                  kk > 0 ? 1u : 0u);
-        umma_commit_warp(mma_done + b);
-        umma_commit_warp(qdo_empty + s);
-        umma_commit_warp(dq_full);
-        TTT_TRACE(4, it);
+          for (int kk = 0; kk < C::BQ / 16; ++kk)
+            umma_ts_warp(tmem + C::COL_DV, tmem + C::COL_PT + 32 * b + kk * 8, dO_mn + so + ((kk * 2048) >> 4),
+                         idDV, (it > 0 || kk > 0) ? 1u : 0u);
+          // dK += dS^T Q~
+#pragma unroll
+          for (int kk = 0; kk < C::BQ / 16; ++kk)
+            umma_ss_warp(tmem + C::COL_DK, dS_k + bo + ((kk * 32) >> 4), dQ_mn + so + ((kk * 2048) >> 4), idDV,
+                         (it > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_warp(qdo_empty + s);  // last readers of this step's q~ / dO tiles
+          TTT_TRACE(2, it);
+          if (it > 0) {
+            if (!wait_warp(dq_free, (it - 1) & 1, wd, kSiteBwdDqFree)) break;
+            tc_fence_after();
+          }
+          TTT_TRACE(3, it);
+          // dQ^T = K~^T dS^T
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk)
+            umma_ss_warp(tmem + C::COL_DQ, dK_mn + ((kk * 2048) >> 4), dS_mn + bo + ((kk * 2048) >> 4), idDQ,
+                         kk > 0 ? 1u : 0u);
+          umma_commit_warp(mma_done + b);
+          umma_commit_warp(dq_full);
+          TTT_TRACE(4, it);
+        }
       }
+      (void)ok;
       umma_commit_warp(final_bar);
       umma_commit_warp(drain);
       wait_drain(drain, 0, wd, kSiteBwdDrain);
@@ -290,13 +310,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     for (int it = 0; it < NIT; ++it) {
       const int s = it % C::ST;
       const int b = it & 1;
-      const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
+      const IterInfo ii = decode_iter(it, nqt, jq0, G, gsz, kvh);
       if (!wait_bounded(sdp_full, it & 1, wd, kSiteBwdSdpFull) ||
           !wait_bounded(qdo_full + s, (it / C::ST) & 1, wd, kSiteBwdQdoFull)) {
         ok = false;
         break;
       }
       if (lane == 0 && warp == 4) TTT_TRACE(5, it);
+      if (lane == 0 && warp == 8) TTT_TRACE(13, it);
       tc_fence_after();
       uint32_t sv[32], dp[32];
       tmem_ld32(lane_base + C::COL_S + 32 * hf, sv);
@@ -304,47 +325,59 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tmem_ld_wait();
       reg_fence32(sv);
       reg_fence32(dp);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sdp_free);
+      if (lane == 0) {
+        constexpr int kSlot[8] = {6, 22, 23, 17, 19, 18, 14, 15};
+        TTT_TRACE(kSlot[warp - 4], it);
+      }
+      const float* ldp = sLD + s * 2 * C::BQ + 32 * hf;
+      // interior tile: every (key, query) pair of this half is visible
+      const int qlo = ii.q0 + 32 * hf;
+      const bool interior = (qlo >= k0 + C::BK - 1) && (qlo + 32 <= len) && (k0 + C::BK <= len);
+      // P = 2^(s*scale*log2e - lse*log2e), dS = P (dP - delta), two columns per
+      // instruction; the bf16 pairs are packed straight from the results
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int c0 = 0; c0 < 32; c0 += 8) {
+        const ulonglong2 nl0 = *reinterpret_cast<const ulonglong2*>(ldp + c0);
+        const ulonglong2 nl1 = *reinterpret_cast<const ulonglong2*>(ldp + c0 + 4);
+        const ulonglong2 dl0 = *reinterpret_cast<const ulonglong2*>(ldp + C::BQ + c0);
+        const ulonglong2 dl1 = *reinterpret_cast<const ulonglong2*>(ldp + C::BQ + c0 + 4);
+        const uint64_t nl[4] = {nl0.x, nl0.y, nl1.x, nl1.y};
+        const uint64_t dl[4] = {dl0.x, dl0.y, dl1.x, dl1.y};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + 2 * u;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nl[u]), x0, x1);
+          float p0 = exp2_approx(x0), p1 = exp2_approx(x1);
+          const uint64_t t = f2_sub(f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), dl[u]);
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
+          if (!interior) {
+            // padding rows of the statistics are never written: select, do not multiply
+            const bool v0 = kvalid && qlo + c < len && kpos <= qlo + c;
+            const bool v1 = kvalid && qlo + c + 1 < len && kpos <= qlo + c + 1;
+            p0 = v0 ? p0 : 0.f;
+            d0 = v0 ? d0 : 0.f;
+            p1 = v1 ? p1 : 0.f;
+            d1 = v1 ? d1 : 0.f;
+          }
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+          dk[c >> 1] = pack_bf16x2(d0, d1);
+        }
+      }
+      if (lane == 0 && warp == 4) TTT_TRACE(8, it);
+      // P^T / dS^T buffer b was last read by the products of step it-2
       if (it >= 2 && !wait_bounded(mma_done + b, ((it >> 1) - 1) & 1, wd, kSiteBwdMmaDone)) {
         ok = false;
         break;
       }
       if (lane == 0 && warp == 4) TTT_TRACE(7, it);
-      const float* ldp = sLD + s * 2 * C::BQ + 32 * hf;
-      // interior tile: every (key, query) pair of this half is visible
-      const int qlo = ii.q0 + 32 * hf;
-      const bool interior = (qlo >= k0 + C::BK - 1) && (qlo + 32 <= len) && (k0 + C::BK <= len);
-      // P and dS overwrite S^T and dP^T in place, 8 columns at a time
-#pragma unroll
-      for (int c0 = 0; c0 < 32; c0 += 8) {
-        const float4 l0 = *reinterpret_cast<const float4*>(ldp + c0);
-        const float4 l1 = *reinterpret_cast<const float4*>(ldp + c0 + 4);
-        const float4 d0 = *reinterpret_cast<const float4*>(ldp + C::BQ + c0);
-        const float4 d1 = *reinterpret_cast<const float4*>(ldp + C::BQ + c0 + 4);
-        const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-        const float dv8[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int c = c0 + u;
-          float pr = exp2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lv[u]));
-          float ds = pr * (__uint_as_float(dp[c]) - dv8[u]);
-          if (!interior) {
-            // padding rows of the statistics are never written: select, do not multiply
-            const int qpos = qlo + c;
-            const bool vis = kvalid && qpos < len && kpos <= qpos;
-            pr = vis ? pr : 0.f;
-            ds = vis ? ds : 0.f;
-          }
-          sv[c] = __float_as_uint(pr);
-          dp[c] = __float_as_uint(ds);
-        }
-      }
-      uint32_t pk[16], dk[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        pk[e] = pack_bf16x2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1]));
-        dk[e] = pack_bf16x2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1]));
-      }
-      if (lane == 0 && warp == 4) TTT_TRACE(8, it);
+      tc_fence_after();
       tmem_st16(lane_base + C::COL_PT + 32 * b + 16 * hf, pk);
       // dS^T row r, 128-byte swizzle: 16-byte chunk c of the row sits at c ^ (r & 7)
       uint8_t* row = sDS + b * C::DSTILE + r * 128;
@@ -358,8 +391,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_ready);
+      if (lane == 0) mbar_arrive(ds_ready + b);
       if (lane == 0 && warp == 4) TTT_TRACE(9, it);
+
     }
     // ---- epilogue: dV (half 0) and dK~ (half 1) of this CTA's keys
     if (ok && wait_bounded(final_bar, 0, wd, kSiteBwdFinal)) {
@@ -399,7 +433,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const int tid = threadIdx.x - 384;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     for (int it = 0; it < NIT; ++it) {
-      const IterInfo ii = decode_iter(it, nqt, jq0, gsz, kvh);
+      const IterInfo ii = decode_iter(it, nqt, jq0, G, gsz, kvh);
       if (!wait_bounded(dq_full, it & 1, wd, kSiteBwdDqFull)) break;
       if (tid == 0) TTT_TRACE(10, it);
       tc_fence_after();
@@ -412,14 +446,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
-      // two halves of 32 query rows through a 16 KB staging buffer
+      if (tid == 0) TTT_TRACE(20, it);
+      // two halves of 32 query rows, each through its own staging buffer; one bulk
+      // group is committed per half (empty past the end of the sequence), so the group
+      // that last read a buffer is always the second most recent one
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
-        if (tid == 0) bulk_wait_read0();  // the staging buffer has been read by the last reduce
+        float* stage = sDQ + hq * (C::DQSTAGE / 4);
+        if (tid == 0) bulk_wait_read1();
         named_bar_sync(1, 128);
         if (d < D) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) sDQ[q * D + d] = __uint_as_float(hq == 0 ? v0[q] : v1[q]);
+          for (int q = 0; q < 32; ++q) stage[q * D + d] = __uint_as_float(hq == 0 ? v0[q] : v1[q]);
         }
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
@@ -428,11 +466,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           const int nrows = min(32, len - r0);
           if (nrows > 0) {
             float* dst = a.dq_acc + ((static_cast<int64_t>(ii.p) * g.H + ii.h) * g.si.T + seq_start + r0) * D;
-            bulk_reduce_add_f32(dst, sDQ, static_cast<uint32_t>(nrows * D * 4));
-            bulk_commit();
+            bulk_reduce_add_f32(dst, stage, static_cast<uint32_t>(nrows * D * 4));
           }
+          bulk_commit();
         }
       }
+      if (tid == 0) TTT_TRACE(21, it);
     }
     if (tid == 0) bulk_wait0();
   }

@@ -30,6 +30,7 @@ enum WaitSite : uint32_t {
   kSiteBwdDqFree = 0x27,
   kSiteBwdFinal = 0x28,
   kSiteBwdDrain = 0x29,
+  kSiteBwdSdpFree = 0x2a,
 };
 
 // Where the sequences are: dense batches (cu_seqlens == nullptr) hold nseq = B

@@ -147,7 +147,7 @@ ttt_status ttt_attn_device_status(void* workspace, void* stream, uint32_t* detai
  *   fwd: [0] status word, [1] q~ bf16 [P][H][Tt][D], [2] k~ bf16 [P][Hkv][Tt][D];
  *   bwd: [0] status, [1] q~, [2] k~, [3] row statistics fp32: for query head (p, h)
  *        and the 64-row query tile j of sequence n, 128 floats at slot
- *        start_n/64 + n + j of row p*H + h (lse * log2(e) of the 64 rows, then their
+ *        start_n/64 + n + j of row p*H + h (-lse * log2(e) of the 64 rows, then their
  *        delta = rowsum(dout * o)), T/64 + nseq + 1 slots per row,
  *        [4] dq~ accumulator fp32 [P][H][Tt][D], [5] dk~_1 accumulator fp32 [Hkv][Tt][D].
  * Tt = B*S (dense) or T (packed).  Returns the number of entries written to
