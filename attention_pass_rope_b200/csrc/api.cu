@@ -237,8 +237,7 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
-    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, stream));
-    TTT_CHECK_CUDA(cudaMemsetAsync(dq_acc, 0, static_cast<size_t>(g.P) * g.H * T * D * 4, stream));
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);

@@ -21,12 +21,6 @@ namespace {
 
 constexpr int kWarpsPerBlock = 8;
 
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
-
 // Lane element map: lane holds E = D/64 consecutive elements of each half of the
 // head dimension, d in [E*lane, E*lane+E) and [D/2 + E*lane, ...), so that each
 // RoPE pair (d, d + D/2) is in one lane.
@@ -79,31 +73,6 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16* row, int lane, con
   }
 }
 
-template <int D>
-__device__ __forceinline__ float dot_row(const float (&a)[2][D / 64], const float (&b)[2][D / 64]) {
-  float s = 0.f;
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-    for (int e = 0; e < D / 64; ++e) s = fmaf(a[hh][e], b[hh][e], s);
-  return warp_sum(s);
-}
-
-// cos/sin of position * theta^(-2d/D) for this lane's E frequencies (double-precision
-// argument, the same recipe as the forward rotation).
-template <int D>
-__device__ __forceinline__ void lane_cos_sin(float theta, int pos, int lane, float (&c)[D / 64], float (&s)[D / 64]) {
-#pragma unroll
-  for (int e = 0; e < D / 64; ++e) {
-    const int d = LaneMap<D>::d(lane, 0, e);
-    const double ang = static_cast<double>(pos) * pow(static_cast<double>(theta), -2.0 * d / D);
-    double sd, cd;
-    sincos(ang, &sd, &cd);
-    c[e] = static_cast<float>(cd);
-    s[e] = static_cast<float>(sd);
-  }
-}
-
 // x <- R(pos)^T x (rotation by the negative angle), in place.
 template <int D>
 __device__ __forceinline__ void rotate_back(float (&x)[2][D / 64], const float (&c)[D / 64], const float (&s)[D / 64]) {
@@ -116,64 +85,77 @@ __device__ __forceinline__ void rotate_back(float (&x)[2][D / 64], const float (
 }
 
 // ---------------------------------------------------------------------------
-// a5: delta = rowsum(dO * O).  Written, with lse * log2(e), into the tile-aligned
-// row-statistics array that the trunk backward fetches one 512-byte slot at a time.
-// Memory bound (reads O and dO once): D/8 lanes per row, one 16-byte load of each
-// per lane, kUnroll rows per lane group in flight.
+// a5: delta = rowsum(dO * O), written with -lse * log2(e) into the tile-aligned
+// row-statistics array that the trunk backward fetches one 512-byte slot at a time;
+// the same pass zeroes the fp32 dq~ accumulator rows that the trunk backward
+// reduces into.  One block per (pass, sequence, 64-token tile, head), head fastest
+// so that neighbouring blocks read neighbouring rows of O and dO.  Memory bound:
+// D/8 lanes per row, 16-byte loads, every row of a warp in flight at once.
 // ---------------------------------------------------------------------------
-constexpr int kUnroll = 4;
+constexpr int kPreRows = 64;
+constexpr int kPreThreads = 256;
 
 template <int D>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(kPreThreads)
     bwd_preprocess_kernel(Geometry g, const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                          const float* __restrict__ lse, float* __restrict__ ld) {
-  constexpr int LPR = D / 8;    // lanes per row
-  constexpr int RPW = 32 / LPR;  // rows per warp and step
-  const int lane = threadIdx.x & 31;
-  const int sub = lane / LPR, c = lane % LPR;
+                          const float* __restrict__ lse, float* __restrict__ ld, float* __restrict__ dq_acc,
+                          int ntile) {
+  constexpr int LPR = D / 8;                            // lanes per row
+  constexpr int RPI = 32 / LPR;                         // rows per warp instruction
+  constexpr int RPWARP = kPreRows / (kPreThreads / 32);  // rows per warp (8)
+  constexpr int NU = RPWARP / RPI;
+  __shared__ float sdelta[kPreRows];
+  const int h = static_cast<int>(blockIdx.x % g.H);
+  int rest = static_cast<int>(blockIdx.x / g.H);
+  const int tile = rest % ntile;
+  rest /= ntile;
+  const int n = rest % g.si.nseq;
+  const int p = rest / g.si.nseq;
+  int start, len;
+  seq_bounds(g.si, n, start, len);
+  const int pos0 = tile * kPreRows;
+  if (pos0 >= len) return;
+  const int nvalid = min(kPreRows, len - pos0);
   const int T = g.si.T;
-  const int64_t nrows = static_cast<int64_t>(g.P) * T * g.H;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
-  const int nslots = ld_slots(g.si);
-  for (int64_t r0 = (static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5)) * RPW * kUnroll;
-       r0 < nrows; r0 += nwarps * RPW * kUnroll) {
-    uint4 a[kUnroll], b[kUnroll];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / LPR, c = lane % LPR;
+
+  uint4 a[NU], b[NU];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t row = r0 + u * RPW + sub;
-      if (row < nrows) {
-        a[u] = __ldg(reinterpret_cast<const uint4*>(o + row * D) + c);
-        b[u] = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + c);
-      } else {
-        a[u] = make_uint4(0, 0, 0, 0);
-        b[u] = make_uint4(0, 0, 0, 0);
-      }
+  for (int u = 0; u < NU; ++u) {
+    const int i = warp * RPWARP + u * RPI + sub;
+    if (i < nvalid) {
+      const int64_t row = (static_cast<int64_t>(p) * T + start + pos0 + i) * g.H + h;
+      a[u] = __ldg(reinterpret_cast<const uint4*>(o + row * D) + c);
+      b[u] = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + c);
+    } else {
+      a[u] = make_uint4(0, 0, 0, 0);
+      b[u] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  // zero this tile's dq~ accumulator rows (contiguous: nvalid rows of D floats)
+  float4* z = reinterpret_cast<float4*>(dq_acc + ((static_cast<int64_t>(p) * g.H + h) * T + start + pos0) * D);
+  for (int i = threadIdx.x; i < nvalid * D / 4; i += kPreThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int u = 0; u < NU; ++u) {
+    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+      acc = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, acc));
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
-      const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
-      float acc = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
-        acc = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, acc));
-      }
-#pragma unroll
-      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      const int64_t row = r0 + u * RPW + sub;
-      if (c == 0 && row < nrows) {
-        const int h = static_cast<int>(row % g.H);
-        const int64_t pt = row / g.H;
-        const int tau = static_cast<int>(pt % T);
-        const int p = static_cast<int>(pt / T);
-        int n, pos;
-        token_position(g.si, tau, n, pos);
-        float* slot = ld + ((static_cast<int64_t>(p) * g.H + h) * nslots + ld_slot(tau - pos, n, pos)) * 128;
-        slot[pos & 63] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)] * -1.4426950408889634f;
-        slot[64 + (pos & 63)] = acc;
-      }
-    }
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (c == 0) sdelta[warp * RPWARP + u * RPI + sub] = acc;
+  }
+  __syncthreads();
+  float* slot = ld + ((static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + ld_slot(start, n, pos0)) * 128;
+  if (threadIdx.x < nvalid) {
+    const int i = threadIdx.x;
+    slot[i] = lse[lse_index(g.si, g.H, p, h, n, start + pos0 + i, pos0 + i)] * -1.4426950408889634f;
+    slot[64 + i] = sdelta[i];
   }
 }
 
@@ -186,8 +168,22 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 //     dQ_p = R(i+p)^T (sigma dq~)
 //   dK_j = R(i+j)^T (sigma dk~_j)  for every pass (j = 0 takes dk~_1 from the trunk
 //   backward), dV_j for j >= 1 (dV_1 is written by the trunk backward).
-// Per-warp accumulators for the branch passes live in shared memory.
+// The group heads of a pass are taken kBranchHeads at a time so that their rows are
+// in flight together and each branch k~_j / V_j row is read once per pass.  Shared
+// memory: the block's inverse frequencies (double), then per warp the cos/sin of
+// positions i..i+P-1 and the branch-pass accumulators.
 // ---------------------------------------------------------------------------
+constexpr int kBranchHeads = 4;
+
+// cos/sin of pos * inv_freq: the angle in double, reduced by whole turns in double,
+// then the single-precision sincosf of the remainder (|remainder| <= pi).
+__device__ __forceinline__ void angle_cos_sin(int pos, double inv_freq, float& c, float& s) {
+  const double ang = static_cast<double>(pos) * inv_freq;
+  const double turns = rint(ang * 0.15915494309189535);  // 1 / (2 pi)
+  const double red = fma(-turns, 6.283185307179586, ang);
+  sincosf(static_cast<float>(red), &s, &c);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     branch_bwd_kernel(Geometry g, const __nv_bfloat16* __restrict__ qr, const __nv_bfloat16* __restrict__ kr,
@@ -195,7 +191,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                       const float* __restrict__ lse, const float* __restrict__ ld,
                       const float* __restrict__ dq_acc, const float* __restrict__ dk1_acc,
                       __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
-  extern __shared__ float acc_smem[];
+  constexpr int E = D / 64;
+  extern __shared__ __align__(16) unsigned char branch_smem[];
+  double* inv_freq = reinterpret_cast<double*>(branch_smem);  // [D/2]
+  const int NB = g.P - 1;  // branch passes
+  const int per_warp = g.P * D + (NB > 0 ? NB : 1) * 2 * D;  // floats: cos/sin [P][2][D/2], acc [NB][2][D]
+  for (int d = threadIdx.x; d < D / 2; d += blockDim.x)
+    inv_freq[d] = pow(static_cast<double>(g.theta), -2.0 * d / D);
+  __syncthreads();
+
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + wib;
@@ -206,87 +210,141 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   int n, pos;
   token_position(g.si, tau, n, pos);
   const int gsz = g.H / g.Hkv;
-  const int NB = g.P - 1;  // branch passes
-  // [NB][2 (dk, dv)][D] per warp; lane touches only its own elements
-  float* acc = acc_smem + static_cast<int64_t>(wib) * (NB > 0 ? NB : 1) * 2 * D;
+  float* cs = reinterpret_cast<float*>(branch_smem + (D / 2) * sizeof(double)) + static_cast<int64_t>(wib) * per_warp;
+  float* acc = cs + g.P * D;  // [NB][2 (dk, dv)][D]; a lane touches only its own elements
+  for (int p = 0; p < g.P; ++p)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int d = LaneMap<D>::d(lane, 0, e);
+      angle_cos_sin(pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
+    }
   for (int j = 0; j < NB; ++j)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-      for (int e = 0; e < D / 64; ++e) {
+      for (int e = 0; e < E; ++e) {
         acc[(j * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
         acc[(j * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
       }
+  const int64_t dl_base = static_cast<int64_t>(ld_slots(g.si)) * 128;
+  const int64_t dl_off = static_cast<int64_t>(ld_slot(tau - pos, n, pos)) * 128 + 64 + (pos & 63);
 
   for (int p = 0; p < g.P; ++p) {
-    float cs_c[D / 64], cs_s[D / 64];
-    lane_cos_sin<D>(g.theta, pos + p, lane, cs_c, cs_s);
-    for (int hi = 0; hi < gsz; ++hi) {
-      const int h = kvh * gsz + hi;
-      const int64_t hrow = (static_cast<int64_t>(p) * g.H + h) * T + tau;
-      float dqv[2][D / 64];
-      load_f32_row<D>(dq_acc + hrow * D, lane, dqv);
-      if (p > 0) {
-        float q[2][D / 64], dO[2][D / 64];
-        load_bf16_row<D>(qr + hrow * D, lane, q);
-        load_bf16_row<D>(dout + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D, lane, dO);
-        const int64_t li = lse_index(g.si, g.H, p, h, n, tau, pos);
-        const float lse_v = lse[li];
-        const float dl = ld[((static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + ld_slot(tau - pos, n, pos)) * 128 +
-                            64 + (pos & 63)];
-        for (int j = 1; j <= p; ++j) {
-          float kj[2][D / 64], vj[2][D / 64];
-          load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
-          load_bf16_row<D>(v + ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D, lane, vj);
-          const float pj = __expf(dot_row<D>(q, kj) * g.scale - lse_v);
-          const float dsj = pj * (dot_row<D>(dO, vj) - dl);
-          float* ak = acc + ((j - 1) * 2 + 0) * D;
-          float* av = acc + ((j - 1) * 2 + 1) * D;
+    float c[E], sn[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      c[e] = cs[p * D + LaneMap<D>::d(lane, 0, e)];
+      sn[e] = cs[p * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
+    }
+    for (int h0 = 0; h0 < gsz; h0 += kBranchHeads) {
+      float dqv[kBranchHeads][2][E], q[kBranchHeads][2][E], dO[kBranchHeads][2][E];
+      float lse_v[kBranchHeads], dl[kBranchHeads];
+#pragma unroll
+      for (int u = 0; u < kBranchHeads; ++u) {
+        const int h = kvh * gsz + h0 + u;
+        if (h0 + u < gsz) {
+          const int64_t hrow = (static_cast<int64_t>(p) * g.H + h) * T + tau;
+          load_f32_row<D>(dq_acc + hrow * D, lane, dqv[u]);
+          if (p > 0) {
+            load_bf16_row<D>(qr + hrow * D, lane, q[u]);
+            load_bf16_row<D>(dout + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D, lane, dO[u]);
+            lse_v[u] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)];
+            dl[u] = ld[(static_cast<int64_t>(p) * g.H + h) * dl_base + dl_off];
+          }
+        }
+      }
+      for (int j = 1; j <= p; ++j) {
+        float kj[2][E], vj[2][E];
+        load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
+        load_bf16_row<D>(v + ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D, lane, vj);
+        float sdot[kBranchHeads], tdot[kBranchHeads];
+#pragma unroll
+        for (int u = 0; u < kBranchHeads; ++u) {
+          sdot[u] = 0.f;
+          tdot[u] = 0.f;
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-            for (int e = 0; e < D / 64; ++e) {
-              const int d = LaneMap<D>::d(lane, hh, e);
-              dqv[hh][e] = fmaf(dsj, kj[hh][e], dqv[hh][e]);
-              ak[d] = fmaf(dsj, q[hh][e], ak[d]);
-              av[d] = fmaf(pj, dO[hh][e], av[d]);
+            for (int e = 0; e < E; ++e) {
+              sdot[u] = fmaf(q[u][hh][e], kj[hh][e], sdot[u]);
+              tdot[u] = fmaf(dO[u][hh][e], vj[hh][e], tdot[u]);
             }
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int u = 0; u < kBranchHeads; ++u) {
+            sdot[u] += __shfl_xor_sync(0xffffffffu, sdot[u], o);
+            tdot[u] += __shfl_xor_sync(0xffffffffu, tdot[u], o);
+          }
+        float ak[2][E] = {}, av[2][E] = {};
+#pragma unroll
+        for (int u = 0; u < kBranchHeads; ++u) {
+          if (h0 + u >= gsz) continue;
+          const float pj = __expf(sdot[u] * g.scale - lse_v[u]);
+          const float dsj = pj * (tdot[u] - dl[u]);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              dqv[u][hh][e] = fmaf(dsj, kj[hh][e], dqv[u][hh][e]);
+              ak[hh][e] = fmaf(dsj, q[u][hh][e], ak[hh][e]);
+              av[hh][e] = fmaf(pj, dO[u][hh][e], av[hh][e]);
+            }
+        }
+        float* akp = acc + ((j - 1) * 2 + 0) * D;
+        float* avp = acc + ((j - 1) * 2 + 1) * D;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const int d = LaneMap<D>::d(lane, hh, e);
+            akp[d] += ak[hh][e];
+            avp[d] += av[hh][e];
+          }
       }
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
+      for (int u = 0; u < kBranchHeads; ++u) {
+        if (h0 + u >= gsz) continue;
 #pragma unroll
-        for (int e = 0; e < D / 64; ++e) dqv[hh][e] *= g.scale;
-      rotate_back<D>(dqv, cs_c, cs_s);
-      store_bf16_row<D>(dq + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D, lane, dqv);
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int e = 0; e < E; ++e) dqv[u][hh][e] *= g.scale;
+        rotate_back<D>(dqv[u], c, sn);
+        store_bf16_row<D>(dq + ((static_cast<int64_t>(p) * T + tau) * g.H + kvh * gsz + h0 + u) * D, lane, dqv[u]);
+      }
     }
   }
   // dK of every pass (trunk from the trunk backward), dV of the branch passes
   for (int j = 0; j < g.P; ++j) {
-    float cs_c[D / 64], cs_s[D / 64];
-    lane_cos_sin<D>(g.theta, pos + j, lane, cs_c, cs_s);
-    float kx[2][D / 64];
+    float c[E], sn[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      c[e] = cs[j * D + LaneMap<D>::d(lane, 0, e)];
+      sn[e] = cs[j * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
+    }
+    float kx[2][E];
     if (j == 0) {
       load_f32_row<D>(dk1_acc + (static_cast<int64_t>(kvh) * T + tau) * D, lane, kx);
     } else {
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int e = 0; e < D / 64; ++e) kx[hh][e] = acc[((j - 1) * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)];
+        for (int e = 0; e < E; ++e) kx[hh][e] = acc[((j - 1) * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)];
     }
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-      for (int e = 0; e < D / 64; ++e) kx[hh][e] *= g.scale;
-    rotate_back<D>(kx, cs_c, cs_s);
+      for (int e = 0; e < E; ++e) kx[hh][e] *= g.scale;
+    rotate_back<D>(kx, c, sn);
     const int64_t krow = ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D;
     store_bf16_row<D>(dk + krow, lane, kx);
     if (j > 0) {
-      float vx[2][D / 64];
+      float vx[2][E];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int e = 0; e < D / 64; ++e) vx[hh][e] = acc[((j - 1) * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)];
+        for (int e = 0; e < E; ++e) vx[hh][e] = acc[((j - 1) * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)];
       store_bf16_row<D>(dv + krow, lane, vx);
     }
   }
@@ -318,18 +376,19 @@ inline unsigned blocks_for(int64_t warps) {
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  cudaStream_t stream) {
-  const int64_t rows = static_cast<int64_t>(g.P) * g.si.T * g.H;
-  if (rows == 0) return cudaSuccess;
-  const int rpw = 32 / (g.D / 8);
-  const int64_t warps = (rows + rpw * kUnroll - 1) / (rpw * kUnroll);
-  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(blocks_for(warps), 148 * 32));
+                                  float* dq_acc, cudaStream_t stream) {
+  if (g.si.T == 0 || g.si.nseq == 0 || g.si.max_len == 0) return cudaSuccess;
+  const int ntile = (g.si.max_len + kPreRows - 1) / kPreRows;
+  const long long blocks = static_cast<long long>(g.P) * g.si.nseq * ntile * g.H;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   auto* ob = static_cast<const __nv_bfloat16*>(o);
   auto* db = static_cast<const __nv_bfloat16*>(dout);
   if (g.D == 128)
-    bwd_preprocess_kernel<128><<<blocks, kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
+    bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
+                                                                                       ntile);
   else
-    bwd_preprocess_kernel<64><<<blocks, kWarpsPerBlock * 32, 0, stream>>>(g, ob, db, lse, ld);
+    bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
+                                                                                      ntile);
   return cudaGetLastError();
 }
 
@@ -339,7 +398,8 @@ cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr,
   const int64_t warps = static_cast<int64_t>(g.si.T) * g.Hkv;
   if (warps == 0) return cudaSuccess;
   const int NB = g.P - 1 > 0 ? g.P - 1 : 1;
-  const size_t smem = static_cast<size_t>(kWarpsPerBlock) * NB * 2 * g.D * sizeof(float);
+  const size_t smem = static_cast<size_t>(g.D / 2) * sizeof(double) +
+                      static_cast<size_t>(kWarpsPerBlock) * (g.P * g.D + NB * 2 * g.D) * sizeof(float);
   auto* qb = static_cast<const __nv_bfloat16*>(qr);
   auto* kb = static_cast<const __nv_bfloat16*>(kr);
   auto* vb = static_cast<const __nv_bfloat16*>(v);

@@ -328,10 +328,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sdp_free);
+#ifdef TTT_KERNEL_TRACE
       if (lane == 0) {
         constexpr int kSlot[8] = {6, 22, 23, 17, 19, 18, 14, 15};
         TTT_TRACE(kSlot[warp - 4], it);
       }
+#endif
       const float* ldp = sLD + s * 2 * C::BQ + 32 * hf;
       // interior tile: every (key, query) pair of this half is visible
       const int qlo = ii.q0 + 32 * hf;

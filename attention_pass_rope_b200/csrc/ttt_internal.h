@@ -79,9 +79,10 @@ cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, co
 // start_{n+1}/64 + n + 1.  Padding entries are never written.
 __host__ __device__ inline int ld_slots(const SeqInfo& si) { return si.T / 64 + si.nseq + 1; }
 
-// a5: delta = rowsum(dO * O); writes the tile-aligned (lse*log2e, delta) rows.
+// a5: delta = rowsum(dO * O); writes the tile-aligned (-lse*log2e, delta) rows and
+// zeroes the fp32 dq~ accumulator [P][H][T][D].
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  cudaStream_t stream);
+                                  float* dq_acc, cudaStream_t stream);
 
 struct TrunkBwdArgs {
   Geometry g;
