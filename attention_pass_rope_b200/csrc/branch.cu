@@ -168,12 +168,13 @@ __global__ void __launch_bounds__(kPreThreads)
 //     dQ_p = R(i+p)^T (sigma dq~)
 //   dK_j = R(i+j)^T (sigma dk~_j)  for every pass (j = 0 takes dk~_1 from the trunk
 //   backward), dV_j for j >= 1 (dV_1 is written by the trunk backward).
-// The group heads of a pass are taken kBranchHeads at a time so that their rows are
-// in flight together and each branch k~_j / V_j row is read once per pass.  Shared
-// memory: the block's inverse frequencies (double), then per warp the cos/sin of
-// positions i..i+P-1 and the branch-pass accumulators.
+// The kernel is bound by memory latency, so resident warps matter most: the group
+// heads of a pass go kBranchHeads at a time (one: more heads per warp keep more rows
+// in flight but cost registers, and 64 registers at four blocks per SM measured
+// fastest).  Shared memory: the block's inverse frequencies (double), then per warp
+// the cos/sin of positions i..i+P-1 and the branch-pass accumulators.
 // ---------------------------------------------------------------------------
-constexpr int kBranchHeads = 4;
+constexpr int kBranchHeads = 1;
 
 // cos/sin of pos * inv_freq: the angle in double, reduced by whole turns in double,
 // then the single-precision sincosf of the remainder (|remainder| <= pi).
@@ -185,7 +186,7 @@ __device__ __forceinline__ void angle_cos_sin(int pos, double inv_freq, float& c
 }
 
 template <int D>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
     branch_bwd_kernel(Geometry g, const __nv_bfloat16* __restrict__ qr, const __nv_bfloat16* __restrict__ kr,
                       const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ ld,
