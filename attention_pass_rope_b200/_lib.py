@@ -17,6 +17,8 @@ TTT_ERR_DEVICE_TIMEOUT = 5
 TTT_LAYOUT_BSHD = 0
 TTT_LAYOUT_THD = 1
 
+TTT_FLAG_ROTATED_IN_WORKSPACE = 1
+
 KERNELS = ("rope_fwd", "trunk_fwd", "unused_2", "rope_bwd", "bwd_preprocess", "trunk_bwd", "branch_bwd")
 KERNEL_COUNT = 8
 
@@ -41,13 +43,21 @@ class TTTDesc(ctypes.Structure):
         ("total_tokens", ctypes.c_int),
         ("max_seqlen", ctypes.c_int),
         ("events", ctypes.c_void_p),
+        ("flags", ctypes.c_int),
     ]
 
 
 class TTTError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        msg = f"{what}: {status_string(status)} (status {status})"
+        if status == TTT_ERR_CUDA:
+            try:
+                code = lib().ttt_attn_last_cuda_error()
+                msg += f"; CUDA: {lib().ttt_attn_cuda_error_name(code).decode()} ({code})"
+            except Exception:  # pragma: no cover - only used for messages
+                pass
+        super().__init__(msg)
 
 
 _lib = None
@@ -84,6 +94,10 @@ def lib() -> ctypes.CDLL:
     L.ttt_status_string.restype = ctypes.c_char_p
     L.ttt_attn_version.argtypes = []
     L.ttt_attn_version.restype = ctypes.c_char_p
+    L.ttt_attn_last_cuda_error.argtypes = []
+    L.ttt_attn_last_cuda_error.restype = ctypes.c_int
+    L.ttt_attn_cuda_error_name.argtypes = [ctypes.c_int]
+    L.ttt_attn_cuda_error_name.restype = ctypes.c_char_p
     _lib = L
     return L
 

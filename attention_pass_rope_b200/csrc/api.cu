@@ -37,6 +37,7 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
   if (d->D != 64 && d->D != 128) return TTT_ERR_UNSUPPORTED;  // rotary needs an even D; kernels take 64/128
   if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return TTT_ERR_INVALID_ARG;
   if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return TTT_ERR_INVALID_ARG;
+  if (d->flags & ~static_cast<int>(TTT_FLAG_ROTATED_IN_WORKSPACE)) return TTT_ERR_INVALID_ARG;
   g.P = d->P;
   g.H = d->H;
   g.Hkv = d->Hkv;
@@ -93,6 +94,11 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
   return TTT_OK;
 }
 
+// The error behind the most recent TTT_ERR_CUDA (cudaError_t, or kEncodeErrorBase +
+// CUresult when a TMA descriptor could not be encoded).
+std::atomic<int> g_last_cuda_error{0};
+constexpr int kEncodeErrorBase = 100000;
+
 // ---- TMA descriptors (driver entry point fetched through the runtime)
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -114,14 +120,19 @@ EncodeTiledFn encode_fn() {
 bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
               uint64_t s2_bytes, uint32_t b1, uint32_t b2) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
+  if (!fn) {
+    g_last_cuda_error.store(static_cast<int>(cudaErrorSymbolNotFound));
+    return false;
+  }
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {s1_bytes, s2_bytes};
   const cuuint32_t box[3] = {64, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_cuda_error.store(kEncodeErrorBase + static_cast<int>(r));
+  return r == CUDA_SUCCESS;
 }
 
 struct EventScope {
@@ -136,10 +147,21 @@ struct EventScope {
   }
 };
 
-#define TTT_CHECK_CUDA(expr)                 \
-  do {                                       \
-    if ((expr) != cudaSuccess) return TTT_ERR_CUDA; \
+#define TTT_CHECK_CUDA(expr)                                    \
+  do {                                                          \
+    const cudaError_t e_ = (expr);                              \
+    if (e_ != cudaSuccess) {                                    \
+      g_last_cuda_error.store(static_cast<int>(e_));           \
+      return TTT_ERR_CUDA;                                      \
+    }                                                           \
   } while (0)
+
+// The launchers read a launch's error with cudaGetLastError(), which also returns a
+// non-sticky status left on this host thread by the caller's own runtime calls
+// (cudaErrorNotReady from an event or stream query, for example: autograd worker
+// threads make such queries).  Each entry point clears it before its first CUDA
+// call; a sticky error cannot be cleared and still fails the call.
+inline void clear_stale_error() { (void)cudaGetLastError(); }
 
 }  // namespace
 }  // namespace ttt
@@ -180,13 +202,16 @@ ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k,
   void* kr = ws + pl.off[2];
   const uint64_t T = g.si.T, D = g.D;
 
+  // The first runtime call also makes the current device's primary context current
+  // on this thread, which the driver's tensor-map encoder needs (a thread that has
+  // made no runtime call yet, such as an autograd worker, has none).
+  clear_stale_error();
+  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, qr, D, T, static_cast<uint64_t>(g.P) * g.H, D * 2, T * D * 2, 128, 1) ||
       !make_map(&mk, kr, D, T, g.Hkv, D * 2, T * D * 2, 128, 1) ||
       !make_map(&mv, v, D, g.Hkv, T, D * 2, g.Hkv * D * 2, 1, 128))
     return TTT_ERR_CUDA;
-
-  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   {
     EventScope es(desc->events, TTT_KERNEL_ROPE_FWD, stream);
     TTT_CHECK_CUDA(launch_rope_fwd(g, q, k, qr, kr, stream));
@@ -223,17 +248,20 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   float* dk1_acc = reinterpret_cast<float*>(ws + pl.off[5]);
   const uint64_t T = g.si.T, D = g.D;
 
+  // first runtime call before the tensor-map encoder (see ttt_attn_fwd)
+  clear_stale_error();
+  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, qr, D, T, static_cast<uint64_t>(g.P) * g.H, D * 2, T * D * 2, 64, 1) ||
       !make_map(&mk, kr, D, T, g.Hkv, D * 2, T * D * 2, 128, 1) ||
       !make_map(&mv, v, D, g.Hkv, T, D * 2, g.Hkv * D * 2, 1, 128) ||
       !make_map(&mdo, dout, D, g.H, static_cast<uint64_t>(g.P) * T, D * 2, g.H * D * 2, 1, 64))
     return TTT_ERR_CUDA;
-
-  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   {
+    // the events are recorded either way, so a timing caller sees ~0 when the
+    // forward's rotated q~ / k~ are reused
     EventScope es(desc->events, TTT_KERNEL_ROPE_BWD, stream);
-    TTT_CHECK_CUDA(launch_rope_fwd(g, q, k, qr, kr, stream));
+    if (!(desc->flags & TTT_FLAG_ROTATED_IN_WORKSPACE)) TTT_CHECK_CUDA(launch_rope_fwd(g, q, k, qr, kr, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
@@ -270,6 +298,7 @@ ttt_status ttt_attn_watchdog_selftest(void* workspace, size_t workspace_bytes, u
   if (!workspace || workspace_bytes < 256 || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   uint32_t* status = static_cast<uint32_t*>(workspace);
+  clear_stale_error();
   TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   TTT_CHECK_CUDA(launch_watchdog_selftest(status, budget_ns, stream));
   return TTT_OK;
@@ -291,6 +320,13 @@ const char* ttt_status_string(ttt_status s) {
   return "unknown status";
 }
 
-const char* ttt_attn_version(void) { return "0.1.0"; }
+const char* ttt_attn_version(void) { return "0.2.0"; }
+
+int ttt_attn_last_cuda_error(void) { return g_last_cuda_error.load(); }
+
+const char* ttt_attn_cuda_error_name(int code) {
+  if (code >= kEncodeErrorBase) return "tensor map encoding failed (CUresult = code - 100000)";
+  return cudaGetErrorName(static_cast<cudaError_t>(code));
+}
 
 }  // extern "C"

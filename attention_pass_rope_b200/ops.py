@@ -68,7 +68,7 @@ def _layout(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens, max_s
                   cu_seqlens=cu_seqlens.contiguous())
 
 
-def make_desc(lay: Layout, theta: float, scale: Optional[float], events=None) -> _lib.TTTDesc:
+def make_desc(lay: Layout, theta: float, scale: Optional[float], events=None, flags: int = 0) -> _lib.TTTDesc:
     d = _lib.TTTDesc()
     d.layout = _lib.TTT_LAYOUT_BSHD if lay.dense else _lib.TTT_LAYOUT_THD
     d.P, d.H, d.Hkv, d.D = lay.P, lay.H, lay.Hkv, lay.D
@@ -79,6 +79,7 @@ def make_desc(lay: Layout, theta: float, scale: Optional[float], events=None) ->
         d.cu_seqlens = lay.cu_seqlens.data_ptr()
         d.nseq, d.total_tokens, d.max_seqlen = lay.nseq, lay.T, lay.max_seqlen
     d.events = ctypes.addressof(events) if events is not None else None
+    d.flags = int(flags)
     return d
 
 
@@ -138,8 +139,13 @@ def ttt_attn_fwd(q, k, v, *, theta: float, scale: Optional[float] = None, cu_seq
 
 
 def ttt_attn_bwd(q, k, v, o, lse, dout, *, theta: float, scale: Optional[float] = None, cu_seqlens=None,
-                 max_seqlen=None, workspace: Optional[torch.Tensor] = None, out=None, events=None):
-    """Backward: returns (dq, dk, dv) with respect to the pre-RoPE q, k, v."""
+                 max_seqlen=None, workspace: Optional[torch.Tensor] = None, out=None, events=None,
+                 rotated_in_workspace: bool = False):
+    """Backward: returns (dq, dk, dv) with respect to the pre-RoPE q, k, v.
+    ``rotated_in_workspace``: ``workspace`` still holds what ``ttt_attn_fwd`` wrote
+    into it for these q, k (TTT_FLAG_ROTATED_IN_WORKSPACE); the rotation is reused."""
+    if rotated_in_workspace and workspace is None:
+        raise ValueError("rotated_in_workspace needs the forward's workspace")
     lay = _layout(q, k, v, cu_seqlens, max_seqlen)
     _contig(q, k, v, o, lse, dout)
     if dout.dtype != torch.bfloat16 or o.dtype != torch.bfloat16 or lse.dtype != torch.float32:
@@ -148,7 +154,8 @@ def ttt_attn_bwd(q, k, v, o, lse, dout, *, theta: float, scale: Optional[float] 
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     else:
         dq, dk, dv = out
-    desc = make_desc(lay, theta, scale, events)
+    desc = make_desc(lay, theta, scale, events,
+                     _lib.TTT_FLAG_ROTATED_IN_WORKSPACE if rotated_in_workspace else 0)
     L = _lib.lib()
     need = L.ttt_attn_workspace_size(ctypes.byref(desc), 1)
     if workspace is None:
@@ -179,21 +186,33 @@ def set_wait_budget_ns(budget_ns: int) -> None:
 
 class _TTTAttention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, theta, scale, cu_seqlens, max_seqlen):
-        o, lse = ttt_attn_fwd(q, k, v, theta=theta, scale=scale, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)
+    def forward(ctx, q, k, v, theta, scale, cu_seqlens, max_seqlen, keep_rotated):
+        ws = None
+        if keep_rotated:
+            lay = _layout(q, k, v, cu_seqlens, max_seqlen)
+            ws = alloc_workspace(workspace_bytes(lay, theta, scale, for_backward=True), q.device)
+        o, lse = ttt_attn_fwd(q, k, v, theta=theta, scale=scale, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen,
+                              workspace=ws)
         ctx.save_for_backward(q, k, v, o, lse, cu_seqlens)
         ctx.theta, ctx.scale, ctx.max_seqlen = theta, scale, max_seqlen
         ctx.has_cu = cu_seqlens is not None
+        ctx.ws = ws
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse, cu = ctx.saved_tensors
         dq, dk, dv = ttt_attn_bwd(q, k, v, o, lse, do.contiguous(), theta=ctx.theta, scale=ctx.scale,
-                                  cu_seqlens=cu if ctx.has_cu else None, max_seqlen=ctx.max_seqlen)
-        return dq, dk, dv, None, None, None, None
+                                  cu_seqlens=cu if ctx.has_cu else None, max_seqlen=ctx.max_seqlen,
+                                  workspace=ctx.ws, rotated_in_workspace=ctx.ws is not None)
+        ctx.ws = None
+        return dq, dk, dv, None, None, None, None, None
 
 
-def ttt_attention(q, k, v, *, theta: float, scale: Optional[float] = None, cu_seqlens=None, max_seqlen=None):
-    """Differentiable TTT trunk+branch attention (autograd over the C ABI)."""
-    return _TTTAttention.apply(q, k, v, theta, scale, cu_seqlens, max_seqlen)
+def ttt_attention(q, k, v, *, theta: float, scale: Optional[float] = None, cu_seqlens=None, max_seqlen=None,
+                  keep_rotated: bool = False):
+    """Differentiable TTT trunk+branch attention (autograd over the C ABI).
+    ``keep_rotated`` holds the forward's workspace (rotated q~ / k~, sized for the
+    backward) until the backward, which then skips rotating q and k again: more
+    memory between the two calls, one kernel less in the backward."""
+    return _TTTAttention.apply(q, k, v, theta, scale, cu_seqlens, max_seqlen, keep_rotated)

@@ -173,8 +173,10 @@ def run_ours(args, rank, world, local):
         ev_objs.append(objs)
 
     def step(events=None):
+        # one workspace for both calls: the backward reuses the forward's rotated q~ / k~
         ops.ttt_attn_fwd(q, k, v, workspace=ws, out=(o, lse), events=events, **kw)
-        ops.ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, out=(dq, dk, dv), events=events, **kw)
+        ops.ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, out=(dq, dk, dv), events=events,
+                         rotated_in_workspace=True, **kw)
 
     for _ in range(args.warmup):
         step()
@@ -279,7 +281,7 @@ def run_ours(args, rank, world, local):
                      "traffic": traffic},
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 6 * K,
+        "gpu_launches": 5 * K,  # rope, trunk fwd; preprocess, trunk bwd, branch bwd
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline:

@@ -94,7 +94,19 @@ typedef struct {
   int total_tokens;    /* THD only: T = cu_seqlens[nseq] */
   int max_seqlen;      /* THD only: upper bound on every sequence length */
   const ttt_attn_events* events; /* optional, NULL for none */
+  int flags;           /* TTT_FLAG_* bits, 0 for none; other bits are rejected */
 } ttt_attn_desc;
+
+/* Descriptor flags. */
+typedef enum {
+  /* ttt_attn_bwd: the workspace still holds the rotated q~ / k~ that ttt_attn_fwd
+   * wrote for this descriptor and these q, k (same workspace, untouched since), so
+   * the backward uses them instead of rotating q and k again.  The backward's
+   * workspace layout starts with the forward's (ttt_attn_workspace_layout), so a
+   * workspace sized for the backward and passed to both calls qualifies.  If the
+   * promise is broken the gradients are wrong; nothing is read out of bounds. */
+  TTT_FLAG_ROTATED_IN_WORKSPACE = 1
+} ttt_flag;
 
 /* Bytes of workspace that ttt_attn_fwd (for_backward = 0) or ttt_attn_bwd
  * (for_backward = 1) needs for `desc`; 0 if the descriptor is invalid.  The
@@ -135,6 +147,14 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
  * streams) race on it, so order them on one stream. */
 ttt_status ttt_attn_fwd_noalloc(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, void* o,
                                 float* lse, void* stream);
+
+/* The error behind the most recent TTT_ERR_CUDA returned by any call in this
+ * process: a cudaError_t value, or 100000 + the CUresult when encoding a TMA tensor
+ * map failed; 0 if there was none.  Not reset by later successful calls. */
+int ttt_attn_last_cuda_error(void);
+
+/* Name of a code returned by ttt_attn_last_cuda_error (static string). */
+const char* ttt_attn_cuda_error_name(int code);
 
 /* Synchronises `stream` and returns TTT_OK if no bounded wait of the calls made
  * with this workspace ran out since the last check, TTT_ERR_DEVICE_TIMEOUT (and

@@ -47,14 +47,20 @@ def flat(t: torch.Tensor, w) -> torch.Tensor:
     return t
 
 
-def run_gpu(w, inp, with_grad=True):
-    from attention_pass_rope_b200 import ttt_attn_bwd, ttt_attn_fwd
+def run_gpu(w, inp, with_grad=True, reuse_rotation=False):
+    """Forward (+ backward) through the C ABI.  ``reuse_rotation``: one workspace for
+    both calls and the backward told to reuse the forward's rotated q~ / k~."""
+    from attention_pass_rope_b200 import ops, ttt_attn_bwd, ttt_attn_fwd
     q, k, v, do, cu = gpu_shapes(w, inp)
     kw = dict(theta=w.theta, cu_seqlens=cu, max_seqlen=None if w.dense else w.max_seqlen)
-    o, lse = ttt_attn_fwd(q, k, v, **kw)
+    ws = None
+    if reuse_rotation:
+        lay = ops._layout(q, k, v, cu, kw["max_seqlen"])
+        ws = ops.alloc_workspace(ops.workspace_bytes(lay, w.theta, for_backward=True), q.device)
+    o, lse = ttt_attn_fwd(q, k, v, workspace=ws, **kw)
     out = {"o": flat(o, w), "lse": lse}
     if with_grad:
-        dq, dk, dv = ttt_attn_bwd(q, k, v, o, lse, do, **kw)
+        dq, dk, dv = ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, rotated_in_workspace=reuse_rotation, **kw)
         out.update(dq=flat(dq, w), dk=flat(dk, w), dv=flat(dv, w))
     torch.cuda.synchronize()
     return out

@@ -66,6 +66,8 @@ def test_workspace_size_dense(L):
     ("softmax_scale", -0.5, _lib.TTT_ERR_INVALID_ARG),
     ("layout", 7, _lib.TTT_ERR_INVALID_ARG),
     ("B", -1, _lib.TTT_ERR_INVALID_ARG),
+    ("flags", 2, _lib.TTT_ERR_INVALID_ARG),     # unknown flag bit
+    ("flags", -1, _lib.TTT_ERR_INVALID_ARG),
 ])
 def test_invalid_descriptor(L, field, value, status):
     d = desc(**{field: value})
@@ -73,6 +75,11 @@ def test_invalid_descriptor(L, field, value, status):
     fake = ctypes.c_void_p(1 << 20)
     st = L.ttt_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, fake, 1 << 40, None)
     assert st == status
+
+
+def test_known_flag_accepted(L):
+    d = desc(flags=_lib.TTT_FLAG_ROTATED_IN_WORKSPACE)
+    assert L.ttt_attn_workspace_size(ctypes.byref(d), 1) == L.ttt_attn_workspace_size(ctypes.byref(desc()), 1) > 0
 
 
 def test_null_descriptor(L):

@@ -178,3 +178,43 @@ def test_long_32k_outputs_finite():
     gpu = parity.run_gpu(w, inp, with_grad=False)
     assert torch.isfinite(gpu["o"].float()).all()
     assert torch.isfinite(gpu["lse"]).all()
+
+
+# ----------------------------------------------------------------------------- reuse of the rotation
+
+@needs_cuda
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_backward_reusing_forward_rotation(name):
+    """TTT_FLAG_ROTATED_IN_WORKSPACE: one workspace for forward and backward, the backward
+    skips the rotation.  Against the oracle, and dk/dv bit-identical to the path that
+    rotates again (the rotation is deterministic; dq~ sums in an unfixed order)."""
+    w = ttt_inputs.workloads()["tiny"] if name == "tiny" else \
+        ttt_inputs.thd("ragged", [300, 128, 17, 1], 4, 8, 2, 128, 1e4)
+    inp = ttt_inputs.make_inputs(w)
+    gpu = parity.run_gpu(w, inp, reuse_rotation=True)
+    m = parity.compare_full(w, inp, gpu)
+    print(name, m)
+    parity.assert_within(m)
+    ref = parity.run_gpu(w, inp)
+    assert torch.equal(gpu["dk"], ref["dk"]) and torch.equal(gpu["dv"], ref["dv"])
+    assert torch.equal(gpu["o"], ref["o"]) and torch.equal(gpu["lse"], ref["lse"])
+
+
+@needs_cuda
+@pytest.mark.parametrize("keep_rotated", [False, True])
+def test_autograd_function(keep_rotated):
+    """ttt_attention under torch.autograd (both settings of keep_rotated) against the oracle."""
+    from attention_pass_rope_b200 import ops
+    w = ttt_inputs.workloads()["tiny"]
+    inp = ttt_inputs.make_inputs(w)
+    q, k, v, do, _ = parity.gpu_shapes(w, inp)
+    q, k, v = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = ops.ttt_attention(q, k, v, theta=w.theta, keep_rotated=keep_rotated)
+    o.backward(do)
+    torch.cuda.synchronize()
+    gpu = {"o": parity.flat(o.detach(), w), "lse": ops.ttt_attn_fwd(q.detach(), k.detach(), v.detach(),
+                                                                       theta=w.theta)[1],
+           "dq": parity.flat(q.grad, w), "dk": parity.flat(k.grad, w), "dv": parity.flat(v.grad, w)}
+    m = parity.compare_full(w, inp, gpu)
+    print("autograd", keep_rotated, m)
+    parity.assert_within(m)
