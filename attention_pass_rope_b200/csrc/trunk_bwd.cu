@@ -99,11 +99,22 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (key tile jk, sequence n, KV head), smallest jk (most work) first
-  const int per_jk = g.si.nseq * g.Hkv;
-  const int jk = static_cast<int>(blockIdx.x) / per_jk;
-  const int n = (static_cast<int>(blockIdx.x) % per_jk) / g.Hkv;
-  const int kvh = static_cast<int>(blockIdx.x) % g.Hkv;
+  // ---- work item: (key tile jk, sequence n, KV head).  The (sequence, KV head) groups
+  // go in bands of nb groups, about 256 CTAs per band; inside a band the smallest jk
+  // (most work) comes first.  The CTAs resident at one time then belong to few groups,
+  // so the q~/dO tiles they read and the dq~ rows they reduce into are shared in L2
+  // (with every group in flight at once, a batch of many short sequences streams all
+  // of it from DRAM), while the work per band still runs largest first.
+  const int njk = (g.si.max_len + C::BK - 1) / C::BK;
+  const int ngroups = g.si.nseq * g.Hkv;
+  const int nb = max(1, 256 / njk);
+  const int band = static_cast<int>(blockIdx.x) / (nb * njk);
+  const int in_band = static_cast<int>(blockIdx.x) % (nb * njk);
+  const int members = min(nb, ngroups - band * nb);
+  const int jk = in_band / members;
+  const int gi = band * nb + in_band % members;
+  const int n = gi / g.Hkv;
+  const int kvh = gi % g.Hkv;
   int seq_start, len;
   seq_bounds(g.si, n, seq_start, len);
   const int k0 = jk * C::BK;

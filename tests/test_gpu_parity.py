@@ -218,3 +218,18 @@ def test_autograd_function(keep_rotated):
     m = parity.compare_full(w, inp, gpu)
     print("autograd", keep_rotated, m)
     parity.assert_within(m)
+
+
+# ----------------------------------------------------------------------------- maximum pass count
+
+@needs_cuda
+@pytest.mark.parametrize("layout,D", [("dense", 128), ("dense", 64), ("thd", 128)])
+def test_sixteen_passes(layout, D):
+    """P = 16, the largest pass count the library takes: 15 branch keys per query in the
+    forward epilogue and 15 branch passes in the branch backward (its largest shared-memory
+    layout), every output element against the oracle."""
+    if layout == "dense":
+        w = ttt_inputs.dense("p16", 1, 130, 16, 4, 2, D, 1e4)
+    else:
+        w = ttt_inputs.thd("p16_thd", [70, 1, 129], 16, 4, 1, D, 1e4)
+    _check(w)
