@@ -18,6 +18,7 @@ TTT_LAYOUT_BSHD = 0
 TTT_LAYOUT_THD = 1
 
 TTT_FLAG_ROTATED_IN_WORKSPACE = 1
+TTT_FLAG_DETERMINISTIC_DQ = 2
 
 KERNELS = ("rope_fwd", "trunk_fwd", "unused_2", "rope_bwd", "bwd_preprocess", "trunk_bwd", "branch_bwd")
 KERNEL_COUNT = 8

@@ -37,7 +37,8 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
   if (d->D != 64 && d->D != 128) return TTT_ERR_UNSUPPORTED;  // rotary needs an even D; kernels take 64/128
   if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return TTT_ERR_INVALID_ARG;
   if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return TTT_ERR_INVALID_ARG;
-  if (d->flags & ~static_cast<int>(TTT_FLAG_ROTATED_IN_WORKSPACE)) return TTT_ERR_INVALID_ARG;
+  if (d->flags & ~static_cast<int>(TTT_FLAG_ROTATED_IN_WORKSPACE | TTT_FLAG_DETERMINISTIC_DQ))
+    return TTT_ERR_INVALID_ARG;
   g.P = d->P;
   g.H = d->H;
   g.Hkv = d->Hkv;
@@ -87,7 +88,9 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
     o = align_up(o + P * H * T * D * 4);
     pl.off[5] = o;  // dk~_1 accumulator
     o = align_up(o + Hkv * T * D * 4);
-    pl.noff = 6;
+    pl.off[6] = o;  // order tickets of the dq~ additions, one per statistics slot
+    o = align_up(o + P * H * static_cast<size_t>(ld_slots(g.si)) * 4);
+    pl.noff = 7;
   }
   pl.total = o;
   *out = pl;
@@ -246,6 +249,8 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   float* ld = reinterpret_cast<float*>(ws + pl.off[3]);
   float* dq_acc = reinterpret_cast<float*>(ws + pl.off[4]);
   float* dk1_acc = reinterpret_cast<float*>(ws + pl.off[5]);
+  int* tickets = reinterpret_cast<int*>(ws + pl.off[6]);
+  const bool deterministic = (desc->flags & TTT_FLAG_DETERMINISTIC_DQ) != 0;
   const uint64_t T = g.si.T, D = g.D;
 
   // first runtime call before the tensor-map encoder (see ttt_attn_fwd)
@@ -265,11 +270,11 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
-    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, stream));
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);
-    TrunkBwdArgs a{g, ld, dq_acc, dk1_acc, dv, status, g_wait_budget_ns.load()};
+    TrunkBwdArgs a{g, ld, dq_acc, dk1_acc, dv, deterministic ? tickets : nullptr, status, g_wait_budget_ns.load()};
     TTT_CHECK_CUDA(launch_trunk_bwd(a, mq, mk, mv, mdo, stream));
   }
   {

@@ -99,7 +99,7 @@ template <int D>
 __global__ void __launch_bounds__(kPreThreads)
     bwd_preprocess_kernel(Geometry g, const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                           const float* __restrict__ lse, float* __restrict__ ld, float* __restrict__ dq_acc,
-                          int ntile) {
+                          int* __restrict__ tickets, int ntile) {
   constexpr int LPR = D / 8;                            // lanes per row
   constexpr int RPI = 32 / LPR;                         // rows per warp instruction
   constexpr int RPWARP = kPreRows / (kPreThreads / 32);  // rows per warp (8)
@@ -151,7 +151,9 @@ __global__ void __launch_bounds__(kPreThreads)
     if (c == 0) sdelta[warp * RPWARP + u * RPI + sub] = acc;
   }
   __syncthreads();
-  float* slot = ld + ((static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + ld_slot(start, n, pos0)) * 128;
+  const int64_t slot_index = (static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + ld_slot(start, n, pos0);
+  float* slot = ld + slot_index * 128;
+  if (threadIdx.x == 0) tickets[slot_index] = 0;
   if (threadIdx.x < nvalid) {
     const int i = threadIdx.x;
     slot[i] = lse[lse_index(g.si, g.H, p, h, n, start + pos0 + i, pos0 + i)] * -1.4426950408889634f;
@@ -377,7 +379,7 @@ inline unsigned blocks_for(int64_t warps) {
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  float* dq_acc, cudaStream_t stream) {
+                                  float* dq_acc, int* tickets, cudaStream_t stream) {
   if (g.si.T == 0 || g.si.nseq == 0 || g.si.max_len == 0) return cudaSuccess;
   const int ntile = (g.si.max_len + kPreRows - 1) / kPreRows;
   const long long blocks = static_cast<long long>(g.P) * g.si.nseq * ntile * g.H;
@@ -386,10 +388,10 @@ cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* 
   auto* db = static_cast<const __nv_bfloat16*>(dout);
   if (g.D == 128)
     bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
-                                                                                       ntile);
+                                                                                       tickets, ntile);
   else
     bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
-                                                                                      ntile);
+                                                                                      tickets, ntile);
   return cudaGetLastError();
 }
 

@@ -146,6 +146,24 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
+// Bounded wait until a global counter that other CTAs advance equals `expect`
+// (acquire: their writes before the increment are visible afterwards).
+static __device__ __noinline__ bool wait_counter(const int* counter, int expect, const Watchdog& wd, uint32_t site) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v == expect) return true;
+    if (*reinterpret_cast<volatile uint32_t*>(wd.abort_smem)) return false;
+    if (globaltimer_ns() - t0 > wd.budget_ns) {
+      atomicExch(wd.abort_smem, 1u);
+      if (wd.status_gmem) atomicCAS(wd.status_gmem, 0u, kStatusTimeoutBase | site);
+      return false;
+    }
+    __nanosleep(128);
+  }
+}
+
 // Bounded wait that ignores the abort flag: used on the exit path to let operations
 // already issued to the tensor cores finish before TMEM is released.
 static __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, const Watchdog& wd, uint32_t site) {

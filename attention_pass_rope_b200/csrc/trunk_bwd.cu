@@ -445,9 +445,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const int d = wq * 32 + lane;  // TMEM lane = head dimension
     const int tid = threadIdx.x - 384;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const int nslots = ld_slots(g.si);
+    volatile uint32_t* go = abort_flag + 1;  // lead thread's dq_full outcome, shared through the barrier
     for (int it = 0; it < NIT; ++it) {
       const IterInfo ii = decode_iter(it, nqt, jq0, G, gsz, kvh);
-      if (!wait_bounded(dq_full, it & 1, wd, kSiteBwdDqFull)) break;
+      // one thread waits and the four warps agree on the outcome, so that all of them
+      // take the same named barriers on every path
+      if (tid == 0) *go = wait_bounded(dq_full, it & 1, wd, kSiteBwdDqFull) ? 1u : 0u;
+      named_bar_sync(1, 128);
+      if (!*go) break;
       if (tid == 0) TTT_TRACE(10, it);
       tc_fence_after();
       uint32_t v0[32], v1[32];
@@ -460,6 +466,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
       if (tid == 0) TTT_TRACE(20, it);
+      // ordered mode: the key tiles of this query tile add their dq~ in key-tile order
+      int* ticket = nullptr;
+      bool ordered_ok = true;
+      if (a.tickets && tid == 0) {
+        ticket = a.tickets + (static_cast<int64_t>(ii.p) * g.H + ii.h) * nslots + ld_slot(seq_start, n, ii.q0);
+        ordered_ok = wait_counter(ticket, jk, wd, kSiteBwdTicket);
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
       // two halves of 32 query rows, each through its own staging buffer; one bulk
       // group is committed per half (empty past the end of the sequence), so the group
       // that last read a buffer is always the second most recent one
@@ -477,12 +491,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (tid == 0) {
           const int r0 = ii.q0 + 32 * hq;
           const int nrows = min(32, len - r0);
-          if (nrows > 0) {
+          if (nrows > 0 && ordered_ok) {
             float* dst = a.dq_acc + ((static_cast<int64_t>(ii.p) * g.H + ii.h) * g.si.T + seq_start + r0) * D;
             bulk_reduce_add_f32(dst, stage, static_cast<uint32_t>(nrows * D * 4));
           }
           bulk_commit();
         }
+      }
+      if (ticket && ordered_ok) {
+        // this tile's additions are complete before the next key tile may start its own
+        bulk_wait0();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        atomicAdd(ticket, 1);
       }
       if (tid == 0) TTT_TRACE(21, it);
     }

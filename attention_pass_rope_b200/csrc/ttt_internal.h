@@ -31,6 +31,7 @@ enum WaitSite : uint32_t {
   kSiteBwdFinal = 0x28,
   kSiteBwdDrain = 0x29,
   kSiteBwdSdpFree = 0x2a,
+  kSiteBwdTicket = 0x2b,
 };
 
 // Where the sequences are: dense batches (cu_seqlens == nullptr) hold nseq = B
@@ -80,9 +81,9 @@ cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, co
 __host__ __device__ inline int ld_slots(const SeqInfo& si) { return si.T / 64 + si.nseq + 1; }
 
 // a5: delta = rowsum(dO * O); writes the tile-aligned (-lse*log2e, delta) rows and
-// zeroes the fp32 dq~ accumulator [P][H][T][D].
+// zeroes the fp32 dq~ accumulator [P][H][T][D] and the per-slot order tickets.
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  float* dq_acc, cudaStream_t stream);
+                                  float* dq_acc, int* tickets, cudaStream_t stream);
 
 struct TrunkBwdArgs {
   Geometry g;
@@ -90,6 +91,7 @@ struct TrunkBwdArgs {
   float* dq_acc;       // fp32 [P][H][T][D], zeroed before the launch
   float* dk1_acc;      // fp32 [Hkv][T][D]  (unscaled sum of dS^T q~)
   void* dv;            // bf16 public dv; pass 0 written here
+  int* tickets;        // nullptr, or per statistics slot: key tiles whose dq~ is added (ordered mode)
   uint32_t* status;
   uint64_t budget_ns;
 };

@@ -140,10 +140,11 @@ def ttt_attn_fwd(q, k, v, *, theta: float, scale: Optional[float] = None, cu_seq
 
 def ttt_attn_bwd(q, k, v, o, lse, dout, *, theta: float, scale: Optional[float] = None, cu_seqlens=None,
                  max_seqlen=None, workspace: Optional[torch.Tensor] = None, out=None, events=None,
-                 rotated_in_workspace: bool = False):
+                 rotated_in_workspace: bool = False, deterministic: bool = False):
     """Backward: returns (dq, dk, dv) with respect to the pre-RoPE q, k, v.
     ``rotated_in_workspace``: ``workspace`` still holds what ``ttt_attn_fwd`` wrote
-    into it for these q, k (TTT_FLAG_ROTATED_IN_WORKSPACE); the rotation is reused."""
+    into it for these q, k (TTT_FLAG_ROTATED_IN_WORKSPACE); the rotation is reused.
+    ``deterministic``: bitwise reproducible dq (TTT_FLAG_DETERMINISTIC_DQ), slower."""
     if rotated_in_workspace and workspace is None:
         raise ValueError("rotated_in_workspace needs the forward's workspace")
     lay = _layout(q, k, v, cu_seqlens, max_seqlen)
@@ -154,8 +155,9 @@ def ttt_attn_bwd(q, k, v, o, lse, dout, *, theta: float, scale: Optional[float] 
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     else:
         dq, dk, dv = out
-    desc = make_desc(lay, theta, scale, events,
-                     _lib.TTT_FLAG_ROTATED_IN_WORKSPACE if rotated_in_workspace else 0)
+    flags = (_lib.TTT_FLAG_ROTATED_IN_WORKSPACE if rotated_in_workspace else 0) | \
+        (_lib.TTT_FLAG_DETERMINISTIC_DQ if deterministic else 0)
+    desc = make_desc(lay, theta, scale, events, flags)
     L = _lib.lib()
     need = L.ttt_attn_workspace_size(ctypes.byref(desc), 1)
     if workspace is None:

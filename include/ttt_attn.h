@@ -105,7 +105,13 @@ typedef enum {
    * workspace layout starts with the forward's (ttt_attn_workspace_layout), so a
    * workspace sized for the backward and passed to both calls qualifies.  If the
    * promise is broken the gradients are wrong; nothing is read out of bounds. */
-  TTT_FLAG_ROTATED_IN_WORKSPACE = 1
+  TTT_FLAG_ROTATED_IN_WORKSPACE = 1,
+  /* ttt_attn_bwd: bitwise reproducible dq.  The trunk backward adds the fp32
+   * partial dq~ of the key tiles of a query tile in key-tile order (each waits,
+   * bounded, for its predecessor's sum) instead of in arrival order.  Everything
+   * else in the library is already deterministic.  Slower: the dq~ additions of a
+   * query tile are serialised.  Ignored by ttt_attn_fwd. */
+  TTT_FLAG_DETERMINISTIC_DQ = 2
 } ttt_flag;
 
 /* Bytes of workspace that ttt_attn_fwd (for_backward = 0) or ttt_attn_bwd
@@ -169,7 +175,8 @@ ttt_status ttt_attn_device_status(void* workspace, void* stream, uint32_t* detai
  *        and the 64-row query tile j of sequence n, 128 floats at slot
  *        start_n/64 + n + j of row p*H + h (-lse * log2(e) of the 64 rows, then their
  *        delta = rowsum(dout * o)), T/64 + nseq + 1 slots per row,
- *        [4] dq~ accumulator fp32 [P][H][Tt][D], [5] dk~_1 accumulator fp32 [Hkv][Tt][D].
+ *        [4] dq~ accumulator fp32 [P][H][Tt][D], [5] dk~_1 accumulator fp32 [Hkv][Tt][D],
+ *        [6] int32 order tickets of the dq~ additions, one per statistics slot.
  * Tt = B*S (dense) or T (packed).  Returns the number of entries written to
  * offsets (at most 8), or 0 for an invalid descriptor. */
 int ttt_attn_workspace_layout(const ttt_attn_desc* desc, int for_backward, size_t* offsets);

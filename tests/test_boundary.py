@@ -50,7 +50,7 @@ def test_workspace_size_dense(L):
     assert bwd >= P * T * H * D * 2 + P * T * Hkv * D * 2 + P * H * T * 4 + P * T * H * D * 4 + Hkv * T * D * 4
     offs = (ctypes.c_size_t * 8)()
     n = L.ttt_attn_workspace_layout(ctypes.byref(d), 1, offs)
-    assert n == 6
+    assert n == 7
     assert all(offs[i] % 1024 == 0 for i in range(1, n))
     assert list(offs[:n]) == sorted(offs[:n])
 
@@ -66,7 +66,7 @@ def test_workspace_size_dense(L):
     ("softmax_scale", -0.5, _lib.TTT_ERR_INVALID_ARG),
     ("layout", 7, _lib.TTT_ERR_INVALID_ARG),
     ("B", -1, _lib.TTT_ERR_INVALID_ARG),
-    ("flags", 2, _lib.TTT_ERR_INVALID_ARG),     # unknown flag bit
+    ("flags", 4, _lib.TTT_ERR_INVALID_ARG),     # unknown flag bit
     ("flags", -1, _lib.TTT_ERR_INVALID_ARG),
 ])
 def test_invalid_descriptor(L, field, value, status):
@@ -77,9 +77,11 @@ def test_invalid_descriptor(L, field, value, status):
     assert st == status
 
 
-def test_known_flag_accepted(L):
-    d = desc(flags=_lib.TTT_FLAG_ROTATED_IN_WORKSPACE)
-    assert L.ttt_attn_workspace_size(ctypes.byref(d), 1) == L.ttt_attn_workspace_size(ctypes.byref(desc()), 1) > 0
+def test_known_flags_accepted(L):
+    for f in (_lib.TTT_FLAG_ROTATED_IN_WORKSPACE, _lib.TTT_FLAG_DETERMINISTIC_DQ,
+              _lib.TTT_FLAG_ROTATED_IN_WORKSPACE | _lib.TTT_FLAG_DETERMINISTIC_DQ):
+        d = desc(flags=f)
+        assert L.ttt_attn_workspace_size(ctypes.byref(d), 1) == L.ttt_attn_workspace_size(ctypes.byref(desc()), 1) > 0
 
 
 def test_null_descriptor(L):

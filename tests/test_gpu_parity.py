@@ -233,3 +233,31 @@ def test_sixteen_passes(layout, D):
     else:
         w = ttt_inputs.thd("p16_thd", [70, 1, 129], 16, 4, 1, D, 1e4)
     _check(w)
+
+
+# ----------------------------------------------------------------------------- deterministic dq
+
+@needs_cuda
+@pytest.mark.parametrize("name", ["ragged", "4k"])
+def test_deterministic_dq(name):
+    """TTT_FLAG_DETERMINISTIC_DQ: the backward run twice gives bit-identical dq (and dk,
+    dv), within the oracle's tolerance; on the 4K workload the oracle checks KV head 5."""
+    from attention_pass_rope_b200 import ops
+    if name == "ragged":
+        w, kv = ttt_inputs.thd("ragged", [300, 128, 17, 1, 257], 3, 8, 2, 128, 1e4), None
+    else:
+        w, kv = ttt_inputs.workloads()["qwen3_8b_4k"], [5]
+    inp = ttt_inputs.make_inputs(w)
+    q, k, v, do, cu = parity.gpu_shapes(w, inp)
+    kw = dict(theta=w.theta, cu_seqlens=cu, max_seqlen=None if w.dense else w.max_seqlen)
+    o, lse = ops.ttt_attn_fwd(q, k, v, **kw)
+    runs = [ops.ttt_attn_bwd(q, k, v, o, lse, do, deterministic=True, **kw) for _ in range(2)]
+    torch.cuda.synchronize()
+    for a_, b_ in zip(*runs):
+        assert torch.equal(a_, b_)
+    dq, dk, dv = runs[0]
+    gpu = {"o": parity.flat(o, w), "lse": lse, "dq": parity.flat(dq, w), "dk": parity.flat(dk, w),
+           "dv": parity.flat(dv, w)}
+    m = parity.compare_full(w, inp, gpu, kv_heads=kv)
+    print(name, "deterministic", m)
+    parity.assert_within(m)
