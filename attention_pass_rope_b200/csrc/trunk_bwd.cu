@@ -7,17 +7,19 @@
 //   P = exp(s - lse),  dP = dO V^T,  dS = P (dP - delta),  delta = rowsum(dO * O)
 //   dV_1 += P^T dO,  dk~_1 += dS^T q~,  dq~ += dS k~_1      (sigma applied later)
 //
-// One CTA owns one 128-key tile of one KV head and walks every (pass, group head)
-// query head and every 64-row query tile at or after the tile's diagonal, keeping
-// dK and dV of its keys in TMEM for the whole walk (no atomics on dK/dV).
+// One CTA owns one 128-key tile of one KV head and walks every 64-row query tile at
+// or after the tile's diagonal (the last one first) and, for each, every (pass, group
+// head) query head, keeping dK and dV of its keys in TMEM for the whole walk (no
+// atomics on dK/dV).
 // Transposed products keep the key dimension on the TMEM lanes:
 //   S^T  = K~ Q~^T        (M=128 keys, N=64 queries)      SS
 //   dP^T = V dO^T         (M=128 keys, N=64)              SS
 //   dV  += P^T dO         (M=128, N=D, K=64 queries)      TS  (P^T in TMEM, bf16)
 //   dK  += dS^T Q~        (M=128, N=D, K=64)              SS  (dS^T in smem, bf16)
 //   dQ^T = K~^T dS^T      (M=128 rows of d, N=64, K=128)  SS  (both MN-major)
-// dQ^T goes TMEM -> registers -> smem (fp32, row-major [q][d]) and is added to the
-// fp32 dq~ accumulator with one bulk reduce-add per tile.
+// dQ^T goes TMEM -> registers -> smem (fp32, row-major [q][d], two staging buffers of
+// 32 rows) and is added to the fp32 dq~ accumulator by bulk reduce-adds, in arrival
+// order, or in key-tile order under TTT_FLAG_DETERMINISTIC_DQ (per-tile tickets).
 //
 // CTA = 16 warps: warp 0 TMA producer (+ lse/delta rows), warp 1 TMEM allocator and
 // S^T/dP^T issuer, warp 2 dV/dK/dQ^T issuer, warps 4-7 and 8-11 the two halves (query
