@@ -179,7 +179,7 @@ static __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, c
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled bulk tensor copies, global -> shared, no multicast)
+// TMA (tiled bulk tensor copies, global -> shared of this CTA only)
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,

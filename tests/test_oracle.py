@@ -3,6 +3,8 @@ than itself (a second formulation, a library routine, finite differences,
 closed forms and invariants).  CPU only."""
 
 import math
+import os
+import sys
 
 import numpy as np
 import pytest
@@ -274,3 +276,42 @@ def test_single_row_functions_match_full_oracle():
         dk_r, dv_r = orc.row_dkv(q, k, v, do, 1e4, j0, t, kv)
         np.testing.assert_allclose(dk_r, dk[j0, t, kv], atol=1e-12)
         np.testing.assert_allclose(dv_r, dv[j0, t, kv], atol=1e-12)
+
+
+# ---------------------------------------------------------------- golden fixtures
+
+def _golden(name):
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)
+
+
+def test_staircase_rope_shift_machine_precision():
+    """NeMo-RL PR 3725's self-review reports that the multi-pass staircase visibility and
+    the RoPE-relative shift agree with an independent rotate-half oracle to machine
+    precision in fp64 (the figure is in tests/golden/staircase_rope_shift_fp64.txt).  The
+    oracle's two forms of the same function -- trunk + branch merged by log-sum-exp, and
+    one softmax over the explicit staircase mask -- must agree to within a few times that
+    figure on short sequences; a wrong shift, mask or merge term is off by orders of
+    magnitude more."""
+    with open(_golden("staircase_rope_shift_fp64.txt")) as f:
+        bound = float([ln.split()[1] for ln in f if ln.startswith("max_abs_diff")][0])
+    rng = np.random.default_rng(1)
+    worst = 0.0
+    for P, L, H, Hkv, D in [(1, 5, 2, 1, 8), (3, 7, 4, 2, 16), (4, 17, 2, 2, 8), (2, 1, 3, 1, 4)]:
+        q, k, v = (rng.standard_normal(s) for s in ((P, L, H, D), (P, L, Hkv, D), (P, L, Hkv, D)))
+        O1, l1 = orc.forward_bruteforce(q, k, v, 1e4, rope_round=None)
+        O2, l2 = orc.forward_twopart(q, k, v, 1e4, rope_round=None, block=4)
+        worst = max(worst, float(np.max(np.abs(O2 - O1))), float(np.max(np.abs(l2 - l1))))
+    assert worst <= 4 * bound, worst
+
+
+def test_oracle_matches_its_fixture():
+    """The oracle reproduces tests/golden/oracle_fixture_p3.txt (written by the committed
+    tests/golden/make_oracle_fixture.py, which calls the oracle only): any later change to
+    the oracle's arithmetic shows up here."""
+    sys.path.insert(0, os.path.dirname(_golden("x")))
+    import make_oracle_fixture as mk
+    ref = mk.read(_golden("oracle_fixture_p3.txt"))
+    got = mk.compute()
+    assert set(ref) == set(got)
+    for name in ref:
+        np.testing.assert_allclose(got[name], ref[name], rtol=0, atol=1e-13, err_msg=name)
