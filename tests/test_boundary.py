@@ -139,3 +139,18 @@ def test_status_strings(L):
     for s in range(6):
         assert L.ttt_status_string(s)
     assert L.ttt_attn_version().decode().count(".") == 2
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(P=1, H=4, Hkv=4, D=64), dict(P=16, B=1, S=130),
+                                dict(layout=1, nseq=3, total_tokens=200, max_seqlen=129, cu_seqlens=1 << 20)])
+def test_forward_layout_is_a_prefix_of_backward(L, kw):
+    """TTT_FLAG_ROTATED_IN_WORKSPACE relies on it: the rotated q~ / k~ sit at the same
+    offsets in the forward's and the backward's workspace, and the backward's is larger."""
+    d = desc(**kw)
+    f = (ctypes.c_size_t * 8)()
+    b = (ctypes.c_size_t * 8)()
+    nf = L.ttt_attn_workspace_layout(ctypes.byref(d), 0, f)
+    nb = L.ttt_attn_workspace_layout(ctypes.byref(d), 1, b)
+    assert nf == 3 and nb == 7
+    assert list(f[:nf]) == list(b[:nf])
+    assert L.ttt_attn_workspace_size(ctypes.byref(d), 1) >= L.ttt_attn_workspace_size(ctypes.byref(d), 0) > 0
