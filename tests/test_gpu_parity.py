@@ -36,9 +36,12 @@ def test_tiny_config_full():
     (1, 2, 2, 128, [200, 3, 129]),
     (4, 8, 2, 128, [300, 128, 17, 1]),
     (2, 3, 1, 128, [70, 260]),
+    (3, 4, 2, 64, [5, 0, 70, 0]),      # empty sequences, one of them last
+    (2, 2, 1, 128, [0, 129, 0, 1]),
 ])
 def test_packed_ragged(P, H, Hkv, D, lengths):
-    """THD with lengths that are not multiples of the tiles (1, 3, 17, 129, 257, ...)."""
+    """THD with lengths that are not multiples of the tiles (1, 3, 17, 129, 257, ...) and
+    with empty sequences (equal consecutive cu_seqlens entries)."""
     _check(ttt_inputs.thd("ragged", lengths, P, H, Hkv, D, 1e4))
 
 
