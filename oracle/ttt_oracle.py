@@ -23,7 +23,7 @@ What is computed (sources, by page and section):
   0..i (causal) and, on the staircase diagonal, the branch keys of passes
   2..p at the same position i.
 
-Readings where the pages are silent (all listed in the design doc):
+Readings where the pages are silent:
 
 * RoPE is rotate-half (dimension d pairs with d + D/2) with inverse frequency
   theta**(-2k/D), k < D/2, over the whole head dimension.
