@@ -148,3 +148,18 @@ def test_finite_differences():
             fd[idx] = (np.sum(bd.forward_bruteforce(theta=1e4, **plus)[0] * do) -
                        np.sum(bd.forward_bruteforce(theta=1e4, **minus)[0] * do)) / (2 * eps)
         np.testing.assert_allclose(g, fd, atol=2e-8, err_msg=name)
+
+
+def test_oracle_matches_its_fixture():
+    """The oracle reproduces tests/golden/block_draft_fixture.txt (written by the committed
+    tests/golden/make_block_draft_fixture.py, which calls the oracle only)."""
+    import os
+    import sys
+    golden = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    sys.path.insert(0, golden)
+    import make_block_draft_fixture as mk
+    ref = mk.read(os.path.join(golden, "block_draft_fixture.txt"))
+    got = mk.compute()
+    assert set(ref) == set(got)
+    for name in ref:
+        np.testing.assert_allclose(got[name], ref[name], rtol=0, atol=1e-13, err_msg=name)
