@@ -17,4 +17,4 @@ from .ops import (  # noqa: F401
     workspace_layout,
 )
 
-__version__ = "0.1.0"
+__version__ = "0.3.0"

@@ -89,6 +89,12 @@ def lib() -> ctypes.CDLL:
     L.ttt_attn_device_status.restype = ctypes.c_int
     L.ttt_attn_watchdog_selftest.argtypes = [vp, sz, u64, vp]
     L.ttt_attn_watchdog_selftest.restype = ctypes.c_int
+    L.ttt_attn_fwd_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp]
+    L.ttt_attn_fwd_noalloc.restype = ctypes.c_int
+    L.ttt_attn_fwd_noalloc_status.argtypes = [vp, P(u32)]
+    L.ttt_attn_fwd_noalloc_status.restype = ctypes.c_int
+    L.ttt_attn_noalloc_watchdog_selftest.argtypes = [u64, vp]
+    L.ttt_attn_noalloc_watchdog_selftest.restype = ctypes.c_int
     L.ttt_attn_set_wait_budget_ns.argtypes = [u64]
     L.ttt_attn_set_wait_budget_ns.restype = None
     L.ttt_status_string.argtypes = [ctypes.c_int]

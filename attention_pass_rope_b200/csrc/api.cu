@@ -325,7 +325,7 @@ const char* ttt_status_string(ttt_status s) {
   return "unknown status";
 }
 
-const char* ttt_attn_version(void) { return "0.2.0"; }
+const char* ttt_attn_version(void) { return "0.3.0"; }
 
 int ttt_attn_last_cuda_error(void) { return g_last_cuda_error.load(); }
 

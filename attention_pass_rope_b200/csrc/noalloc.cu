@@ -19,6 +19,10 @@
 // in it.  The forward clears what must start at zero (its status word) itself.  Two
 // calls whose work overlaps on the GPU (different streams, no ordering between
 // them) race on the array and give undefined results; order them on one stream.
+//
+// The forward's bounded in-kernel waits record a timeout in the first word of the
+// array, as the workspace forward does in the first word of its workspace; this
+// caller has no pointer to it, so ttt_attn_fwd_noalloc_status reads it instead.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -54,6 +58,20 @@ ttt_status scratch_on_current_device(void** out) {
 }
 
 }  // namespace
+
+extern "C" ttt_status ttt_attn_fwd_noalloc_status(void* stream, uint32_t* detail) {
+  void* scratch = nullptr;
+  const ttt_status st = scratch_on_current_device(&scratch);
+  if (st != TTT_OK) return st;
+  return ttt_attn_device_status(scratch, stream, detail);
+}
+
+extern "C" ttt_status ttt_attn_noalloc_watchdog_selftest(uint64_t budget_ns, void* stream) {
+  void* scratch = nullptr;
+  const ttt_status st = scratch_on_current_device(&scratch);
+  if (st != TTT_OK) return st;
+  return ttt_attn_watchdog_selftest(scratch, kNoallocScratchBytes, budget_ns, stream);
+}
 
 extern "C" ttt_status ttt_attn_fwd_noalloc(const ttt_attn_desc* desc, const void* q, const void* k, const void* v,
                                            void* o, float* lse, void* stream) {

@@ -33,7 +33,12 @@
  *
  * Ownership.  Every pointer is device memory owned by the caller, including the
  * workspace, whose size ttt_attn_workspace_size() returns.  The library allocates
- * nothing and keeps no state between calls.  Outputs must not alias inputs.
+ * nothing and keeps no per-call state between calls, with these exceptions: the
+ * no-allocation forward (ttt_attn_fwd_noalloc) uses a fixed 32 MiB array in the
+ * library's own device memory, held by every GPU that loads the library, whose device
+ * address is looked up once per device and cached; the in-kernel wait limit
+ * (ttt_attn_set_wait_budget_ns) and the last CUDA error (ttt_attn_last_cuda_error)
+ * are process-wide.  Outputs must not alias inputs.
  *
  * Asynchrony and errors.  Calls enqueue work on `stream` (a cudaStream_t; NULL is
  * the legacy default stream) and return without synchronising.  Argument errors
@@ -154,6 +159,18 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
 ttt_status ttt_attn_fwd_noalloc(const ttt_attn_desc* desc, const void* q, const void* k, const void* v, void* o,
                                 float* lse, void* stream);
 
+/* ttt_attn_device_status() for ttt_attn_fwd_noalloc, whose status word is the first
+ * word of the library's scratch array on the current device (the caller has no pointer
+ * to it): synchronises `stream`, returns TTT_OK or TTT_ERR_DEVICE_TIMEOUT (raw word in
+ * *detail if non-NULL) and clears the word.  Allocates nothing.  Like the forward, its
+ * first call on a device looks up the array's address. */
+ttt_status ttt_attn_fwd_noalloc_status(void* stream, uint32_t* detail);
+
+/* ttt_attn_watchdog_selftest() with its status word in that scratch array: lets a
+ * caller of the no-allocation forward check that a wait that runs out is reported
+ * through ttt_attn_fwd_noalloc_status(). */
+ttt_status ttt_attn_noalloc_watchdog_selftest(uint64_t budget_ns, void* stream);
+
 /* The error behind the most recent TTT_ERR_CUDA returned by any call in this
  * process: a cudaError_t value, or 100000 + the CUresult when encoding a TMA tensor
  * map failed; 0 if there was none.  Not reset by later successful calls. */
@@ -193,7 +210,7 @@ void ttt_attn_set_wait_budget_ns(uint64_t budget_ns);
 
 const char* ttt_status_string(ttt_status status);
 
-/* Library version, e.g. "0.1.0". */
+/* Library version, e.g. "0.3.0". */
 const char* ttt_attn_version(void);
 
 #ifdef __cplusplus

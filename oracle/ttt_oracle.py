@@ -509,3 +509,57 @@ def row_dkv(q, k, v, do, theta, j0, t, kv, scale=None, rope_round="bf16"):
             dv += Pr[c] * do[p0, i, h].astype(np.float64)
     dk = rope_rotate(dkr[None, None, :], [t + j0], theta, inverse=True)[0, 0]
     return dk, dv
+
+
+def tail_trunk_dkv(q, k, v, do, theta, kv, t0, scale=None, rope_round="bf16"):
+    """dK[0, t0:, kv, :] (pre-RoPE) and dV[0, t0:, kv, :] of one sequence: the trunk
+    keys t >= t0 of KV head kv, summed over every query row that sees them (rows
+    i >= t0 of every pass and every query head of the group).
+
+    Plain definition, vectorised over the rows i = t0..L-1 of one (pass, head) at a
+    time: each row's softmax runs over all its visible keys (trunk 0..i and the
+    branch keys of passes 2..p at position i), dS = P (dP - delta) with delta the sum
+    of P dP over those keys, then dk~_1[t] = sigma * sum_rows dS[., t] q~,
+    dV_1[t] = sum_rows P[., t] dO, and dK = R(t)^T dk~.  Used on the last keys of
+    long sequences, where few rows see them."""
+    P_, L, H, D = q.shape
+    g = H // k.shape[2]
+    sc = _scale(D, scale)
+    rows = np.arange(t0, L)
+    kt = rope_rotate(k[0, :, kv][:, None, :].astype(np.float64), np.arange(L), theta)[:, 0]
+    if rope_round == "bf16":
+        kt = bf16_round(kt)
+    v1 = v[0, :, kv].astype(np.float64)
+    causal = np.arange(L)[None, :] <= rows[:, None]                       # [R, L]
+    dkr = np.zeros((L - t0, D))
+    dv = np.zeros((L - t0, D))
+    for h in range(kv * g, (kv + 1) * g):
+        for p0 in range(P_):
+            qr = rope_rotate(q[p0, t0:, h][:, None, :].astype(np.float64), rows + p0, theta)[:, 0]
+            if rope_round == "bf16":
+                qr = bf16_round(qr)
+            dO = do[p0, t0:, h].astype(np.float64)
+            s_t = np.where(causal, sc * (qr @ kt.T), -np.inf)                  # [R, L]
+            dp_t = dO @ v1.T
+            if p0 > 0:                                                          # branch keys j = 1..p0
+                kb = np.stack([rope_rotate(k[j, t0:, kv][:, None, :].astype(np.float64), rows + j, theta)[:, 0]
+                               for j in range(1, p0 + 1)], axis=1)              # [R, p0, D]
+                if rope_round == "bf16":
+                    kb = bf16_round(kb)
+                vb = np.stack([v[j, t0:, kv] for j in range(1, p0 + 1)], axis=1).astype(np.float64)
+                s_b = sc * np.einsum("rd,rjd->rj", qr, kb)
+                dp_b = np.einsum("rd,rjd->rj", dO, vb)
+            else:
+                s_b = np.zeros((L - t0, 0))
+                dp_b = np.zeros((L - t0, 0))
+            s_all = np.concatenate([s_t, s_b], axis=1)
+            m = s_all.max(axis=1, keepdims=True)
+            e = np.exp(s_all - m)
+            Pr = e / e.sum(axis=1, keepdims=True)
+            dp_all = np.concatenate([dp_t, dp_b], axis=1)
+            delta = (Pr * dp_all).sum(axis=1, keepdims=True)
+            dS_t = Pr[:, :L] * (dp_t - delta)
+            dkr += sc * (dS_t[:, t0:].T @ qr)
+            dv += Pr[:, t0:L].T @ dO
+    dk = rope_rotate(dkr[:, None, :], rows, theta, inverse=True)[:, 0]
+    return dk, dv

@@ -74,3 +74,33 @@ def test_reference_arm_line_rank0_small():
     for k in ("impl", "metric", "value", "unit", "cpu_baseline", "e2e", "higher_is_better"):
         assert k in line
     assert line["impl"] == "reference" and line["value"] > 0
+
+
+def test_applicable_peak_burst_for_short_regions():
+    """A timed region under a second is held to the burst peak, a longer one to the
+    sustained (power-capped) peak; the label says which."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1683.8, "bf16_tflops_sustained": 1391.3}
+    p, why = bench.applicable_peak(peaks, "measured", 0.074)
+    assert p == 1683.8 and "burst" in why
+    p, why = bench.applicable_peak(peaks, "measured", 1.5)
+    assert p == 1391.3 and "sustained" in why
+
+
+def test_clock_record_of_a_region_shorter_than_the_period():
+    """No sample falls inside a 20 ms region between two samples: the record keeps the
+    nearest sample on each side instead of reporting none; reasons are unioned."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cs = bench.ClockSampler(0)
+    cs.source = "nvml"
+    cs.samples = [(10.00, 1965.0, 1965.0, set()), (10.10, 1950.0, 1965.0, {"sw_power_cap"}),
+                  (10.20, 1965.0, 1965.0, set())]
+    cs.t_begin, cs.t_end = 10.12, 10.14
+    r = cs.stop()
+    assert r["samples"] == 2 and r["sm_mhz"] == (1950.0 + 1965.0) / 2 and r["reasons"] == ["sw_power_cap"]
+    assert "nearest" in r["kept"]
+    cs.samples.append((10.13, 1900.0, 1965.0, set()))
+    r = cs.stop()
+    assert r["samples"] == 1 and r["sm_mhz"] == 1900.0 and r["kept"] == "inside the timed region"

@@ -141,6 +141,14 @@ def test_status_strings(L):
     assert L.ttt_attn_version().decode().count(".") == 2
 
 
+def test_one_version_string(L):
+    """The library, the Python package and the header's example name the same version."""
+    import attention_pass_rope_b200 as pkg
+    v = L.ttt_attn_version().decode()
+    assert pkg.__version__ == v
+    assert f'"{v}"' in open(HEADER).read()
+
+
 @pytest.mark.parametrize("kw", [dict(), dict(P=1, H=4, Hkv=4, D=64), dict(P=16, B=1, S=130),
                                 dict(layout=1, nseq=3, total_tokens=200, max_seqlen=129, cu_seqlens=1 << 20)])
 def test_forward_layout_is_a_prefix_of_backward(L, kw):

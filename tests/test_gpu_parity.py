@@ -15,11 +15,11 @@ pytestmark = pytest.mark.gpu
 needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 
 
-def _check(w, kv_heads=None, seqs=None, with_grad=True):
+def _check(w, kv_heads=None, seqs=None, with_grad=True, scale=None):
     inp = ttt_inputs.make_inputs(w)
-    gpu = parity.run_gpu(w, inp, with_grad=with_grad)
-    m = parity.compare_full(w, inp, gpu, with_grad=with_grad, kv_heads=kv_heads, seqs=seqs)
-    print(w.name, m)
+    gpu = parity.run_gpu(w, inp, with_grad=with_grad, scale=scale)
+    m = parity.compare_full(w, inp, gpu, with_grad=with_grad, kv_heads=kv_heads, seqs=seqs, scale=scale)
+    print(w.name, "scale", scale, m)
     parity.assert_within(m)
     return m
 
@@ -49,6 +49,22 @@ def test_packed_ragged(P, H, Hkv, D, lengths):
 @pytest.mark.parametrize("B,S,P,H,Hkv,D", [(2, 200, 3, 4, 4, 128), (3, 64, 5, 2, 1, 64), (1, 384, 2, 8, 2, 128)])
 def test_dense_tails(B, S, P, H, Hkv, D):
     _check(ttt_inputs.dense("dense_tail", B, S, P, H, Hkv, D, 1e6))
+
+
+@needs_cuda
+@pytest.mark.parametrize("layout,D", [("dense", 128), ("dense", 64), ("thd", 128), ("thd", 64)])
+def test_non_default_softmax_scale(layout, D):
+    """ttt_attn_desc.softmax_scale != 0: the trunk forward, the branch keys and merge of
+    its epilogue, the trunk backward and the branch backward all take the descriptor's
+    scale instead of 1/sqrt(D).  0.37/sqrt(D) and 2.5/sqrt(D) (sharper rows, so the
+    forward's running-max rescale of O is exercised too), forward and backward, every
+    element against the oracle run with the same scale."""
+    for factor in (0.37, 2.5):
+        if layout == "dense":
+            w = ttt_inputs.dense("scale", 2, 200, 3, 4, 2, D, 1e4)
+        else:
+            w = ttt_inputs.thd("scale_thd", [129, 1, 300, 64], 4, 4, 1, D, 1e6)
+        _check(w, scale=factor / D ** 0.5)
 
 
 @needs_cuda
@@ -135,42 +151,65 @@ def test_thd_packed_sampled_sequences():
     _check(ttt_inputs.workloads()["thd_packed"], kv_heads=[2], seqs=[4, 5])
 
 
+# positions at the edges of the 64-row and 128-row tiles and of the sequence
+EDGE_POSITIONS_32K = [0, 1, 63, 64, 127, 128, 129, 255, 256, 4095, 4096, 4097, 8191, 8192, 16383, 16384,
+                      24575, 32639, 32640, 32703, 32704, 32766, 32767]
+
+
 @needs_cuda
 def test_long_32k_sampled_rows():
-    """B=1, S=32768, P=5, 32/8 heads, D=128, inputs scaled by 0.5: single rows computed
-    one by one by the oracle -- outputs and dQ of query rows across the sequence, dK/dV
-    of trunk keys near the end (seen by few queries) and of branch keys anywhere."""
+    """B=1, S=32768, P=5, 32/8 heads, D=128, inputs scaled by 0.5, against the oracle's
+    per-row forms: outputs, lse and dQ of ~300 query rows (every pass at the tile-edge
+    positions, plus seeded random rows); dK/dV of the last 130 trunk keys of two KV heads
+    (they cross the 128- and 64-row tile edges at 32640 and 32704), computed over every
+    query row that sees them; dK/dV of branch keys at tile edges across the sequence."""
     w = ttt_inputs.workloads()["long_32k"]
     inp = ttt_inputs.make_inputs(w)
     gpu = parity.run_gpu(w, inp, with_grad=True)
     # float32 copies hold the bf16 values exactly; the oracle widens the rows it uses
     q, k, v, do = (t.float().numpy() for t in (inp.q, inp.k, inp.v, inp.do))
     g = w.H // w.Hkv
+    L = w.lengths[0]
+    rng = np.random.default_rng(0)
+    rows = [(p0, i, (7 * n + 3 * p0) % w.H) for n, i in enumerate(EDGE_POSITIONS_32K) for p0 in range(w.P)]
+    rows += [(int(rng.integers(w.P)), int(rng.integers(L)), int(rng.integers(w.H))) for _ in range(185)]
     kts = {}
-    o_err, l_err, dq_ref, dq_got = 0.0, 0.0, [], []
-    for (p0, i, h) in [(0, 0, 0), (4, 0, 31), (1, 127, 5), (2, 128, 9), (3, 4097, 14), (0, 20000, 22),
-                       (4, 32767, 7), (2, 32766, 30)]:
+    o_err, l_err = 0.0, 0.0
+    dq_ref, dq_got = [[] for _ in range(w.P)], [[] for _ in range(w.P)]
+    for (p0, i, h) in rows:
         kv = h // g
         if kv not in kts:
             kts[kv] = orc.rotate_trunk_keys(k, kv, w.theta)
         o_r, l_r = orc.row_forward(q, k, v, w.theta, p0, i, h, kt=kts[kv])
         o_err = max(o_err, float(np.max(np.abs(parity.to64(gpu["o"][p0, i, h]) - o_r))))
         l_err = max(l_err, abs(float(gpu["lse"][p0, 0, h, i]) - l_r))
-        dq_ref.append(orc.row_dq(q, k, v, do, w.theta, p0, i, h, kt=kts[kv]))
-        dq_got.append(parity.to64(gpu["dq"][p0, i, h]))
+        dq_ref[p0].append(orc.row_dq(q, k, v, do, w.theta, p0, i, h, kt=kts[kv]))
+        dq_got[p0].append(parity.to64(gpu["dq"][p0, i, h]))
+    t0 = L - 130
     dk_ref, dk_got, dv_ref, dv_got = [], [], [], []
-    for (j0, t, kv) in [(0, 32767, 0), (0, 32760, 5), (1, 0, 2), (2, 9000, 7), (4, 32767, 1), (3, 15, 4)]:
+    for kv in (0, 5):
+        dk_t, dv_t = orc.tail_trunk_dkv(q, k, v, do, w.theta, kv, t0)
+        dk_ref.append(dk_t)
+        dv_ref.append(dv_t)
+        dk_got.append(parity.to64(gpu["dk"][0, t0:, kv]))
+        dv_got.append(parity.to64(gpu["dv"][0, t0:, kv]))
+    bk_ref, bk_got, bv_ref, bv_got = [], [], [], []
+    for (j0, t, kv) in [(1, 0, 2), (4, 127, 1), (2, 128, 7), (3, 4095, 4), (1, 4096, 6), (2, 9000, 7),
+                        (4, 16384, 3), (3, 32703, 0), (1, 32767, 5), (4, 32767, 1)]:
         dk_r, dv_r = orc.row_dkv(q, k, v, do, w.theta, j0, t, kv)
-        dk_ref.append(dk_r)
-        dv_ref.append(dv_r)
-        dk_got.append(parity.to64(gpu["dk"][j0, t, kv]))
-        dv_got.append(parity.to64(gpu["dv"][j0, t, kv]))
-    m = {"o_max_abs": o_err, "lse_max_abs": l_err,
-         "dq_rel_l2": parity.rel_l2(np.array(dq_got), np.array(dq_ref)),
-         "dk_rel_l2": parity.rel_l2(np.array(dk_got), np.array(dk_ref)),
-         "dv_rel_l2": parity.rel_l2(np.array(dv_got), np.array(dv_ref))}
+        bk_ref.append(dk_r)
+        bv_ref.append(dv_r)
+        bk_got.append(parity.to64(gpu["dk"][j0, t, kv]))
+        bv_got.append(parity.to64(gpu["dv"][j0, t, kv]))
+    rel = lambda a_, b_: parity.rel_l2(np.array(a_), np.array(b_))
+    dq_pass = [rel(dq_got[p], dq_ref[p]) for p in range(w.P) if dq_ref[p]]
+    m = {"rows": len(rows), "o_max_abs": o_err, "lse_max_abs": l_err,
+         "dq_rel_l2": rel(sum(dq_got, []), sum(dq_ref, [])), "dq_rel_l2_per_pass": dq_pass,
+         "dk_rel_l2": rel(dk_got, dk_ref), "dv_rel_l2": rel(dv_got, dv_ref),
+         "branch_dk_rel_l2": rel(bk_got, bk_ref), "branch_dv_rel_l2": rel(bv_got, bv_ref)}
     print("long_32k", m)
     parity.assert_within(m)
+    assert m["branch_dk_rel_l2"] <= parity.GRAD_REL_L2 and m["branch_dv_rel_l2"] <= parity.GRAD_REL_L2, m
 
 
 @needs_cuda

@@ -278,6 +278,20 @@ def test_single_row_functions_match_full_oracle():
         np.testing.assert_allclose(dv_r, dv[j0, t, kv], atol=1e-12)
 
 
+@pytest.mark.parametrize("t0", [0, 5, 8])
+def test_tail_trunk_dkv_matches_full_oracle(t0):
+    """The vectorised gradient of the last trunk keys (used on 32K-token samples)
+    agrees with the two-part oracle's full backward on every key t >= t0."""
+    P, L, H, Hkv, D = 3, 9, 4, 2, 8
+    q, k, v, do = rnd(P, L, H, D), rnd(P, L, Hkv, D), rnd(P, L, Hkv, D), rnd(P, L, H, D)
+    O, lse = orc.forward_twopart(q, k, v, 1e4)
+    dq, dk, dv = orc.backward_twopart(q, k, v, do, lse, 1e4)
+    for kv in range(Hkv):
+        dk_t, dv_t = orc.tail_trunk_dkv(q, k, v, do, 1e4, kv, t0)
+        np.testing.assert_allclose(dk_t, dk[0, t0:, kv], atol=1e-12)
+        np.testing.assert_allclose(dv_t, dv[0, t0:, kv], atol=1e-12)
+
+
 # ---------------------------------------------------------------- golden fixtures
 
 def _golden(name):
