@@ -45,6 +45,8 @@ class TTTDesc(ctypes.Structure):
         ("max_seqlen", ctypes.c_int),
         ("events", ctypes.c_void_p),
         ("flags", ctypes.c_int),
+        ("pass_stride_q", ctypes.c_int64),
+        ("pass_stride_kv", ctypes.c_int64),
     ]
 
 

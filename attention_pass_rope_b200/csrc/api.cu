@@ -69,6 +69,22 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
   // per-pass offsets in int32 where they are formed that way
   const long long rows = static_cast<long long>(g.P) * g.H * g.si.T;
   if (rows * g.D > (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+  // per-pass strides of the public tensors (0: packed); passes never overlap
+  const int64_t packed_q = static_cast<int64_t>(g.si.T) * g.H * g.D;
+  const int64_t packed_kv = static_cast<int64_t>(g.si.T) * g.Hkv * g.D;
+  g.sq = packed_q;
+  g.skv = packed_kv;
+  if (g.P > 1) {
+    if (d->pass_stride_q != 0) {
+      if (d->pass_stride_q < packed_q || d->pass_stride_q % 8 != 0) return TTT_ERR_INVALID_ARG;
+      g.sq = d->pass_stride_q;
+    }
+    if (d->pass_stride_kv != 0) {
+      if (d->pass_stride_kv < packed_kv || d->pass_stride_kv % 8 != 0) return TTT_ERR_INVALID_ARG;
+      g.skv = d->pass_stride_kv;
+    }
+    if (g.sq > (1LL << 44) / g.P || g.skv > (1LL << 44) / g.P) return TTT_ERR_UNSUPPORTED;
+  }
 
   const size_t T = static_cast<size_t>(g.si.T);
   const size_t P = g.P, H = g.H, Hkv = g.Hkv, D = g.D;
@@ -132,6 +148,25 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
   const cuuint32_t box[3] = {64, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_cuda_error.store(kEncodeErrorBase + static_cast<int>(r));
+  return r == CUDA_SUCCESS;
+}
+
+// 4-D bf16 tensor map, 128-byte swizzle, box {64, b1, b2, b3}; dims/strides innermost first.
+bool make_map4(CUtensorMap* m, const void* base, const uint64_t (&dims)[4], const uint64_t (&strides_bytes)[3],
+               const uint32_t (&box_outer)[3]) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    g_last_cuda_error.store(static_cast<int>(cudaErrorSymbolNotFound));
+    return false;
+  }
+  const cuuint64_t d4[4] = {dims[0], dims[1], dims[2], dims[3]};
+  const cuuint64_t s3[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+  const cuuint32_t box[4] = {64, box_outer[0], box_outer[1], box_outer[2]};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d4, s3, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) g_last_cuda_error.store(kEncodeErrorBase + static_cast<int>(r));
@@ -260,7 +295,8 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   if (!make_map(&mq, qr, D, T, static_cast<uint64_t>(g.P) * g.H, D * 2, T * D * 2, 64, 1) ||
       !make_map(&mk, kr, D, T, g.Hkv, D * 2, T * D * 2, 128, 1) ||
       !make_map(&mv, v, D, g.Hkv, T, D * 2, g.Hkv * D * 2, 1, 128) ||
-      !make_map(&mdo, dout, D, g.H, static_cast<uint64_t>(g.P) * T, D * 2, g.H * D * 2, 1, 64))
+      !make_map4(&mdo, dout, {D, static_cast<uint64_t>(g.H), T, static_cast<uint64_t>(g.P)},
+                 {D * 2, g.H * D * 2, static_cast<uint64_t>(g.sq) * 2}, {1, 64, 1}))
     return TTT_ERR_CUDA;
   {
     // the events are recorded either way, so a timing caller sees ~0 when the

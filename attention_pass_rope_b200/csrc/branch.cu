@@ -125,9 +125,9 @@ __global__ void __launch_bounds__(kPreThreads)
   for (int u = 0; u < NU; ++u) {
     const int i = warp * RPWARP + u * RPI + sub;
     if (i < nvalid) {
-      const int64_t row = (static_cast<int64_t>(p) * T + start + pos0 + i) * g.H + h;
-      a[u] = __ldg(reinterpret_cast<const uint4*>(o + row * D) + c);
-      b[u] = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + c);
+      const int64_t row = p * g.sq + (static_cast<int64_t>(start + pos0 + i) * g.H + h) * D;
+      a[u] = __ldg(reinterpret_cast<const uint4*>(o + row) + c);
+      b[u] = __ldg(reinterpret_cast<const uint4*>(dout + row) + c);
     } else {
       a[u] = make_uint4(0, 0, 0, 0);
       b[u] = make_uint4(0, 0, 0, 0);
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
           load_f32_row<D>(dq_acc + hrow * D, lane, dqv[u]);
           if (p > 0) {
             load_bf16_row<D>(qr + hrow * D, lane, q[u]);
-            load_bf16_row<D>(dout + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D, lane, dO[u]);
+            load_bf16_row<D>(dout + p * g.sq + (static_cast<int64_t>(tau) * g.H + h) * D, lane, dO[u]);
             lse_v[u] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)];
             dl[u] = ld[(static_cast<int64_t>(p) * g.H + h) * dl_base + dl_off];
           }
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
       for (int j = 1; j <= p; ++j) {
         float kj[2][E], vj[2][E];
         load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
-        load_bf16_row<D>(v + ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D, lane, vj);
+        load_bf16_row<D>(v + j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D, lane, vj);
         float sdot[kBranchHeads], tdot[kBranchHeads];
 #pragma unroll
         for (int u = 0; u < kBranchHeads; ++u) {
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
 #pragma unroll
           for (int e = 0; e < E; ++e) dqv[u][hh][e] *= g.scale;
         rotate_back<D>(dqv[u], c, sn);
-        store_bf16_row<D>(dq + ((static_cast<int64_t>(p) * T + tau) * g.H + kvh * gsz + h0 + u) * D, lane, dqv[u]);
+        store_bf16_row<D>(dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz + h0 + u) * D, lane, dqv[u]);
       }
     }
   }
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
 #pragma unroll
       for (int e = 0; e < E; ++e) kx[hh][e] *= g.scale;
     rotate_back<D>(kx, c, sn);
-    const int64_t krow = ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D;
+    const int64_t krow = j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D;
     store_bf16_row<D>(dk + krow, lane, kx);
     if (j > 0) {
       float vx[2][E];

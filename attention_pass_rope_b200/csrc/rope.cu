@@ -5,7 +5,8 @@
 // offset itself (pass p, position i -> i+p-1) and rotate-half ("bounded multi-pass
 // EAGLE-3 TTT provider", self-review) fix the rotation.
 //
-// Memory bound: reads q [P][T][H][D] and k [P][T][Hkv][D] once, writes the rotated
+// Memory bound: reads q [P][T][H][D] and k [P][T][Hkv][D] once (consecutive passes
+// g.sq and g.skv elements apart), writes the rotated
 // copies head-major (q~ [P][H][T][D], k~ [P][Hkv][T][D]) so that the attention
 // kernels fetch a (head, 128-token) tile as one contiguous block.  cos/sin depend
 // on (position, frequency) only: each CTA computes them once per token in double
@@ -60,11 +61,11 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
     const __nv_bfloat16* src;
     __nv_bfloat16* dst;
     if (head < g.H) {
-      src = q + ((static_cast<int64_t>(p) * T + tau) * g.H + head) * D;
+      src = q + p * g.sq + (static_cast<int64_t>(tau) * g.H + head) * D;
       dst = qr + ((static_cast<int64_t>(p) * g.H + head) * T + tau) * D;
     } else {
       const int hk = head - g.H;
-      src = k + ((static_cast<int64_t>(p) * T + tau) * g.Hkv + hk) * D;
+      src = k + p * g.skv + (static_cast<int64_t>(tau) * g.Hkv + hk) * D;
       dst = kr + ((static_cast<int64_t>(p) * g.Hkv + hk) * T + tau) * D;
     }
     const int d0 = part * 8;

@@ -206,8 +206,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int c = 0; c < C::KCH; ++c) {
           tma_load_3d(sQ + s * C::QTILE + c * C::QCHUNK, &map_q, qdo_full + s, c * 64, seq_start + ii.q0,
                       ii.p * g.H + ii.h);
-          tma_load_3d(sDO + s * C::QTILE + c * C::QCHUNK, &map_do, qdo_full + s, c * 64, ii.h,
-                      ii.p * g.si.T + seq_start + ii.q0);
+          tma_load_4d(sDO + s * C::QTILE + c * C::QCHUNK, &map_do, qdo_full + s, c * 64, ii.h, seq_start + ii.q0,
+                      ii.p);
         }
         const float* src =
             a.ld + ((static_cast<int64_t>(ii.p) * g.H + ii.h) * nslots + ld_slot(seq_start, n, ii.q0)) * 128;

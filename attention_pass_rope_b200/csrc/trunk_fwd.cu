@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         l += bs[j];
       }
       const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + p * g.sq + (static_cast<int64_t>(tau) * g.H + h) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int j = 1; j <= kMaxBranch; ++j) {
             if (j <= p) {
               const uint4* vj = reinterpret_cast<const uint4*>(
-                  static_cast<const __nv_bfloat16*>(a.v) + ((static_cast<int64_t>(j) * T + tau) * g.Hkv + kvh) * D +
+                  static_cast<const __nv_bfloat16*>(a.v) + j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D +
                   32 * c);
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4) {

@@ -49,6 +49,8 @@ struct Geometry {
   int P, H, Hkv, D;
   float theta;
   float scale;  // softmax scale sigma
+  int64_t sq;   // elements between passes of the public q, o, dout, dq
+  int64_t skv;  // elements between passes of the public k, v, dk, dv
 };
 
 // ----------------------------------------------------------------- launchers
@@ -61,8 +63,8 @@ cudaError_t launch_rope_fwd(const Geometry& g, const void* q, const void* k, voi
 struct TrunkFwdArgs {
   Geometry g;
   const void* kr;  // bf16 k~ head-major [P][Hkv][T][D] (branch keys, passes >= 1)
-  const void* v;   // bf16 V, public layout [P][T][Hkv][D] (branch values)
-  void* o;         // bf16 output, public layout [P][T][H][D]
+  const void* v;   // bf16 V, public layout [P][T][Hkv][D] (branch values; passes g.skv apart)
+  void* o;         // bf16 output, public layout [P][T][H][D] (passes g.sq apart)
   float* lse;      // fp32 merged lse, public layout
   uint32_t* status;
   uint64_t budget_ns;
@@ -96,7 +98,7 @@ struct TrunkBwdArgs {
   uint64_t budget_ns;
 };
 // a6: trunk backward on tcgen05; maps: q~ (box 64 rows), k~_1 (box 128 rows),
-// V_1 (box 128 rows), dO (3D {D, H, P*T}, box 64 rows).
+// V_1 (box 128 rows), dO (4D {D, H, T, P}, pass stride g.sq, box 64 rows).
 cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
                              const CUtensorMap& map_v, const CUtensorMap& map_do, cudaStream_t stream);
 

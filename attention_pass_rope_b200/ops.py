@@ -9,6 +9,10 @@ Shapes (pass-major, trunk = index 0 along P):
   dense:  q [P, B, S, H, D], k/v [P, B, S, Hkv, D]    -> o like q, lse [P, B, H, S]
   packed: q [P, T, H, D],    k/v [P, T, Hkv, D] with cu_seqlens (int32, cuda)
                                                       -> o like q, lse [P, H, T]
+Each pass of a tensor must be contiguous; the passes themselves may sit at any common
+stride (a multiple of 8 elements, no overlap), e.g. slices of one larger buffer that a
+caller filled one pass at a time: q, o, dout, dq share one pass stride, k, v, dk, dv
+another.  Outputs that are not given are allocated at the inputs' pass strides.
 """
 
 from __future__ import annotations
@@ -35,10 +39,25 @@ class Layout:
     nseq: int = 0
     max_seqlen: int = 0
     cu_seqlens: Optional[torch.Tensor] = None
+    stride_q: int = 0    # elements between passes of q-shaped tensors (packed: T*H*D)
+    stride_kv: int = 0   # elements between passes of k-shaped tensors (packed: T*Hkv*D)
 
     @property
     def lse_shape(self):
         return (self.P, self.B, self.H, self.S) if self.dense else (self.P, self.H, self.T)
+
+
+def pass_stride(t: torch.Tensor) -> int:
+    """Elements between consecutive passes of a pass-major tensor whose every pass is
+    contiguous (raises otherwise)."""
+    if not t[0].is_contiguous():
+        raise ValueError("every pass of a tensor must be contiguous")
+    if t.shape[0] == 1:
+        return t[0].numel()
+    st = t.stride(0)
+    if st < t[0].numel() or st % 8 != 0:
+        raise ValueError(f"pass stride {st} must be a multiple of 8 elements and at least {t[0].numel()}")
+    return st
 
 
 def _layout(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens, max_seqlen) -> Layout:
@@ -53,19 +72,51 @@ def _layout(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens, max_s
         Hkv = k.shape[3]
         if k.shape != (P, B, S, Hkv, D) or v.shape != k.shape:
             raise ValueError("k, v must be [P, B, S, Hkv, D]")
-        return Layout(P, H, Hkv, D, True, B=B, S=S, T=B * S, nseq=B, max_seqlen=S)
-    if q.dim() != 4:
-        raise ValueError("packed q must be [P, T, H, D]")
-    P, T, H, D = q.shape
-    Hkv = k.shape[2]
-    if k.shape != (P, T, Hkv, D) or v.shape != k.shape:
-        raise ValueError("k, v must be [P, T, Hkv, D]")
-    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
-        raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
-    if max_seqlen is None:
-        raise ValueError("max_seqlen is required with cu_seqlens")
-    return Layout(P, H, Hkv, D, False, T=T, nseq=cu_seqlens.numel() - 1, max_seqlen=int(max_seqlen),
-                  cu_seqlens=cu_seqlens.contiguous())
+        lay = Layout(P, H, Hkv, D, True, B=B, S=S, T=B * S, nseq=B, max_seqlen=S)
+    else:
+        if q.dim() != 4:
+            raise ValueError("packed q must be [P, T, H, D]")
+        P, T, H, D = q.shape
+        Hkv = k.shape[2]
+        if k.shape != (P, T, Hkv, D) or v.shape != k.shape:
+            raise ValueError("k, v must be [P, T, Hkv, D]")
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        lay = Layout(P, H, Hkv, D, False, T=T, nseq=cu_seqlens.numel() - 1, max_seqlen=int(max_seqlen),
+                     cu_seqlens=cu_seqlens.contiguous())
+    if q.numel() == 0 or k.numel() == 0:
+        return lay
+    lay.stride_q = pass_stride(q)
+    lay.stride_kv = pass_stride(k)
+    if pass_stride(v) != lay.stride_kv:
+        raise ValueError("k and v must share one pass stride")
+    return lay
+
+
+def _check_strides(lay: Layout, q_like=(), kv_like=()):
+    """Every q-shaped tensor at the layout's q pass stride, every k-shaped one at its kv
+    stride (the descriptor carries one stride per kind)."""
+    if lay.T == 0:
+        return
+    for t in q_like:
+        if pass_stride(t) != lay.stride_q:
+            raise ValueError("q, o, dout and dq must share one pass stride")
+    for t in kv_like:
+        if pass_stride(t) != lay.stride_kv:
+            raise ValueError("k, v, dk and dv must share one pass stride")
+
+
+def empty_at_pass_stride(like: torch.Tensor, stride: int, dtype=None) -> torch.Tensor:
+    """Uninitialised tensor of like's shape whose passes are ``stride`` elements apart."""
+    P = like.shape[0]
+    per = like[0].numel()
+    if P <= 1 or stride == per:
+        return torch.empty(like.shape, dtype=dtype or like.dtype, device=like.device)
+    buf = torch.empty((P - 1) * stride + per, dtype=dtype or like.dtype, device=like.device)
+    inner = torch.empty(like.shape[1:], dtype=buf.dtype, device="meta").stride()
+    return buf.as_strided(like.shape, (stride,) + tuple(inner))
 
 
 def make_desc(lay: Layout, theta: float, scale: Optional[float], events=None, flags: int = 0) -> _lib.TTTDesc:
@@ -80,6 +131,9 @@ def make_desc(lay: Layout, theta: float, scale: Optional[float], events=None, fl
         d.nseq, d.total_tokens, d.max_seqlen = lay.nseq, lay.T, lay.max_seqlen
     d.events = ctypes.addressof(events) if events is not None else None
     d.flags = int(flags)
+    packed_q, packed_kv = lay.T * lay.H * lay.D, lay.T * lay.Hkv * lay.D
+    d.pass_stride_q = 0 if lay.stride_q in (0, packed_q) else lay.stride_q
+    d.pass_stride_kv = 0 if lay.stride_kv in (0, packed_kv) else lay.stride_kv
     return d
 
 
@@ -111,22 +165,18 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def _contig(*ts):
-    for t in ts:
-        if t is not None and not t.is_contiguous():
-            raise ValueError("tensors must be contiguous")
-
-
 def ttt_attn_fwd(q, k, v, *, theta: float, scale: Optional[float] = None, cu_seqlens=None, max_seqlen=None,
                  workspace: Optional[torch.Tensor] = None, out=None, events=None):
     """Forward: returns (o, lse).  ``out=(o, lse)`` writes into given tensors."""
     lay = _layout(q, k, v, cu_seqlens, max_seqlen)
-    _contig(q, k, v)
     if out is None:
-        o = torch.empty_like(q)
+        o = empty_at_pass_stride(q, lay.stride_q)
         lse = torch.empty(lay.lse_shape, dtype=torch.float32, device=q.device)
     else:
         o, lse = out
+    _check_strides(lay, q_like=(o,))
+    if not lse.is_contiguous():
+        raise ValueError("lse must be contiguous")
     desc = make_desc(lay, theta, scale, events)
     L = _lib.lib()
     need = L.ttt_attn_workspace_size(ctypes.byref(desc), 0)
@@ -148,13 +198,17 @@ def ttt_attn_bwd(q, k, v, o, lse, dout, *, theta: float, scale: Optional[float] 
     if rotated_in_workspace and workspace is None:
         raise ValueError("rotated_in_workspace needs the forward's workspace")
     lay = _layout(q, k, v, cu_seqlens, max_seqlen)
-    _contig(q, k, v, o, lse, dout)
     if dout.dtype != torch.bfloat16 or o.dtype != torch.bfloat16 or lse.dtype != torch.float32:
         raise TypeError("o, dout must be bfloat16 and lse float32")
+    if not lse.is_contiguous():
+        raise ValueError("lse must be contiguous")
     if out is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dq = empty_at_pass_stride(q, lay.stride_q)
+        dk = empty_at_pass_stride(k, lay.stride_kv)
+        dv = empty_at_pass_stride(v, lay.stride_kv)
     else:
         dq, dk, dv = out
+    _check_strides(lay, q_like=(o, dout, dq), kv_like=(dk, dv))
     flags = (_lib.TTT_FLAG_ROTATED_IN_WORKSPACE if rotated_in_workspace else 0) | \
         (_lib.TTT_FLAG_DETERMINISTIC_DQ if deterministic else 0)
     desc = make_desc(lay, theta, scale, events, flags)
@@ -204,7 +258,14 @@ class _TTTAttention(torch.autograd.Function):
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse, cu = ctx.saved_tensors
-        dq, dk, dv = ttt_attn_bwd(q, k, v, o, lse, do.contiguous(), theta=ctx.theta, scale=ctx.scale,
+        if do.shape[0] > 0 and do.numel() > 0:
+            try:
+                same = pass_stride(do) == pass_stride(o)
+            except ValueError:
+                same = False
+            if not same:
+                do = empty_at_pass_stride(o, pass_stride(o)).copy_(do)
+        dq, dk, dv = ttt_attn_bwd(q, k, v, o, lse, do, theta=ctx.theta, scale=ctx.scale,
                                   cu_seqlens=cu if ctx.has_cu else None, max_seqlen=ctx.max_seqlen,
                                   workspace=ctx.ws, rotated_in_workspace=ctx.ws is not None)
         ctx.ws = None

@@ -19,7 +19,7 @@
  *   k~ are computed in fp32 and rounded to bf16 before the dot products.
  *   R(m) pairs dimension d with d + D/2 and rotates by m * theta^(-2d/D).
  *
- * Layouts (all pass-major, the trunk is index 0 along P, row-major, contiguous):
+ * Layouts (all pass-major, the trunk is index 0 along P, row-major):
  *   dense (TTT_LAYOUT_BSHD):  q, o, dout, dq  [P][B][S][H][D]    bf16
  *                             k, v, dk, dv    [P][B][S][Hkv][D]  bf16
  *                             lse             [P][B][H][S]       fp32 (natural log)
@@ -29,6 +29,12 @@
  *                             non-decreasing, cu_seqlens[nseq] = T); positions restart
  *                             at 0 at every sequence start and no attention crosses
  *                             a sequence boundary.
+ *   Within a pass every tensor is contiguous.  Consecutive passes of q, o, dout and dq
+ *   are desc->pass_stride_q elements apart, those of k, v, dk and dv
+ *   desc->pass_stride_kv elements apart (0 selects the packed value, T*H*D and
+ *   T*Hkv*D; T = B*S for dense batches), so a caller that produces the passes one at a
+ *   time can place them at a common stride in one allocation instead of
+ *   concatenating them.  lse is always packed.
  *   Supported: D in {64, 128}; H a multiple of Hkv; 1 <= P <= 16.
  *
  * Ownership.  Every pointer is device memory owned by the caller, including the
@@ -100,6 +106,14 @@ typedef struct {
   int max_seqlen;      /* THD only: upper bound on every sequence length */
   const ttt_attn_events* events; /* optional, NULL for none */
   int flags;           /* TTT_FLAG_* bits, 0 for none; other bits are rejected */
+  /* Elements between consecutive passes of q, o, dout, dq (pass_stride_q) and of k, v,
+   * dk, dv (pass_stride_kv); 0 = packed.  A non-zero stride must be a multiple of 8
+   * (16 bytes) and at least the packed value (passes never overlap); with P = 1 it is
+   * ignored.  Source: the boundary of the "DFlash/DSpark and EAGLE-3 TTT draft
+   * co-training" roadmap (NeMo-RL issue 3698), items 1 and 4: passes run one after
+   * another and hand their q/k/v to the attention as they are produced. */
+  int64_t pass_stride_q;
+  int64_t pass_stride_kv;
 } ttt_attn_desc;
 
 /* Descriptor flags. */

@@ -77,6 +77,25 @@ def test_invalid_descriptor(L, field, value, status):
     assert st == status
 
 
+@pytest.mark.parametrize("field", ["pass_stride_q", "pass_stride_kv"])
+def test_pass_stride_validation(L, field):
+    """A non-zero pass stride must be a multiple of 8 elements and no shorter than a packed
+    pass; it does not change the workspace (the rotated copies are packed); with P = 1 it
+    is ignored."""
+    packed = 8192 * (32 if field == "pass_stride_q" else 8) * 128
+    base = L.ttt_attn_workspace_size(ctypes.byref(desc()), 1)
+    for value, ok in ((packed, True), (packed + 8, True), (3 * packed, True), (packed - 8, False),
+                      (packed + 4, False), (-8, False)):
+        d = desc(**{field: value})
+        assert (L.ttt_attn_workspace_size(ctypes.byref(d), 1) == base) == ok, value
+        if not ok:
+            fake = ctypes.c_void_p(1 << 20)
+            st = L.ttt_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, fake, 1 << 40, None)
+            assert st == _lib.TTT_ERR_INVALID_ARG
+    d = desc(P=1, **{field: 5})
+    assert L.ttt_attn_workspace_size(ctypes.byref(d), 0) > 0
+
+
 def test_known_flags_accepted(L):
     for f in (_lib.TTT_FLAG_ROTATED_IN_WORKSPACE, _lib.TTT_FLAG_DETERMINISTIC_DQ,
               _lib.TTT_FLAG_ROTATED_IN_WORKSPACE | _lib.TTT_FLAG_DETERMINISTIC_DQ):

@@ -222,6 +222,59 @@ def test_long_32k_outputs_finite():
     assert torch.isfinite(gpu["lse"]).all()
 
 
+# ----------------------------------------------------------------------------- per-pass strides
+
+def _pass_slots(t: torch.Tensor, pad: int) -> torch.Tensor:
+    """Each pass written into its own slot of one larger buffer, slots `pad` elements apart
+    beyond a packed pass: what a caller that produces the passes one at a time does
+    instead of concatenating them."""
+    P = t.shape[0]
+    per = t[0].numel()
+    buf = torch.full(((P - 1) * (per + pad) + per,), float("nan"), dtype=t.dtype, device=t.device)
+    view = buf.as_strided(t.shape, (per + pad,) + t[0].stride())
+    for p in range(P):
+        view[p].copy_(t[p])
+    return view
+
+
+@needs_cuda
+@pytest.mark.parametrize("layout", ["dense", "thd"])
+def test_pass_strided_inputs(layout):
+    """pass_stride_q / pass_stride_kv: q, k, v, dO with their passes at a padded common
+    stride (different for the q and the kv kind), outputs allocated at the same strides.
+    Against the oracle, and o, lse, dk, dv bit-identical to the packed call (same kernels;
+    dq sums its fp32 partials in an unfixed order); the padding is never written."""
+    from attention_pass_rope_b200 import ops
+    if layout == "dense":
+        w = ttt_inputs.dense("strided", 2, 200, 3, 4, 2, 128, 1e4)
+    else:
+        w = ttt_inputs.thd("strided_thd", [129, 1, 300, 64], 4, 8, 2, 64, 1e6)
+    inp = ttt_inputs.make_inputs(w)
+    q, k, v, do, cu = parity.gpu_shapes(w, inp)
+    kw = dict(theta=w.theta, cu_seqlens=cu, max_seqlen=None if w.dense else w.max_seqlen)
+    qs, dos = _pass_slots(q, 8 * 37), _pass_slots(do, 8 * 37)
+    ks, vs = _pass_slots(k, 8 * 5), _pass_slots(v, 8 * 5)
+    assert not qs.is_contiguous() and not ks.is_contiguous()
+    o, lse = ops.ttt_attn_fwd(qs, ks, vs, **kw)
+    dq, dk, dv = ops.ttt_attn_bwd(qs, ks, vs, o, lse, dos, **kw)
+    torch.cuda.synchronize()
+    assert o.stride(0) == qs.stride(0) and dq.stride(0) == qs.stride(0) and dk.stride(0) == ks.stride(0)
+    gpu = {"o": parity.flat(o, w), "lse": lse, "dq": parity.flat(dq, w), "dk": parity.flat(dk, w),
+           "dv": parity.flat(dv, w)}
+    m = parity.compare_full(w, inp, gpu)
+    print(layout, "strided", m)
+    parity.assert_within(m)
+    o_ref, lse_ref = ops.ttt_attn_fwd(q, k, v, **kw)
+    _, dk_ref, dv_ref = ops.ttt_attn_bwd(q, k, v, o_ref, lse_ref, do, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    assert torch.equal(dk, dk_ref) and torch.equal(dv, dv_ref)
+    # the inputs' padding is untouched (still NaN) and nothing was read from it
+    per = qs[0].numel()
+    gap = qs.as_strided((qs.shape[0] - 1, qs.stride(0) - per), (qs.stride(0), 1), per)
+    assert torch.isnan(gap.float()).all()
+
+
 # ----------------------------------------------------------------------------- reuse of the rotation
 
 @needs_cuda
