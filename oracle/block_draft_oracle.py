@@ -24,6 +24,11 @@ The page gives the pattern in one line.  Readings where it is silent:
 * RoPE is rotate-half at the token's position (trunk key t at t, block token j
   at a+j), the same frequencies as the TTT attention; the softmax scale is
   1/sqrt(D) unless given; query head h reads KV head h // (H // Hkv).
+* ``rope_round="bf16"`` rounds the rotated queries and keys to bf16 (round to
+  nearest even) before the dot products, the library's defined semantics for
+  this attention as for the TTT attention (bf16 operands into the tensor cores);
+  the default ``None`` keeps them exact.  Gradients treat the rounding as the
+  identity.
 
 Array conventions (one sequence): trunk k_ctx, v_ctx [L, Hkv, D]; anchors [nb]
 (ints in 0..L-1); block qb [nb, Bs, H, D], kb, vb [nb, Bs, Hkv, D].  Outputs:
@@ -44,21 +49,26 @@ import math
 
 import numpy as np
 
-from oracle.ttt_oracle import rope_rotate
+from oracle.ttt_oracle import bf16_round, rope_rotate
 
 
 def _scale(D, scale):
     return 1.0 / math.sqrt(D) if scale is None else float(scale)
 
 
-def _rotate(k_ctx, anchors, qb, kb, theta, pos_offset=0):
-    """RoPE at the tokens' positions: trunk key t at t, block token j at anchor + j."""
+def _rotate(k_ctx, anchors, qb, kb, theta, pos_offset=0, rope_round=None):
+    """RoPE at the tokens' positions: trunk key t at t, block token j at anchor + j;
+    ``rope_round="bf16"`` rounds the rotated arrays to bf16."""
     L = k_ctx.shape[0]
     nb, Bs = qb.shape[:2]
     kt = rope_rotate(k_ctx, np.arange(L) + pos_offset, theta)
     pos_b = (np.asarray(anchors)[:, None] + np.arange(Bs)[None, :] + pos_offset).reshape(-1)
     qr = rope_rotate(qb.reshape(nb * Bs, *qb.shape[2:]), pos_b, theta).reshape(qb.shape)
     kr = rope_rotate(kb.reshape(nb * Bs, *kb.shape[2:]), pos_b, theta).reshape(kb.shape)
+    if rope_round == "bf16":
+        kt, qr, kr = bf16_round(kt), bf16_round(qr), bf16_round(kr)
+    elif rope_round is not None:
+        raise ValueError(rope_round)
     return kt, qr, kr
 
 
@@ -74,12 +84,12 @@ def block_mask(L, anchors, Bs):
     return m
 
 
-def forward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_offset=0):
+def forward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_offset=0, rope_round=None):
     L, Hkv, D = k_ctx.shape
     nb, Bs, H, _ = qb.shape
     g = H // Hkv
     sc = _scale(D, scale)
-    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset)
+    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset, rope_round)
     K = np.concatenate([kt, kr.reshape(nb * Bs, Hkv, D)])      # [L + nb*Bs, Hkv, D]
     V = np.concatenate([v_ctx, vb.reshape(nb * Bs, Hkv, D)])
     Q = qr.reshape(nb * Bs, H, D)
@@ -97,13 +107,14 @@ def forward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos
     return O.reshape(nb, Bs, H, D), lse.reshape(H, nb, Bs).transpose(1, 0, 2)
 
 
-def backward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, do, theta, scale=None, pos_offset=0):
+def backward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, do, theta, scale=None, pos_offset=0,
+                        rope_round=None):
     """Gradients with respect to the pre-RoPE inputs: (dqb, dk_ctx, dv_ctx, dkb, dvb)."""
     L, Hkv, D = k_ctx.shape
     nb, Bs, H, _ = qb.shape
     g = H // Hkv
     sc = _scale(D, scale)
-    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset)
+    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset, rope_round)
     K = np.concatenate([kt, kr.reshape(nb * Bs, Hkv, D)])
     V = np.concatenate([v_ctx, vb.reshape(nb * Bs, Hkv, D)])
     Q = qr.reshape(nb * Bs, H, D)
@@ -130,13 +141,14 @@ def backward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, do, theta, scale=None
     return dqb, dk_ctx, dV[:L], dkb, dV[L:].reshape(vb.shape)
 
 
-def forward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_offset=0, return_parts=False):
+def forward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_offset=0, return_parts=False,
+                    rope_round=None):
     """Per block: trunk softmax over t <= anchor, block softmax over its Bs keys, merged."""
     L, Hkv, D = k_ctx.shape
     nb, Bs, H, _ = qb.shape
     g = H // Hkv
     sc = _scale(D, scale)
-    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset)
+    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset, rope_round)
     O = np.zeros((nb, Bs, H, D))
     lse = np.zeros((nb, H, Bs))
     parts = []
@@ -160,14 +172,15 @@ def forward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_of
     return (O, lse, parts) if return_parts else (O, lse)
 
 
-def backward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, do, O, lse, theta, scale=None, pos_offset=0):
+def backward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, do, O, lse, theta, scale=None, pos_offset=0,
+                     rope_round=None):
     """Gradients from the merged lse: P = exp(s - lse) for both parts,
     delta = rowsum(dO * O), dS = P (dP - delta)."""
     L, Hkv, D = k_ctx.shape
     nb, Bs, H, _ = qb.shape
     g = H // Hkv
     sc = _scale(D, scale)
-    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset)
+    kt, qr, kr = _rotate(k_ctx, anchors, qb, kb, theta, pos_offset, rope_round)
     dqr = np.zeros_like(qr)
     dkt = np.zeros_like(kt)
     dvt = np.zeros_like(v_ctx)

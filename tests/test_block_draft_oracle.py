@@ -44,23 +44,48 @@ def test_twopart_equals_bruteforce(shape):
         np.testing.assert_allclose(a, b, atol=1e-12)
 
 
-def test_equals_masked_sdpa():
+@pytest.mark.parametrize("shape", [dict(), dict(L=9, nb=2, Bs=7, H=3, Hkv=1, D=16)])
+def test_bf16_rounded_rotation_forms_agree(shape):
+    """rope_round="bf16": the brute-force and two-part forms round the same rotated
+    arrays, so they still agree, forward and backward."""
+    c = case(**shape)
+    O1, l1 = bd.forward_bruteforce(theta=1e4, rope_round="bf16", **c)
+    O2, l2 = bd.forward_twopart(theta=1e4, rope_round="bf16", **c)
+    np.testing.assert_allclose(O2, O1, atol=1e-13)
+    np.testing.assert_allclose(l2, l1, atol=1e-13)
+    do = rnd(*O1.shape)
+    g1 = bd.backward_bruteforce(theta=1e4, do=do, rope_round="bf16", **c)
+    g2 = bd.backward_twopart(theta=1e4, do=do, O=O2, lse=l2, rope_round="bf16", **c)
+    for a, b in zip(g2, g1):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+def _bf16_ste(x):
+    """torch's own bf16 cast in the forward, identity in the backward."""
+    return x + (x.to(torch.bfloat16).double() - x).detach()
+
+
+@pytest.mark.parametrize("rope_round", [None, "bf16"])
+def test_equals_masked_sdpa(rope_round):
     """The block pattern is one masked softmax: torch SDPA (fp64) over the trunk keys and
     the block keys, rotated independently, with the visibility mask written out here,
-    outputs and autograd gradients."""
+    outputs and autograd gradients.  With rope_round="bf16" the rotated tensors go
+    through torch's bf16 cast (the gradient passing through unchanged), an independent
+    restatement of the oracle's rounding step."""
     L, Bs, H, Hkv, D, theta = 10, 3, 4, 2, 8, 1e4
     anchors = [0, 6, 9]
     c = case(L=L, Bs=Bs, H=H, Hkv=Hkv, D=D, anchors=anchors)
     nb = len(anchors)
-    O, lse = bd.forward_bruteforce(theta=theta, **c)
+    O, lse = bd.forward_bruteforce(theta=theta, rope_round=rope_round, **c)
     do = rnd(*O.shape)
-    grads = bd.backward_bruteforce(theta=theta, do=do, **c)
+    grads = bd.backward_bruteforce(theta=theta, do=do, rope_round=rope_round, **c)
+    rnd_ = _bf16_ste if rope_round == "bf16" else (lambda x: x)
 
     t = {n: torch.tensor(c[n], requires_grad=True) for n in ("k_ctx", "v_ctx", "qb", "kb", "vb")}
     pos_b = [a + j for a in anchors for j in range(Bs)]
-    q = torch_rope(t["qb"].reshape(nb * Bs, H, D), pos_b, theta)
-    k = torch.cat([torch_rope(t["k_ctx"], list(range(L)), theta),
-                   torch_rope(t["kb"].reshape(nb * Bs, Hkv, D), pos_b, theta)])
+    q = rnd_(torch_rope(t["qb"].reshape(nb * Bs, H, D), pos_b, theta))
+    k = torch.cat([rnd_(torch_rope(t["k_ctx"], list(range(L)), theta)),
+                   rnd_(torch_rope(t["kb"].reshape(nb * Bs, Hkv, D), pos_b, theta))])
     v = torch.cat([t["v_ctx"], t["vb"].reshape(nb * Bs, Hkv, D)])
     mask = torch.zeros(nb * Bs, L + nb * Bs, dtype=torch.bool)
     for b, a in enumerate(anchors):
