@@ -6,7 +6,11 @@ is its thin PyTorch binding.  Build the library with
 """
 
 from .ops import (  # noqa: F401
+    BlockLayout,
     Layout,
+    block_attention,
+    block_attn_bwd,
+    block_attn_fwd,
     device_status,
     set_wait_budget_ns,
     ttt_attention,

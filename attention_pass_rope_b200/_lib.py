@@ -50,6 +50,31 @@ class TTTDesc(ctypes.Structure):
     ]
 
 
+class TTTBlockDesc(ctypes.Structure):
+    _fields_ = [
+        ("layout", ctypes.c_int),
+        ("B", ctypes.c_int),
+        ("S", ctypes.c_int),
+        ("nblk", ctypes.c_int),
+        ("H", ctypes.c_int),
+        ("Hkv", ctypes.c_int),
+        ("D", ctypes.c_int),
+        ("Bs", ctypes.c_int),
+        ("rope_theta", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float),
+        ("anchors", ctypes.c_void_p),
+        ("cu_ctx", ctypes.c_void_p),
+        ("cu_blocks", ctypes.c_void_p),
+        ("nseq", ctypes.c_int),
+        ("total_ctx", ctypes.c_int),
+        ("total_blocks", ctypes.c_int),
+        ("max_ctx", ctypes.c_int),
+        ("max_blocks", ctypes.c_int),
+        ("events", ctypes.c_void_p),
+        ("flags", ctypes.c_int),
+    ]
+
+
 class TTTError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -99,6 +124,15 @@ def lib() -> ctypes.CDLL:
     L.ttt_attn_noalloc_watchdog_selftest.restype = ctypes.c_int
     L.ttt_attn_set_wait_budget_ns.argtypes = [u64]
     L.ttt_attn_set_wait_budget_ns.restype = None
+    BD = P(TTTBlockDesc)
+    L.ttt_block_workspace_size.argtypes = [BD, ctypes.c_int]
+    L.ttt_block_workspace_size.restype = sz
+    L.ttt_block_workspace_layout.argtypes = [BD, ctypes.c_int, P(sz)]
+    L.ttt_block_workspace_layout.restype = ctypes.c_int
+    L.ttt_block_attn_fwd.argtypes = [BD, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.ttt_block_attn_fwd.restype = ctypes.c_int
+    L.ttt_block_attn_bwd.argtypes = [BD] + [vp] * 14 + [sz, vp]
+    L.ttt_block_attn_bwd.restype = ctypes.c_int
     L.ttt_status_string.argtypes = [ctypes.c_int]
     L.ttt_status_string.restype = ctypes.c_char_p
     L.ttt_attn_version.argtypes = []

@@ -65,6 +65,10 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
     g.si.T = d->total_tokens;
     g.si.max_len = d->max_seqlen;
   }
+  g.si.mult = 1;
+  g.ksi = g.si;  // queries and keys index the same tokens
+  g.Bs = 0;
+  g.anchors = nullptr;
   // index arithmetic in the kernels: P*H*T*D elements must fit comfortably in int64,
   // per-pass offsets in int32 where they are formed that way
   const long long rows = static_cast<long long>(g.P) * g.H * g.si.T;
@@ -102,11 +106,83 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
     o = align_up(o + P * H * static_cast<size_t>(ld_slots(g.si)) * 128 * 4);
     pl.off[4] = o;  // dq~ accumulator
     o = align_up(o + P * H * T * D * 4);
-    pl.off[5] = o;  // dk~_1 accumulator
-    o = align_up(o + Hkv * T * D * 4);
-    pl.off[6] = o;  // order tickets of the dq~ additions, one per statistics slot
+    pl.off[5] = o;  // order tickets of the dq~ additions, one per statistics slot
     o = align_up(o + P * H * static_cast<size_t>(ld_slots(g.si)) * 4);
-    pl.noff = 7;
+    pl.noff = 6;
+  }
+  pl.total = o;
+  *out = pl;
+  return TTT_OK;
+}
+
+// Block-draft attention: validate, derive the two index spaces (block rows, context)
+// and the workspace layout.
+ttt_status make_block_plan(const ttt_block_desc* d, int for_backward, Plan* out) {
+  if (!d) return TTT_ERR_INVALID_ARG;
+  Plan pl{};
+  Geometry& g = pl.g;
+  if (d->layout != TTT_LAYOUT_BSHD && d->layout != TTT_LAYOUT_THD) return TTT_ERR_INVALID_ARG;
+  if (d->H < 1 || d->Hkv < 1 || d->D < 1 || d->Bs < 1) return TTT_ERR_INVALID_ARG;
+  if (d->H % d->Hkv != 0) return TTT_ERR_INVALID_ARG;
+  if (d->Bs > 16) return TTT_ERR_UNSUPPORTED;
+  if (d->D != 64 && d->D != 128) return TTT_ERR_UNSUPPORTED;
+  if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return TTT_ERR_INVALID_ARG;
+  if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return TTT_ERR_INVALID_ARG;
+  if (d->flags & ~static_cast<int>(TTT_FLAG_ROTATED_IN_WORKSPACE | TTT_FLAG_DETERMINISTIC_DQ))
+    return TTT_ERR_INVALID_ARG;
+  g.P = 1;
+  g.H = d->H;
+  g.Hkv = d->Hkv;
+  g.D = d->D;
+  g.theta = d->rope_theta;
+  g.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt(static_cast<float>(d->D));
+  g.Bs = d->Bs;
+  g.anchors = d->anchors;
+  if (d->layout == TTT_LAYOUT_BSHD) {
+    if (d->B < 0 || d->S < 0 || d->nblk < 0) return TTT_ERR_INVALID_ARG;
+    const long long Tc = static_cast<long long>(d->B) * d->S;
+    const long long NQ = static_cast<long long>(d->B) * d->nblk * d->Bs;
+    if (Tc > (1LL << 30) || NQ > (1LL << 30)) return TTT_ERR_UNSUPPORTED;
+    if (d->nblk > 0 && d->S < 1) return TTT_ERR_INVALID_ARG;  // a block needs a context to anchor in
+    g.ksi = SeqInfo{nullptr, d->B, d->S, static_cast<int>(Tc), d->S, 1};
+    g.si = SeqInfo{nullptr, d->B, d->nblk * d->Bs, static_cast<int>(NQ), d->nblk * d->Bs, 1};
+  } else {
+    if (d->nseq < 0 || d->total_ctx < 0 || d->total_blocks < 0 || d->max_ctx < 0 || d->max_blocks < 0)
+      return TTT_ERR_INVALID_ARG;
+    if (d->total_blocks > 0 && (!d->cu_ctx || !d->cu_blocks || d->nseq < 1 || d->max_blocks < 1 || d->max_ctx < 1))
+      return TTT_ERR_INVALID_ARG;
+    if (d->max_ctx > d->total_ctx || d->max_blocks > d->total_blocks) return TTT_ERR_INVALID_ARG;
+    const long long NQ = static_cast<long long>(d->total_blocks) * d->Bs;
+    if (d->total_ctx > (1 << 30) || NQ > (1LL << 30)) return TTT_ERR_UNSUPPORTED;
+    g.ksi = SeqInfo{d->cu_ctx, d->nseq, 0, d->total_ctx, d->max_ctx, 1};
+    g.si = SeqInfo{d->cu_blocks, d->nseq, 0, static_cast<int>(NQ), d->max_blocks * d->Bs, d->Bs};
+  }
+  if (g.si.T > 0 && !g.anchors) return TTT_ERR_INVALID_ARG;
+  g.sq = static_cast<int64_t>(g.si.T) * g.H * g.D;
+  g.skv = static_cast<int64_t>(g.ksi.T) * g.Hkv * g.D;
+  const size_t NQ = static_cast<size_t>(g.si.T), Tc = static_cast<size_t>(g.ksi.T);
+  const size_t H = g.H, Hkv = g.Hkv, D = g.D;
+  size_t o = 0;
+  pl.off[0] = 0;
+  o = align_up(256);
+  pl.off[1] = o;  // q~ of the block tokens
+  o = align_up(o + H * NQ * D * 2);
+  pl.off[2] = o;  // k~ of the context
+  o = align_up(o + Hkv * Tc * D * 2);
+  pl.off[3] = o;  // k~ of the block tokens
+  o = align_up(o + Hkv * NQ * D * 2);
+  if (!for_backward) {
+    pl.noff = 4;
+  } else {
+    pl.off[4] = o;  // row statistics over the block rows
+    o = align_up(o + H * static_cast<size_t>(ld_slots(g.si)) * 128 * 4);
+    pl.off[5] = o;  // dq~ accumulator
+    o = align_up(o + H * NQ * D * 4);
+    pl.off[6] = o;  // order tickets
+    o = align_up(o + H * static_cast<size_t>(ld_slots(g.si)) * 4);
+    pl.off[7] = o;  // trunk-key limit of every block row
+    o = align_up(o + NQ * 4);
+    pl.noff = 8;
   }
   pl.total = o;
   *out = pl;
@@ -283,8 +359,7 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   void* kr = ws + pl.off[2];
   float* ld = reinterpret_cast<float*>(ws + pl.off[3]);
   float* dq_acc = reinterpret_cast<float*>(ws + pl.off[4]);
-  float* dk1_acc = reinterpret_cast<float*>(ws + pl.off[5]);
-  int* tickets = reinterpret_cast<int*>(ws + pl.off[6]);
+  int* tickets = reinterpret_cast<int*>(ws + pl.off[5]);
   const bool deterministic = (desc->flags & TTT_FLAG_DETERMINISTIC_DQ) != 0;
   const uint64_t T = g.si.T, D = g.D;
 
@@ -306,16 +381,136 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
-    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, stream));
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, nullptr, status, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);
-    TrunkBwdArgs a{g, ld, dq_acc, dk1_acc, dv, deterministic ? tickets : nullptr, status, g_wait_budget_ns.load()};
+    TrunkBwdArgs a{g, ld, dq_acc, dk, dv, deterministic ? tickets : nullptr, nullptr, status, g_wait_budget_ns.load()};
     TTT_CHECK_CUDA(launch_trunk_bwd(a, mq, mk, mv, mdo, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BRANCH_BWD, stream);
-    TTT_CHECK_CUDA(launch_branch_bwd(g, qr, kr, v, dout, lse, ld, dq_acc, dk1_acc, dq, dk, dv, stream));
+    TTT_CHECK_CUDA(launch_branch_bwd(g, qr, kr, v, dout, lse, ld, dq_acc, dq, dk, dv, stream));
+  }
+  return TTT_OK;
+}
+
+size_t ttt_block_workspace_size(const ttt_block_desc* desc, int for_backward) {
+  Plan pl;
+  if (make_block_plan(desc, for_backward, &pl) != TTT_OK) return 0;
+  return pl.total;
+}
+
+int ttt_block_workspace_layout(const ttt_block_desc* desc, int for_backward, size_t* offsets) {
+  Plan pl;
+  if (!offsets || make_block_plan(desc, for_backward, &pl) != TTT_OK) return 0;
+  for (int i = 0; i < pl.noff; ++i) offsets[i] = pl.off[i];
+  return pl.noff;
+}
+
+ttt_status ttt_block_attn_fwd(const ttt_block_desc* desc, const void* k_ctx, const void* v_ctx, const void* qb,
+                              const void* kb, const void* vb, void* o, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream_) {
+  Plan pl;
+  ttt_status st = make_block_plan(desc, 0, &pl);
+  if (st != TTT_OK) return st;
+  const Geometry& g = pl.g;
+  if (g.si.T == 0) return TTT_OK;
+  if (!k_ctx || !v_ctx || !qb || !kb || !vb || !o || !lse) return TTT_ERR_INVALID_ARG;
+  if (!ptr_aligned(k_ctx, 16) || !ptr_aligned(v_ctx, 16) || !ptr_aligned(qb, 16) || !ptr_aligned(kb, 16) ||
+      !ptr_aligned(vb, 16) || !ptr_aligned(o, 16) || !ptr_aligned(lse, 4))
+    return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + pl.off[0]);
+  void* qr = ws + pl.off[1];
+  void* kr_ctx = ws + pl.off[2];
+  void* kr_blk = ws + pl.off[3];
+  const uint64_t NQ = g.si.T, Tc = g.ksi.T, D = g.D;
+  clear_stale_error();
+  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, qr, D, NQ, g.H, D * 2, NQ * D * 2, 128, 1) ||
+      !make_map(&mk, kr_ctx, D, Tc, g.Hkv, D * 2, Tc * D * 2, 128, 1) ||
+      !make_map(&mv, v_ctx, D, g.Hkv, Tc, D * 2, g.Hkv * D * 2, 1, 128))
+    return TTT_ERR_CUDA;
+  {
+    EventScope es(desc->events, TTT_KERNEL_ROPE_FWD, stream);
+    TTT_CHECK_CUDA(launch_rope_rows(g, false, g.ksi.T, k_ctx, g.Hkv, kr_ctx, nullptr, 0, nullptr, stream));
+    TTT_CHECK_CUDA(launch_rope_rows(g, true, g.si.T, qb, g.H, qr, kb, g.Hkv, kr_blk, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
+    TrunkFwdArgs a{g, kr_blk, vb, o, lse, status, g_wait_budget_ns.load()};
+    TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
+  }
+  return TTT_OK;
+}
+
+ttt_status ttt_block_attn_bwd(const ttt_block_desc* desc, const void* k_ctx, const void* v_ctx, const void* qb,
+                              const void* kb, const void* vb, const void* o, const float* lse, const void* dout,
+                              void* dk_ctx, void* dv_ctx, void* dqb, void* dkb, void* dvb, void* workspace,
+                              size_t workspace_bytes, void* stream_) {
+  Plan pl;
+  ttt_status st = make_block_plan(desc, 1, &pl);
+  if (st != TTT_OK) return st;
+  const Geometry& g = pl.g;
+  if (g.si.T == 0 && g.ksi.T == 0) return TTT_OK;
+  if (!k_ctx || !v_ctx || !o || !lse || !dout || !dk_ctx || !dv_ctx) return TTT_ERR_INVALID_ARG;
+  if (g.si.T > 0 && (!qb || !kb || !vb || !dqb || !dkb || !dvb)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {k_ctx, v_ctx, qb, kb, vb, o, dout, dk_ctx, dv_ctx, dqb, dkb, dvb};
+  for (const void* p : ptrs)
+    if (!ptr_aligned(p, 16)) return TTT_ERR_INVALID_ARG;
+  if (!ptr_aligned(lse, 4)) return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + pl.off[0]);
+  void* qr = ws + pl.off[1];
+  void* kr_ctx = ws + pl.off[2];
+  void* kr_blk = ws + pl.off[3];
+  float* ld = reinterpret_cast<float*>(ws + pl.off[4]);
+  float* dq_acc = reinterpret_cast<float*>(ws + pl.off[5]);
+  int* tickets = reinterpret_cast<int*>(ws + pl.off[6]);
+  int* qlim = reinterpret_cast<int*>(ws + pl.off[7]);
+  const bool deterministic = (desc->flags & TTT_FLAG_DETERMINISTIC_DQ) != 0;
+  const uint64_t NQ = g.si.T, Tc = g.ksi.T, D = g.D;
+  clear_stale_error();
+  TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  if (g.si.T == 0) {
+    // no block: no context key is seen
+    TTT_CHECK_CUDA(cudaMemsetAsync(dk_ctx, 0, Tc * g.Hkv * D * 2, stream));
+    TTT_CHECK_CUDA(cudaMemsetAsync(dv_ctx, 0, Tc * g.Hkv * D * 2, stream));
+    return TTT_OK;
+  }
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, qr, D, NQ, g.H, D * 2, NQ * D * 2, 64, 1) ||
+      !make_map(&mk, kr_ctx, D, Tc, g.Hkv, D * 2, Tc * D * 2, 128, 1) ||
+      !make_map(&mv, v_ctx, D, g.Hkv, Tc, D * 2, g.Hkv * D * 2, 1, 128) ||
+      !make_map4(&mdo, dout, {D, static_cast<uint64_t>(g.H), NQ, 1}, {D * 2, g.H * D * 2, NQ * g.H * D * 2},
+                 {1, 64, 1}))
+    return TTT_ERR_CUDA;
+  {
+    EventScope es(desc->events, TTT_KERNEL_ROPE_BWD, stream);
+    if (!(desc->flags & TTT_FLAG_ROTATED_IN_WORKSPACE)) {
+      TTT_CHECK_CUDA(launch_rope_rows(g, false, g.ksi.T, k_ctx, g.Hkv, kr_ctx, nullptr, 0, nullptr, stream));
+      TTT_CHECK_CUDA(launch_rope_rows(g, true, g.si.T, qb, g.H, qr, kb, g.Hkv, kr_blk, stream));
+    }
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, qlim, status, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);
+    TrunkBwdArgs a{g, ld, dq_acc, dk_ctx, dv_ctx, deterministic ? tickets : nullptr, qlim, status,
+                   g_wait_budget_ns.load()};
+    TTT_CHECK_CUDA(launch_trunk_bwd(a, mq, mk, mv, mdo, stream));
+  }
+  {
+    EventScope es(desc->events, TTT_KERNEL_BRANCH_BWD, stream);
+    TTT_CHECK_CUDA(launch_block_bwd(g, qr, kr_blk, vb, dout, lse, ld, dq_acc, dqb, dkb, dvb, stream));
   }
   return TTT_OK;
 }
@@ -332,7 +527,7 @@ ttt_status ttt_attn_device_status(void* workspace, void* stream_, uint32_t* deta
   if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), stream) != cudaSuccess ||
       cudaStreamSynchronize(stream) != cudaSuccess)
     return TTT_ERR_CUDA;
-  return TTT_ERR_DEVICE_TIMEOUT;
+  return word == kStatusBadAnchors ? TTT_ERR_INVALID_ARG : TTT_ERR_DEVICE_TIMEOUT;
 }
 
 ttt_status ttt_attn_watchdog_selftest(void* workspace, size_t workspace_bytes, uint64_t budget_ns, void* stream_) {

@@ -99,7 +99,7 @@ template <int D>
 __global__ void __launch_bounds__(kPreThreads)
     bwd_preprocess_kernel(Geometry g, const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                           const float* __restrict__ lse, float* __restrict__ ld, float* __restrict__ dq_acc,
-                          int* __restrict__ tickets, int ntile) {
+                          int* __restrict__ tickets, int ntile, int* __restrict__ qlim, uint32_t* status) {
   constexpr int LPR = D / 8;                            // lanes per row
   constexpr int RPI = 32 / LPR;                         // rows per warp instruction
   constexpr int RPWARP = kPreRows / (kPreThreads / 32);  // rows per warp (8)
@@ -154,6 +154,16 @@ __global__ void __launch_bounds__(kPreThreads)
   const int64_t slot_index = (static_cast<int64_t>(p) * g.H + h) * ld_slots(g.si) + ld_slot(start, n, pos0);
   float* slot = ld + slot_index * 128;
   if (threadIdx.x == 0) tickets[slot_index] = 0;
+  if (qlim && h == 0 && threadIdx.x < nvalid) {
+    // block-draft rows: the trunk-key limit of each row (its block's clamped anchor), and
+    // the anchors' order, which the trunk backward's tile walk relies on
+    int kstart, klen;
+    seq_bounds(g.ksi, n, kstart, klen);
+    const int r = pos0 + threadIdx.x;
+    qlim[start + r] = block_row_limit(g, start, r, klen);
+    if (r % g.Bs == 0 && r >= g.Bs && g.anchors[(start + r) / g.Bs] < g.anchors[(start + r) / g.Bs - 1])
+      atomicCAS(status, 0u, kStatusBadAnchors);
+  }
   if (threadIdx.x < nvalid) {
     const int i = threadIdx.x;
     slot[i] = lse[lse_index(g.si, g.H, p, h, n, start + pos0 + i, pos0 + i)] * -1.4426950408889634f;
@@ -168,8 +178,8 @@ __global__ void __launch_bounds__(kPreThreads)
 //     dS_j = P_j (dO . V_j - delta),  P_j = exp(sigma q~ . k~_j - lse)
 //     dk~_j += dS_j q~,  dV_j += P_j dO                   (accumulated over p >= j, h)
 //     dQ_p = R(i+p)^T (sigma dq~)
-//   dK_j = R(i+j)^T (sigma dk~_j)  for every pass (j = 0 takes dk~_1 from the trunk
-//   backward), dV_j for j >= 1 (dV_1 is written by the trunk backward).
+//   dK_j = R(i+j)^T (sigma dk~_j) and dV_j for the branch passes j >= 1 (dK_1 and dV_1
+//   are written by the trunk backward).
 // The kernel is bound by memory latency, so resident warps matter most: the group
 // heads of a pass go kBranchHeads at a time (one: more heads per warp keep more rows
 // in flight but cost registers, and 64 registers at four blocks per SM measured
@@ -178,21 +188,12 @@ __global__ void __launch_bounds__(kPreThreads)
 // ---------------------------------------------------------------------------
 constexpr int kBranchHeads = 1;
 
-// cos/sin of pos * inv_freq: the angle in double, reduced by whole turns in double,
-// then the single-precision sincosf of the remainder (|remainder| <= pi).
-__device__ __forceinline__ void angle_cos_sin(int pos, double inv_freq, float& c, float& s) {
-  const double ang = static_cast<double>(pos) * inv_freq;
-  const double turns = rint(ang * 0.15915494309189535);  // 1 / (2 pi)
-  const double red = fma(-turns, 6.283185307179586, ang);
-  sincosf(static_cast<float>(red), &s, &c);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
     branch_bwd_kernel(Geometry g, const __nv_bfloat16* __restrict__ qr, const __nv_bfloat16* __restrict__ kr,
                       const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ ld,
-                      const float* __restrict__ dq_acc, const float* __restrict__ dk1_acc,
+                      const float* __restrict__ dq_acc,
                       __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
   constexpr int E = D / 64;
   extern __shared__ __align__(16) unsigned char branch_smem[];
@@ -318,38 +319,26 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
       }
     }
   }
-  // dK of every pass (trunk from the trunk backward), dV of the branch passes
-  for (int j = 0; j < g.P; ++j) {
+  // dK and dV of the branch passes (those of the trunk pass come from the trunk backward)
+  for (int j = 1; j < g.P; ++j) {
     float c[E], sn[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       c[e] = cs[j * D + LaneMap<D>::d(lane, 0, e)];
       sn[e] = cs[j * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
     }
-    float kx[2][E];
-    if (j == 0) {
-      load_f32_row<D>(dk1_acc + (static_cast<int64_t>(kvh) * T + tau) * D, lane, kx);
-    } else {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int e = 0; e < E; ++e) kx[hh][e] = acc[((j - 1) * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)];
-    }
+    float kx[2][E], vx[2][E];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-      for (int e = 0; e < E; ++e) kx[hh][e] *= g.scale;
+      for (int e = 0; e < E; ++e) {
+        kx[hh][e] = acc[((j - 1) * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] * g.scale;
+        vx[hh][e] = acc[((j - 1) * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)];
+      }
     rotate_back<D>(kx, c, sn);
     const int64_t krow = j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D;
     store_bf16_row<D>(dk + krow, lane, kx);
-    if (j > 0) {
-      float vx[2][E];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int e = 0; e < E; ++e) vx[hh][e] = acc[((j - 1) * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)];
-      store_bf16_row<D>(dv + krow, lane, vx);
-    }
+    store_bf16_row<D>(dv + krow, lane, vx);
   }
 }
 
@@ -379,7 +368,7 @@ inline unsigned blocks_for(int64_t warps) {
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  float* dq_acc, int* tickets, cudaStream_t stream) {
+                                  float* dq_acc, int* tickets, int* qlim, uint32_t* status, cudaStream_t stream) {
   if (g.si.T == 0 || g.si.nseq == 0 || g.si.max_len == 0) return cudaSuccess;
   const int ntile = (g.si.max_len + kPreRows - 1) / kPreRows;
   const long long blocks = static_cast<long long>(g.P) * g.si.nseq * ntile * g.H;
@@ -388,16 +377,16 @@ cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* 
   auto* db = static_cast<const __nv_bfloat16*>(dout);
   if (g.D == 128)
     bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
-                                                                                       tickets, ntile);
+                                                                                       tickets, ntile, qlim, status);
   else
     bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
-                                                                                      tickets, ntile);
+                                                                                      tickets, ntile, qlim, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr, const void* v, const void* dout,
-                              const float* lse, const float* ld, const float* dq_acc, const float* dk1_acc,
-                              void* dq, void* dk, void* dv, cudaStream_t stream) {
+                              const float* lse, const float* ld, const float* dq_acc, void* dq, void* dk, void* dv,
+                              cudaStream_t stream) {
   const int64_t warps = static_cast<int64_t>(g.si.T) * g.Hkv;
   if (warps == 0) return cudaSuccess;
   const int NB = g.P - 1 > 0 ? g.P - 1 : 1;
@@ -415,12 +404,12 @@ cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr,
     e = cudaFuncSetAttribute(branch_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     branch_bwd_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, ld,
-                                                                                      dq_acc, dk1_acc, dqb, dkb, dvb);
+                                                                                      dq_acc, dqb, dkb, dvb);
   } else {
     e = cudaFuncSetAttribute(branch_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     branch_bwd_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, ld,
-                                                                                     dq_acc, dk1_acc, dqb, dkb, dvb);
+                                                                                     dq_acc, dqb, dkb, dvb);
   }
   return cudaGetLastError();
 }

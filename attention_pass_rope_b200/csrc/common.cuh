@@ -400,8 +400,8 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
 // packed (THD) batches read cu_seqlens.
 __device__ __forceinline__ void seq_bounds(const SeqInfo& si, int n, int& start, int& len) {
   if (si.cu_seqlens) {
-    start = si.cu_seqlens[n];
-    len = si.cu_seqlens[n + 1] - start;
+    start = si.cu_seqlens[n] * si.mult;
+    len = si.cu_seqlens[n + 1] * si.mult - start;
   } else {
     start = n * si.S;
     len = si.S;
@@ -414,13 +414,13 @@ __device__ __forceinline__ void token_position(const SeqInfo& si, int tau, int& 
     int lo = 0, hi = si.nseq - 1;
     while (lo < hi) {
       int mid = (lo + hi + 1) >> 1;
-      if (si.cu_seqlens[mid] <= tau)
+      if (si.cu_seqlens[mid] * si.mult <= tau)
         lo = mid;
       else
         hi = mid - 1;
     }
     n = lo;
-    pos = tau - si.cu_seqlens[lo];
+    pos = tau - si.cu_seqlens[lo] * si.mult;
   } else {
     n = tau / si.S;
     pos = tau - n * si.S;
@@ -432,6 +432,29 @@ __device__ __forceinline__ void token_position(const SeqInfo& si, int tau, int& 
 __device__ __forceinline__ int64_t lse_index(const SeqInfo& si, int H, int p, int h, int n, int tau, int pos) {
   if (si.cu_seqlens) return (static_cast<int64_t>(p) * H + h) * si.T + tau;
   return ((static_cast<int64_t>(p) * si.nseq + n) * H + h) * si.S + pos;
+}
+
+// cos/sin of pos * inv_freq: the angle in double, reduced by whole turns in double,
+// then the single-precision sincosf of the remainder (|remainder| <= pi).
+__device__ __forceinline__ void angle_cos_sin(int pos, double inv_freq, float& c, float& s) {
+  const double ang = static_cast<double>(pos) * inv_freq;
+  const double turns = rint(ang * 0.15915494309189535);  // 1 / (2 pi)
+  const double red = fma(-turns, 6.283185307179586, ang);
+  sincosf(static_cast<float>(red), &s, &c);
+}
+
+// Trunk-key limit of block-draft query row r of a sequence whose block rows start at
+// qstart (a multiple of Bs) and whose context has klen keys: its block's anchor,
+// clamped to [0, klen - 1] (-1, no trunk key, for an empty context).
+__device__ __forceinline__ int block_row_limit(const Geometry& g, int qstart, int r, int klen) {
+  const int a = __ldg(g.anchors + (qstart + r) / g.Bs);
+  return min(max(a, 0), klen - 1);
+}
+
+// RoPE position of that row: the clamped anchor (0 for an empty context) plus the
+// row's index in its block.
+__device__ __forceinline__ int block_row_position(const Geometry& g, int qstart, int r, int klen) {
+  return max(block_row_limit(g, qstart, r, klen), 0) + r % g.Bs;
 }
 
 }  // namespace ttt

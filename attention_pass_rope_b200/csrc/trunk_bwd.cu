@@ -88,7 +88,58 @@ __device__ __forceinline__ IterInfo decode_iter(int it, int nqt, int jq0, int G,
   return r;
 }
 
+// First 64-row query tile of a block-draft sequence whose last row sees key k0
+// (anchors non-decreasing within a sequence, so the tiles that see k0 are a suffix).
+__device__ int first_tile_seeing(const Geometry& g, const int* qlim, int qstart, int qlen, int k0) {
+  int lo = 0, hi = (qlen + 63) / 64;  // answer in [lo, hi]; hi = no tile
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int last = min(mid * 64 + 63, qlen - 1);
+    if (__ldg(qlim + qstart + last) >= k0)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  return lo;
+}
+
+// dK of the trunk keys, finalised: sigma * R(pos)^T dk~ in bf16, for one key row held
+// by the calling thread as 32-column chunks (c, c + D/2 pair the RoPE dimensions).
 template <int D>
+__device__ __forceinline__ void store_dk_row(__nv_bfloat16* dst, int pos, float theta, float scale,
+                                             const uint32_t (&lo)[32], const uint32_t (&hi)[32], int c) {
+  // inverse frequencies theta^(-2d/D) for d = 32c .. 32c+31: one pow, then a ratio
+  const double ratio = pow(static_cast<double>(theta), -2.0 / D);
+  double f = pow(static_cast<double>(theta), -2.0 * (32 * c) / D);
+  uint32_t out_lo[16], out_hi[16];
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float r[2][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float cs, sn;
+      angle_cos_sin(pos, f, cs, sn);
+      f *= ratio;
+      const float x1 = __uint_as_float(lo[e + u]) * scale, x2 = __uint_as_float(hi[e + u]) * scale;
+      r[0][u] = fmaf(x1, cs, x2 * sn);
+      r[1][u] = fmaf(x2, cs, -x1 * sn);
+    }
+    out_lo[e >> 1] = pack_bf16x2(r[0][0], r[0][1]);
+    out_hi[e >> 1] = pack_bf16x2(r[1][0], r[1][1]);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    *reinterpret_cast<uint4*>(dst + 32 * c + 8 * q) =
+        make_uint4(out_lo[4 * q], out_lo[4 * q + 1], out_lo[4 * q + 2], out_lo[4 * q + 3]);
+    *reinterpret_cast<uint4*>(dst + D / 2 + 32 * c + 8 * q) =
+        make_uint4(out_hi[4 * q], out_hi[4 * q + 1], out_hi[4 * q + 2], out_hi[4 * q + 3]);
+  }
+}
+
+// MODE 0: TTT trunk (queries and keys are the same tokens, causal).  MODE 1: block-draft
+// trunk (queries are block rows, keys the context; a query row sees the keys up to its
+// block's anchor, a.qlim).
+template <int D, int MODE>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     trunk_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
@@ -107,7 +158,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   // so the q~/dO tiles they read and the dq~ rows they reduce into are shared in L2
   // (with every group in flight at once, a batch of many short sequences streams all
   // of it from DRAM), while the work per band still runs largest first.
-  const int njk = (g.si.max_len + C::BK - 1) / C::BK;
+  const int njk = (g.ksi.max_len + C::BK - 1) / C::BK;
   const int ngroups = g.si.nseq * g.Hkv;
   const int nb = max(1, 256 / njk);
   const int band = static_cast<int>(blockIdx.x) / (nb * njk);
@@ -117,15 +168,27 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int gi = band * nb + in_band % members;
   const int n = gi / g.Hkv;
   const int kvh = gi % g.Hkv;
-  int seq_start, len;
-  seq_bounds(g.si, n, seq_start, len);
+  int seq_start, len, kstart, klen;
+  seq_bounds(g.si, n, seq_start, len);  // query rows
+  seq_bounds(g.ksi, n, kstart, klen);   // key rows (the same tokens in MODE 0)
   const int k0 = jk * C::BK;
-  if (k0 >= len) return;
+  if (k0 >= klen) return;
   const int gsz = g.H / g.Hkv;
   const int G = g.P * gsz;
-  const int jq0 = k0 / C::BQ;
+  const int jq0 = MODE == 0 ? k0 / C::BQ : first_tile_seeing(g, a.qlim, seq_start, len, k0);
   const int nqt = (len + C::BQ - 1) / C::BQ - jq0;
   const int NIT = G * nqt;
+  if (NIT <= 0) {
+    // block-draft keys that no query row sees: zero gradients
+    for (int i = threadIdx.x; i < C::BK * (D / 8); i += blockDim.x) {
+      const int r = i / (D / 8), c8 = i % (D / 8);
+      if (k0 + r >= klen) continue;
+      const int64_t row = (static_cast<int64_t>(kstart + k0 + r) * g.Hkv + kvh) * D + 8 * c8;
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dk) + row) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dv) + row) = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_bar = bars + 0;
@@ -191,8 +254,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&map_do);
       mbar_arrive_expect_tx(kv_bar, 2 * C::KCH * C::KCHUNK);
       for (int c = 0; c < C::KCH; ++c) {
-        tma_load_3d(sK + c * C::KCHUNK, &map_k, kv_bar, c * 64, seq_start + k0, kvh);
-        tma_load_3d(sV + c * C::KCHUNK, &map_v, kv_bar, c * 64, kvh, seq_start + k0);
+        tma_load_3d(sK + c * C::KCHUNK, &map_k, kv_bar, c * 64, kstart + k0, kvh);
+        tma_load_3d(sV + c * C::KCHUNK, &map_v, kv_bar, c * 64, kvh, kstart + k0);
       }
     }
     if (lane == 0) {
@@ -316,7 +379,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;    // key row
     const int kpos = k0 + r;
-    const bool kvalid = kpos < len;
+    const bool kvalid = kpos < klen;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = g.scale * kLog2e;
     bool ok = true;
@@ -350,7 +413,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const float* ldp = sLD + s * 2 * C::BQ + 32 * hf;
       // interior tile: every (key, query) pair of this half is visible
       const int qlo = ii.q0 + 32 * hf;
-      const bool interior = (qlo >= k0 + C::BK - 1) && (qlo + 32 <= len) && (k0 + C::BK <= len);
+      const bool interior =
+          (qlo + 32 <= len) && (k0 + C::BK <= klen) &&
+          (MODE == 0 ? qlo >= k0 + C::BK - 1 : __ldg(a.qlim + seq_start + qlo) >= k0 + C::BK - 1);
       // P = 2^(s*scale*log2e - lse*log2e), dS = P (dP - delta), two columns per
       // instruction; the bf16 pairs are packed straight from the results
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -374,8 +439,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
           if (!interior) {
             // padding rows of the statistics are never written: select, do not multiply
-            const bool v0 = kvalid && qlo + c < len && kpos <= qlo + c;
-            const bool v1 = kvalid && qlo + c + 1 < len && kpos <= qlo + c + 1;
+            int lim0 = qlo + c, lim1 = qlo + c + 1;
+            if (MODE == 1) {
+              lim0 = qlo + c < len ? __ldg(a.qlim + seq_start + qlo + c) : -1;
+              lim1 = qlo + c + 1 < len ? __ldg(a.qlim + seq_start + qlo + c + 1) : -1;
+            }
+            const bool v0 = kvalid && qlo + c < len && kpos <= lim0;
+            const bool v1 = kvalid && qlo + c + 1 < len && kpos <= lim1;
             p0 = v0 ? p0 : 0.f;
             d0 = v0 ? d0 : 0.f;
             p1 = v1 ? p1 : 0.f;
@@ -410,18 +480,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (lane == 0 && warp == 4) TTT_TRACE(9, it);
 
     }
-    // ---- epilogue: dV (half 0) and dK~ (half 1) of this CTA's keys
+    // ---- epilogue: dV (half 0) and dK (half 1) of this CTA's keys, final: dV in bf16,
+    // dK = sigma * R(pos)^T dk~ in bf16 (the trunk keys' rotation at their own position)
     if (ok && wait_bounded(final_bar, 0, wd, kSiteBwdFinal)) {
       tc_fence_after();
-      const int64_t tau = seq_start + kpos;
+      const int64_t tau = kstart + kpos;
+      if (hf == 0) {
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(lane_base + (hf == 0 ? C::COL_DV : C::COL_DK) + 32 * c, v);
-        tmem_ld_wait();
-        reg_fence32(v);
-        if (!kvalid) continue;
-        if (hf == 0) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + C::COL_DV + 32 * c, v);
+          tmem_ld_wait();
+          reg_fence32(v);
+          if (!kvalid) continue;
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dv) + (tau * g.Hkv + kvh) * D + 32 * c;
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
@@ -431,13 +502,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                                  pack_bf16x2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
             *reinterpret_cast<uint4*>(dst + e) = w;
           }
-        } else {
-          float* dst = a.dk1_acc + (static_cast<int64_t>(kvh) * g.si.T + tau) * D + 32 * c;
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + e) =
-                make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
-                            __uint_as_float(v[e + 3]));
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t lo[32], hi[32];
+          tmem_ld32(lane_base + C::COL_DK + 32 * c, lo);
+          tmem_ld32(lane_base + C::COL_DK + D / 2 + 32 * c, hi);
+          tmem_ld_wait();
+          reg_fence32(lo);
+          reg_fence32(hi);
+          if (!kvalid) continue;
+          store_dk_row<D>(static_cast<__nv_bfloat16*>(a.dk) + (tau * g.Hkv + kvh) * D, kpos, g.theta, g.scale, lo,
+                          hi, c);
         }
       }
     }
@@ -518,17 +595,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int D>
+template <int D, int MODE>
 cudaError_t launch(const TrunkBwdArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const CUtensorMap& mdo, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(trunk_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t e =
+      cudaFuncSetAttribute(trunk_bwd_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const int njk = (a.g.si.max_len + C::BK - 1) / C::BK;
-  const long long blocks = static_cast<long long>(njk) * a.g.si.nseq * a.g.Hkv;
+  const int njk = (a.g.ksi.max_len + C::BK - 1) / C::BK;
+  const long long blocks = static_cast<long long>(njk) * a.g.ksi.nseq * a.g.Hkv;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  trunk_bwd_kernel<D><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, a);
+  trunk_bwd_kernel<D, MODE><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, a);
   return cudaGetLastError();
 }
 
@@ -536,8 +614,11 @@ cudaError_t launch(const TrunkBwdArgs& a, const CUtensorMap& mq, const CUtensorM
 
 cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
                              const CUtensorMap& map_v, const CUtensorMap& map_do, cudaStream_t stream) {
-  return a.g.D == 128 ? launch<128>(a, map_q, map_k, map_v, map_do, stream)
-                      : launch<64>(a, map_q, map_k, map_v, map_do, stream);
+  if (a.g.Bs > 0)
+    return a.g.D == 128 ? launch<128, 1>(a, map_q, map_k, map_v, map_do, stream)
+                        : launch<64, 1>(a, map_q, map_k, map_v, map_do, stream);
+  return a.g.D == 128 ? launch<128, 0>(a, map_q, map_k, map_v, map_do, stream)
+                      : launch<64, 0>(a, map_q, map_k, map_v, map_do, stream);
 }
 
 }  // namespace ttt

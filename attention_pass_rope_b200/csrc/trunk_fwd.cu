@@ -52,13 +52,22 @@ struct FwdCfg {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kMaxBranch = 15;             // P <= 16 passes: at most 15 branch keys per query
 
-template <int D>
+// MODE 0: TTT trunk+branch attention (epilogue keys: the branch keys of passes 2..p at
+// the query's position).  MODE 1: block-draft attention (query rows are block tokens,
+// trunk keys the context up to the block's anchor, epilogue keys the Bs keys of the
+// row's own block).
+template <int MODE>
+struct EpiKeys {
+  static constexpr int kMax = MODE == 0 ? 15 : 16;  // P <= 16 passes; Bs <= 16
+};
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     trunk_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const TrunkFwdArgs a) {
   using C = FwdCfg<D>;
+  constexpr int kMaxBranch = EpiKeys<MODE>::kMax;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
@@ -79,11 +88,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   rem %= g.Hkv * npairs;
   const int kvh = rem / npairs;
   const int pair = rem % npairs;
-  int seq_start, len;
-  seq_bounds(g.si, n, seq_start, len);
+  int seq_start, len, kstart, klen;
+  seq_bounds(g.si, n, seq_start, len);  // query rows
+  seq_bounds(g.ksi, n, kstart, klen);   // key rows (the same tokens in MODE 0)
   if (jq * C::BM >= len) return;  // the whole CTA leaves before touching TMEM
   const int nq_tiles = (2 * pair + 1 < G) ? 2 : 1;
-  const int nkv = jq + 1;
   const int q0 = jq * C::BM;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -98,6 +107,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   uint64_t* drain = o_final + C::NQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   uint32_t* abort_flag = tmem_slot + 1;
+  int* nkv_slot = reinterpret_cast<int*>(abort_flag + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -119,10 +129,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  if (MODE == 1 && warp == 2) {
+    // key tiles to stream: up to the largest anchor among this tile's rows
+    // (none for an empty context: the rows see their block's keys only)
+    const int rows = min(C::BM, len - q0);
+    int mx = -1;
+    for (int r = lane * g.Bs; r < rows; r += 32 * g.Bs) mx = max(mx, block_row_limit(g, seq_start, q0 + r, klen));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) *nkv_slot = (mx + C::BN) / C::BN;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int nkv = MODE == 0 ? jq + 1 : *nkv_slot;
   const Watchdog wd{abort_flag, a.status, a.budget_ns};
 
   int p_of[2], h_of[2];
@@ -148,7 +169,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &map_q, q_full, c * 64, seq_start + q0,
                       p_of[t] * g.H + h_of[t]);
       for (int j = 0; j < nkv; ++j) {
-        const int krow = seq_start + j * C::BN;
+        const int krow = kstart + j * C::BN;
         const int ks = j % C::KST;
         if (j >= C::KST && !wait_bounded(k_empty + ks, ((j / C::KST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
         TTT_TRACE(14, j);
@@ -241,6 +262,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const uint32_t colS = C::COL_S0 + 128 * t;
     const uint32_t colO = C::COL_O0 + D * t;
     const float sl2 = g.scale * kLog2e;
+    // last visible key of this row: its own position (causal) or its block's anchor
+    const int lim = MODE == 0 ? qpos : (qpos < len ? block_row_limit(g, seq_start, qpos, klen) : 0);
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
@@ -258,12 +281,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
       const int k0 = j * C::BN;
-      if (k0 + C::BN - 1 > qpos) {
+      if (k0 + C::BN - 1 > lim) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (k0 + 32 * c + e > qpos) sr[c][e] = __float_as_uint(-INFINITY);
+            if (k0 + 32 * c + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
       }
       // row max: 8 independent chains, then a tree
       float mxv[8];
@@ -331,24 +354,38 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       if (lane == 0) mbar_arrive(p_full + t);
       if (lane == 0 && wq == 0) TTT_TRACE(12 + t, j);
     }
-    if (ok && wait_bounded(o_final + t, 0, wd, kSiteFwdOFinal)) {
+    if (ok && (nkv == 0 || wait_bounded(o_final + t, 0, wd, kSiteFwdOFinal))) {
       tc_fence_after();
       // ---- epilogue: branch keys (a3) and the exact joint-LSE merge (a4).
-      // Query (pass p, position qpos) also sees k~_j[tau], V_j[tau] of the branch passes
-      // j = 1..p (0-based) at its own position; scores on the CUDA cores.  The trunk
-      // partial is (m_run, l_run, unnormalised O in TMEM), all in log2 units.
+      // MODE 0: query (pass p, position qpos) also sees k~_j[tau], V_j[tau] of the branch
+      // passes j = 1..p (0-based) at its own position.  MODE 1: a block token also sees
+      // the Bs keys of its own block (bidirectional).  Scores on the CUDA cores.  The
+      // trunk partial is (m_run, l_run, unnormalised O in TMEM), all in log2 units.
       const bool valid = qpos < len;
       const int p = p_of[t], h = h_of[t];
       const int tau = seq_start + qpos;
       const int T = g.si.T;
+      const int nkeys = MODE == 0 ? p : g.Bs;      // epilogue keys of this row
+      const int bstart = MODE == 0 ? 0 : tau - qpos % g.Bs;  // first row of the block
+      // key u (0-based) of the epilogue: k~ row and V row
+      auto krow_of = [&](int u) -> const uint4* {
+        const int64_t r = MODE == 0 ? (static_cast<int64_t>(u + 1) * g.Hkv + kvh) * T + tau
+                                    : static_cast<int64_t>(kvh) * T + bstart + u;
+        return reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + r * D);
+      };
+      auto vrow_of = [&](int u) -> const __nv_bfloat16* {
+        return MODE == 0 ? static_cast<const __nv_bfloat16*>(a.v) + (u + 1) * g.skv +
+                               (static_cast<int64_t>(tau) * g.Hkv + kvh) * D
+                         : static_cast<const __nv_bfloat16*>(a.v) +
+                               (static_cast<int64_t>(bstart + u) * g.Hkv + kvh) * D;
+      };
       float bs[kMaxBranch];
       float m = m_run;
 #pragma unroll
       for (int j = 1; j <= kMaxBranch; ++j) {
         bs[j - 1] = -INFINITY;
-        if (j <= p && valid) {
-          const uint4* kj = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) +
-                                                           ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D);
+        if (j <= nkeys && valid) {
+          const uint4* kj = krow_of(j - 1);
           const uint8_t* qrow = sQ + t * C::TILE + row * 128;
           float acc = 0.f;
 #pragma unroll 4
@@ -380,19 +417,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(lane_base + colO + 32 * c, o);
-        tmem_ld_wait();
-        reg_fence32(o);
+        if (nkv > 0) {  // CTA-uniform: no trunk key at all leaves O in TMEM unwritten
+          tmem_ld32(lane_base + colO + 32 * c, o);
+          tmem_ld_wait();
+          reg_fence32(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
         if (valid) {
           float acc[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * scale_t;
 #pragma unroll
           for (int j = 1; j <= kMaxBranch; ++j) {
-            if (j <= p) {
-              const uint4* vj = reinterpret_cast<const uint4*>(
-                  static_cast<const __nv_bfloat16*>(a.v) + j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D +
-                  32 * c);
+            if (j <= nkeys) {
+              const uint4* vj = reinterpret_cast<const uint4*>(vrow_of(j - 1) + 32 * c);
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4) {
                 const uint4 vv = __ldg(vj + q4);
@@ -425,11 +465,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int D>
+template <int D, int MODE>
 cudaError_t launch(const TrunkFwdArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    cudaStream_t stream) {
   using C = FwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(trunk_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t e =
+      cudaFuncSetAttribute(trunk_fwd_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int G = a.g.P * (a.g.H / a.g.Hkv);
   const int npairs = (G + 1) / 2;
@@ -437,7 +478,7 @@ cudaError_t launch(const TrunkFwdArgs& a, const CUtensorMap& mq, const CUtensorM
   const long long blocks = static_cast<long long>(njq) * a.g.si.nseq * a.g.Hkv * npairs;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  trunk_fwd_kernel<D><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, a);
+  trunk_fwd_kernel<D, MODE><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -445,7 +486,9 @@ cudaError_t launch(const TrunkFwdArgs& a, const CUtensorMap& mq, const CUtensorM
 
 cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
                              const CUtensorMap& map_v, cudaStream_t stream) {
-  return a.g.D == 128 ? launch<128>(a, map_q, map_k, map_v, stream) : launch<64>(a, map_q, map_k, map_v, stream);
+  if (a.g.Bs > 0)
+    return a.g.D == 128 ? launch<128, 1>(a, map_q, map_k, map_v, stream) : launch<64, 1>(a, map_q, map_k, map_v, stream);
+  return a.g.D == 128 ? launch<128, 0>(a, map_q, map_k, map_v, stream) : launch<64, 0>(a, map_q, map_k, map_v, stream);
 }
 
 }  // namespace ttt

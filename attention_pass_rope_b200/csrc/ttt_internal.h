@@ -40,18 +40,31 @@ struct SeqInfo {
   const int32_t* cu_seqlens;  // device, nullptr for dense
   int nseq;                   // B (dense) or number of sequences
   int S;                      // dense sequence length (0 for packed)
-  int T;                      // total tokens (B*S or cu_seqlens[nseq])
+  int T;                      // total tokens (B*S or mult * cu_seqlens[nseq])
   int max_len;                // longest sequence
+  int mult;                   // packed: row counts are mult * the cu_seqlens entries (1 for tokens)
 };
 
+// The attention has two index spaces: query rows (si) and key rows (ksi), one sequence
+// of each per batch entry.  For the TTT attention they are the same tokens.  For the
+// block-draft attention (Bs > 0) query row r of sequence n is token r % Bs of block
+// (start_n + r) / Bs, and the keys are the context tokens: the row sees the context
+// keys 0..anchor of its block (qlim) and the Bs keys of its own block.
 struct Geometry {
-  SeqInfo si;
+  SeqInfo si;   // query rows (TTT: tokens; block draft: block rows)
+  SeqInfo ksi;  // key rows (TTT: = si; block draft: context tokens)
   int P, H, Hkv, D;
   float theta;
   float scale;  // softmax scale sigma
   int64_t sq;   // elements between passes of the public q, o, dout, dq
   int64_t skv;  // elements between passes of the public k, v, dk, dv
+  int Bs;                    // block-draft: tokens per block (0: TTT attention)
+  const int32_t* anchors;    // block-draft: device int32, anchor position of every block
 };
+
+// Status word of an argument error that only the device can see (block-draft anchors
+// not non-decreasing within a sequence); reported as TTT_ERR_INVALID_ARG.
+constexpr uint32_t kStatusBadAnchors = 0x7200'0001u;
 
 // ----------------------------------------------------------------- launchers
 // All launchers enqueue on `stream` and return the launch error.
@@ -84,16 +97,19 @@ __host__ __device__ inline int ld_slots(const SeqInfo& si) { return si.T / 64 + 
 
 // a5: delta = rowsum(dO * O); writes the tile-aligned (-lse*log2e, delta) rows and
 // zeroes the fp32 dq~ accumulator [P][H][T][D] and the per-slot order tickets.
+// Block-draft geometry (g.Bs > 0): also writes qlim (the trunk-key limit of every query
+// row) and records kStatusBadAnchors in *status if a sequence's anchors decrease.
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  float* dq_acc, int* tickets, cudaStream_t stream);
+                                  float* dq_acc, int* tickets, int* qlim, uint32_t* status, cudaStream_t stream);
 
 struct TrunkBwdArgs {
   Geometry g;
   const float* ld;     // tile-aligned (lse*log2e, delta) rows, see ld_slots
-  float* dq_acc;       // fp32 [P][H][T][D], zeroed before the launch
-  float* dk1_acc;      // fp32 [Hkv][T][D]  (unscaled sum of dS^T q~)
-  void* dv;            // bf16 public dv; pass 0 written here
+  float* dq_acc;       // fp32 [P][H][Tq][D], zeroed before the launch
+  void* dk;            // bf16 public dk of the trunk keys (pass 0 / the context): written here
+  void* dv;            // bf16 public dv of the trunk keys: written here
   int* tickets;        // nullptr, or per statistics slot: key tiles whose dq~ is added (ordered mode)
+  const int* qlim;     // block-draft: trunk-key limit of every query row; nullptr otherwise
   uint32_t* status;
   uint64_t budget_ns;
 };
@@ -102,10 +118,23 @@ struct TrunkBwdArgs {
 cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
                              const CUtensorMap& map_v, const CUtensorMap& map_do, cudaStream_t stream);
 
-// a7+a8: branch backward, dq finalize (inverse RoPE), dk of every pass.
+// a7+a8: branch backward, dq finalize (inverse RoPE), dk/dv of the branch passes.
 cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr, const void* v,
                               const void* dout, const float* lse, const float* ld, const float* dq_acc,
-                              const float* dk1_acc, void* dq, void* dk, void* dv, cudaStream_t stream);
+                              void* dq, void* dk, void* dv, cudaStream_t stream);
+
+// Block-draft: head-major rotated copies dst[head][tau][:] = R(pos(tau)) src[tau][head][:]
+// of up to two tensors sharing the rows' positions: context tokens (block_rows = false,
+// rows of g.ksi, position in the sequence) or block tokens (rows of g.si, position =
+// the block's clamped anchor + the token's index in the block).
+cudaError_t launch_rope_rows(const Geometry& g, bool block_rows, int T, const void* src_a, int nha, void* dst_a,
+                             const void* src_b, int nhb, void* dst_b, cudaStream_t stream);
+
+// Block-draft: backward of the block part, dq of the block tokens (adding the trunk part
+// from dq_acc), dk and dv of the block tokens.
+cudaError_t launch_block_bwd(const Geometry& g, const void* qr, const void* kr, const void* vb, const void* dout,
+                             const float* lse, const float* ld, const float* dq_acc, void* dq, void* dk, void* dv,
+                             cudaStream_t stream);
 
 cudaError_t launch_watchdog_selftest(uint32_t* status, uint64_t budget_ns, cudaStream_t stream);
 

@@ -279,3 +279,162 @@ def ttt_attention(q, k, v, *, theta: float, scale: Optional[float] = None, cu_se
     backward) until the backward, which then skips rotating q and k again: more
     memory between the two calls, one kernel less in the backward."""
     return _TTTAttention.apply(q, k, v, theta, scale, cu_seqlens, max_seqlen, keep_rotated)
+
+
+# ----------------------------------------------------------------------------- block-draft attention
+
+@dataclasses.dataclass
+class BlockLayout:
+    """Shapes of a block-draft call.  dense: k_ctx [B, S, Hkv, D], qb [B, nblk, Bs, H, D],
+    kb/vb [B, nblk, Bs, Hkv, D], anchors [B, nblk], lse [B, H, nblk*Bs].  packed:
+    k_ctx [Tc, Hkv, D], qb [NB, Bs, H, D], kb/vb [NB, Bs, Hkv, D], anchors [NB], lse
+    [H, NB*Bs], with cu_ctx / cu_blocks prefix sums (int32, cuda)."""
+    H: int
+    Hkv: int
+    D: int
+    Bs: int
+    dense: bool
+    B: int = 0
+    S: int = 0
+    nblk: int = 0
+    nseq: int = 0
+    Tc: int = 0
+    NB: int = 0
+    max_ctx: int = 0
+    max_blocks: int = 0
+    cu_ctx: Optional[torch.Tensor] = None
+    cu_blocks: Optional[torch.Tensor] = None
+
+    @property
+    def lse_shape(self):
+        return (self.B, self.H, self.nblk * self.Bs) if self.dense else (self.H, self.NB * self.Bs)
+
+
+def _block_layout(k_ctx, v_ctx, qb, kb, vb, anchors, cu_ctx, cu_blocks, max_ctx, max_blocks) -> BlockLayout:
+    for t in (k_ctx, v_ctx, qb, kb, vb):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("k_ctx, v_ctx, qb, kb, vb must be contiguous bfloat16 CUDA tensors")
+    if anchors.dtype != torch.int32 or not anchors.is_cuda or not anchors.is_contiguous():
+        raise ValueError("anchors must be a contiguous int32 CUDA tensor")
+    if cu_ctx is None:
+        B, S, Hkv, D = k_ctx.shape
+        _, nblk, Bs, H, _ = qb.shape
+        if qb.shape[:1] != (B,) or qb.shape[4] != D or kb.shape != (B, nblk, Bs, Hkv, D) or vb.shape != kb.shape \
+                or v_ctx.shape != k_ctx.shape or anchors.shape != (B, nblk):
+            raise ValueError("inconsistent dense block-draft shapes")
+        return BlockLayout(H, Hkv, D, Bs, True, B=B, S=S, nblk=nblk, nseq=B, Tc=B * S, NB=B * nblk)
+    Tc, Hkv, D = k_ctx.shape
+    NB, Bs, H, _ = qb.shape
+    if kb.shape != (NB, Bs, Hkv, D) or vb.shape != kb.shape or v_ctx.shape != k_ctx.shape or \
+            anchors.shape != (NB,) or qb.shape[3] != D:
+        raise ValueError("inconsistent packed block-draft shapes")
+    for c in (cu_ctx, cu_blocks):
+        if c is None or c.dtype != torch.int32 or not c.is_cuda or c.dim() != 1:
+            raise ValueError("cu_ctx and cu_blocks must be 1-D int32 CUDA tensors")
+    if max_ctx is None or max_blocks is None:
+        raise ValueError("max_ctx and max_blocks are required with cu_ctx / cu_blocks")
+    return BlockLayout(H, Hkv, D, Bs, False, nseq=cu_ctx.numel() - 1, Tc=Tc, NB=NB, max_ctx=int(max_ctx),
+                       max_blocks=int(max_blocks), cu_ctx=cu_ctx.contiguous(), cu_blocks=cu_blocks.contiguous())
+
+
+def make_block_desc(lay: BlockLayout, anchors, theta: float, scale: Optional[float], events=None,
+                    flags: int = 0) -> _lib.TTTBlockDesc:
+    d = _lib.TTTBlockDesc()
+    d.layout = _lib.TTT_LAYOUT_BSHD if lay.dense else _lib.TTT_LAYOUT_THD
+    d.B, d.S, d.nblk = lay.B, lay.S, lay.nblk
+    d.H, d.Hkv, d.D, d.Bs = lay.H, lay.Hkv, lay.D, lay.Bs
+    d.rope_theta = float(theta)
+    d.softmax_scale = 0.0 if scale is None else float(scale)
+    d.anchors = anchors.data_ptr() if anchors is not None else None
+    if not lay.dense:
+        d.cu_ctx, d.cu_blocks = lay.cu_ctx.data_ptr(), lay.cu_blocks.data_ptr()
+        d.nseq, d.total_ctx, d.total_blocks = lay.nseq, lay.Tc, lay.NB
+        d.max_ctx, d.max_blocks = lay.max_ctx, lay.max_blocks
+    d.events = ctypes.addressof(events) if events is not None else None
+    d.flags = int(flags)
+    return d
+
+
+def block_workspace_bytes(lay: BlockLayout, anchors, theta: float, scale=None, for_backward=False) -> int:
+    d = make_block_desc(lay, anchors, theta, scale)
+    n = _lib.lib().ttt_block_workspace_size(ctypes.byref(d), int(for_backward))
+    if n == 0 and lay.NB > 0:
+        raise _lib.TTTError(_lib.TTT_ERR_INVALID_ARG, "ttt_block_workspace_size")
+    return int(n)
+
+
+def block_attn_fwd(k_ctx, v_ctx, qb, kb, vb, anchors, *, theta: float, scale: Optional[float] = None, cu_ctx=None,
+                   cu_blocks=None, max_ctx=None, max_blocks=None, workspace: Optional[torch.Tensor] = None, out=None,
+                   events=None):
+    """Block-draft forward: returns (o, lse)."""
+    lay = _block_layout(k_ctx, v_ctx, qb, kb, vb, anchors, cu_ctx, cu_blocks, max_ctx, max_blocks)
+    if out is None:
+        o = torch.empty_like(qb)
+        lse = torch.empty(lay.lse_shape, dtype=torch.float32, device=qb.device)
+    else:
+        o, lse = out
+    desc = make_block_desc(lay, anchors, theta, scale, events)
+    L = _lib.lib()
+    if workspace is None:
+        workspace = alloc_workspace(L.ttt_block_workspace_size(ctypes.byref(desc), 0), qb.device)
+    st = L.ttt_block_attn_fwd(ctypes.byref(desc), _ptr(k_ctx), _ptr(v_ctx), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(o),
+                              _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream())
+    _lib.check(st, "ttt_block_attn_fwd")
+    return o, lse
+
+
+def block_attn_bwd(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse, dout, *, theta: float, scale: Optional[float] = None,
+                   cu_ctx=None, cu_blocks=None, max_ctx=None, max_blocks=None,
+                   workspace: Optional[torch.Tensor] = None, out=None, events=None, rotated_in_workspace=False,
+                   deterministic=False):
+    """Block-draft backward: returns (dk_ctx, dv_ctx, dqb, dkb, dvb) with respect to the
+    pre-RoPE inputs."""
+    if rotated_in_workspace and workspace is None:
+        raise ValueError("rotated_in_workspace needs the forward's workspace")
+    lay = _block_layout(k_ctx, v_ctx, qb, kb, vb, anchors, cu_ctx, cu_blocks, max_ctx, max_blocks)
+    for t in (o, dout):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != qb.shape:
+            raise ValueError("o and dout must be contiguous bfloat16 tensors shaped like qb")
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor")
+    if out is None:
+        out = tuple(torch.empty_like(t) for t in (k_ctx, v_ctx, qb, kb, vb))
+    flags = (_lib.TTT_FLAG_ROTATED_IN_WORKSPACE if rotated_in_workspace else 0) | \
+        (_lib.TTT_FLAG_DETERMINISTIC_DQ if deterministic else 0)
+    desc = make_block_desc(lay, anchors, theta, scale, events, flags)
+    L = _lib.lib()
+    if workspace is None:
+        workspace = alloc_workspace(L.ttt_block_workspace_size(ctypes.byref(desc), 1), qb.device)
+    dk_ctx, dv_ctx, dqb, dkb, dvb = out
+    st = L.ttt_block_attn_bwd(ctypes.byref(desc), _ptr(k_ctx), _ptr(v_ctx), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(o),
+                              _ptr(lse), _ptr(dout), _ptr(dk_ctx), _ptr(dv_ctx), _ptr(dqb), _ptr(dkb), _ptr(dvb),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream())
+    _lib.check(st, "ttt_block_attn_bwd")
+    return out
+
+
+class _BlockAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, k_ctx, v_ctx, qb, kb, vb, anchors, theta, scale, cu_ctx, cu_blocks, max_ctx, max_blocks):
+        o, lse = block_attn_fwd(k_ctx, v_ctx, qb, kb, vb, anchors, theta=theta, scale=scale, cu_ctx=cu_ctx,
+                                cu_blocks=cu_blocks, max_ctx=max_ctx, max_blocks=max_blocks)
+        ctx.save_for_backward(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse,
+                              *(t for t in (cu_ctx, cu_blocks) if t is not None))
+        ctx.kw = dict(theta=theta, scale=scale, max_ctx=max_ctx, max_blocks=max_blocks)
+        ctx.packed = cu_ctx is not None
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        saved = ctx.saved_tensors
+        k_ctx, v_ctx, qb, kb, vb, anchors, o, lse = saved[:8]
+        cu = dict(cu_ctx=saved[8], cu_blocks=saved[9]) if ctx.packed else {}
+        grads = block_attn_bwd(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse, do.contiguous(), **cu, **ctx.kw)
+        return (*grads, None, None, None, None, None, None, None)
+
+
+def block_attention(k_ctx, v_ctx, qb, kb, vb, anchors, *, theta: float, scale: Optional[float] = None, cu_ctx=None,
+                    cu_blocks=None, max_ctx=None, max_blocks=None):
+    """Differentiable block-draft attention (autograd over the C ABI); returns o."""
+    return _BlockAttention.apply(k_ctx, v_ctx, qb, kb, vb, anchors, theta, scale, cu_ctx, cu_blocks, max_ctx,
+                                 max_blocks)

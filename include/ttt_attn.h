@@ -185,6 +185,81 @@ ttt_status ttt_attn_fwd_noalloc_status(void* stream, uint32_t* detail);
  * through ttt_attn_fwd_noalloc_status(). */
 ttt_status ttt_attn_noalloc_watchdog_selftest(uint64_t budget_ns, void* stream);
 
+/* ------------------------------------------------------------------------------
+ * Block-draft attention of DFlash/DSpark drafters.  Source: "DFlash/DSpark and EAGLE-3
+ * TTT draft co-training ..." (NeMo-RL issue 3698), "What I'm working on", item 2
+ * (anchor + mask-token block drafting: bidirectional in-block attention, trunk
+ * truncated at the anchor) and item 4 (packed THD layout).
+ *
+ *   A block b of Bs tokens starts at the anchor position a_b of its sequence; its
+ *   token j sits at position a_b + j and has its own q, k, v.  With kv(h) = h / (H/Hkv):
+ *     q~ = R(a_b + j) q,  k~ = R(a_b + j) k (block tokens),  k~_ctx[t] = R(t) k_ctx[t]
+ *     trunk keys: k~_ctx[t], v_ctx[t] for t = 0..a_b            (truncated at the anchor)
+ *     block keys: k~, v of the Bs tokens of block b             (bidirectional)
+ *     lse = logaddexp(lse_trunk, lse_block), O = the exact merge of the two partial
+ *     softmaxes, i.e. one softmax over the (a_b + 1) + Bs visible keys.
+ *   Rotated q~ / k~ are rounded to bf16 before the dot products, as in the TTT call.
+ *
+ * Layouts (row-major, contiguous; NB = total blocks, Tc = total context tokens):
+ *   dense (TTT_LAYOUT_BSHD): B sequences of S context tokens and nblk blocks each:
+ *     k_ctx, v_ctx, dk_ctx, dv_ctx [B][S][Hkv][D];  qb, o, dout, dqb [B][nblk][Bs][H][D];
+ *     kb, vb, dkb, dvb [B][nblk][Bs][Hkv][D];  anchors int32 [B][nblk];
+ *     lse fp32 [B][H][nblk*Bs].
+ *   packed (TTT_LAYOUT_THD): cu_ctx (context tokens) and cu_blocks (blocks), device
+ *     int32[nseq+1] prefix sums: k_ctx.. [Tc][Hkv][D], qb.. [NB][Bs][H][D],
+ *     kb.. [NB][Bs][Hkv][D], anchors [NB], lse [H][NB*Bs].
+ *   anchors: device int32, each block's anchor position within its sequence, in
+ *   [0, its context length) (values outside are clamped to it) and non-decreasing
+ *   within a sequence (the backward relies on the order and reports a violation as
+ *   TTT_ERR_INVALID_ARG through ttt_attn_device_status; the forward is exact for any
+ *   order).  Supported: D in {64, 128}, H a multiple of Hkv, 1 <= Bs <= 16.
+ * Ownership, asynchrony, errors and the workspace contract are those of the TTT calls
+ * above; descriptor flags TTT_FLAG_ROTATED_IN_WORKSPACE and TTT_FLAG_DETERMINISTIC_DQ
+ * mean the same (the forward's workspace layout is a prefix of the backward's).
+ * ------------------------------------------------------------------------------ */
+typedef struct {
+  int layout;                /* ttt_layout */
+  int B, S, nblk;            /* dense: sequences, context length, blocks per sequence */
+  int H, Hkv, D;             /* query heads, KV heads, head dimension */
+  int Bs;                    /* tokens per block, 1..16 */
+  float rope_theta;          /* RoPE base, > 0 */
+  float softmax_scale;       /* 0 selects 1/sqrt(D) */
+  const int32_t* anchors;    /* device int32[NB] */
+  const int32_t* cu_ctx;     /* THD: device int32[nseq+1], context tokens */
+  const int32_t* cu_blocks;  /* THD: device int32[nseq+1], blocks */
+  int nseq;                  /* THD: sequences */
+  int total_ctx;             /* THD: Tc = cu_ctx[nseq] */
+  int total_blocks;          /* THD: NB = cu_blocks[nseq] */
+  int max_ctx;               /* THD: upper bound on every context length */
+  int max_blocks;            /* THD: upper bound on every sequence's block count */
+  const ttt_attn_events* events; /* optional: TTT_KERNEL_ROPE_FWD, _TRUNK_FWD, _ROPE_BWD,
+                                    _BWD_PREPROCESS, _TRUNK_BWD, _BRANCH_BWD (block part) */
+  int flags;                 /* TTT_FLAG_* bits */
+} ttt_block_desc;
+
+/* Workspace bytes of ttt_block_attn_fwd (for_backward = 0) or ttt_block_attn_bwd (1); 0
+ * for an invalid descriptor.  256-byte aligned. */
+size_t ttt_block_workspace_size(const ttt_block_desc* desc, int for_backward);
+
+/* Sub-buffers: fwd [0] status word, [1] q~ of the block tokens bf16 [H][NB*Bs][D],
+ * [2] k~_ctx bf16 [Hkv][Tc][D], [3] k~ of the block tokens bf16 [Hkv][NB*Bs][D];
+ * bwd adds [4] row statistics (as for the TTT call, over the block rows), [5] dq~
+ * accumulator fp32 [H][NB*Bs][D], [6] order tickets, [7] int32 trunk-key limit of
+ * every block row.  Returns the number of entries (at most 8), 0 if invalid. */
+int ttt_block_workspace_layout(const ttt_block_desc* desc, int for_backward, size_t* offsets);
+
+/* Forward: o (bf16, like qb) and lse (fp32 natural log). */
+ttt_status ttt_block_attn_fwd(const ttt_block_desc* desc, const void* k_ctx, const void* v_ctx, const void* qb,
+                              const void* kb, const void* vb, void* o, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Backward, recomputing the probabilities from lse: gradients with respect to the
+ * pre-RoPE inputs (bf16).  dk_ctx / dv_ctx of context keys no block sees are zero. */
+ttt_status ttt_block_attn_bwd(const ttt_block_desc* desc, const void* k_ctx, const void* v_ctx, const void* qb,
+                              const void* kb, const void* vb, const void* o, const float* lse, const void* dout,
+                              void* dk_ctx, void* dv_ctx, void* dqb, void* dkb, void* dvb, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* The error behind the most recent TTT_ERR_CUDA returned by any call in this
  * process: a cudaError_t value, or 100000 + the CUresult when encoding a TMA tensor
  * map failed; 0 if there was none.  Not reset by later successful calls. */
@@ -195,8 +270,9 @@ const char* ttt_attn_cuda_error_name(int code);
 
 /* Synchronises `stream` and returns TTT_OK if no bounded wait of the calls made
  * with this workspace ran out since the last check, TTT_ERR_DEVICE_TIMEOUT (and
- * the raw status word in *detail if non-NULL) otherwise, or TTT_ERR_CUDA.  The
- * status word is cleared. */
+ * the raw status word in *detail if non-NULL) otherwise, TTT_ERR_INVALID_ARG for an
+ * argument error only the device could see (block-draft anchors out of order), or
+ * TTT_ERR_CUDA.  The status word is cleared. */
 ttt_status ttt_attn_device_status(void* workspace, void* stream, uint32_t* detail);
 
 /* Workspace sub-buffers (byte offsets from the workspace base), for inspection of
@@ -206,8 +282,8 @@ ttt_status ttt_attn_device_status(void* workspace, void* stream, uint32_t* detai
  *        and the 64-row query tile j of sequence n, 128 floats at slot
  *        start_n/64 + n + j of row p*H + h (-lse * log2(e) of the 64 rows, then their
  *        delta = rowsum(dout * o)), T/64 + nseq + 1 slots per row,
- *        [4] dq~ accumulator fp32 [P][H][Tt][D], [5] dk~_1 accumulator fp32 [Hkv][Tt][D],
- *        [6] int32 order tickets of the dq~ additions, one per statistics slot.
+ *        [4] dq~ accumulator fp32 [P][H][Tt][D], [5] int32 order tickets of the dq~
+ *        additions, one per statistics slot.
  * Tt = B*S (dense) or T (packed).  Returns the number of entries written to
  * offsets (at most 8), or 0 for an invalid descriptor. */
 int ttt_attn_workspace_layout(const ttt_attn_desc* desc, int for_backward, size_t* offsets);

@@ -142,3 +142,117 @@ def make_inputs(w: Workload, with_grad: bool = True, seed: Optional[int] = None)
     v = draw(w.P, T, w.Hkv, w.D)
     do = draw(w.P, T, w.H, w.D) if with_grad else None
     return Inputs(q, k, v, do)
+
+
+# ----------------------------------------------------------------------------- block-draft attention
+
+@dataclasses.dataclass(frozen=True)
+class BlockWorkload:
+    """Shape of one block-draft call: per sequence a context of ``ctx_lengths[n]`` tokens
+    and ``nblocks[n]`` blocks of ``Bs`` tokens.  Anchors are drawn per sequence (sorted
+    uniform positions of its context) unless ``anchors`` lists them (flat, per block)."""
+
+    name: str
+    H: int
+    Hkv: int
+    D: int
+    Bs: int
+    theta: float
+    ctx_lengths: tuple
+    nblocks: tuple
+    dense: bool
+    scale: float = 1.0
+    seed: int = 0
+    anchors: tuple = ()
+
+    @property
+    def nseq(self) -> int:
+        return len(self.ctx_lengths)
+
+    @property
+    def Tc(self) -> int:
+        return int(sum(self.ctx_lengths))
+
+    @property
+    def NB(self) -> int:
+        return int(sum(self.nblocks))
+
+    @property
+    def cu_ctx(self) -> list:
+        out = [0]
+        for n in self.ctx_lengths:
+            out.append(out[-1] + int(n))
+        return out
+
+    @property
+    def cu_blocks(self) -> list:
+        out = [0]
+        for n in self.nblocks:
+            out.append(out[-1] + int(n))
+        return out
+
+    def flops_fwd_bwd(self, anchors, per_pair: int = 14) -> float:
+        """Algorithmic flops: ``per_pair * D`` per visible (block token, key) pair and query
+        head: (anchor + 1) trunk keys and Bs block keys per block token."""
+        keys = sum((int(a) + 1 + self.Bs) * self.Bs for a in anchors)
+        return float(per_pair * self.D * keys * self.H)
+
+
+def block_dense(name, B, S, nblk, Bs, H, Hkv, D, theta, scale=1.0, seed=0, anchors=()) -> BlockWorkload:
+    return BlockWorkload(name, H, Hkv, D, Bs, float(theta), tuple([S] * B), tuple([nblk] * B), True, scale, seed,
+                         tuple(anchors))
+
+
+def block_thd(name, ctx_lengths, nblocks, Bs, H, Hkv, D, theta, scale=1.0, seed=0, anchors=()) -> BlockWorkload:
+    return BlockWorkload(name, H, Hkv, D, Bs, float(theta), tuple(int(x) for x in ctx_lengths),
+                         tuple(int(x) for x in nblocks), False, scale, seed, tuple(anchors))
+
+
+def block_workloads() -> dict:
+    """Block-draft workloads with the draft layer's head shapes (32/8 heads, D = 128)."""
+    return {
+        "block_tiny": block_dense("block_tiny", B=1, S=128, nblk=8, Bs=4, H=4, Hkv=2, D=64, theta=1e4),
+        "block_draft_4k": block_dense("block_draft_4k", B=2, S=4096, nblk=256, Bs=16, H=32, Hkv=8, D=128,
+                                      theta=1e6),
+    }
+
+
+@dataclasses.dataclass
+class BlockInputs:
+    """bf16 tensors on the CPU (packed layouts) and int32 anchors (flat, per block)."""
+
+    k_ctx: torch.Tensor   # [Tc, Hkv, D]
+    v_ctx: torch.Tensor   # [Tc, Hkv, D]
+    qb: torch.Tensor      # [NB, Bs, H, D]
+    kb: torch.Tensor      # [NB, Bs, Hkv, D]
+    vb: torch.Tensor      # [NB, Bs, Hkv, D]
+    do: torch.Tensor      # [NB, Bs, H, D]
+    anchors: torch.Tensor  # [NB] int32
+
+
+def make_block_inputs(w: BlockWorkload) -> BlockInputs:
+    """One generator seeded with ``w.seed``: the anchors first (per sequence, sorted
+    ``randint(0, L_n)`` draws, unless given), then K_ctx, V_ctx, Qb, Kb, Vb and dO, each
+    fp32 N(0, 1) times ``scale`` rounded to bf16."""
+    g = torch.Generator().manual_seed(w.seed)
+    if w.anchors:
+        anchors = torch.tensor(w.anchors, dtype=torch.int32)
+        assert anchors.numel() == w.NB
+    else:
+        parts = [torch.sort(torch.randint(0, max(L, 1), (nb,), generator=g)).values
+                 for L, nb in zip(w.ctx_lengths, w.nblocks)]
+        anchors = (torch.cat(parts) if parts else torch.zeros(0, dtype=torch.int64)).to(torch.int32)
+
+    def draw(*shape):
+        x = torch.randn(*shape, generator=g, dtype=torch.float32)
+        if w.scale != 1.0:
+            x.mul_(w.scale)
+        return x.to(torch.bfloat16)
+
+    k_ctx = draw(w.Tc, w.Hkv, w.D)
+    v_ctx = draw(w.Tc, w.Hkv, w.D)
+    qb = draw(w.NB, w.Bs, w.H, w.D)
+    kb = draw(w.NB, w.Bs, w.Hkv, w.D)
+    vb = draw(w.NB, w.Bs, w.Hkv, w.D)
+    do = draw(w.NB, w.Bs, w.H, w.D)
+    return BlockInputs(k_ctx, v_ctx, qb, kb, vb, do, anchors)
