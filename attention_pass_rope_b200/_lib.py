@@ -75,6 +75,22 @@ class TTTBlockDesc(ctypes.Structure):
     ]
 
 
+class TTTRingDesc(ctypes.Structure):
+    _fields_ = [
+        ("P", ctypes.c_int),
+        ("H", ctypes.c_int),
+        ("Hkv", ctypes.c_int),
+        ("D", ctypes.c_int),
+        ("rope_theta", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float),
+        ("q_len", ctypes.c_int),
+        ("q_start", ctypes.c_int),
+        ("kv_len", ctypes.c_int),
+        ("kv_start", ctypes.c_int),
+        ("include_branch", ctypes.c_int),
+    ]
+
+
 class TTTError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -133,6 +149,15 @@ def lib() -> ctypes.CDLL:
     L.ttt_block_attn_fwd.restype = ctypes.c_int
     L.ttt_block_attn_bwd.argtypes = [BD] + [vp] * 14 + [sz, vp]
     L.ttt_block_attn_bwd.restype = ctypes.c_int
+    RD = P(TTTRingDesc)
+    L.ttt_ring_rotate.argtypes = [RD, vp, vp, vp, vp, vp]
+    L.ttt_ring_rotate.restype = ctypes.c_int
+    L.ttt_ring_step.argtypes = [RD, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.ttt_ring_step.restype = ctypes.c_int
+    L.ttt_ring_merge.argtypes = [RD, vp, vp, vp, vp, ctypes.c_int, vp]
+    L.ttt_ring_merge.restype = ctypes.c_int
+    L.ttt_ring_finish.argtypes = [RD, vp, vp, vp]
+    L.ttt_ring_finish.restype = ctypes.c_int
     L.ttt_status_string.argtypes = [ctypes.c_int]
     L.ttt_status_string.restype = ctypes.c_char_p
     L.ttt_attn_version.argtypes = []

@@ -69,6 +69,9 @@ ttt_status make_plan(const ttt_attn_desc* d, int for_backward, Plan* out) {
   g.ksi = g.si;  // queries and keys index the same tokens
   g.Bs = 0;
   g.anchors = nullptr;
+  g.ring = 0;
+  g.limit_off = 0;
+  g.pos0 = 0;
   // index arithmetic in the kernels: P*H*T*D elements must fit comfortably in int64,
   // per-pass offsets in int32 where they are formed that way
   const long long rows = static_cast<long long>(g.P) * g.H * g.si.T;
@@ -138,6 +141,9 @@ ttt_status make_block_plan(const ttt_block_desc* d, int for_backward, Plan* out)
   g.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt(static_cast<float>(d->D));
   g.Bs = d->Bs;
   g.anchors = d->anchors;
+  g.ring = 0;
+  g.limit_off = 0;
+  g.pos0 = 0;
   if (d->layout == TTT_LAYOUT_BSHD) {
     if (d->B < 0 || d->S < 0 || d->nblk < 0) return TTT_ERR_INVALID_ARG;
     const long long Tc = static_cast<long long>(d->B) * d->S;
@@ -186,6 +192,35 @@ ttt_status make_block_plan(const ttt_block_desc* d, int for_backward, Plan* out)
   }
   pl.total = o;
   *out = pl;
+  return TTT_OK;
+}
+
+// Ring step geometry: the local query chunk is one dense sequence of q_len rows (B = 1),
+// the visiting keys another of kv_len rows.
+ttt_status make_ring_geometry(const ttt_ring_desc* d, Geometry* out) {
+  if (!d) return TTT_ERR_INVALID_ARG;
+  if (d->P < 1 || d->H < 1 || d->Hkv < 1 || d->H % d->Hkv != 0) return TTT_ERR_INVALID_ARG;
+  if (d->P > 16) return TTT_ERR_UNSUPPORTED;
+  if (d->D != 64 && d->D != 128) return TTT_ERR_UNSUPPORTED;
+  if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return TTT_ERR_INVALID_ARG;
+  if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return TTT_ERR_INVALID_ARG;
+  if (d->q_len < 0 || d->kv_len < 0 || d->q_start < 0 || d->kv_start < 0) return TTT_ERR_INVALID_ARG;
+  if (d->q_len > (1 << 28) || d->kv_len > (1 << 28)) return TTT_ERR_UNSUPPORTED;
+  Geometry g{};
+  g.P = d->P;
+  g.H = d->H;
+  g.Hkv = d->Hkv;
+  g.D = d->D;
+  g.theta = d->rope_theta;
+  g.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt(static_cast<float>(d->D));
+  g.si = SeqInfo{nullptr, 1, d->q_len, d->q_len, d->q_len, 1};
+  g.ksi = SeqInfo{nullptr, 1, d->kv_len, d->kv_len, d->kv_len, 1};
+  g.sq = static_cast<int64_t>(d->q_len) * d->H * d->D;
+  g.skv = static_cast<int64_t>(d->q_len) * d->Hkv * d->D;
+  g.ring = d->include_branch ? 2 : 1;
+  g.limit_off = d->q_start - d->kv_start;
+  g.pos0 = d->q_start;
+  *out = g;
   return TTT_OK;
 }
 
@@ -332,7 +367,7 @@ ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k,
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
-    TrunkFwdArgs a{g, kr, v, o, lse, status, g_wait_budget_ns.load()};
+    TrunkFwdArgs a{g, nullptr, kr, v, o, lse, status, g_wait_budget_ns.load()};
     TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
   }
   return TTT_OK;
@@ -442,7 +477,7 @@ ttt_status ttt_block_attn_fwd(const ttt_block_desc* desc, const void* k_ctx, con
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
-    TrunkFwdArgs a{g, kr_blk, vb, o, lse, status, g_wait_budget_ns.load()};
+    TrunkFwdArgs a{g, nullptr, kr_blk, vb, o, lse, status, g_wait_budget_ns.load()};
     TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
   }
   return TTT_OK;
@@ -512,6 +547,77 @@ ttt_status ttt_block_attn_bwd(const ttt_block_desc* desc, const void* k_ctx, con
     EventScope es(desc->events, TTT_KERNEL_BRANCH_BWD, stream);
     TTT_CHECK_CUDA(launch_block_bwd(g, qr, kr_blk, vb, dout, lse, ld, dq_acc, dqb, dkb, dvb, stream));
   }
+  return TTT_OK;
+}
+
+ttt_status ttt_ring_rotate(const ttt_ring_desc* desc, const void* q, const void* k, void* qr, void* kr,
+                           void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0) return TTT_OK;
+  if (!q || !k || !qr || !kr) return TTT_ERR_INVALID_ARG;
+  if (!ptr_aligned(q, 16) || !ptr_aligned(k, 16) || !ptr_aligned(qr, 16) || !ptr_aligned(kr, 16))
+    return TTT_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  clear_stale_error();
+  TTT_CHECK_CUDA(launch_rope_fwd(g, q, k, qr, kr, stream));
+  return TTT_OK;
+}
+
+ttt_status ttt_ring_step(const ttt_ring_desc* desc, const void* qr, const void* kr_local, const void* v_local,
+                         const void* kr_visit, const void* v_visit, float* o_part, float* lse_part, void* status,
+                         void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0) return TTT_OK;
+  if (desc->kv_start > desc->q_start || desc->kv_len == 0) return TTT_ERR_INVALID_ARG;  // no visible key
+  if (!qr || !kr_visit || !v_visit || !o_part || !lse_part || !status) return TTT_ERR_INVALID_ARG;
+  if (desc->include_branch && desc->P > 1 && (!kr_local || !v_local)) return TTT_ERR_INVALID_ARG;
+  if (!ptr_aligned(qr, 16) || !ptr_aligned(kr_visit, 16) || !ptr_aligned(v_visit, 16) || !ptr_aligned(o_part, 16) ||
+      !ptr_aligned(lse_part, 4) || !ptr_aligned(status, 4) || (kr_local && !ptr_aligned(kr_local, 16)) ||
+      (v_local && !ptr_aligned(v_local, 16)))
+    return TTT_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const uint64_t Lq = desc->q_len, Lk = desc->kv_len, D = g.D;
+  clear_stale_error();
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, qr, D, Lq, static_cast<uint64_t>(g.P) * g.H, D * 2, Lq * D * 2, 128, 1) ||
+      !make_map(&mk, kr_visit, D, Lk, g.Hkv, D * 2, Lk * D * 2, 128, 1) ||
+      !make_map(&mv, v_visit, D, g.Hkv, Lk, D * 2, g.Hkv * D * 2, 1, 128))
+    return TTT_ERR_CUDA;
+  TrunkFwdArgs a{g, o_part, kr_local, v_local, nullptr, lse_part, static_cast<uint32_t*>(status),
+                 g_wait_budget_ns.load()};
+  TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
+  return TTT_OK;
+}
+
+ttt_status ttt_ring_merge(const ttt_ring_desc* desc, float* o_acc, float* lse_acc, const float* o_part,
+                          const float* lse_part, int first, void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0) return TTT_OK;
+  if (!o_acc || !lse_acc || !o_part || !lse_part || !ptr_aligned(o_acc, 16) || !ptr_aligned(o_part, 16))
+    return TTT_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(g.P) * desc->q_len * g.H;
+  if (rows > 0x7FFFFFFFLL) return TTT_ERR_UNSUPPORTED;
+  clear_stale_error();
+  TTT_CHECK_CUDA(launch_ring_merge(static_cast<int>(rows), g.D, g.H, desc->q_len, o_acc, lse_acc, o_part, lse_part,
+                                   first != 0, static_cast<cudaStream_t>(stream_)));
+  return TTT_OK;
+}
+
+ttt_status ttt_ring_finish(const ttt_ring_desc* desc, const float* o_acc, void* o, void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0) return TTT_OK;
+  if (!o_acc || !o || !ptr_aligned(o_acc, 16) || !ptr_aligned(o, 16)) return TTT_ERR_INVALID_ARG;
+  clear_stale_error();
+  TTT_CHECK_CUDA(launch_ring_finish(static_cast<int64_t>(g.P) * desc->q_len * g.H * g.D, o_acc, o,
+                                    static_cast<cudaStream_t>(stream_)));
   return TTT_OK;
 }
 

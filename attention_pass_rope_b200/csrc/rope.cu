@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
   for (int e = threadIdx.x; e < kRopeTok * HALF; e += blockDim.x) {
     const int tok = e / HALF, d = e % HALF;
     const double inv_freq = pow(static_cast<double>(g.theta), -2.0 * d / D);
-    const double ang = static_cast<double>(i0 + tok + p) * inv_freq;
+    const double ang = static_cast<double>(g.pos0 + i0 + tok + p) * inv_freq;
     double s, c;
     sincos(ang, &s, &c);
     cs[tok][d] = make_float2(static_cast<float>(c), static_cast<float>(s));

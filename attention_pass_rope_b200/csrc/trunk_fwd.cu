@@ -56,10 +56,12 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // MODE 0: TTT trunk+branch attention (epilogue keys: the branch keys of passes 2..p at
 // the query's position).  MODE 1: block-draft attention (query rows are block tokens,
 // trunk keys the context up to the block's anchor, epilogue keys the Bs keys of the
-// row's own block).
+// row's own block).  MODE 2: one step of the context-parallel ring (query rows are a
+// chunk of the sequence, trunk keys a visiting chunk, causal by global position; the
+// branch keys only in the step that meets the chunk's own keys; fp32 partial output).
 template <int MODE>
 struct EpiKeys {
-  static constexpr int kMax = MODE == 0 ? 15 : 16;  // P <= 16 passes; Bs <= 16
+  static constexpr int kMax = MODE == 1 ? 16 : 15;  // P <= 16 passes; Bs <= 16
 };
 
 template <int D, int MODE>
@@ -143,7 +145,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nkv = MODE == 0 ? jq + 1 : *nkv_slot;
+  const int nkv = MODE == 0 ? jq + 1
+                  : MODE == 1 ? *nkv_slot
+                              : min(q0 + min(C::BM, len - q0) - 1 + g.limit_off, klen - 1) / C::BN + 1;
   const Watchdog wd{abort_flag, a.status, a.budget_ns};
 
   int p_of[2], h_of[2];
@@ -263,7 +267,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const uint32_t colO = C::COL_O0 + D * t;
     const float sl2 = g.scale * kLog2e;
     // last visible key of this row: its own position (causal) or its block's anchor
-    const int lim = MODE == 0 ? qpos : (qpos < len ? block_row_limit(g, seq_start, qpos, klen) : 0);
+    const int lim = MODE == 0   ? qpos
+                    : MODE == 1 ? (qpos < len ? block_row_limit(g, seq_start, qpos, klen) : 0)
+                                : min(qpos + g.limit_off, klen - 1);
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
@@ -365,16 +371,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const int p = p_of[t], h = h_of[t];
       const int tau = seq_start + qpos;
       const int T = g.si.T;
-      const int nkeys = MODE == 0 ? p : g.Bs;      // epilogue keys of this row
-      const int bstart = MODE == 0 ? 0 : tau - qpos % g.Bs;  // first row of the block
+      const int nkeys = MODE == 0 ? p : MODE == 1 ? g.Bs : (g.ring == 2 ? p : 0);  // epilogue keys of this row
+      const int bstart = MODE == 1 ? tau - qpos % g.Bs : 0;  // first row of the block
       // key u (0-based) of the epilogue: k~ row and V row
       auto krow_of = [&](int u) -> const uint4* {
-        const int64_t r = MODE == 0 ? (static_cast<int64_t>(u + 1) * g.Hkv + kvh) * T + tau
+        const int64_t r = MODE != 1 ? (static_cast<int64_t>(u + 1) * g.Hkv + kvh) * T + tau
                                     : static_cast<int64_t>(kvh) * T + bstart + u;
         return reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + r * D);
       };
       auto vrow_of = [&](int u) -> const __nv_bfloat16* {
-        return MODE == 0 ? static_cast<const __nv_bfloat16*>(a.v) + (u + 1) * g.skv +
+        return MODE != 1 ? static_cast<const __nv_bfloat16*>(a.v) + (u + 1) * g.skv +
                                (static_cast<int64_t>(tau) * g.Hkv + kvh) * D
                          : static_cast<const __nv_bfloat16*>(a.v) +
                                (static_cast<int64_t>(bstart + u) * g.Hkv + kvh) * D;
@@ -446,13 +452,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               }
             }
           }
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+          if (MODE == 2) {
+            float4* dst = reinterpret_cast<float4*>(a.o_part + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D +
+                                                    32 * c);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            dst[q4] = make_uint4(pack_bf16x2(acc[8 * q4] * inv_l, acc[8 * q4 + 1] * inv_l),
-                                 pack_bf16x2(acc[8 * q4 + 2] * inv_l, acc[8 * q4 + 3] * inv_l),
-                                 pack_bf16x2(acc[8 * q4 + 4] * inv_l, acc[8 * q4 + 5] * inv_l),
-                                 pack_bf16x2(acc[8 * q4 + 6] * inv_l, acc[8 * q4 + 7] * inv_l));
+            for (int q4 = 0; q4 < 8; ++q4)
+              dst[q4] = make_float4(acc[4 * q4] * inv_l, acc[4 * q4 + 1] * inv_l, acc[4 * q4 + 2] * inv_l,
+                                    acc[4 * q4 + 3] * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              dst[q4] = make_uint4(pack_bf16x2(acc[8 * q4] * inv_l, acc[8 * q4 + 1] * inv_l),
+                                   pack_bf16x2(acc[8 * q4 + 2] * inv_l, acc[8 * q4 + 3] * inv_l),
+                                   pack_bf16x2(acc[8 * q4 + 4] * inv_l, acc[8 * q4 + 5] * inv_l),
+                                   pack_bf16x2(acc[8 * q4 + 6] * inv_l, acc[8 * q4 + 7] * inv_l));
+          }
         }
       }
       if (valid) a.lse[lse_index(g.si, g.H, p, h, n, tau, qpos)] = (m + __log2f(l)) * kLn2;
@@ -486,6 +501,8 @@ cudaError_t launch(const TrunkFwdArgs& a, const CUtensorMap& mq, const CUtensorM
 
 cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
                              const CUtensorMap& map_v, cudaStream_t stream) {
+  if (a.g.ring > 0)
+    return a.g.D == 128 ? launch<128, 2>(a, map_q, map_k, map_v, stream) : launch<64, 2>(a, map_q, map_k, map_v, stream);
   if (a.g.Bs > 0)
     return a.g.D == 128 ? launch<128, 1>(a, map_q, map_k, map_v, stream) : launch<64, 1>(a, map_q, map_k, map_v, stream);
   return a.g.D == 128 ? launch<128, 0>(a, map_q, map_k, map_v, stream) : launch<64, 0>(a, map_q, map_k, map_v, stream);

@@ -60,6 +60,12 @@ struct Geometry {
   int64_t skv;  // elements between passes of the public k, v, dk, dv
   int Bs;                    // block-draft: tokens per block (0: TTT attention)
   const int32_t* anchors;    // block-draft: device int32, anchor position of every block
+  // context-parallel ring step (ring > 0): the queries are one chunk of a sequence, the
+  // keys another chunk of the same sequence; query row r sees key row t iff
+  // t <= r + limit_off (global positions: limit_off = q_start - kv_start >= 0)
+  int ring;                  // 0: not a ring step; 1: without, 2: with the branch keys
+  int limit_off;
+  int pos0;                  // RoPE position of the first row (global position of a chunk)
 };
 
 // Status word of an argument error that only the device can see (block-draft anchors
@@ -75,6 +81,7 @@ cudaError_t launch_rope_fwd(const Geometry& g, const void* q, const void* k, voi
 
 struct TrunkFwdArgs {
   Geometry g;
+  float* o_part;   // ring step: fp32 partial output [P][Tq][H][D] (normalised over the step's keys)
   const void* kr;  // bf16 k~ head-major [P][Hkv][T][D] (branch keys, passes >= 1)
   const void* v;   // bf16 V, public layout [P][T][Hkv][D] (branch values; passes g.skv apart)
   void* o;         // bf16 output, public layout [P][T][H][D] (passes g.sq apart)
@@ -135,6 +142,12 @@ cudaError_t launch_rope_rows(const Geometry& g, bool block_rows, int T, const vo
 cudaError_t launch_block_bwd(const Geometry& g, const void* qr, const void* kr, const void* vb, const void* dout,
                              const float* lse, const float* ld, const float* dq_acc, void* dq, void* dk, void* dv,
                              cudaStream_t stream);
+
+// Ring: running merge of partial results (acc <- acc (+) part by log-sum-exp; `first`
+// copies), and the final bf16 output.  O rows are [P][Lq][H][D] fp32, lse [P][H][Lq].
+cudaError_t launch_ring_merge(int rows, int D, int H, int Lq, float* o_acc, float* lse_acc, const float* o_part,
+                              const float* lse_part, bool first, cudaStream_t stream);
+cudaError_t launch_ring_finish(int64_t n, const float* o_acc, void* o, cudaStream_t stream);
 
 cudaError_t launch_watchdog_selftest(uint32_t* status, uint64_t budget_ns, cudaStream_t stream);
 

@@ -260,6 +260,56 @@ ttt_status ttt_block_attn_bwd(const ttt_block_desc* desc, const void* k_ctx, con
                               void* dk_ctx, void* dv_ctx, void* dqb, void* dkb, void* dvb, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------------
+ * Context-parallel ring over the pass-1 trunk K/V.  Source: "DFlash/DSpark and EAGLE-3
+ * TTT draft co-training ..." (NeMo-RL issue 3698), "What I'm working on", item 4 (pass-1
+ * trunk K/V on a zigzag ring, exact joint-LSE merge).
+ *
+ * The sequence is cut into chunks held by different ranks.  A rank rotates its query
+ * chunks (ttt_ring_rotate: every pass of q and k at the chunk's global positions), and
+ * in each ring step computes the attention of a local query chunk against a visiting
+ * chunk of rotated pass-1 keys and of pass-1 values, causal by global position
+ * (ttt_ring_step), merging the partial into a running result (ttt_ring_merge); the last
+ * step writes the bf16 output (ttt_ring_finish).  The chunk that meets its own trunk
+ * keys also takes the branch keys (include_branch).  After every visiting chunk whose
+ * start is at or before the query chunk's has been merged, the result equals
+ * ttt_attn_fwd's on the whole sequence (up to rounding).  Moving chunks between ranks
+ * is the caller's (e.g. NCCL send/recv into this GPU's memory); these calls read this
+ * GPU's memory only.  Rows: queries [P][q_len][H][D], local k/v [P][q_len][Hkv][D];
+ * rotated local qr [P][H][q_len][D], kr [P][Hkv][q_len][D]; visiting keys
+ * kr_visit [Hkv][kv_len][D] (rotated, i.e. pass 0 of the owner's kr) and values
+ * v_visit [kv_len][Hkv][D]; partial and running outputs fp32 [P][q_len][H][D] with lse
+ * fp32 [P][H][q_len]. */
+typedef struct {
+  int P, H, Hkv, D;
+  float rope_theta;
+  float softmax_scale;       /* 0 selects 1/sqrt(D) */
+  int q_len, q_start;        /* local query chunk: rows, global position of its first row */
+  int kv_len, kv_start;      /* visiting key chunk: rows, global position of its first row */
+  int include_branch;        /* 1: this step also takes the branch keys (the local chunk's) */
+} ttt_ring_desc;
+
+/* qr, kr <- the rotated local chunk (positions q_start + i + p), head-major. */
+ttt_status ttt_ring_rotate(const ttt_ring_desc* desc, const void* q, const void* k, void* qr, void* kr, void* stream);
+
+/* One ring step: partial (o_part, lse_part) of the local queries over the visiting
+ * chunk's keys (and the branch keys with include_branch).  Requires kv_start <= q_start
+ * (a chunk that starts later holds no visible key: skip it).  kr_local / v_local (the
+ * local chunk's rotated keys and public-layout values) are read only with
+ * include_branch.  status: a device word for the bounded waits (read it with
+ * ttt_attn_device_status). */
+ttt_status ttt_ring_step(const ttt_ring_desc* desc, const void* qr, const void* kr_local, const void* v_local,
+                         const void* kr_visit, const void* v_visit, float* o_part, float* lse_part, void* status,
+                         void* stream);
+
+/* o_acc, lse_acc <- their exact log-sum-exp merge with o_part, lse_part (first != 0:
+ * copy). */
+ttt_status ttt_ring_merge(const ttt_ring_desc* desc, float* o_acc, float* lse_acc, const float* o_part,
+                          const float* lse_part, int first, void* stream);
+
+/* o (bf16 [P][q_len][H][D]) <- o_acc; the lse is lse_acc itself. */
+ttt_status ttt_ring_finish(const ttt_ring_desc* desc, const float* o_acc, void* o, void* stream);
+
 /* The error behind the most recent TTT_ERR_CUDA returned by any call in this
  * process: a cudaError_t value, or 100000 + the CUresult when encoding a TMA tensor
  * map failed; 0 if there was none.  Not reset by later successful calls. */

@@ -563,3 +563,55 @@ def tail_trunk_dkv(q, k, v, do, theta, kv, t0, scale=None, rope_round="bf16"):
             dv += Pr[:, t0:L].T @ dO
     dk = rope_rotate(dkr[:, None, :], rows, theta, inverse=True)[:, 0]
     return dk, dv
+
+
+# --------------------------------------------------------------------------
+# context-parallel ring: the partial attention of one query chunk over one
+# chunk of trunk keys (NeMo-RL issue 3698, "What I'm working on", item 4)
+# --------------------------------------------------------------------------
+
+
+def chunk_partial(qc, kt, vt, theta, q_start, kv_start, branch_k=None, branch_v=None, scale=None,
+                  rope_round="bf16"):
+    """Partial attention of the query chunk qc [P, Lq, H, D] (pre-RoPE; row i of pass p0
+    at global position q_start + i + p0) over the trunk-key chunk kt, vt [Lk, Hkv, D]
+    (pass-1 keys at global positions kv_start + t): trunk key t is visible to row i iff
+    kv_start + t <= q_start + i.  With branch_k / branch_v ([P, Lq, Hkv, D], the chunk's
+    own keys and values of every pass) the branch keys of passes 2..p at the row's own
+    position join the partial.  Returns O [P, Lq, H, D] normalised over the visible keys
+    and lse [P, H, Lq] (-inf, with O = 0, for a row that sees no key)."""
+    P, Lq, H, D = qc.shape
+    Lk, Hkv = kt.shape[0], kt.shape[1]
+    g = H // Hkv
+    sc = _scale(D, scale)
+    ktr = rope_rotate(kt.astype(np.float64), np.arange(Lk) + kv_start, theta)
+    if branch_k is not None:
+        kbr = np.stack([rope_rotate(branch_k[j].astype(np.float64), np.arange(Lq) + q_start + j, theta)
+                        for j in range(P)])
+    qr = np.stack([rope_rotate(qc[p0].astype(np.float64), np.arange(Lq) + q_start + p0, theta) for p0 in range(P)])
+    if rope_round == "bf16":
+        ktr, qr = bf16_round(ktr), bf16_round(qr)
+        if branch_k is not None:
+            kbr = bf16_round(kbr)
+    visible = (kv_start + np.arange(Lk))[None, :] <= (q_start + np.arange(Lq))[:, None]   # [Lq, Lk]
+    O = np.zeros((P, Lq, H, D))
+    lse = np.full((P, H, Lq), -np.inf)
+    for h in range(H):
+        kv = h // g
+        for p0 in range(P):
+            s = np.where(visible, sc * (qr[p0, :, h] @ ktr[:, kv].T), -np.inf)              # [Lq, Lk]
+            vals = [vt[:, kv].astype(np.float64)]
+            if branch_k is not None and p0 > 0:
+                sb = sc * np.einsum("ld,jld->lj", qr[p0, :, h], kbr[1:p0 + 1, :, kv])      # [Lq, p0]
+                s = np.concatenate([s, sb], axis=1)
+            m = s.max(axis=1, keepdims=True)
+            has = np.isfinite(m[:, 0])
+            e = np.exp(s - np.where(np.isfinite(m), m, 0.0))
+            z = e.sum(axis=1)
+            w = e / np.where(z > 0, z, 1.0)[:, None]
+            out = w[:, :Lk] @ vals[0]
+            if branch_k is not None and p0 > 0:
+                out += np.einsum("lj,jld->ld", w[:, Lk:], branch_v[1:p0 + 1, :, kv].astype(np.float64))
+            O[p0, :, h] = out
+            lse[p0, h] = np.where(has, m[:, 0] + np.log(np.where(z > 0, z, 1.0)), -np.inf)
+    return O, lse

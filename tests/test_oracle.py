@@ -292,6 +292,46 @@ def test_tail_trunk_dkv_matches_full_oracle(t0):
         np.testing.assert_allclose(dv_t, dv[0, t0:, kv], atol=1e-12)
 
 
+def test_chunk_partial_whole_sequence_equals_the_oracle():
+    """One chunk holding the whole sequence, with its branch keys, is the full attention."""
+    P, L, H, Hkv, D = 3, 11, 4, 2, 8
+    q, k, v = rnd(P, L, H, D), rnd(P, L, Hkv, D), rnd(P, L, Hkv, D)
+    O, lse = orc.forward_twopart(q, k, v, 1e4)
+    Oc, lc = orc.chunk_partial(q, k[0], v[0], 1e4, 0, 0, branch_k=k, branch_v=v)
+    np.testing.assert_allclose(Oc, O, atol=1e-13)
+    np.testing.assert_allclose(lc, lse, atol=1e-13)
+
+
+@pytest.mark.parametrize("cuts", [(4, 7), (1, 10), (5,)])
+def test_chunk_partials_merge_to_the_oracle(cuts):
+    """Partials of every query chunk over every trunk-key chunk (its own chunk taking the
+    branch keys), merged by log-sum-exp (written out here), equal the full attention;
+    chunks that start after the query chunk contribute lse = -inf."""
+    P, L, H, Hkv, D = 3, 11, 4, 2, 8
+    q, k, v = rnd(P, L, H, D), rnd(P, L, Hkv, D), rnd(P, L, Hkv, D)
+    O, lse = orc.forward_twopart(q, k, v, 1e4)
+    bounds = [0, *cuts, L]
+    for qa, qb in zip(bounds[:-1], bounds[1:]):
+        acc_o, acc_l = None, None
+        for ka, kb in zip(bounds[:-1], bounds[1:]):
+            own = ka == qa
+            Op, lp = orc.chunk_partial(q[:, qa:qb], k[0, ka:kb], v[0, ka:kb], 1e4, qa, ka,
+                                       branch_k=k[:, qa:qb] if own else None, branch_v=v[:, qa:qb] if own else None)
+            if ka > qa:
+                assert np.all(lp == -np.inf) and np.all(Op == 0.0)
+            if acc_o is None:
+                acc_o, acc_l = Op, lp
+                continue
+            m = np.maximum(acc_l, lp)
+            ms = np.where(np.isfinite(m), m, 0.0)
+            l = ms + np.log(np.exp(acc_l - ms) + np.exp(lp - ms))
+            wa = np.exp(acc_l - l).transpose(0, 2, 1)[..., None]
+            wb = np.exp(lp - l).transpose(0, 2, 1)[..., None]
+            acc_o, acc_l = wa * acc_o + wb * Op, l
+        np.testing.assert_allclose(acc_o, O[:, qa:qb], atol=1e-12)
+        np.testing.assert_allclose(acc_l, lse[:, :, qa:qb], atol=1e-12)
+
+
 # ---------------------------------------------------------------- golden fixtures
 
 def _golden(name):
