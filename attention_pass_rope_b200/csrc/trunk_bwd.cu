@@ -387,8 +387,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int s = it % C::ST;
       const int b = it & 1;
       const IterInfo ii = decode_iter(it, nqt, jq0, G, gsz, kvh);
-      if (!wait_bounded(sdp_full, it & 1, wd, kSiteBwdSdpFull) ||
-          !wait_bounded(qdo_full + s, (it / C::ST) & 1, wd, kSiteBwdQdoFull)) {
+      // warp-agreed waits: the TMEM loads and stores that follow are warp-wide instructions
+      if (!wait_warp(sdp_full, it & 1, wd, kSiteBwdSdpFull) ||
+          !wait_warp(qdo_full + s, (it / C::ST) & 1, wd, kSiteBwdQdoFull)) {
         ok = false;
         break;
       }
@@ -457,7 +458,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       }
       if (lane == 0 && warp == 4) TTT_TRACE(8, it);
       // P^T / dS^T buffer b was last read by the products of step it-2
-      if (it >= 2 && !wait_bounded(mma_done + b, ((it >> 1) - 1) & 1, wd, kSiteBwdMmaDone)) {
+      if (it >= 2 && !wait_warp(mma_done + b, ((it >> 1) - 1) & 1, wd, kSiteBwdMmaDone)) {
         ok = false;
         break;
       }
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     // ---- epilogue: dV (half 0) and dK (half 1) of this CTA's keys, final: dV in bf16,
     // dK = sigma * R(pos)^T dk~ in bf16 (the trunk keys' rotation at their own position)
-    if (ok && wait_bounded(final_bar, 0, wd, kSiteBwdFinal)) {
+    if (ok && wait_warp(final_bar, 0, wd, kSiteBwdFinal)) {
       tc_fence_after();
       const int64_t tau = kstart + kpos;
       if (hf == 0) {

@@ -106,7 +106,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   uint64_t* s_full = v_empty + C::VST;     // [NQ]
   uint64_t* p_full = s_full + C::NQ;       // [NQ]
   uint64_t* o_final = p_full + C::NQ;      // [NQ]
-  uint64_t* drain = o_final + C::NQ;
+  uint64_t* p_half = o_final + C::NQ;      // [NQ]: P of the first 64 keys written
+  uint64_t* drain = p_half + C::NQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   uint32_t* abort_flag = tmem_slot + 1;
   int* nkv_slot = reinterpret_cast<int*>(abort_flag + 1);
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     for (int t = 0; t < C::NQ; ++t) {
       mbar_init(s_full + t, 1);
       mbar_init(p_full + t, 4);  // one arrival per softmax warp
+      mbar_init(p_half + t, 4);
       mbar_init(o_final + t, 1);
     }
     mbar_init(drain, 1);
@@ -208,12 +210,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           umma_ss_warp(d_tmem, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int s, bool acc) {
+      // O += P V over keys [16*k0, 16*k1) of the tile
+      auto issue_pv = [&](int t, int s, bool acc, int k0, int k1) {
         const uint64_t vd = dv0 + static_cast<uint32_t>((s * C::TILE) >> 4);
         const uint32_t d_tmem = tmem + C::COL_O0 + D * t;
         const uint32_t a_tmem = tmem + C::COL_S0 + 128 * t;
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
+        for (int kk = k0; kk < k1; ++kk)
           umma_ts_warp(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), idO, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_warp(q_full, 0, wd, kSiteFwdQ);
@@ -223,17 +226,25 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       for (int j = 0; ok && j <= nkv; ++j) {
         for (int t = 0; t < nq_tiles; ++t) {
           if (j > 0) {
-            if (!wait_warp(p_full + t, (j - 1) & 1, wd, kSiteFwdPFull)) {
+            // the first half of O += P V as soon as P of the first 64 keys is written, the
+            // second half when the whole of P is
+            if (!wait_warp(p_half + t, (j - 1) & 1, wd, kSiteFwdPFull)) {
               ok = false;
               break;
             }
-            TTT_TRACE(0 + t, j);
             if (t == 0 && !wait_warp(v_full + (j - 1) % C::VST, ((j - 1) / C::VST) & 1, wd, kSiteFwdKvFull)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_pv(t, (j - 1) % C::VST, j - 1 > 0);
+            issue_pv(t, (j - 1) % C::VST, j - 1 > 0, 0, C::BN / 32);
+            if (!wait_warp(p_full + t, (j - 1) & 1, wd, kSiteFwdPFull)) {
+              ok = false;
+              break;
+            }
+            TTT_TRACE(0 + t, j);
+            tc_fence_after();
+            issue_pv(t, (j - 1) % C::VST, true, C::BN / 32, C::BN / 16);
             if (j == nkv) umma_commit_warp(o_final + t);
             if (t == nq_tiles - 1) umma_commit_warp(v_empty + (j - 1) % C::VST);
           }
@@ -274,7 +285,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      if (!wait_bounded(s_full + t, j & 1, wd, kSiteFwdSFull)) {
+      if (!wait_warp(s_full + t, j & 1, wd, kSiteFwdSFull)) {  // warp-agreed: TMEM access follows
         ok = false;
         break;
       }
@@ -320,8 +331,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         l_run *= alpha;
         m_run = m_new;
       }
+      // a warp with a row whose O needs rescaling releases P only after the rescale (rare:
+      // the running max grew by more than 2^8); the others release the first 64 keys early
+      const bool warp_rescale = __any_sync(0xffffffffu, rescale && j > 0);
       float rsv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      // P = 2^(s*scale*log2e - m), bf16 pairs into the first 64 columns of S_t
+      // P = 2^(s*scale*log2e - m), bf16 pairs into the first 64 columns of S_t; the first
+      // 64 keys are released to the MMA warp before the last 64 are computed
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -334,6 +349,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(lane_base + colS + 16 * c, pk);
+        if (c == 1 && !warp_rescale) {
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_half + t);
+        }
       }
 #pragma unroll
       for (int u = 4; u > 0; u >>= 1)
@@ -341,8 +362,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int v = 0; v < u; ++v) rsv[v] += rsv[v + u];
       l_run += rsv[0];
       if (lane == 0 && wq == 0) TTT_TRACE(10 + t, j);
-      if (rescale && j > 0) {
-        // O of this row was complete up to tile j-1 when s_full fired (in-order MMAs)
+      if (warp_rescale) {
+        // O of this row was complete up to tile j-1 when s_full fired (in-order MMAs), and
+        // no O += P V of this tile runs before this warp releases P.  TMEM loads and
+        // stores are warp-wide instructions: the whole warp runs them, rows that need no
+        // rescaling with alpha = 1 (exact)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -357,10 +381,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + t);
+      if (lane == 0) {
+        if (warp_rescale) mbar_arrive(p_half + t);
+        mbar_arrive(p_full + t);
+      }
       if (lane == 0 && wq == 0) TTT_TRACE(12 + t, j);
     }
-    if (ok && (nkv == 0 || wait_bounded(o_final + t, 0, wd, kSiteFwdOFinal))) {
+    if (ok && (nkv == 0 || wait_warp(o_final + t, 0, wd, kSiteFwdOFinal))) {
       tc_fence_after();
       // ---- epilogue: branch keys (a3) and the exact joint-LSE merge (a4).
       // MODE 0: query (pass p, position qpos) also sees k~_j[tau], V_j[tau] of the branch

@@ -15,6 +15,7 @@ workload (one sequence and one KV head group), scaled to the metric's unit.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -181,16 +182,16 @@ def applicable_peak(peaks, peak_src, timed_s):
 
 # ----------------------------------------------------------------------------- ours
 
-def run_ours(args, rank, world, local):
-    from attention_pass_rope_b200 import _lib, ops
+class Job:
+    """One workload's step on the device: `step(events)` runs every kernel of the path once
+    over resident inputs; `host_in` / `dev_in` / `outputs` serve the end-to-end leg."""
 
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=device)
-    w = workload(args)
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def ttt_job(args, w, device, rank):
+    from attention_pass_rope_b200 import ops
     # every rank draws its own batch (weak scaling); the sizes are the workload's
     inp = ttt_inputs.make_inputs(w, seed=w.seed + rank)
 
@@ -210,6 +211,70 @@ def run_ours(args, rank, world, local):
     lse = torch.empty(lay.lse_shape, dtype=torch.float32, device=device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
 
+    def step(events=None):
+        # one workspace for both calls: the backward reuses the forward's rotated q~ / k~
+        ops.ttt_attn_fwd(q, k, v, workspace=ws, out=(o, lse), events=events, **kw)
+        ops.ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, out=(dq, dk, dv), events=events,
+                         rotated_in_workspace=True, **kw)
+
+    desc = (f"{w.name}: B={len(w.lengths)} S={w.lengths[0]} P={w.P} H={w.H}/{w.Hkv} D={w.D} theta={w.theta:g}"
+            if w.dense else
+            f"{w.name}: THD nseq={w.nseq} T={w.T} P={w.P} H={w.H}/{w.Hkv} D={w.D} theta={w.theta:g}")
+    return Job(step=step, ws=ws, host_src=(inp.q, inp.k, inp.v, inp.do), dev_in=(q, k, v, do),
+               outputs=(o, lse, dq, dk, dv), flops=w.flops_fwd_bwd(),
+               trunk_bwd_flops=10 * w.D * w.trunk_pairs * w.H * w.P, tokens=w.T, desc=desc,
+               launches=5, unit_note="tokens = B*S (or T) positions, each carrying P passes", name=w.name)
+
+
+def block_job(args, w, device, rank):
+    from attention_pass_rope_b200 import ops
+    inp = ttt_inputs.make_block_inputs(dataclasses.replace(w, seed=w.seed + rank))
+    B, S, nblk = w.nseq, w.ctx_lengths[0], w.nblocks[0]
+
+    def dev(t, shape):
+        return t.to(device).view(*shape).contiguous()
+
+    k_ctx, v_ctx = dev(inp.k_ctx, (B, S, w.Hkv, w.D)), dev(inp.v_ctx, (B, S, w.Hkv, w.D))
+    qb, do = dev(inp.qb, (B, nblk, w.Bs, w.H, w.D)), dev(inp.do, (B, nblk, w.Bs, w.H, w.D))
+    kb, vb = dev(inp.kb, (B, nblk, w.Bs, w.Hkv, w.D)), dev(inp.vb, (B, nblk, w.Bs, w.Hkv, w.D))
+    anchors = inp.anchors.to(device).view(B, nblk).contiguous()
+    lay = ops._block_layout(k_ctx, v_ctx, qb, kb, vb, anchors, None, None, None, None)
+    ws = ops.alloc_workspace(ops.block_workspace_bytes(lay, anchors, w.theta, for_backward=True), device)
+    o = torch.empty_like(qb)
+    lse = torch.empty(lay.lse_shape, dtype=torch.float32, device=device)
+    grads = tuple(torch.empty_like(t) for t in (k_ctx, v_ctx, qb, kb, vb))
+    args_ = (k_ctx, v_ctx, qb, kb, vb, anchors)
+
+    def step(events=None):
+        ops.block_attn_fwd(*args_, theta=w.theta, workspace=ws, out=(o, lse), events=events)
+        ops.block_attn_bwd(*args_, o, lse, do, theta=w.theta, workspace=ws, out=grads, events=events,
+                           rotated_in_workspace=True)
+
+    a = inp.anchors.tolist()
+    trunk_pairs = sum((x + 1) * w.Bs for x in a)  # per query head
+    desc = (f"{w.name}: block-draft B={B} context S={S} blocks={nblk} x Bs={w.Bs} H={w.H}/{w.Hkv} D={w.D} "
+            f"theta={w.theta:g}, anchors sorted uniform")
+    return Job(step=step, ws=ws, host_src=(inp.k_ctx, inp.v_ctx, inp.qb, inp.kb, inp.vb, inp.do),
+               dev_in=(k_ctx, v_ctx, qb, kb, vb, do), outputs=(o, lse) + grads, flops=w.flops_fwd_bwd(a),
+               trunk_bwd_flops=10 * w.D * trunk_pairs * w.H, tokens=w.NB * w.Bs, desc=desc, launches=6,
+               unit_note="tokens = block tokens", name=w.name)
+
+
+def run_ours(args, rank, world, local):
+    from attention_pass_rope_b200 import _lib, ops
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    if args.workload in ttt_inputs.block_workloads():
+        job = block_job(args, ttt_inputs.block_workloads()[args.workload], device, rank)
+    else:
+        job = ttt_job(args, workload(args), device, rank)
+    step, ws = job.step, job.ws
+
     # per-kernel CUDA events, recorded by the library on the launching stream
     K = args.steps
     evs = [_lib.TTTEvents() for _ in range(K)]
@@ -224,12 +289,6 @@ def run_ours(args, rank, world, local):
             e.stop[kk] = b.cuda_event
             objs.append((a, b))
         ev_objs.append(objs)
-
-    def step(events=None):
-        # one workspace for both calls: the backward reuses the forward's rotated q~ / k~
-        ops.ttt_attn_fwd(q, k, v, workspace=ws, out=(o, lse), events=events, **kw)
-        ops.ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, out=(dq, dk, dv), events=events,
-                         rotated_in_workspace=True, **kw)
 
     for _ in range(args.warmup):
         step()
@@ -266,17 +325,16 @@ def run_ours(args, rank, world, local):
         raise RuntimeError(f"device status after timing: {st} {word:#x}")
 
     # end to end: pinned host inputs -> device, fwd+bwd, results back to pinned host memory
-    host_in = [t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.do)]
-    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+    host_in = [t.pin_memory() for t in job.host_src]
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in job.outputs]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
-    dev_in = [q, k, v, do]
 
     def e2e_step():
-        for hsrc, dst in zip(host_in, dev_in):
+        for hsrc, dst in zip(host_in, job.dev_in):
             dst.view(-1).copy_(hsrc.view(-1), non_blocking=True)
         step()
-        for src, hdst in zip((o, lse, dq, dk, dv), host_out):
+        for src, hdst in zip(job.outputs, host_out):
             hdst.copy_(src, non_blocking=True)
 
     E = max(1, min(K, 5))
@@ -296,16 +354,15 @@ def run_ours(args, rank, world, local):
         ms, e2e_ms = max_over_ranks([ms, e2e_ms], device)
 
     ms_step = ms / K
-    flops = w.flops_fwd_bwd()
+    flops = job.flops
     tflops = whole_job_tflops(flops, world, ms_step)
     peaks, peak_src = load_peaks()
     peak, peak_kind = applicable_peak(peaks, peak_src, ms * 1e-3)
     # dominant kernel: the trunk backward (tensor bound); its algorithmic flops per launch
-    # are 10*D per visible trunk pair per query head and pass
-    bwd_flops = 10 * w.D * w.trunk_pairs * w.H * w.P
+    # are 10*D per visible trunk pair per query head (and pass)
     bwd_ms = per_kernel["trunk_bwd"]
-    achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
-    traffic = read_traffic("trunk_bwd", w.name)
+    achieved = job.trunk_bwd_flops / (bwd_ms * 1e-3) / 1e12
+    traffic = read_traffic("trunk_bwd", job.name)
     line = {
         "metric": METRIC,
         "value": round(tflops, 2),
@@ -319,12 +376,10 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={len(w.lengths)} S={w.lengths[0]} P={w.P} H={w.H}/{w.Hkv} D={w.D} "
-                               f"theta={w.theta:g}" if w.dense else
-                   f"{w.name}: THD nseq={w.nseq} T={w.T} P={w.P} H={w.H}/{w.Hkv} D={w.D} theta={w.theta:g}",
-                   "tokens_per_step": w.T, "flops_per_step": flops, "parallelism": f"replicas{world}",
-                   "l2": "inputs per step (q,k,v,dO: %.0f MB) exceed L2 (126 MB)" % (h2d / 1e6)},
-        "tokens_per_s": round(w.T * world / (ms_step * 1e-3), 1),
+        "config": {"workload": job.desc, "tokens_per_step": job.tokens, "tokens": job.unit_note,
+                   "flops_per_step": flops, "parallelism": f"replicas{world}",
+                   "l2": "inputs per step (%.0f MB) exceed L2 (126 MB)" % (h2d / 1e6)},
+        "tokens_per_s": round(job.tokens * world / (ms_step * 1e-3), 1),
         "pct_of_peak": round(100.0 * tflops / world / peak, 2),
         "peak": {"tflops": peak, "source": peak_kind, "pct_of_burst": round(100.0 * tflops / world / peaks["bf16_tflops"], 2),
                  "pct_of_sustained": round(100.0 * tflops / world / peaks["bf16_tflops_sustained"], 2)},
@@ -337,11 +392,14 @@ def run_ours(args, rank, world, local):
                      "traffic": traffic},
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * K,  # rope, trunk fwd; preprocess, trunk bwd, branch bwd
+        "gpu_launches": job.launches * K,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        if args.workload in ttt_inputs.block_workloads():
+            line["cpu_baseline"] = block_cpu_baseline(ttt_inputs.block_workloads()[args.workload])
+        else:
+            line["cpu_baseline"] = cpu_baseline(workload(args), budget_s=args.cpu_budget)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
@@ -418,19 +476,47 @@ def cpu_baseline(w, budget_s=30.0):
             "seconds": round(dt, 2)}
 
 
+def block_cpu_baseline(w):
+    """The fp64 block-draft oracle on one sequence and one KV-head group of the workload."""
+    import numpy as np
+    from oracle import block_draft_oracle as bd
+    inp = ttt_inputs.make_block_inputs(w)
+    g = w.H // w.Hkv
+    b1 = w.cu_blocks[1]
+    f64 = lambda x: x.float().numpy().astype(np.float64)
+    c = dict(k_ctx=f64(inp.k_ctx[:w.cu_ctx[1], :1]), v_ctx=f64(inp.v_ctx[:w.cu_ctx[1], :1]),
+             anchors=inp.anchors[:b1].tolist(), qb=f64(inp.qb[:b1, :, :g]), kb=f64(inp.kb[:b1, :, :1]),
+             vb=f64(inp.vb[:b1, :, :1]))
+    t0 = time.perf_counter()
+    O, lse = bd.forward_twopart(theta=w.theta, rope_round="bf16", **c)
+    bd.backward_twopart(do=f64(inp.do[:b1, :, :g]), O=O, lse=lse, theta=w.theta, rope_round="bf16", **c)
+    dt = time.perf_counter() - t0
+    sub = dataclasses.replace(w, H=g, Hkv=1, ctx_lengths=w.ctx_lengths[:1], nblocks=w.nblocks[:1])
+    fl = sub.flops_fwd_bwd(inp.anchors[:b1].tolist())
+    cores = blas_threads() or len(os.sched_getaffinity(0))
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 block-draft oracle, fwd+bwd of sequence 0 and KV head 0 = 1/{w.nseq * w.Hkv} of the "
+                      f"workload, {dt:.1f} s", "seconds": round(dt, 2)}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = workload(args)
-    for _ in range(args.warmup and 1):
-        pass  # the oracle has no warm-up state; one untimed sample below warms the BLAS pool
-    oracle_sample(ttt_inputs.thd("warm", [256], w.P, w.H // w.Hkv, 1, w.D, w.theta))
-    times, fl = [], None
-    for _ in range(args.steps):
-        dt, fl, _ = oracle_sample(w)
-        times.append(dt)
-    dt = sum(times) / len(times)
-    value = fl / dt / 1e12
+    if args.workload in ttt_inputs.block_workloads():
+        wb = ttt_inputs.block_workloads()[args.workload]
+        runs = [block_cpu_baseline(wb) for _ in range(args.steps)]
+        dt = sum(r["seconds"] for r in runs) / len(runs)
+        value = sum(r["value"] for r in runs) / len(runs)
+    else:
+        w = workload(args)
+        # the oracle has no warm-up state; one untimed sample warms the BLAS pool
+        oracle_sample(ttt_inputs.thd("warm", [256], w.P, w.H // w.Hkv, 1, w.D, w.theta))
+        times, fl = [], None
+        for _ in range(args.steps):
+            dt, fl, _ = oracle_sample(w)
+            times.append(dt)
+        dt = sum(times) / len(times)
+        value = fl / dt / 1e12
     cores = blas_threads() or len(os.sched_getaffinity(0))
     line = {
         "impl": "reference",
@@ -460,7 +546,8 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ttt_inputs.workloads()))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(ttt_inputs.workloads()) + sorted(ttt_inputs.block_workloads()))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=30.0)
     ap.add_argument("--batch", type=int, default=0, help="override B of a dense workload (profiling)")
