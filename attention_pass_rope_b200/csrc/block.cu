@@ -40,7 +40,7 @@ struct RowPositions {
 };
 
 // dst_x[head][tau][:] = R(pos(tau)) src_x[tau][head][:] for the heads of up to two
-// tensors that share the rows' positions (rotate-half RoPE, fp32 math, bf16 out;
+// tensors that share the rows' positions (rotate-half RoPE, double math, bf16 out;
 // outputs head-major so that a (head, 128-row) tile is one contiguous block for TMA).
 template <int D>
 __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int T, RowPositions posf,
@@ -50,16 +50,16 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
                                                                  __nv_bfloat16* __restrict__ dst_b) {
   constexpr int HALF = D / 2;
   constexpr int PARTS = HALF / 8;
-  __shared__ float2 cs[kRopeRows][HALF];
+  __shared__ double2 cs[kRopeRows][HALF];
   const int r0 = blockIdx.x * kRopeRows;
   const int nrows = min(kRopeRows, T - r0);
   for (int e = threadIdx.x; e < kRopeRows * HALF; e += blockDim.x) {
     const int r = e / HALF, d = e % HALF;
     if (r >= nrows) continue;
     const double inv_freq = pow(static_cast<double>(g.theta), -2.0 * d / D);
-    float c, s;
-    angle_cos_sin(posf(g, r0 + r), inv_freq, c, s);
-    cs[r][d] = make_float2(c, s);
+    double s, c;
+    sincos(static_cast<double>(posf(g, r0 + r)) * inv_freq, &s, &c);
+    cs[r][d] = make_double2(c, s);
   }
   __syncthreads();
   const int NH = nha + nhb;
@@ -89,11 +89,9 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float2 rr = cs[r][d0 + e];
-      const float x1 = __bfloat162float(xa[e]);
-      const float x2 = __bfloat162float(xb[e]);
-      ya[e] = __float2bfloat16_rn(fmaf(x1, rr.x, -x2 * rr.y));
-      yb[e] = __float2bfloat16_rn(fmaf(x2, rr.x, x1 * rr.y));
+      const double2 rr = cs[r][d0 + e];
+      ya[e] = rotate_round(xa[e], xb[e], rr, false);
+      yb[e] = rotate_round(xa[e], xb[e], rr, true);
     }
     *reinterpret_cast<uint4*>(dst + d0) = oa;
     *reinterpret_cast<uint4*>(dst + HALF + d0) = ob;

@@ -180,13 +180,16 @@ __global__ void __launch_bounds__(kPreThreads)
 //     dQ_p = R(i+p)^T (sigma dq~)
 //   dK_j = R(i+j)^T (sigma dk~_j) and dV_j for the branch passes j >= 1 (dK_1 and dV_1
 //   are written by the trunk backward).
-// The kernel is bound by memory latency: each warp keeps the next (pass, head) row's
-// loads in flight while it computes the current one.  Shared memory: the block's
-// inverse frequencies (double), then per warp the cos/sin of positions i..i+P-1 and the
-// branch-pass accumulators.
+// The kernel is bound by memory latency, so resident warps matter most: the group
+// heads of a pass go kBranchHeads at a time (one: more heads per warp keep more rows
+// in flight but cost registers, and 64 registers at four blocks per SM measured
+// fastest).  Shared memory: the block's inverse frequencies (double), then per warp
+// the cos/sin of positions i..i+P-1 and the branch-pass accumulators.
 // ---------------------------------------------------------------------------
+constexpr int kBranchHeads = 1;
+
 template <int D>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32, 3)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
     branch_bwd_kernel(Geometry g, const __nv_bfloat16* __restrict__ qr, const __nv_bfloat16* __restrict__ kr,
                       const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ ld,
@@ -230,76 +233,91 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 3)
   const int64_t dl_base = static_cast<int64_t>(ld_slots(g.si)) * 128;
   const int64_t dl_off = static_cast<int64_t>(ld_slot(tau - pos, n, pos)) * 128 + 64 + (pos & 63);
 
-  // The rows of the (pass, head) pairs go one after another; the loads of the next row
-  // are issued before the current one is computed (memory latency bounds this kernel,
-  // so the bytes in flight per warp are what count).
-  struct Row {
-    float dqv[2][E], q[2][E], dO[2][E];
-    float lse, dl;
-  };
-  auto load_row = [&](int it, Row& r) {
-    const int p = it / gsz;
-    const int h = kvh * gsz + it % gsz;
-    const int64_t hrow = (static_cast<int64_t>(p) * g.H + h) * T + tau;
-    load_f32_row<D>(dq_acc + hrow * D, lane, r.dqv);
-    if (p > 0) {
-      load_bf16_row<D>(qr + hrow * D, lane, r.q);
-      load_bf16_row<D>(dout + p * g.sq + (static_cast<int64_t>(tau) * g.H + h) * D, lane, r.dO);
-      r.lse = lse[lse_index(g.si, g.H, p, h, n, tau, pos)];
-      r.dl = ld[(static_cast<int64_t>(p) * g.H + h) * dl_base + dl_off];
-    }
-  };
-  const int NIT = g.P * gsz;
-  Row cur, nxt;
-  load_row(0, cur);
-  for (int it = 0; it < NIT; ++it) {
-    if (it + 1 < NIT) load_row(it + 1, nxt);
-    const int p = it / gsz;
-    const int h = kvh * gsz + it % gsz;
-    for (int j = 1; j <= p; ++j) {
-      float kj[2][E], vj[2][E];
-      load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
-      load_bf16_row<D>(v + j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D, lane, vj);
-      float sdot = 0.f, tdot = 0.f;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          sdot = fmaf(cur.q[hh][e], kj[hh][e], sdot);
-          tdot = fmaf(cur.dO[hh][e], vj[hh][e], tdot);
-        }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
-        tdot += __shfl_xor_sync(0xffffffffu, tdot, o);
-      }
-      const float pj = __expf(sdot * g.scale - cur.lse);
-      const float dsj = pj * (tdot - cur.dl);
-      float* akp = acc + ((j - 1) * 2 + 0) * D;
-      float* avp = acc + ((j - 1) * 2 + 1) * D;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int d = LaneMap<D>::d(lane, hh, e);
-          cur.dqv[hh][e] = fmaf(dsj, kj[hh][e], cur.dqv[hh][e]);
-          akp[d] = fmaf(dsj, cur.q[hh][e], akp[d]);
-          avp[d] = fmaf(pj, cur.dO[hh][e], avp[d]);
-        }
-    }
+  for (int p = 0; p < g.P; ++p) {
     float c[E], sn[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       c[e] = cs[p * D + LaneMap<D>::d(lane, 0, e)];
       sn[e] = cs[p * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
     }
+    for (int h0 = 0; h0 < gsz; h0 += kBranchHeads) {
+      float dqv[kBranchHeads][2][E], q[kBranchHeads][2][E], dO[kBranchHeads][2][E];
+      float lse_v[kBranchHeads], dl[kBranchHeads];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
+      for (int u = 0; u < kBranchHeads; ++u) {
+        const int h = kvh * gsz + h0 + u;
+        if (h0 + u < gsz) {
+          const int64_t hrow = (static_cast<int64_t>(p) * g.H + h) * T + tau;
+          load_f32_row<D>(dq_acc + hrow * D, lane, dqv[u]);
+          if (p > 0) {
+            load_bf16_row<D>(qr + hrow * D, lane, q[u]);
+            load_bf16_row<D>(dout + p * g.sq + (static_cast<int64_t>(tau) * g.H + h) * D, lane, dO[u]);
+            lse_v[u] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)];
+            dl[u] = ld[(static_cast<int64_t>(p) * g.H + h) * dl_base + dl_off];
+          }
+        }
+      }
+      for (int j = 1; j <= p; ++j) {
+        float kj[2][E], vj[2][E];
+        load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
+        load_bf16_row<D>(v + j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D, lane, vj);
+        float sdot[kBranchHeads], tdot[kBranchHeads];
 #pragma unroll
-      for (int e = 0; e < E; ++e) cur.dqv[hh][e] *= g.scale;
-    rotate_back<D>(cur.dqv, c, sn);
-    store_bf16_row<D>(dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + h) * D, lane, cur.dqv);
-    cur = nxt;
+        for (int u = 0; u < kBranchHeads; ++u) {
+          sdot[u] = 0.f;
+          tdot[u] = 0.f;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              sdot[u] = fmaf(q[u][hh][e], kj[hh][e], sdot[u]);
+              tdot[u] = fmaf(dO[u][hh][e], vj[hh][e], tdot[u]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int u = 0; u < kBranchHeads; ++u) {
+            sdot[u] += __shfl_xor_sync(0xffffffffu, sdot[u], o);
+            tdot[u] += __shfl_xor_sync(0xffffffffu, tdot[u], o);
+          }
+        float ak[2][E] = {}, av[2][E] = {};
+#pragma unroll
+        for (int u = 0; u < kBranchHeads; ++u) {
+          if (h0 + u >= gsz) continue;
+          const float pj = __expf(sdot[u] * g.scale - lse_v[u]);
+          const float dsj = pj * (tdot[u] - dl[u]);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              dqv[u][hh][e] = fmaf(dsj, kj[hh][e], dqv[u][hh][e]);
+              ak[hh][e] = fmaf(dsj, q[u][hh][e], ak[hh][e]);
+              av[hh][e] = fmaf(pj, dO[u][hh][e], av[hh][e]);
+            }
+        }
+        float* akp = acc + ((j - 1) * 2 + 0) * D;
+        float* avp = acc + ((j - 1) * 2 + 1) * D;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const int d = LaneMap<D>::d(lane, hh, e);
+            akp[d] += ak[hh][e];
+            avp[d] += av[hh][e];
+          }
+      }
+#pragma unroll
+      for (int u = 0; u < kBranchHeads; ++u) {
+        if (h0 + u >= gsz) continue;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int e = 0; e < E; ++e) dqv[u][hh][e] *= g.scale;
+        rotate_back<D>(dqv[u], c, sn);
+        store_bf16_row<D>(dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz + h0 + u) * D, lane, dqv[u]);
+      }
+    }
   }
   // dK and dV of the branch passes (those of the trunk pass come from the trunk backward)
   for (int j = 1; j < g.P; ++j) {

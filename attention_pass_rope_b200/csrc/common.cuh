@@ -443,6 +443,21 @@ __device__ __forceinline__ void angle_cos_sin(int pos, double inv_freq, float& c
   sincosf(static_cast<float>(red), &s, &c);
 }
 
+// One output of the rotate-half rotation of the pair (x1, x2) by (cos, sin) = r:
+// x1 cos - x2 sin (first half) or x2 cos + x1 sin (second half), each product and the
+// sum rounded in double (no fused multiply-add), the result rounded to fp32 and then to
+// bf16 (round to nearest even).  Evaluating in double leaves the bf16 result equal to
+// rounding the exact rotation, except when it lies within a few double ulps of a bf16
+// rounding boundary.
+__device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bfloat16 x2b, double2 r,
+                                                      bool second) {
+  const double x1 = static_cast<double>(__bfloat162float(x1b));
+  const double x2 = static_cast<double>(__bfloat162float(x2b));
+  const double y = second ? __dadd_rn(__dmul_rn(x2, r.x), __dmul_rn(x1, r.y))
+                          : __dsub_rn(__dmul_rn(x1, r.x), __dmul_rn(x2, r.y));
+  return __float2bfloat16_rn(static_cast<float>(y));
+}
+
 // Trunk-key limit of block-draft query row r of a sequence whose block rows start at
 // qstart (a multiple of Bs) and whose context has klen keys: its block's anchor,
 // clamped to [0, klen - 1] (-1, no trunk key, for an empty context).

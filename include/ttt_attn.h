@@ -16,7 +16,8 @@
  *     the branch keys (empty for p = 1: lse_b = -inf);
  *     lse = logaddexp(lse_t, lse_b),  O = e^(lse_t-lse) O_t + e^(lse_b-lse) O_b.
  *   This equals one softmax over the (i+1)+(p-1) visible keys.  The rotated q~ and
- *   k~ are computed in fp32 and rounded to bf16 before the dot products.
+ *   k~ are evaluated in double precision and rounded to bf16 (through fp32) before the
+ *   dot products, which run on bf16 tensor-core operands with fp32 accumulation.
  *   R(m) pairs dimension d with d + D/2 and rotates by m * theta^(-2d/D).
  *
  * Layouts (all pass-major, the trunk is index 0 along P, row-major):

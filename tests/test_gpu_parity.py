@@ -97,11 +97,13 @@ def test_rotated_inputs_tiny():
     kr = view(2, P * Hkv * T * D, torch.bfloat16).view(P, Hkv, T, D).permute(0, 2, 1, 3)
     qn, kn, vn, _ = parity.oracle_np(inp)
     qr_ref, kr_ref = orc.rotate_inputs(qn, kn, w.theta, rope_round="bf16")
-    # fp32 rotation vs fp64 rotation, both rounded to bf16: a rare one-ulp flip
+    # both evaluate the rotation in double and round it to bf16 through fp32: equal except
+    # where the exact value sits within a few double ulps of a bf16 rounding boundary
     dq_ = np.abs(parity.to64(qr) - qr_ref)
-    assert np.mean(dq_ > 0) < 2e-3 and np.max(dq_) <= 2.0 ** -7 * np.max(np.abs(qr_ref))
     dk_ = np.abs(parity.to64(kr) - kr_ref)
-    assert np.mean(dk_ > 0) < 2e-3
+    print("rotated q~ / k~ elements that differ:", int(np.sum(dq_ > 0)), int(np.sum(dk_ > 0)), "of", dq_.size, dk_.size)
+    assert np.sum(dq_ > 0) <= 2 and np.sum(dk_ > 0) <= 2
+    assert np.max(dq_) <= 2.0 ** -7 * np.max(np.abs(qr_ref))
 
 
 @needs_cuda
