@@ -40,7 +40,7 @@ struct RowPositions {
 };
 
 // dst_x[head][tau][:] = R(pos(tau)) src_x[tau][head][:] for the heads of up to two
-// tensors that share the rows' positions (rotate-half RoPE, double math, bf16 out;
+// tensors that share the rows' positions (rotate-half RoPE rounded as in fp64, bf16 out;
 // outputs head-major so that a (head, 128-row) tile is one contiguous block for TMA).
 template <int D>
 __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int T, RowPositions posf,
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
                                                                  __nv_bfloat16* __restrict__ dst_b) {
   constexpr int HALF = D / 2;
   constexpr int PARTS = HALF / 8;
-  __shared__ double2 cs[kRopeRows][HALF];
+  __shared__ float4 cs[kRopeRows][HALF];
   const int r0 = blockIdx.x * kRopeRows;
   const int nrows = min(kRopeRows, T - r0);
   for (int e = threadIdx.x; e < kRopeRows * HALF; e += blockDim.x) {
@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     const double inv_freq = pow(static_cast<double>(g.theta), -2.0 * d / D);
     double s, c;
     sincos(static_cast<double>(posf(g, r0 + r)) * inv_freq, &s, &c);
-    cs[r][d] = make_double2(c, s);
+    cs[r][d] = cos_sin_split(c, s);
   }
   __syncthreads();
   const int NH = nha + nhb;
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const double2 rr = cs[r][d0 + e];
+      const float4 rr = cs[r][d0 + e];
       ya[e] = rotate_round(xa[e], xb[e], rr, false);
       yb[e] = rotate_round(xa[e], xb[e], rr, true);
     }
@@ -105,19 +105,40 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
 //   dq~_i = (trunk part, from the trunk backward) + sum_j dS_ij k~_j
 //   dk~_j += sum_i dS_ij q~_i,  dV_j += sum_i P_ij dO_i         (over the group's heads)
 // then dQ_i = sigma R(a+i)^T dq~_i, dK_j = sigma R(a+j)^T dk~_j, dV_j, all bf16.
+// The group's heads are stacked into up to 64 query rows (r = head * Bs + i) so that
+// every product is a small matrix product over shared memory; each thread computes a
+// register block of it (4x4 scores, 4 rows x 16 columns of dq, 4 keys x 8 columns of
+// dk~ / dV), which keeps shared-memory traffic per multiply-add low.
 // ---------------------------------------------------------------------------
 constexpr int kBlockThreads = 128;
+constexpr int kBlockRows = 64;  // stacked query rows per pass over the group's heads
 
 template <int D>
 struct BlockSmem {
-  static constexpr int LD = D + 1;  // padded rows: a column walk touches distinct banks
-  static constexpr int kMaxBs = 16;
-  // K, V, Q, dO, accK, accV rows; S and dP [Bs][Bs]; cos/sin [Bs][D/2]
-  static constexpr size_t bytes(int Bs) {
-    return (6 * static_cast<size_t>(Bs) * LD + 2 * static_cast<size_t>(Bs) * Bs + 2 * static_cast<size_t>(Bs) * (D / 2)) *
-           sizeof(float);
-  }
+  static constexpr int LD = D + 4;  // row stride (floats): 16-byte aligned rows, staggered banks
+  static constexpr int BP = 16;     // block keys, padded
+  // Q, dO [64][LD]; K, V [16][LD]; P, dS [64][16]; cos, sin [16][D/2]; lse, delta [64]
+  static constexpr size_t kFloats = 2 * kBlockRows * LD + 2 * BP * LD + 2 * kBlockRows * BP + 2 * BP * (D / 2) +
+                                    2 * kBlockRows;
+  static constexpr size_t bytes = kFloats * sizeof(float);
 };
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void fma4(float (&acc)[4], float a, const float4& b) {
+  acc[0] = fmaf(a, b.x, acc[0]);
+  acc[1] = fmaf(a, b.y, acc[1]);
+  acc[2] = fmaf(a, b.z, acc[2]);
+  acc[3] = fmaf(a, b.w, acc[3]);
+}
+__device__ __forceinline__ float dot4(const float4& a, const float4& b, float acc) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+__device__ __forceinline__ float4 bf4(const __nv_bfloat16* p) {  // 4 bf16 -> float4 (8-byte aligned)
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kBlockThreads)
@@ -127,20 +148,21 @@ __global__ void __launch_bounds__(kBlockThreads)
                      __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
   using SM = BlockSmem<D>;
   constexpr int LD = SM::LD;
+  constexpr int BP = SM::BP;
   constexpr int HALF = D / 2;
   extern __shared__ __align__(16) float blk_smem[];
-  const int Bs = g.Bs;
-  float* sK = blk_smem;
-  float* sV = sK + Bs * LD;
-  float* sQ = sV + Bs * LD;
-  float* sO = sQ + Bs * LD;  // dO
-  float* aK = sO + Bs * LD;
-  float* aV = aK + Bs * LD;
-  float* sS = aV + Bs * LD;  // S, then P
-  float* sP = sS + Bs * Bs;  // dP, then dS
-  float* sC = sP + Bs * Bs;  // cos [Bs][D/2]
-  float* sN = sC + Bs * HALF;  // sin
+  float* sQ = blk_smem;                  // [64][LD]
+  float* sO = sQ + kBlockRows * LD;      // [64][LD] dO
+  float* sK = sO + kBlockRows * LD;      // [16][LD]
+  float* sV = sK + BP * LD;              // [16][LD]
+  float* sP = sV + BP * LD;              // [64][16] scores, then P
+  float* sD = sP + kBlockRows * BP;      // [64][16] dP, then dS
+  float* sC = sD + kBlockRows * BP;      // [16][D/2] cos
+  float* sN = sC + BP * HALF;            // [16][D/2] sin
+  float* sL = sN + BP * HALF;            // [64] lse
+  float* sDl = sL + kBlockRows;          // [64] delta
 
+  const int Bs = g.Bs;
   const int b = static_cast<int>(blockIdx.x) / g.Hkv;
   const int kvh = static_cast<int>(blockIdx.x) % g.Hkv;
   const int T = g.si.T;  // block rows
@@ -152,15 +174,20 @@ __global__ void __launch_bounds__(kBlockThreads)
   const int qstart = row0 - pos0;
   const int anchor = block_row_position(g, qstart, pos0, klen);  // position of token 0
   const int gsz = g.H / g.Hkv;
+  const int hc = max(1, min(gsz, kBlockRows / Bs));  // heads per pass
   const int nslots = ld_slots(g.si);
   const int tid = threadIdx.x;
 
-  for (int e = tid; e < Bs * D; e += blockDim.x) {
-    const int j = e / D, d = e % D;
-    sK[j * LD + d] = __bfloat162float(kr[(static_cast<int64_t>(kvh) * T + row0 + j) * D + d]);
-    sV[j * LD + d] = __bfloat162float(vb[(static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D + d]);
-    aK[j * LD + d] = 0.f;
-    aV[j * LD + d] = 0.f;
+  // block keys / values (rows >= Bs zero), cos / sin of the block's positions
+  for (int e = tid; e < BP * (D / 4); e += blockDim.x) {
+    const int j = e / (D / 4), d = 4 * (e % (D / 4));
+    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), v4 = k4;
+    if (j < Bs) {
+      k4 = bf4(kr + (static_cast<int64_t>(kvh) * T + row0 + j) * D + d);
+      v4 = bf4(vb + (static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D + d);
+    }
+    *reinterpret_cast<float4*>(sK + j * LD + d) = k4;
+    *reinterpret_cast<float4*>(sV + j * LD + d) = v4;
   }
   for (int e = tid; e < Bs * HALF; e += blockDim.x) {
     const int i = e / HALF, d = e % HALF;
@@ -170,72 +197,167 @@ __global__ void __launch_bounds__(kBlockThreads)
     sN[i * HALF + d] = s;
   }
 
-  for (int hh = 0; hh < gsz; ++hh) {
-    const int h = kvh * gsz + hh;
-    __syncthreads();  // previous head's readers of sQ / sO / sS / sP are done
-    for (int e = tid; e < Bs * D; e += blockDim.x) {
-      const int i = e / D, d = e % D;
-      sQ[i * LD + d] = __bfloat162float(qr[(static_cast<int64_t>(h) * T + row0 + i) * D + d]);
-      sO[i * LD + d] = __bfloat162float(dout[(static_cast<int64_t>(row0 + i) * g.H + h) * D + d]);
-    }
-    __syncthreads();
-    // scores and dP of every (i, j) pair
-    for (int e = tid; e < Bs * Bs; e += blockDim.x) {
-      const int i = e / Bs, j = e % Bs;
-      float s = 0.f, t = 0.f;
-#pragma unroll 8
-      for (int d = 0; d < D; ++d) {
-        s = fmaf(sQ[i * LD + d], sK[j * LD + d], s);
-        t = fmaf(sO[i * LD + d], sV[j * LD + d], t);
+  // dk~ / dV accumulators: thread -> (4 keys, 8 columns) of dk~ (tid < 64) or of dV
+  const bool acc_v = tid >= 64;
+  const int akb = (tid & 63) / (D / 8);        // key block (4 keys)
+  const int acol = 8 * ((tid & 63) % (D / 8));  // 8 consecutive columns
+  const bool acc_on = akb < BP / 4;
+  float acc[4][8] = {};
+
+  for (int h0 = 0; h0 < gsz; h0 += hc) {
+    const int nh = min(hc, gsz - h0);
+    const int R = nh * Bs;
+    const int RP = (R + 3) & ~3;
+    __syncthreads();  // the previous pass's readers of sQ / sO / sP / sD are done
+    for (int e = tid; e < RP * (D / 4); e += blockDim.x) {
+      const int r = e / (D / 4), d = 4 * (e % (D / 4));
+      float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), o4 = q4;
+      if (r < R) {
+        const int h = kvh * gsz + h0 + r / Bs, i = r % Bs;
+        q4 = bf4(qr + (static_cast<int64_t>(h) * T + row0 + i) * D + d);
+        o4 = bf4(dout + (static_cast<int64_t>(row0 + i) * g.H + h) * D + d);
       }
-      const int pos = pos0 + i;
-      const float l = lse[lse_index(g.si, g.H, 0, h, n, row0 + i, pos)];
-      const float delta = ld[(static_cast<int64_t>(h) * nslots + ld_slot(qstart, n, pos)) * 128 + 64 + (pos & 63)];
-      const float p = __expf(s * g.scale - l);
-      sS[e] = p;
-      sP[e] = p * (t - delta);
+      *reinterpret_cast<float4*>(sQ + r * LD + d) = q4;
+      *reinterpret_cast<float4*>(sO + r * LD + d) = o4;
+    }
+    for (int r = tid; r < RP; r += blockDim.x) {
+      float l = 0.f, dl = 0.f;
+      if (r < R) {
+        const int h = kvh * gsz + h0 + r / Bs, pos = pos0 + r % Bs;
+        l = lse[lse_index(g.si, g.H, 0, h, n, row0 + r % Bs, pos)];
+        dl = ld[(static_cast<int64_t>(h) * nslots + ld_slot(qstart, n, pos)) * 128 + 64 + (pos & 63)];
+      }
+      sL[r] = l;
+      sDl[r] = dl;
     }
     __syncthreads();
-    // dq of the block tokens: trunk part + block part, then sigma and R^T
-    for (int e = tid; e < Bs * HALF; e += blockDim.x) {
-      const int i = e / HALF, d = e % HALF;
-      const float* acc = dq_acc + (static_cast<int64_t>(h) * T + row0 + i) * D;
-      float x1 = acc[d], x2 = acc[d + HALF];
+    // scores (threads 0..63) and dP (64..127), 4x4 blocks of (rows, keys)
+    {
+      const int blk = tid & 63;
+      const int rb = blk / (BP / 4), cb = blk % (BP / 4);
+      if (4 * rb < RP) {
+        const float* A = tid < 64 ? sQ : sO;
+        const float* Bm = tid < 64 ? sK : sV;
+        float s[4][4] = {};
+#pragma unroll 4
+        for (int d = 0; d < D; d += 4) {
+          float4 a[4], bb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) a[u] = ld4(A + (4 * rb + u) * LD + d);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) bb[v] = ld4(Bm + (4 * cb + v) * LD + d);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) s[u][v] = dot4(a[u], bb[v], s[u][v]);
+        }
+        float* out = tid < 64 ? sP : sD;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<float4*>(out + (4 * rb + u) * BP + 4 * cb) = make_float4(s[u][0], s[u][1], s[u][2], s[u][3]);
+      }
+    }
+    __syncthreads();
+    // P = exp(sigma s - lse), dS = P (dP - delta); padding rows and keys give 0
+    for (int e = tid; e < RP * BP; e += blockDim.x) {
+      const int r = e / BP, j = e % BP;
+      float p = 0.f, ds = 0.f;
+      if (r < R && j < Bs) {
+        p = __expf(sP[e] * g.scale - sL[r]);
+        ds = p * (sD[e] - sDl[r]);
+      }
+      sP[e] = p;
+      sD[e] = ds;
+    }
+    __syncthreads();
+    // dq of the rows: 4 rows x (8 + 8 paired) columns per item
+    for (int item = tid; item < (RP / 4) * (HALF / 8); item += blockDim.x) {
+      const int rb = item / (HALF / 8), c = 8 * (item % (HALF / 8));
+      float lo[4][8] = {}, hi[4][8] = {};
       for (int j = 0; j < Bs; ++j) {
-        const float ds = sP[i * Bs + j];
-        x1 = fmaf(ds, sK[j * LD + d], x1);
-        x2 = fmaf(ds, sK[j * LD + d + HALF], x2);
+        const float4 k0 = ld4(sK + j * LD + c), k1 = ld4(sK + j * LD + c + 4);
+        const float4 k2 = ld4(sK + j * LD + HALF + c), k3 = ld4(sK + j * LD + HALF + c + 4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float ds = sD[(4 * rb + u) * BP + j];
+          float (&l4a)[4] = *reinterpret_cast<float(*)[4]>(&lo[u][0]);
+          float (&l4b)[4] = *reinterpret_cast<float(*)[4]>(&lo[u][4]);
+          float (&h4a)[4] = *reinterpret_cast<float(*)[4]>(&hi[u][0]);
+          float (&h4b)[4] = *reinterpret_cast<float(*)[4]>(&hi[u][4]);
+          fma4(l4a, ds, k0);
+          fma4(l4b, ds, k1);
+          fma4(h4a, ds, k2);
+          fma4(h4b, ds, k3);
+        }
       }
-      x1 *= g.scale;
-      x2 *= g.scale;
-      const float c = sC[i * HALF + d], s = sN[i * HALF + d];
-      __nv_bfloat16* out = dq + (static_cast<int64_t>(row0 + i) * g.H + h) * D;
-      out[d] = __float2bfloat16_rn(fmaf(x1, c, x2 * s));
-      out[d + HALF] = __float2bfloat16_rn(fmaf(x2, c, -x1 * s));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = 4 * rb + u;
+        if (r >= R) continue;
+        const int h = kvh * gsz + h0 + r / Bs, i = r % Bs;
+        const float* acc_row = dq_acc + (static_cast<int64_t>(h) * T + row0 + i) * D;
+        __nv_bfloat16* out = dq + (static_cast<int64_t>(row0 + i) * g.H + h) * D;
+        uint32_t plo[4], phi[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          float y[2][2];
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int d = c + e + w;
+            const float x1 = (acc_row[d] + lo[u][e + w]) * g.scale;
+            const float x2 = (acc_row[d + HALF] + hi[u][e + w]) * g.scale;
+            const float cs = sC[i * HALF + d], sn = sN[i * HALF + d];
+            y[0][w] = fmaf(x1, cs, x2 * sn);
+            y[1][w] = fmaf(x2, cs, -x1 * sn);
+          }
+          plo[e >> 1] = pack_bf16x2(y[0][0], y[0][1]);
+          phi[e >> 1] = pack_bf16x2(y[1][0], y[1][1]);
+        }
+        *reinterpret_cast<uint4*>(out + c) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
+        *reinterpret_cast<uint4*>(out + HALF + c) = make_uint4(phi[0], phi[1], phi[2], phi[3]);
+      }
     }
-    // dk~ and dV of the block keys, summed over the group's heads
-    for (int e = tid; e < Bs * D; e += blockDim.x) {
-      const int j = e / D, d = e % D;
-      float xk = aK[j * LD + d], xv = aV[j * LD + d];
-      for (int i = 0; i < Bs; ++i) {
-        xk = fmaf(sP[i * Bs + j], sQ[i * LD + d], xk);
-        xv = fmaf(sS[i * Bs + j], sO[i * LD + d], xv);
+    // dk~ (sum of dS q~) and dV (sum of P dO) over this pass's rows
+    if (acc_on) {
+      const float* W = acc_v ? sP : sD;  // P for dV, dS for dk~
+      const float* X = acc_v ? sO : sQ;
+      for (int r = 0; r < R; ++r) {
+        const float4 w4 = ld4(W + r * BP + 4 * akb);
+        const float4 x0 = ld4(X + r * LD + acol), x1 = ld4(X + r * LD + acol + 4);
+        const float w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          float (&a0)[4] = *reinterpret_cast<float(*)[4]>(&acc[v][0]);
+          float (&a1)[4] = *reinterpret_cast<float(*)[4]>(&acc[v][4]);
+          fma4(a0, w[v], x0);
+          fma4(a1, w[v], x1);
+        }
       }
-      aK[j * LD + d] = xk;
-      aV[j * LD + d] = xv;
+    }
+  }
+  // dk~ and dV to shared memory (over sQ / sO), then dK = sigma R^T dk~ and dV in bf16
+  __syncthreads();
+  if (acc_on) {
+    float* dst = acc_v ? sO : sQ;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      *reinterpret_cast<float4*>(dst + (4 * akb + v) * LD + acol) =
+          make_float4(acc[v][0], acc[v][1], acc[v][2], acc[v][3]);
+      *reinterpret_cast<float4*>(dst + (4 * akb + v) * LD + acol + 4) =
+          make_float4(acc[v][4], acc[v][5], acc[v][6], acc[v][7]);
     }
   }
   __syncthreads();
   for (int e = tid; e < Bs * HALF; e += blockDim.x) {
     const int j = e / HALF, d = e % HALF;
-    const float x1 = aK[j * LD + d] * g.scale, x2 = aK[j * LD + d + HALF] * g.scale;
+    const float x1 = sQ[j * LD + d] * g.scale, x2 = sQ[j * LD + d + HALF] * g.scale;
     const float c = sC[j * HALF + d], s = sN[j * HALF + d];
     __nv_bfloat16* ok = dk + (static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D;
     ok[d] = __float2bfloat16_rn(fmaf(x1, c, x2 * s));
     ok[d + HALF] = __float2bfloat16_rn(fmaf(x2, c, -x1 * s));
     __nv_bfloat16* ov = dv + (static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D;
-    ov[d] = __float2bfloat16_rn(aV[j * LD + d]);
-    ov[d + HALF] = __float2bfloat16_rn(aV[j * LD + d + HALF]);
+    ov[d] = __float2bfloat16_rn(sO[j * LD + d]);
+    ov[d + HALF] = __float2bfloat16_rn(sO[j * LD + d + HALF]);
   }
 }
 
@@ -272,13 +394,13 @@ cudaError_t launch_block_bwd(const Geometry& g, const void* qr, const void* kr, 
   auto* c = static_cast<__nv_bfloat16*>(dv);
   cudaError_t e;
   if (g.D == 128) {
-    const size_t smem = BlockSmem<128>::bytes(g.Bs);
+    const size_t smem = BlockSmem<128>::bytes;
     e = cudaFuncSetAttribute(block_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     block_bwd_kernel<128><<<static_cast<unsigned>(nblocks), kBlockThreads, smem, stream>>>(g, q, k, v, o, lse, ld,
                                                                                           dq_acc, a, b, c);
   } else {
-    const size_t smem = BlockSmem<64>::bytes(g.Bs);
+    const size_t smem = BlockSmem<64>::bytes;
     e = cudaFuncSetAttribute(block_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     block_bwd_kernel<64><<<static_cast<unsigned>(nblocks), kBlockThreads, smem, stream>>>(g, q, k, v, o, lse, ld,

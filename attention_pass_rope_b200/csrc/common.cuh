@@ -443,19 +443,38 @@ __device__ __forceinline__ void angle_cos_sin(int pos, double inv_freq, float& c
   sincosf(static_cast<float>(red), &s, &c);
 }
 
-// One output of the rotate-half rotation of the pair (x1, x2) by (cos, sin) = r:
-// x1 cos - x2 sin (first half) or x2 cos + x1 sin (second half), each product and the
-// sum rounded in double (no fused multiply-add), the result rounded to fp32 and then to
-// bf16 (round to nearest even).  Evaluating in double leaves the bf16 result equal to
-// rounding the exact rotation, except when it lies within a few double ulps of a bf16
-// rounding boundary.
-__device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bfloat16 x2b, double2 r,
-                                                      bool second) {
-  const double x1 = static_cast<double>(__bfloat162float(x1b));
-  const double x2 = static_cast<double>(__bfloat162float(x2b));
-  const double y = second ? __dadd_rn(__dmul_rn(x2, r.x), __dmul_rn(x1, r.y))
-                          : __dsub_rn(__dmul_rn(x1, r.x), __dmul_rn(x2, r.y));
-  return __float2bfloat16_rn(static_cast<float>(y));
+// cos and sin of one rotation angle, each split into a float pair (hi + lo carries
+// about 48 significant bits of the double value): {c_hi, c_lo, s_hi, s_lo}.
+__device__ __forceinline__ float4 cos_sin_split(double c, double s) {
+  const float ch = static_cast<float>(c), sh = static_cast<float>(s);
+  return make_float4(ch, static_cast<float>(c - static_cast<double>(ch)), sh,
+                     static_cast<float>(s - static_cast<double>(sh)));
+}
+
+// One output of the rotate-half rotation of the pair (x1, x2) by (cos, sin):
+// x1 cos - x2 sin (first half) or x2 cos + x1 sin (second half), rounded to fp32 and then
+// to bf16 (round to nearest even), the chain of an fp64 evaluation.  The value is formed
+// to about 2^-48 relative in float-float arithmetic: each product of a bf16 input with
+// the high part of cos / sin is split exactly into a rounded product and its error
+// (fma), the two products are added with an exact two-sum, and the small terms (the
+// errors and the low parts) are added to the error; the final fp32 addition then rounds
+// the value the way an fp64 evaluation would, except within ~2^-48 of an fp32 rounding
+// midpoint, and the bf16 result differs only if that also sits on a bf16 tie.
+__device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bfloat16 x2b, float4 cs, bool second) {
+  const float x1 = __bfloat162float(x1b), x2 = __bfloat162float(x2b);
+  // first half: a*c - b*s with (a, b) = (x1, x2); second half: a*c + b*s with (a, b) = (x2, x1)
+  const float a = second ? x2 : x1;
+  const float bneg = second ? -x1 : x2;  // the term subtracted: b * s with b = bneg
+  const float p1 = __fmul_rn(a, cs.x);
+  const float e1 = __fmaf_rn(a, cs.x, -p1);
+  const float p2 = __fmul_rn(bneg, cs.z);
+  const float e2 = __fmaf_rn(bneg, cs.z, -p2);
+  // two-sum of p1 - p2
+  const float t = __fsub_rn(p1, p2);
+  const float bv = __fsub_rn(t, p1);
+  const float err = __fadd_rn(__fsub_rn(p1, __fsub_rn(t, bv)), __fsub_rn(-p2, bv));
+  const float small = __fmaf_rn(a, cs.y, __fmaf_rn(-bneg, cs.w, __fsub_rn(e1, e2)));
+  return __float2bfloat16_rn(__fadd_rn(t, __fadd_rn(err, small)));
 }
 
 // Trunk-key limit of block-draft query row r of a sequence whose block rows start at
