@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
                                                                  __nv_bfloat16* __restrict__ dst_b) {
   constexpr int HALF = D / 2;
   constexpr int PARTS = HALF / 8;
-  __shared__ float4 cs[kRopeRows][HALF];
+  __shared__ float2 cs_hi[kRopeRows][HALF], cs_lo[kRopeRows][HALF];
   const int r0 = blockIdx.x * kRopeRows;
   const int nrows = min(kRopeRows, T - r0);
   for (int e = threadIdx.x; e < kRopeRows * HALF; e += blockDim.x) {
@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     const double inv_freq = pow(static_cast<double>(g.theta), -2.0 * d / D);
     double s, c;
     sincos(static_cast<double>(posf(g, r0 + r)) * inv_freq, &s, &c);
-    cs[r][d] = cos_sin_split(c, s);
+    cos_sin_split(c, s, cs_hi[r][d], cs_lo[r][d]);
   }
   __syncthreads();
   const int NH = nha + nhb;
@@ -89,9 +89,9 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float4 rr = cs[r][d0 + e];
-      ya[e] = rotate_round(xa[e], xb[e], rr, false);
-      yb[e] = rotate_round(xa[e], xb[e], rr, true);
+      const float2 rh = cs_hi[r][d0 + e], rl = cs_lo[r][d0 + e];
+      ya[e] = rotate_round(xa[e], xb[e], rh, rl, false);
+      yb[e] = rotate_round(xa[e], xb[e], rh, rl, true);
     }
     *reinterpret_cast<uint4*>(dst + d0) = oa;
     *reinterpret_cast<uint4*>(dst + HALF + d0) = ob;

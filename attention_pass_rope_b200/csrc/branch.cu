@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kPreThreads)
 }
 
 // ---------------------------------------------------------------------------
-// a7 + a8: branch backward and finalisation.  One warp per (token, KV head):
+// a7 + a8: branch backward and finalisation.  One warp per (token, KV head) item:
 //   for every pass p and group head h:
 //     dq~ = dq_acc (trunk part) + sum_j dS_j k~_j        (j = passes 1..p, 0-based)
 //     dS_j = P_j (dO . V_j - delta),  P_j = exp(sigma q~ . k~_j - lse)
@@ -180,165 +180,230 @@ __global__ void __launch_bounds__(kPreThreads)
 //     dQ_p = R(i+p)^T (sigma dq~)
 //   dK_j = R(i+j)^T (sigma dk~_j) and dV_j for the branch passes j >= 1 (dK_1 and dV_1
 //   are written by the trunk backward).
-// The kernel is bound by memory latency, so resident warps matter most: the group
-// heads of a pass go kBranchHeads at a time (one: more heads per warp keep more rows
-// in flight but cost registers, and 64 registers at four blocks per SM measured
-// fastest).  Shared memory: the block's inverse frequencies (double), then per warp
-// the cos/sin of positions i..i+P-1 and the branch-pass accumulators.
+// The kernel is bound by memory latency, so what counts is the bytes each warp keeps in
+// flight.  A warp works through (item, pass) units -- the unit's dq~ rows, q~ rows, dO
+// rows, lse and delta of the group's heads and the branch keys / values it needs -- and
+// fetches the next unit into the other half of a two-stage shared-memory buffer with
+// cp.async while it computes the current one (no registers hold data in flight).  Each
+// warp takes items w, w + W, ... (W = warps in the grid) so that neighbouring warps read
+// neighbouring rows.  Shared memory: the block's inverse frequencies (double), then per
+// warp the cos/sin of positions i..i+P-1, the branch-pass accumulators and the stages.
 // ---------------------------------------------------------------------------
-constexpr int kBranchHeads = 1;
+struct BranchLayout {
+  int cs, acc, stage, dqa, q, o, kj, vj, lse, dl, stage_bytes, warp_bytes;
+};
+
+// byte offsets inside one warp's shared-memory region (every part 16-byte aligned)
+__host__ __device__ inline BranchLayout branch_layout(int D, int gsz, int P) {
+  const int NB = P > 1 ? P - 1 : 1;
+  BranchLayout L{};
+  L.cs = 0;                                // float [P][D]: cos [D/2], sin [D/2]
+  L.acc = L.cs + P * D * 4;                // float [NB][2][D]
+  L.stage = L.acc + NB * 2 * D * 4;        // two stages
+  L.dqa = 0;                               // float [gsz][D]
+  L.q = L.dqa + gsz * D * 4;               // bf16 [gsz][D]
+  L.o = L.q + gsz * D * 2;                 // bf16 [gsz][D]
+  L.kj = L.o + gsz * D * 2;                // bf16 [NB][D]
+  L.vj = L.kj + NB * D * 2;                // bf16 [NB][D]
+  L.lse = L.vj + NB * D * 2;               // float [gsz]
+  L.dl = L.lse + ((gsz * 4 + 15) / 16) * 16;  // float [gsz]
+  L.stage_bytes = L.dl + ((gsz * 4 + 15) / 16) * 16;
+  L.warp_bytes = L.stage + 2 * L.stage_bytes;
+  return L;
+}
+
+constexpr int kBranchItemsPerWarp = 8;
+constexpr int kBranchFreqBytes = 512;  // inverse frequencies (double [D/2]), padded
 
 template <int D>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
     branch_bwd_kernel(Geometry g, const __nv_bfloat16* __restrict__ qr, const __nv_bfloat16* __restrict__ kr,
                       const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ ld,
                       const float* __restrict__ dq_acc,
-                      __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
+                      __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                      int warps_per_block) {
   constexpr int E = D / 64;
   extern __shared__ __align__(16) unsigned char branch_smem[];
   double* inv_freq = reinterpret_cast<double*>(branch_smem);  // [D/2]
-  const int NB = g.P - 1;  // branch passes
-  const int per_warp = g.P * D + (NB > 0 ? NB : 1) * 2 * D;  // floats: cos/sin [P][2][D/2], acc [NB][2][D]
-  for (int d = threadIdx.x; d < D / 2; d += blockDim.x)
-    inv_freq[d] = pow(static_cast<double>(g.theta), -2.0 * d / D);
+  for (int d = threadIdx.x; d < D / 2; d += blockDim.x) inv_freq[d] = pow(static_cast<double>(g.theta), -2.0 * d / D);
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
-  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + wib;
-  const int T = g.si.T;
-  if (w >= static_cast<int64_t>(T) * g.Hkv) return;
-  const int tau = static_cast<int>(w / g.Hkv);
-  const int kvh = static_cast<int>(w % g.Hkv);
-  int n, pos;
-  token_position(g.si, tau, n, pos);
+  if (wib >= warps_per_block) return;
   const int gsz = g.H / g.Hkv;
-  float* cs = reinterpret_cast<float*>(branch_smem + (D / 2) * sizeof(double)) + static_cast<int64_t>(wib) * per_warp;
-  float* acc = cs + g.P * D;  // [NB][2 (dk, dv)][D]; a lane touches only its own elements
-  for (int p = 0; p < g.P; ++p)
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int d = LaneMap<D>::d(lane, 0, e);
-      angle_cos_sin(pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
-    }
-  for (int j = 0; j < NB; ++j)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        acc[(j * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
-        acc[(j * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
-      }
+  const int NB = g.P > 1 ? g.P - 1 : 1;
+  const BranchLayout Lo = branch_layout(D, gsz, g.P);
+  unsigned char* wsm = branch_smem + kBranchFreqBytes + static_cast<size_t>(wib) * Lo.warp_bytes;
+  float* cs = reinterpret_cast<float*>(wsm + Lo.cs);
+  float* acc = reinterpret_cast<float*>(wsm + Lo.acc);
+  auto stage = [&](int st) { return wsm + Lo.stage + st * Lo.stage_bytes; };
+  const int T = g.si.T;
+  const int64_t nitems = static_cast<int64_t>(T) * g.Hkv;
+  const int64_t W = static_cast<int64_t>(gridDim.x) * warps_per_block;
   const int64_t dl_base = static_cast<int64_t>(ld_slots(g.si)) * 128;
-  const int64_t dl_off = static_cast<int64_t>(ld_slot(tau - pos, n, pos)) * 128 + 64 + (pos & 63);
 
-  for (int p = 0; p < g.P; ++p) {
-    float c[E], sn[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      c[e] = cs[p * D + LaneMap<D>::d(lane, 0, e)];
-      sn[e] = cs[p * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
+  // queue the copies of unit (item, p) into stage st (one commit group per unit)
+  auto issue = [&](int64_t item, int p, int st) {
+    const int tau = static_cast<int>(item / g.Hkv);
+    const int kvh = static_cast<int>(item % g.Hkv);
+    unsigned char* sb = stage(st);
+    constexpr int RC32 = D / 4;  // 16-byte chunks of an fp32 row
+    constexpr int RC16 = D / 8;  // 16-byte chunks of a bf16 row
+    for (int c = lane; c < gsz * RC32; c += 32) {
+      const int hh = c / RC32, k = c % RC32;
+      const int64_t row = (static_cast<int64_t>(p) * g.H + kvh * gsz + hh) * T + tau;
+      cp_async16(sb + Lo.dqa + (hh * D + 4 * k) * 4, dq_acc + row * D + 4 * k);
     }
-    for (int h0 = 0; h0 < gsz; h0 += kBranchHeads) {
-      float dqv[kBranchHeads][2][E], q[kBranchHeads][2][E], dO[kBranchHeads][2][E];
-      float lse_v[kBranchHeads], dl[kBranchHeads];
-#pragma unroll
-      for (int u = 0; u < kBranchHeads; ++u) {
-        const int h = kvh * gsz + h0 + u;
-        if (h0 + u < gsz) {
-          const int64_t hrow = (static_cast<int64_t>(p) * g.H + h) * T + tau;
-          load_f32_row<D>(dq_acc + hrow * D, lane, dqv[u]);
-          if (p > 0) {
-            load_bf16_row<D>(qr + hrow * D, lane, q[u]);
-            load_bf16_row<D>(dout + p * g.sq + (static_cast<int64_t>(tau) * g.H + h) * D, lane, dO[u]);
-            lse_v[u] = lse[lse_index(g.si, g.H, p, h, n, tau, pos)];
-            dl[u] = ld[(static_cast<int64_t>(p) * g.H + h) * dl_base + dl_off];
-          }
-        }
+    if (p > 0) {
+      int n, pos;
+      token_position(g.si, tau, n, pos);
+      const int64_t dl_off = static_cast<int64_t>(ld_slot(tau - pos, n, pos)) * 128 + 64 + (pos & 63);
+      for (int c = lane; c < gsz * RC16; c += 32) {
+        const int hh = c / RC16, k = c % RC16;
+        const int64_t row = (static_cast<int64_t>(p) * g.H + kvh * gsz + hh) * T + tau;
+        cp_async16(sb + Lo.q + (hh * D + 8 * k) * 2, qr + row * D + 8 * k);
       }
-      for (int j = 1; j <= p; ++j) {
-        float kj[2][E], vj[2][E];
-        load_bf16_row<D>(kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D, lane, kj);
-        load_bf16_row<D>(v + j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D, lane, vj);
-        float sdot[kBranchHeads], tdot[kBranchHeads];
-#pragma unroll
-        for (int u = 0; u < kBranchHeads; ++u) {
-          sdot[u] = 0.f;
-          tdot[u] = 0.f;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-              sdot[u] = fmaf(q[u][hh][e], kj[hh][e], sdot[u]);
-              tdot[u] = fmaf(dO[u][hh][e], vj[hh][e], tdot[u]);
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-          for (int u = 0; u < kBranchHeads; ++u) {
-            sdot[u] += __shfl_xor_sync(0xffffffffu, sdot[u], o);
-            tdot[u] += __shfl_xor_sync(0xffffffffu, tdot[u], o);
-          }
-        float ak[2][E] = {}, av[2][E] = {};
-#pragma unroll
-        for (int u = 0; u < kBranchHeads; ++u) {
-          if (h0 + u >= gsz) continue;
-          const float pj = __expf(sdot[u] * g.scale - lse_v[u]);
-          const float dsj = pj * (tdot[u] - dl[u]);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-              dqv[u][hh][e] = fmaf(dsj, kj[hh][e], dqv[u][hh][e]);
-              ak[hh][e] = fmaf(dsj, q[u][hh][e], ak[hh][e]);
-              av[hh][e] = fmaf(pj, dO[u][hh][e], av[hh][e]);
-            }
-        }
-        float* akp = acc + ((j - 1) * 2 + 0) * D;
-        float* avp = acc + ((j - 1) * 2 + 1) * D;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            const int d = LaneMap<D>::d(lane, hh, e);
-            akp[d] += ak[hh][e];
-            avp[d] += av[hh][e];
-          }
+      const __nv_bfloat16* orow = dout + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz) * D;
+      for (int c = lane; c < gsz * RC16; c += 32) cp_async16(sb + Lo.o + c * 16, orow + 8 * c);
+      for (int c = lane; c < p * RC16; c += 32) {
+        const int j = 1 + c / RC16, k = c % RC16;
+        cp_async16(sb + Lo.kj + ((j - 1) * D + 8 * k) * 2, kr + ((static_cast<int64_t>(j) * g.Hkv + kvh) * T + tau) * D + 8 * k);
+        cp_async16(sb + Lo.vj + ((j - 1) * D + 8 * k) * 2,
+                   v + j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D + 8 * k);
       }
-#pragma unroll
-      for (int u = 0; u < kBranchHeads; ++u) {
-        if (h0 + u >= gsz) continue;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int e = 0; e < E; ++e) dqv[u][hh][e] *= g.scale;
-        rotate_back<D>(dqv[u], c, sn);
-        store_bf16_row<D>(dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz + h0 + u) * D, lane, dqv[u]);
+      if (lane < gsz) {
+        const int h = kvh * gsz + lane;
+        cp_async4(sb + Lo.lse + lane * 4, lse + lse_index(g.si, g.H, p, h, n, tau, pos));
+        cp_async4(sb + Lo.dl + lane * 4, ld + (static_cast<int64_t>(p) * g.H + h) * dl_base + dl_off);
       }
     }
-  }
-  // dK and dV of the branch passes (those of the trunk pass come from the trunk backward)
-  for (int j = 1; j < g.P; ++j) {
-    float c[E], sn[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      c[e] = cs[j * D + LaneMap<D>::d(lane, 0, e)];
-      sn[e] = cs[j * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
-    }
-    float kx[2][E], vx[2][E];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
+    cp_async_commit();
+  };
+
+  int64_t item = static_cast<int64_t>(blockIdx.x) * warps_per_block + wib;
+  if (item >= nitems) return;
+  int st = 0;
+  issue(item, 0, 0);
+  while (true) {
+    const int tau = static_cast<int>(item / g.Hkv);
+    const int kvh = static_cast<int>(item % g.Hkv);
+    int n, pos;
+    token_position(g.si, tau, n, pos);
+    // cos / sin of this token's positions, zeroed branch accumulators
+    for (int p = 0; p < g.P; ++p)
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        kx[hh][e] = acc[((j - 1) * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] * g.scale;
-        vx[hh][e] = acc[((j - 1) * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)];
+        const int d = LaneMap<D>::d(lane, 0, e);
+        angle_cos_sin(pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
       }
-    rotate_back<D>(kx, c, sn);
-    const int64_t krow = j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D;
-    store_bf16_row<D>(dk + krow, lane, kx);
-    store_bf16_row<D>(dv + krow, lane, vx);
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          acc[(j * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
+          acc[(j * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
+        }
+    const int64_t next_item = item + W;
+    for (int p = 0; p < g.P; ++p) {
+      // fetch the next unit while this one is computed
+      const bool more = p + 1 < g.P || next_item < nitems;
+      if (more) {
+        issue(p + 1 < g.P ? item : next_item, p + 1 < g.P ? p + 1 : 0, st ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncwarp();
+      const unsigned char* sb = stage(st);
+      const float* sdqa = reinterpret_cast<const float*>(sb + Lo.dqa);
+      const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(sb + Lo.q);
+      const __nv_bfloat16* so = reinterpret_cast<const __nv_bfloat16*>(sb + Lo.o);
+      const __nv_bfloat16* skj = reinterpret_cast<const __nv_bfloat16*>(sb + Lo.kj);
+      const __nv_bfloat16* svj = reinterpret_cast<const __nv_bfloat16*>(sb + Lo.vj);
+      const float* slse = reinterpret_cast<const float*>(sb + Lo.lse);
+      const float* sdl = reinterpret_cast<const float*>(sb + Lo.dl);
+      float c[E], sn[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        c[e] = cs[p * D + LaneMap<D>::d(lane, 0, e)];
+        sn[e] = cs[p * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
+      }
+      for (int hh = 0; hh < gsz; ++hh) {
+        float dqv[2][E], q[2][E], dO[2][E];
+        load_f32_row<D>(sdqa + hh * D, lane, dqv);
+        if (p > 0) {
+          load_bf16_row<D>(sq + hh * D, lane, q);
+          load_bf16_row<D>(so + hh * D, lane, dO);
+          const float lse_v = slse[hh], dl = sdl[hh];
+          for (int j = 1; j <= p; ++j) {
+            float kj[2][E], vj[2][E];
+            load_bf16_row<D>(skj + (j - 1) * D, lane, kj);
+            load_bf16_row<D>(svj + (j - 1) * D, lane, vj);
+            float sdot = 0.f, tdot = 0.f;
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+              for (int e = 0; e < E; ++e) {
+                sdot = fmaf(q[x][e], kj[x][e], sdot);
+                tdot = fmaf(dO[x][e], vj[x][e], tdot);
+              }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+              tdot += __shfl_xor_sync(0xffffffffu, tdot, o);
+            }
+            const float pj = __expf(sdot * g.scale - lse_v);
+            const float dsj = pj * (tdot - dl);
+            float* akp = acc + ((j - 1) * 2 + 0) * D;
+            float* avp = acc + ((j - 1) * 2 + 1) * D;
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+              for (int e = 0; e < E; ++e) {
+                const int d = LaneMap<D>::d(lane, x, e);
+                dqv[x][e] = fmaf(dsj, kj[x][e], dqv[x][e]);
+                akp[d] = fmaf(dsj, q[x][e], akp[d]);
+                avp[d] = fmaf(pj, dO[x][e], avp[d]);
+              }
+          }
+        }
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int e = 0; e < E; ++e) dqv[x][e] *= g.scale;
+        rotate_back<D>(dqv, c, sn);
+        store_bf16_row<D>(dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz + hh) * D, lane, dqv);
+      }
+      __syncwarp();  // every lane is done with stage st before it is refilled
+      st ^= 1;
+    }
+    // dK and dV of the branch passes (those of the trunk pass come from the trunk backward)
+    for (int j = 1; j < g.P; ++j) {
+      float c[E], sn[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        c[e] = cs[j * D + LaneMap<D>::d(lane, 0, e)];
+        sn[e] = cs[j * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
+      }
+      float kx[2][E], vx[2][E];
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          kx[x][e] = acc[((j - 1) * 2 + 0) * D + LaneMap<D>::d(lane, x, e)] * g.scale;
+          vx[x][e] = acc[((j - 1) * 2 + 1) * D + LaneMap<D>::d(lane, x, e)];
+        }
+      rotate_back<D>(kx, c, sn);
+      const int64_t krow = j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D;
+      store_bf16_row<D>(dk + krow, lane, kx);
+      store_bf16_row<D>(dv + krow, lane, vx);
+    }
+    __syncwarp();  // cos / sin and the accumulators are rewritten for the next item
+    item = next_item;
+    if (item >= nitems) break;
   }
 }
 
@@ -359,10 +424,6 @@ __global__ void watchdog_selftest_kernel(uint32_t* status, uint64_t budget_ns) {
     wait_bounded(&bar, 0, wd, kSiteSelftest);
   }
   __syncthreads();
-}
-
-inline unsigned blocks_for(int64_t warps) {
-  return static_cast<unsigned>((warps + kWarpsPerBlock - 1) / kWarpsPerBlock);
 }
 
 }  // namespace
@@ -387,11 +448,16 @@ cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* 
 cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr, const void* v, const void* dout,
                               const float* lse, const float* ld, const float* dq_acc, void* dq, void* dk, void* dv,
                               cudaStream_t stream) {
-  const int64_t warps = static_cast<int64_t>(g.si.T) * g.Hkv;
-  if (warps == 0) return cudaSuccess;
-  const int NB = g.P - 1 > 0 ? g.P - 1 : 1;
-  const size_t smem = static_cast<size_t>(g.D / 2) * sizeof(double) +
-                      static_cast<size_t>(kWarpsPerBlock) * (g.P * g.D + NB * 2 * g.D) * sizeof(float);
+  const int64_t items = static_cast<int64_t>(g.si.T) * g.Hkv;
+  if (items == 0) return cudaSuccess;
+  const BranchLayout Lo = branch_layout(g.D, g.H / g.Hkv, g.P);
+  // as many warps per block as 227 KB of shared memory holds (at most kWarpsPerBlock)
+  const int wpb = static_cast<int>(std::min<int64_t>(kWarpsPerBlock, (227 * 1024 - kBranchFreqBytes) / Lo.warp_bytes));
+  if (wpb < 1) return cudaErrorInvalidConfiguration;
+  const size_t smem = kBranchFreqBytes + static_cast<size_t>(wpb) * Lo.warp_bytes;
+  const int64_t per_block = static_cast<int64_t>(wpb) * kBranchItemsPerWarp;
+  const int64_t blocks = (items + per_block - 1) / per_block;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   auto* qb = static_cast<const __nv_bfloat16*>(qr);
   auto* kb = static_cast<const __nv_bfloat16*>(kr);
   auto* vb = static_cast<const __nv_bfloat16*>(v);
@@ -403,13 +469,13 @@ cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr,
   if (g.D == 128) {
     e = cudaFuncSetAttribute(branch_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    branch_bwd_kernel<128><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, ld,
-                                                                                      dq_acc, dqb, dkb, dvb);
+    branch_bwd_kernel<128><<<static_cast<unsigned>(blocks), wpb * 32, smem, stream>>>(
+        g, qb, kb, vb, db, lse, ld, dq_acc, dqb, dkb, dvb, wpb);
   } else {
     e = cudaFuncSetAttribute(branch_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    branch_bwd_kernel<64><<<blocks_for(warps), kWarpsPerBlock * 32, smem, stream>>>(g, qb, kb, vb, db, lse, ld,
-                                                                                     dq_acc, dqb, dkb, dvb);
+    branch_bwd_kernel<64><<<static_cast<unsigned>(blocks), wpb * 32, smem, stream>>>(
+        g, qb, kb, vb, db, lse, ld, dq_acc, dqb, dkb, dvb, wpb);
   }
   return cudaGetLastError();
 }

@@ -252,6 +252,20 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return d;
 }
 
+// asynchronous copies global -> shared of this thread (16 or 4 bytes, aligned), completed
+// by cp.async.wait_group
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* sdst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // all but the most recent bulk group have finished reading their shared-memory source
 __device__ __forceinline__ void bulk_wait_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
@@ -444,11 +458,14 @@ __device__ __forceinline__ void angle_cos_sin(int pos, double inv_freq, float& c
 }
 
 // cos and sin of one rotation angle, each split into a float pair (hi + lo carries
-// about 48 significant bits of the double value): {c_hi, c_lo, s_hi, s_lo}.
-__device__ __forceinline__ float4 cos_sin_split(double c, double s) {
+// about 48 significant bits of the double value): hi = {c_hi, s_hi}, lo = {c_lo, s_lo}.
+// Kept as two float2 arrays in shared memory (8-byte entries: a warp reading 32
+// consecutive entries spreads over the banks; 16-byte entries at a stride of 8 would
+// put every lane on the same four banks).
+__device__ __forceinline__ void cos_sin_split(double c, double s, float2& hi, float2& lo) {
   const float ch = static_cast<float>(c), sh = static_cast<float>(s);
-  return make_float4(ch, static_cast<float>(c - static_cast<double>(ch)), sh,
-                     static_cast<float>(s - static_cast<double>(sh)));
+  hi = make_float2(ch, sh);
+  lo = make_float2(static_cast<float>(c - static_cast<double>(ch)), static_cast<float>(s - static_cast<double>(sh)));
 }
 
 // One output of the rotate-half rotation of the pair (x1, x2) by (cos, sin):
@@ -460,7 +477,9 @@ __device__ __forceinline__ float4 cos_sin_split(double c, double s) {
 // errors and the low parts) are added to the error; the final fp32 addition then rounds
 // the value the way an fp64 evaluation would, except within ~2^-48 of an fp32 rounding
 // midpoint, and the bf16 result differs only if that also sits on a bf16 tie.
-__device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bfloat16 x2b, float4 cs, bool second) {
+__device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bfloat16 x2b, float2 hi, float2 lo,
+                                                      bool second) {
+  const float4 cs = make_float4(hi.x, lo.x, hi.y, lo.y);
   const float x1 = __bfloat162float(x1b), x2 = __bfloat162float(x2b);
   // first half: a*c - b*s with (a, b) = (x1, x2); second half: a*c + b*s with (a, b) = (x2, x1)
   const float a = second ? x2 : x1;

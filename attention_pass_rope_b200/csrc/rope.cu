@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
                                                                 __nv_bfloat16* __restrict__ kr) {
   constexpr int HALF = D / 2;
   constexpr int PARTS = HALF / 8;  // threads per row (8 elements of each half each)
-  __shared__ float4 cs[kRopeTok][HALF];
+  __shared__ float2 cs_hi[kRopeTok][HALF], cs_lo[kRopeTok][HALF];
 
   const int n = blockIdx.y;
   const int p = blockIdx.z;
@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
     const double ang = static_cast<double>(g.pos0 + i0 + tok + p) * inv_freq;
     double s, c;
     sincos(ang, &s, &c);
-    cs[tok][d] = cos_sin_split(c, s);
+    cos_sin_split(c, s, cs_hi[tok][d], cs_lo[tok][d]);
   }
   __syncthreads();
 
@@ -78,9 +78,9 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float4 r = cs[tok][d0 + e];
-      ya[e] = rotate_round(xa[e], xb[e], r, false);
-      yb[e] = rotate_round(xa[e], xb[e], r, true);
+      const float2 rh = cs_hi[tok][d0 + e], rl = cs_lo[tok][d0 + e];
+      ya[e] = rotate_round(xa[e], xb[e], rh, rl, false);
+      yb[e] = rotate_round(xa[e], xb[e], rh, rl, true);
     }
     *reinterpret_cast<uint4*>(dst + d0) = oa;
     *reinterpret_cast<uint4*>(dst + HALF + d0) = ob;
