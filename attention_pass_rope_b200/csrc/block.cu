@@ -62,13 +62,24 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     cos_sin_split(c, s, cs_hi[r][d], cs_lo[r][d]);
   }
   __syncthreads();
+  // every thread keeps one (row, 8-element part) slot and walks the heads, so that it
+  // reads its cos / sin from shared memory once
+  static_assert(kRopeThreads % (kRopeRows * PARTS) == 0, "threads must cover whole slots");
+  constexpr int kHeadLanes = kRopeThreads / (kRopeRows * PARTS);
   const int NH = nha + nhb;
-  for (int task = threadIdx.x; task < NH * kRopeRows * PARTS; task += blockDim.x) {
-    const int part = task % PARTS;
-    const int r = (task / PARTS) % kRopeRows;
-    const int head = task / (PARTS * kRopeRows);
-    if (r >= nrows) continue;
-    const int tau = r0 + r;
+  const int slot = threadIdx.x % (kRopeRows * PARTS);
+  const int part = slot % PARTS;
+  const int r = slot / PARTS;
+  if (r >= nrows) return;
+  const int d0 = part * 8;
+  float2 rh[8], rl[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    rh[e] = cs_hi[r][d0 + e];
+    rl[e] = cs_lo[r][d0 + e];
+  }
+  const int tau = r0 + r;
+  for (int head = threadIdx.x / (kRopeRows * PARTS); head < NH; head += kHeadLanes) {
     const __nv_bfloat16* src;
     __nv_bfloat16* dst;
     if (head < nha) {
@@ -79,7 +90,6 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
       src = src_b + (static_cast<int64_t>(tau) * nhb + hb) * D;
       dst = dst_b + (static_cast<int64_t>(hb) * T + tau) * D;
     }
-    const int d0 = part * 8;
     const uint4 av = *reinterpret_cast<const uint4*>(src + d0);
     const uint4 bv = *reinterpret_cast<const uint4*>(src + HALF + d0);
     const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&av);
@@ -89,9 +99,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float2 rh = cs_hi[r][d0 + e], rl = cs_lo[r][d0 + e];
-      ya[e] = rotate_round(xa[e], xb[e], rh, rl, false);
-      yb[e] = rotate_round(xa[e], xb[e], rh, rl, true);
+      ya[e] = rotate_round(xa[e], xb[e], rh[e], rl[e], false);
+      yb[e] = rotate_round(xa[e], xb[e], rh[e], rl[e], true);
     }
     *reinterpret_cast<uint4*>(dst + d0) = oa;
     *reinterpret_cast<uint4*>(dst + HALF + d0) = ob;

@@ -49,15 +49,25 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
   }
   __syncthreads();
 
+  // every thread keeps one (token, 8-element part) slot and walks the heads, so that it
+  // reads its cos / sin from shared memory once
+  static_assert(kRopeThreads % (kRopeTok * PARTS) == 0, "threads must cover whole slots");
+  constexpr int kHeadLanes = kRopeThreads / (kRopeTok * PARTS);
   const int NH = g.H + g.Hkv;
   const int T = g.si.T;
-  const int tasks = NH * kRopeTok * PARTS;
-  for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
-    const int part = task % PARTS;
-    const int tok = (task / PARTS) % kRopeTok;
-    const int head = task / (PARTS * kRopeTok);
-    if (tok >= ntok) continue;
-    const int tau = start + i0 + tok;
+  const int slot = threadIdx.x % (kRopeTok * PARTS);
+  const int part = slot % PARTS;
+  const int tok = slot / PARTS;
+  if (tok >= ntok) return;
+  const int d0 = part * 8;
+  float2 rh[8], rl[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    rh[e] = cs_hi[tok][d0 + e];
+    rl[e] = cs_lo[tok][d0 + e];
+  }
+  const int tau = start + i0 + tok;
+  for (int head = threadIdx.x / (kRopeTok * PARTS); head < NH; head += kHeadLanes) {
     const __nv_bfloat16* src;
     __nv_bfloat16* dst;
     if (head < g.H) {
@@ -68,7 +78,6 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
       src = k + p * g.skv + (static_cast<int64_t>(tau) * g.Hkv + hk) * D;
       dst = kr + ((static_cast<int64_t>(p) * g.Hkv + hk) * T + tau) * D;
     }
-    const int d0 = part * 8;
     const uint4 a = *reinterpret_cast<const uint4*>(src + d0);
     const uint4 b = *reinterpret_cast<const uint4*>(src + HALF + d0);
     const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&a);
@@ -78,9 +87,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_fwd_kernel(Geometry g, cons
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float2 rh = cs_hi[tok][d0 + e], rl = cs_lo[tok][d0 + e];
-      ya[e] = rotate_round(xa[e], xb[e], rh, rl, false);
-      yb[e] = rotate_round(xa[e], xb[e], rh, rl, true);
+      ya[e] = rotate_round(xa[e], xb[e], rh[e], rl[e], false);
+      yb[e] = rotate_round(xa[e], xb[e], rh[e], rl[e], true);
     }
     *reinterpret_cast<uint4*>(dst + d0) = oa;
     *reinterpret_cast<uint4*>(dst + HALF + d0) = ob;
