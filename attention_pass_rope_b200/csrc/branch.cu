@@ -21,6 +21,69 @@ namespace {
 
 constexpr int kWarpsPerBlock = 8;
 
+// Lane element map: lane holds E = D/64 consecutive elements of each half of the
+// head dimension, d in [E*lane, E*lane+E) and [D/2 + E*lane, ...), so that each
+// RoPE pair (d, d + D/2) is in one lane.
+template <int D>
+struct LaneMap {
+  static constexpr int E = D / 64;
+  __device__ static int d(int lane, int half, int e) { return half * (D / 2) + E * lane + e; }
+};
+
+template <int D>
+__device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* row, int lane, float (&x)[2][D / 64]) {
+  constexpr int E = D / 64;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    if constexpr (E == 2) {
+      const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(row + LaneMap<D>::d(lane, hh, 0));
+      x[hh][0] = __low2float(v);
+      x[hh][1] = __high2float(v);
+    } else {
+      x[hh][0] = __bfloat162float(row[LaneMap<D>::d(lane, hh, 0)]);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void load_f32_row(const float* row, int lane, float (&x)[2][D / 64]) {
+  constexpr int E = D / 64;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    if constexpr (E == 2) {
+      const float2 v = *reinterpret_cast<const float2*>(row + LaneMap<D>::d(lane, hh, 0));
+      x[hh][0] = v.x;
+      x[hh][1] = v.y;
+    } else {
+      x[hh][0] = row[LaneMap<D>::d(lane, hh, 0)];
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16* row, int lane, const float (&x)[2][D / 64]) {
+  constexpr int E = D / 64;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    if constexpr (E == 2) {
+      *reinterpret_cast<__nv_bfloat162*>(row + LaneMap<D>::d(lane, hh, 0)) = __floats2bfloat162_rn(x[hh][0], x[hh][1]);
+    } else {
+      row[LaneMap<D>::d(lane, hh, 0)] = __float2bfloat16_rn(x[hh][0]);
+    }
+  }
+}
+
+// x <- R(pos)^T x (rotation by the negative angle), in place.
+template <int D>
+__device__ __forceinline__ void rotate_back(float (&x)[2][D / 64], const float (&c)[D / 64], const float (&s)[D / 64]) {
+#pragma unroll
+  for (int e = 0; e < D / 64; ++e) {
+    const float x1 = x[0][e], x2 = x[1][e];
+    x[0][e] = fmaf(x1, c[e], x2 * s[e]);
+    x[1][e] = fmaf(x2, c[e], -x1 * s[e]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // a5: delta = rowsum(dO * O), written with -lse * log2(e) into the tile-aligned
 // row-statistics array that the trunk backward fetches one 512-byte slot at a time;
@@ -121,9 +184,7 @@ __global__ void __launch_bounds__(kPreThreads)
 // flight.  A warp works through (item, pass) units -- the unit's dq~ rows, q~ rows, dO
 // rows, lse and delta of the group's heads and the branch keys / values it needs -- and
 // fetches the next unit into the other half of a two-stage shared-memory buffer with
-// cp.async while it computes the current one (no registers hold data in flight).  The
-// compute is instruction-bound: each half-warp takes one head's row (16 lanes, a row's
-// dot products reduce in 4 shuffle steps), two rows per warp instruction.  Each
+// cp.async while it computes the current one (no registers hold data in flight).  Each
 // warp takes items w, w + W, ... (W = warps in the grid) so that neighbouring warps read
 // neighbouring rows.  Shared memory: the block's inverse frequencies (double), then per
 // warp the cos/sin of positions i..i+P-1, the branch-pass accumulators and the stages.
@@ -137,8 +198,8 @@ __host__ __device__ inline BranchLayout branch_layout(int D, int gsz, int P) {
   const int NB = P > 1 ? P - 1 : 1;
   BranchLayout L{};
   L.cs = 0;                                // float [P][D]: cos [D/2], sin [D/2]
-  L.acc = L.cs + P * D * 4;                // float [2 half-warps][NB][2][D]
-  L.stage = L.acc + 2 * NB * 2 * D * 4;    // two stages
+  L.acc = L.cs + P * D * 4;                // float [NB][2][D]
+  L.stage = L.acc + NB * 2 * D * 4;        // two stages
   L.dqa = 0;                               // float [gsz][D]
   L.q = L.dqa + gsz * D * 4;               // bf16 [gsz][D]
   L.o = L.q + gsz * D * 2;                 // bf16 [gsz][D]
@@ -162,6 +223,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                       const float* __restrict__ dq_acc,
                       __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                       int warps_per_block) {
+  constexpr int E = D / 64;
   extern __shared__ __align__(16) unsigned char branch_smem[];
   double* inv_freq = reinterpret_cast<double*>(branch_smem);  // [D/2]
   for (int d = threadIdx.x; d < D / 2; d += blockDim.x) inv_freq[d] = pow(static_cast<double>(g.theta), -2.0 * d / D);
@@ -220,41 +282,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     cp_async_commit();
   };
 
-  // compute mapping: half-warp hw takes one head's row at a time; its lane l16 holds
-  // the EL elements [EL*l16, EL*l16+EL) of each half of the head dimension, so that every
-  // RoPE pair (d, d + D/2) stays in one lane and a row's dot products reduce over 16 lanes
-  constexpr int EL = D / 32;
-  const int hw = lane >> 4, l16 = lane & 15;
-  const int dlo = EL * l16, dhi = D / 2 + EL * l16;
-  float* acc_h = acc + hw * NB * 2 * D;  // this half-warp's accumulators
-  auto lds_f32 = [](const float* row, int d, float (&x)[EL]) {
-    if constexpr (EL == 4) {
-      const float4 v4 = *reinterpret_cast<const float4*>(row + d);
-      x[0] = v4.x; x[1] = v4.y; x[2] = v4.z; x[3] = v4.w;
-    } else {
-      const float2 v2 = *reinterpret_cast<const float2*>(row + d);
-      x[0] = v2.x; x[1] = v2.y;
-    }
-  };
-  auto lds_bf16 = [](const __nv_bfloat16* row, int d, float (&x)[EL]) {
-    if constexpr (EL == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(row + d);
-      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-      x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-    } else {
-      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(row + d));
-      x[0] = a.x; x[1] = a.y;
-    }
-  };
-  auto stg_bf16 = [](__nv_bfloat16* row, int d, const float (&x)[EL]) {
-    if constexpr (EL == 4) {
-      *reinterpret_cast<uint2*>(row + d) = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
-    } else {
-      *reinterpret_cast<uint32_t*>(row + d) = pack_bf16x2(x[0], x[1]);
-    }
-  };
-
   int64_t item = static_cast<int64_t>(blockIdx.x) * warps_per_block + wib;
   if (item >= nitems) return;
   int st = 0;
@@ -264,13 +291,21 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     const int kvh = static_cast<int>(item % g.Hkv);
     int n, pos;
     token_position(g.si, tau, n, pos);
-    // cos / sin of this token's positions, zeroed branch accumulators (both copies)
-    for (int e = lane; e < g.P * (D / 2); e += 32) {
-      const int p = e / (D / 2), d = e % (D / 2);
-      angle_cos_sin(pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
-    }
-    for (int e = lane; e < 2 * NB * 2 * D; e += 32) acc[e] = 0.f;
-    __syncwarp();
+    // cos / sin of this token's positions, zeroed branch accumulators
+    for (int p = 0; p < g.P; ++p)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int d = LaneMap<D>::d(lane, 0, e);
+        angle_cos_sin(pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
+      }
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          acc[(j * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
+          acc[(j * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
+        }
     const int64_t next_item = item + W;
     for (int p = 0; p < g.P; ++p) {
       // fetch the next unit while this one is computed
@@ -290,116 +325,81 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       const __nv_bfloat16* svj = reinterpret_cast<const __nv_bfloat16*>(sb + Lo.vj);
       const float* slse = reinterpret_cast<const float*>(sb + Lo.lse);
       const float* sdl = reinterpret_cast<const float*>(sb + Lo.dl);
-      float c[EL], sn[EL];
-      lds_f32(cs + p * D, dlo, c);
-      lds_f32(cs + p * D + D / 2, dlo, sn);
-      for (int h2 = 0; h2 < gsz; h2 += 2) {
-        const int hh = h2 + hw;
-        const bool on = hh < gsz;  // an odd group leaves the second half-warp idle on its last pair
-        const int hr = on ? hh : h2;
-        float x1[EL], x2[EL];
-        lds_f32(sdqa + hr * D, dlo, x1);
-        lds_f32(sdqa + hr * D, dhi, x2);
+      float c[E], sn[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        c[e] = cs[p * D + LaneMap<D>::d(lane, 0, e)];
+        sn[e] = cs[p * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
+      }
+      for (int hh = 0; hh < gsz; ++hh) {
+        float dqv[2][E], q[2][E], dO[2][E];
+        load_f32_row<D>(sdqa + hh * D, lane, dqv);
         if (p > 0) {
-          float q1[EL], q2[EL], o1[EL], o2[EL];
-          lds_bf16(sq + hr * D, dlo, q1);
-          lds_bf16(sq + hr * D, dhi, q2);
-          lds_bf16(so + hr * D, dlo, o1);
-          lds_bf16(so + hr * D, dhi, o2);
-          const float lse_v = slse[hr], dl = sdl[hr];
+          load_bf16_row<D>(sq + hh * D, lane, q);
+          load_bf16_row<D>(so + hh * D, lane, dO);
+          const float lse_v = slse[hh], dl = sdl[hh];
           for (int j = 1; j <= p; ++j) {
-            float k1[EL], k2[EL], v1[EL], v2[EL];
-            lds_bf16(skj + (j - 1) * D, dlo, k1);
-            lds_bf16(skj + (j - 1) * D, dhi, k2);
-            lds_bf16(svj + (j - 1) * D, dlo, v1);
-            lds_bf16(svj + (j - 1) * D, dhi, v2);
+            float kj[2][E], vj[2][E];
+            load_bf16_row<D>(skj + (j - 1) * D, lane, kj);
+            load_bf16_row<D>(svj + (j - 1) * D, lane, vj);
             float sdot = 0.f, tdot = 0.f;
 #pragma unroll
-            for (int e = 0; e < EL; ++e) {
-              sdot = fmaf(q1[e], k1[e], fmaf(q2[e], k2[e], sdot));
-              tdot = fmaf(o1[e], v1[e], fmaf(o2[e], v2[e], tdot));
-            }
+            for (int x = 0; x < 2; ++x)
 #pragma unroll
-            for (int o = 8; o > 0; o >>= 1) {
+              for (int e = 0; e < E; ++e) {
+                sdot = fmaf(q[x][e], kj[x][e], sdot);
+                tdot = fmaf(dO[x][e], vj[x][e], tdot);
+              }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
               sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
               tdot += __shfl_xor_sync(0xffffffffu, tdot, o);
             }
-            float pj = __expf(sdot * g.scale - lse_v);
-            float dsj = pj * (tdot - dl);
-            if (!on) pj = dsj = 0.f;
-            float* ak = acc_h + ((j - 1) * 2 + 0) * D;
-            float* av = acc_h + ((j - 1) * 2 + 1) * D;
-            float a1[EL], a2[EL], b1[EL], b2[EL];
-            lds_f32(ak, dlo, a1);
-            lds_f32(ak, dhi, a2);
-            lds_f32(av, dlo, b1);
-            lds_f32(av, dhi, b2);
+            const float pj = __expf(sdot * g.scale - lse_v);
+            const float dsj = pj * (tdot - dl);
+            float* akp = acc + ((j - 1) * 2 + 0) * D;
+            float* avp = acc + ((j - 1) * 2 + 1) * D;
 #pragma unroll
-            for (int e = 0; e < EL; ++e) {
-              x1[e] = fmaf(dsj, k1[e], x1[e]);
-              x2[e] = fmaf(dsj, k2[e], x2[e]);
-              a1[e] = fmaf(dsj, q1[e], a1[e]);
-              a2[e] = fmaf(dsj, q2[e], a2[e]);
-              b1[e] = fmaf(pj, o1[e], b1[e]);
-              b2[e] = fmaf(pj, o2[e], b2[e]);
-            }
-            if constexpr (EL == 4) {
-              *reinterpret_cast<float4*>(ak + dlo) = make_float4(a1[0], a1[1], a1[2], a1[3]);
-              *reinterpret_cast<float4*>(ak + dhi) = make_float4(a2[0], a2[1], a2[2], a2[3]);
-              *reinterpret_cast<float4*>(av + dlo) = make_float4(b1[0], b1[1], b1[2], b1[3]);
-              *reinterpret_cast<float4*>(av + dhi) = make_float4(b2[0], b2[1], b2[2], b2[3]);
-            } else {
-              *reinterpret_cast<float2*>(ak + dlo) = make_float2(a1[0], a1[1]);
-              *reinterpret_cast<float2*>(ak + dhi) = make_float2(a2[0], a2[1]);
-              *reinterpret_cast<float2*>(av + dlo) = make_float2(b1[0], b1[1]);
-              *reinterpret_cast<float2*>(av + dhi) = make_float2(b2[0], b2[1]);
-            }
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+              for (int e = 0; e < E; ++e) {
+                const int d = LaneMap<D>::d(lane, x, e);
+                dqv[x][e] = fmaf(dsj, kj[x][e], dqv[x][e]);
+                akp[d] = fmaf(dsj, q[x][e], akp[d]);
+                avp[d] = fmaf(pj, dO[x][e], avp[d]);
+              }
           }
         }
-        if (on) {
-          // dQ = R(pos + p)^T (sigma dq~)
-          float y1[EL], y2[EL];
 #pragma unroll
-          for (int e = 0; e < EL; ++e) {
-            const float a = x1[e] * g.scale, b = x2[e] * g.scale;
-            y1[e] = fmaf(a, c[e], b * sn[e]);
-            y2[e] = fmaf(b, c[e], -a * sn[e]);
-          }
-          __nv_bfloat16* out = dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz + hh) * D;
-          stg_bf16(out, dlo, y1);
-          stg_bf16(out, dhi, y2);
-        }
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int e = 0; e < E; ++e) dqv[x][e] *= g.scale;
+        rotate_back<D>(dqv, c, sn);
+        store_bf16_row<D>(dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz + hh) * D, lane, dqv);
       }
       __syncwarp();  // every lane is done with stage st before it is refilled
       st ^= 1;
     }
-    // dK and dV of the branch passes: the two half-warps' sums, sigma and R^T for dK
-    // (those of the trunk pass come from the trunk backward); half-warp hw takes the
-    // branch passes j = 1 + hw, 3 + hw, ...
-    for (int j = 1 + hw; j < g.P; j += 2) {
-      const float* k0 = acc + ((j - 1) * 2 + 0) * D;
-      const float* k1b = acc + NB * 2 * D + ((j - 1) * 2 + 0) * D;
-      const float* v0 = acc + ((j - 1) * 2 + 1) * D;
-      const float* v1b = acc + NB * 2 * D + ((j - 1) * 2 + 1) * D;
-      float a1[EL], a2[EL], t1[EL], t2[EL], b1[EL], b2[EL], u1[EL], u2[EL], c[EL], sn[EL];
-      lds_f32(k0, dlo, a1); lds_f32(k0, dhi, a2); lds_f32(k1b, dlo, t1); lds_f32(k1b, dhi, t2);
-      lds_f32(v0, dlo, b1); lds_f32(v0, dhi, b2); lds_f32(v1b, dlo, u1); lds_f32(v1b, dhi, u2);
-      lds_f32(cs + j * D, dlo, c);
-      lds_f32(cs + j * D + D / 2, dlo, sn);
-      float y1[EL], y2[EL], w1[EL], w2[EL];
+    // dK and dV of the branch passes (those of the trunk pass come from the trunk backward)
+    for (int j = 1; j < g.P; ++j) {
+      float c[E], sn[E];
 #pragma unroll
-      for (int e = 0; e < EL; ++e) {
-        const float a = (a1[e] + t1[e]) * g.scale, b = (a2[e] + t2[e]) * g.scale;
-        y1[e] = fmaf(a, c[e], b * sn[e]);
-        y2[e] = fmaf(b, c[e], -a * sn[e]);
-        w1[e] = b1[e] + u1[e];
-        w2[e] = b2[e] + u2[e];
+      for (int e = 0; e < E; ++e) {
+        c[e] = cs[j * D + LaneMap<D>::d(lane, 0, e)];
+        sn[e] = cs[j * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
       }
+      float kx[2][E], vx[2][E];
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          kx[x][e] = acc[((j - 1) * 2 + 0) * D + LaneMap<D>::d(lane, x, e)] * g.scale;
+          vx[x][e] = acc[((j - 1) * 2 + 1) * D + LaneMap<D>::d(lane, x, e)];
+        }
+      rotate_back<D>(kx, c, sn);
       const int64_t krow = j * g.skv + (static_cast<int64_t>(tau) * g.Hkv + kvh) * D;
-      stg_bf16(dk + krow, dlo, y1);
-      stg_bf16(dk + krow, dhi, y2);
-      stg_bf16(dv + krow, dlo, w1);
-      stg_bf16(dv + krow, dhi, w2);
+      store_bf16_row<D>(dk + krow, lane, kx);
+      store_bf16_row<D>(dv + krow, lane, vx);
     }
     __syncwarp();  // cos / sin and the accumulators are rewritten for the next item
     item = next_item;

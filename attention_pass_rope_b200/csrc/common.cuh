@@ -477,10 +477,8 @@ __device__ __forceinline__ void cos_sin_split(double c, double s, float2& hi, fl
 // errors and the low parts) are added to the error; the final fp32 addition then rounds
 // the value the way an fp64 evaluation would, except within ~2^-48 of an fp32 rounding
 // midpoint, and the bf16 result differs only if that also sits on a bf16 tie.
-__device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bfloat16 x2b, float2 hi, float2 lo,
-                                                      bool second) {
+__device__ __forceinline__ __nv_bfloat16 rotate_round_exact(float x1, float x2, float2 hi, float2 lo, bool second) {
   const float4 cs = make_float4(hi.x, lo.x, hi.y, lo.y);
-  const float x1 = __bfloat162float(x1b), x2 = __bfloat162float(x2b);
   // first half: a*c - b*s with (a, b) = (x1, x2); second half: a*c + b*s with (a, b) = (x2, x1)
   const float a = second ? x2 : x1;
   const float bneg = second ? -x1 : x2;  // the term subtracted: b * s with b = bneg
@@ -494,6 +492,20 @@ __device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bf
   const float err = __fadd_rn(__fsub_rn(p1, __fsub_rn(t, bv)), __fsub_rn(-p2, bv));
   const float small = __fmaf_rn(a, cs.y, __fmaf_rn(-bneg, cs.w, __fsub_rn(e1, e2)));
   return __float2bfloat16_rn(__fadd_rn(t, __fadd_rn(err, small)));
+}
+
+// The same rounding, fast in the common case.  The plain fp32 evaluation differs from
+// the exact value by less than (|x1| + |x2|) * 2^-21 (two rounded products, cos / sin
+// rounded to fp32), so its bf16 rounding is the exact value's unless it lies that close
+// to a bf16 rounding midpoint (the value with the dropped 16 bits equal to 0x8000);
+// about 1.4e-3 of the elements do, and take the float-float path above.
+__device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bfloat16 x2b, float2 hi, float2 lo,
+                                                      bool second) {
+  const float x1 = __bfloat162float(x1b), x2 = __bfloat162float(x2b);
+  const float y = second ? fmaf(x2, hi.x, x1 * hi.y) : fmaf(x1, hi.x, -x2 * hi.y);
+  const float mid = __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
+  if (fabsf(y - mid) > (fabsf(x1) + fabsf(x2)) * 4.76837158203125e-07f) return __float2bfloat16_rn(y);  // 2^-21
+  return rotate_round_exact(x1, x2, hi, lo, second);
 }
 
 // Trunk-key limit of block-draft query row r of a sequence whose block rows start at
