@@ -126,10 +126,11 @@ template <int D>
 struct BlockSmem {
   static constexpr int LD = D + 4;  // row stride (floats): 16-byte aligned rows, staggered banks
   static constexpr int BP = 16;     // block keys, padded
-  // Q, dO [64][LD]; K, V [16][LD]; P, dS [64][16]; cos, sin [16][D/2]; lse, delta [64]
+  // Q, dO [64][LD]; K, V [16][LD]; P, dS [64][16]; cos, sin [16][D/2]; lse, delta [64];
+  // then the inverse frequencies (double [D/2])
   static constexpr size_t kFloats = 2 * kBlockRows * LD + 2 * BP * LD + 2 * kBlockRows * BP + 2 * BP * (D / 2) +
                                     2 * kBlockRows;
-  static constexpr size_t bytes = kFloats * sizeof(float);
+  static constexpr size_t bytes = kFloats * sizeof(float) + (D / 2) * sizeof(double);
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(kBlockThreads)
   float* sN = sC + BP * HALF;            // [16][D/2] sin
   float* sL = sN + BP * HALF;            // [64] lse
   float* sDl = sL + kBlockRows;          // [64] delta
+  double* sF = reinterpret_cast<double*>(blk_smem + SM::kFloats);  // [D/2] inverse frequencies
 
   const int Bs = g.Bs;
   const int b = static_cast<int>(blockIdx.x) / g.Hkv;
@@ -198,10 +200,12 @@ __global__ void __launch_bounds__(kBlockThreads)
     *reinterpret_cast<float4*>(sK + j * LD + d) = k4;
     *reinterpret_cast<float4*>(sV + j * LD + d) = v4;
   }
+  for (int d = tid; d < HALF; d += blockDim.x) sF[d] = pow(static_cast<double>(g.theta), -2.0 * d / D);
+  __syncthreads();
   for (int e = tid; e < Bs * HALF; e += blockDim.x) {
     const int i = e / HALF, d = e % HALF;
     float c, s;
-    angle_cos_sin(anchor + i, pow(static_cast<double>(g.theta), -2.0 * d / D), c, s);
+    angle_cos_sin(anchor + i, sF[d], c, s);
     sC[i * HALF + d] = c;
     sN[i * HALF + d] = s;
   }
