@@ -356,10 +356,14 @@ ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k,
   // made no runtime call yet, such as an autograd worker, has none).
   clear_stale_error();
   TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, qr, D, T, static_cast<uint64_t>(g.P) * g.H, D * 2, T * D * 2, 128, 1) ||
-      !make_map(&mk, kr, D, T, g.Hkv, D * 2, T * D * 2, 128, 1) ||
-      !make_map(&mv, v, D, g.Hkv, T, D * 2, g.Hkv * D * 2, 1, 128))
+  CUtensorMap mq, mk, mv, mo, mek, mev;
+  const uint64_t P = g.P, H = g.H, Hkv = g.Hkv;
+  if (!make_map(&mq, qr, D, T, P * H, D * 2, T * D * 2, 128, 1) ||
+      !make_map(&mk, kr, D, T, Hkv, D * 2, T * D * 2, 128, 1) ||
+      !make_map(&mv, v, D, Hkv, T, D * 2, Hkv * D * 2, 1, 128) ||
+      !make_map4(&mo, o, {D, H, T, P}, {D * 2, H * D * 2, static_cast<uint64_t>(g.sq) * 2}, {1, 32, 1}) ||
+      !make_map(&mek, kr, D, T, P * Hkv, D * 2, T * D * 2, 128, 1) ||
+      !make_map4(&mev, v, {D, Hkv, T, P}, {D * 2, Hkv * D * 2, static_cast<uint64_t>(g.skv) * 2}, {1, 128, 1}))
     return TTT_ERR_CUDA;
   {
     EventScope es(desc->events, TTT_KERNEL_ROPE_FWD, stream);
@@ -368,7 +372,7 @@ ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k,
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
     TrunkFwdArgs a{g, nullptr, kr, v, o, lse, status, g_wait_budget_ns.load()};
-    TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
+    TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, mo, mek, mev, stream));
   }
   return TTT_OK;
 }
@@ -465,10 +469,14 @@ ttt_status ttt_block_attn_fwd(const ttt_block_desc* desc, const void* k_ctx, con
   const uint64_t NQ = g.si.T, Tc = g.ksi.T, D = g.D;
   clear_stale_error();
   TTT_CHECK_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, qr, D, NQ, g.H, D * 2, NQ * D * 2, 128, 1) ||
-      !make_map(&mk, kr_ctx, D, Tc, g.Hkv, D * 2, Tc * D * 2, 128, 1) ||
-      !make_map(&mv, v_ctx, D, g.Hkv, Tc, D * 2, g.Hkv * D * 2, 1, 128))
+  CUtensorMap mq, mk, mv, mo, mek, mev;
+  const uint64_t H = g.H, Hkv = g.Hkv;
+  if (!make_map(&mq, qr, D, NQ, H, D * 2, NQ * D * 2, 128, 1) ||
+      !make_map(&mk, kr_ctx, D, Tc, Hkv, D * 2, Tc * D * 2, 128, 1) ||
+      !make_map(&mv, v_ctx, D, Hkv, Tc, D * 2, Hkv * D * 2, 1, 128) ||
+      !make_map4(&mo, o, {D, H, NQ, 1}, {D * 2, H * D * 2, NQ * H * D * 2}, {1, 32, 1}) ||
+      !make_map(&mek, kr_blk, D, NQ, Hkv, D * 2, NQ * D * 2, 128, 1) ||
+      !make_map4(&mev, vb, {D, Hkv, NQ, 1}, {D * 2, Hkv * D * 2, NQ * Hkv * D * 2}, {1, 128, 1}))
     return TTT_ERR_CUDA;
   {
     EventScope es(desc->events, TTT_KERNEL_ROPE_FWD, stream);
@@ -478,7 +486,7 @@ ttt_status ttt_block_attn_fwd(const ttt_block_desc* desc, const void* k_ctx, con
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
     TrunkFwdArgs a{g, nullptr, kr_blk, vb, o, lse, status, g_wait_budget_ns.load()};
-    TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
+    TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, mo, mek, mev, stream));
   }
   return TTT_OK;
 }
@@ -582,14 +590,25 @@ ttt_status ttt_ring_step(const ttt_ring_desc* desc, const void* qr, const void* 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   const uint64_t Lq = desc->q_len, Lk = desc->kv_len, D = g.D;
   clear_stale_error();
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, qr, D, Lq, static_cast<uint64_t>(g.P) * g.H, D * 2, Lq * D * 2, 128, 1) ||
-      !make_map(&mk, kr_visit, D, Lk, g.Hkv, D * 2, Lk * D * 2, 128, 1) ||
-      !make_map(&mv, v_visit, D, g.Hkv, Lk, D * 2, g.Hkv * D * 2, 1, 128))
+  CUtensorMap mq, mk, mv, mek, mev;
+  const uint64_t P = g.P, Hkv = g.Hkv;
+  if (!make_map(&mq, qr, D, Lq, P * g.H, D * 2, Lq * D * 2, 128, 1) ||
+      !make_map(&mk, kr_visit, D, Lk, Hkv, D * 2, Lk * D * 2, 128, 1) ||
+      !make_map(&mv, v_visit, D, Hkv, Lk, D * 2, Hkv * D * 2, 1, 128))
+    return TTT_ERR_CUDA;
+  // the branch keys' tiles (this chunk's own passes 2..P); without them the maps are
+  // never used and stand in as copies of the query map
+  mek = mq;
+  mev = mq;
+  if (g.ring == 2 && g.P > 1 &&
+      (!make_map(&mek, kr_local, D, Lq, P * Hkv, D * 2, Lq * D * 2, 128, 1) ||
+       !make_map4(&mev, v_local, {D, Hkv, Lq, P}, {D * 2, Hkv * D * 2, static_cast<uint64_t>(g.skv) * 2},
+                  {1, 128, 1})))
     return TTT_ERR_CUDA;
   TrunkFwdArgs a{g, o_part, kr_local, v_local, nullptr, lse_part, static_cast<uint32_t*>(status),
                  g_wait_budget_ns.load()};
-  TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, stream));
+  // fp32 partial output: the bf16 output map is not used
+  TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, mq, mek, mev, stream));
   return TTT_OK;
 }
 

@@ -92,16 +92,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_rows_kernel(Geometry g, int
     }
     const uint4 av = *reinterpret_cast<const uint4*>(src + d0);
     const uint4 bv = *reinterpret_cast<const uint4*>(src + HALF + d0);
-    const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&av);
-    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&bv);
     uint4 oa, ob;
-    __nv_bfloat16* ya = reinterpret_cast<__nv_bfloat16*>(&oa);
-    __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      ya[e] = rotate_round(xa[e], xb[e], rh[e], rl[e], false);
-      yb[e] = rotate_round(xa[e], xb[e], rh[e], rl[e], true);
-    }
+    rotate8_round(av, bv, rh, rl, oa, ob);
     *reinterpret_cast<uint4*>(dst + d0) = oa;
     *reinterpret_cast<uint4*>(dst + HALF + d0) = ob;
   }

@@ -29,13 +29,41 @@ __device__ __forceinline__ void trace_point(int slot, int j) {
     g_trace[slot][j] = t;
   }
 }
+// Every CTA (up to kCtaTrace) also records its SM, its work count and %clock64 /
+// %globaltimer at four points: entry, first tile ready, last tile done, exit.
+constexpr int kCtaTrace = 8192;
+static __device__ long long g_cta[kCtaTrace][10];
+__device__ __forceinline__ void cta_mark(int point) {
+  if (blockIdx.x < kCtaTrace) {
+    long long t;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+    g_cta[blockIdx.x][point] = t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    g_cta[blockIdx.x][4 + point] = t;
+  }
+}
+__device__ __forceinline__ void cta_info(int work) {
+  if (blockIdx.x < kCtaTrace) {
+    unsigned sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    g_cta[blockIdx.x][8] = sm;
+    g_cta[blockIdx.x][9] = work;
+  }
+}
 #define TTT_TRACE(slot, j) ::ttt::trace_point((slot), (j))
+#define TTT_CTA_MARK(point) ::ttt::cta_mark(point)
+#define TTT_CTA_INFO(work) ::ttt::cta_info(work)
 #define TTT_TRACE_READER(name)                                                                       \
   extern "C" int name(void* host) {                                                                  \
     return static_cast<int>(cudaMemcpyFromSymbol(host, ::ttt::g_trace, sizeof(::ttt::g_trace)));     \
+  }                                                                                                  \
+  extern "C" int name##_cta(void* host) {                                                            \
+    return static_cast<int>(cudaMemcpyFromSymbol(host, ::ttt::g_cta, sizeof(::ttt::g_cta)));         \
   }
 #else
 #define TTT_TRACE(slot, j) ((void)0)
+#define TTT_CTA_MARK(point) ((void)0)
+#define TTT_CTA_INFO(work) ((void)0)
 #define TTT_TRACE_READER(name)
 #endif
 
@@ -200,6 +228,15 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Tiled bulk tensor store shared -> global (bulk-group completion; coordinates >= 0).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                             int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -271,6 +308,10 @@ __device__ __forceinline__ void bulk_wait_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// every bulk group has finished reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 
 // ---------------------------------------------------------------------------
 // tcgen05: shared-memory matrix descriptors, instruction descriptor, MMA
@@ -506,6 +547,46 @@ __device__ __forceinline__ __nv_bfloat16 rotate_round(__nv_bfloat16 x1b, __nv_bf
   const float mid = __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
   if (fabsf(y - mid) > (fabsf(x1) + fabsf(x2)) * 4.76837158203125e-07f) return __float2bfloat16_rn(y);  // 2^-21
   return rotate_round_exact(x1, x2, hi, lo, second);
+}
+
+// Eight (x1, x2) pairs of one head row (x1 = a[e] in the first half, x2 = b[e] in the
+// second): oa[e] = x1 c - x2 s, ob[e] = x2 c + x1 s, rounded as rotate_round rounds them.
+// All sixteen results are first evaluated in plain fp32 and packed; the elements within
+// the error bound of a bf16 midpoint are only flagged, and redone after the packing in
+// float-float arithmetic, so the common path carries no branch per element.
+// lo is read in the rare path only: a register array or a pointer to shared memory.
+template <typename LoT>
+__device__ __forceinline__ void rotate8_round(const uint4& av, const uint4& bv, const float2 (&hi)[8], const LoT& lo,
+                                              uint4& oa, uint4& ob) {
+  const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&av);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&bv);
+  float y1[8], y2[8];
+  uint32_t near = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float x1 = __bfloat162float(xa[e]), x2 = __bfloat162float(xb[e]);
+    y1[e] = fmaf(x1, hi[e].x, -x2 * hi[e].y);
+    y2[e] = fmaf(x2, hi[e].x, x1 * hi[e].y);
+    const float bound = (fabsf(x1) + fabsf(x2)) * 4.76837158203125e-07f;  // 2^-21
+    const float m1 = __uint_as_float((__float_as_uint(y1[e]) & 0xFFFF0000u) | 0x8000u);
+    const float m2 = __uint_as_float((__float_as_uint(y2[e]) & 0xFFFF0000u) | 0x8000u);
+    near |= (fabsf(y1[e] - m1) > bound ? 0u : 1u) << e;
+    near |= (fabsf(y2[e] - m2) > bound ? 0u : 1u) << (8 + e);
+  }
+  oa = make_uint4(pack_bf16x2(y1[0], y1[1]), pack_bf16x2(y1[2], y1[3]), pack_bf16x2(y1[4], y1[5]),
+                  pack_bf16x2(y1[6], y1[7]));
+  ob = make_uint4(pack_bf16x2(y2[0], y2[1]), pack_bf16x2(y2[2], y2[3]), pack_bf16x2(y2[4], y2[5]),
+                  pack_bf16x2(y2[6], y2[7]));
+  if (near != 0u) {
+    __nv_bfloat16* ya = reinterpret_cast<__nv_bfloat16*>(&oa);
+    __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(&ob);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x1 = __bfloat162float(xa[e]), x2 = __bfloat162float(xb[e]);
+      if (near & (1u << e)) ya[e] = rotate_round_exact(x1, x2, hi[e], lo[e], false);
+      if (near & (1u << (8 + e))) yb[e] = rotate_round_exact(x1, x2, hi[e], lo[e], true);
+    }
+  }
 }
 
 // Trunk-key limit of block-draft query row r of a sequence whose block rows start at

@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const Geometry& g = a.g;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) TTT_CTA_MARK(0);
 
   // ---- work item: (key tile jk, sequence n, KV head).  The (sequence, KV head) groups
   // go in bands of nb groups, about 256 CTAs per band; inside a band the smallest jk
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int jq0 = MODE == 0 ? k0 / C::BQ : first_tile_seeing(g, a.qlim, seq_start, len, k0);
   const int nqt = (len + C::BQ - 1) / C::BQ - jq0;
   const int NIT = G * nqt;
+  if (threadIdx.x == 0) TTT_CTA_INFO(NIT);
   if (NIT <= 0) {
     // block-draft keys that no query row sees: zero gradients
     for (int i = threadIdx.x; i < C::BK * (D / 8); i += blockDim.x) {
@@ -394,6 +396,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         break;
       }
       if (lane == 0 && warp == 4) TTT_TRACE(5, it);
+      if (lane == 0 && warp == 4 && it == 0) TTT_CTA_MARK(1);
       if (lane == 0 && warp == 8) TTT_TRACE(13, it);
       tc_fence_after();
       uint32_t sv[32], dp[32];
@@ -485,6 +488,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     // dK = sigma * R(pos)^T dk~ in bf16 (the trunk keys' rotation at their own position)
     if (ok && wait_warp(final_bar, 0, wd, kSiteBwdFinal)) {
       tc_fence_after();
+      if (lane == 0 && warp == 4) TTT_CTA_MARK(2);
       const int64_t tau = kstart + kpos;
       if (hf == 0) {
 #pragma unroll 1
@@ -593,6 +597,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) TTT_CTA_MARK(3);
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 

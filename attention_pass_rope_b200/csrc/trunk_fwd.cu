@@ -52,6 +52,7 @@ struct FwdCfg {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kEpiTiles = 2;               // epilogue keys staged through the ring stages
 
 // MODE 0: TTT trunk+branch attention (epilogue keys: the branch keys of passes 2..p at
 // the query's position).  MODE 1: block-draft attention (query rows are block tokens,
@@ -59,23 +60,23 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // row's own block).  MODE 2: one step of the context-parallel ring (query rows are a
 // chunk of the sequence, trunk keys a visiting chunk, causal by global position; the
 // branch keys only in the step that meets the chunk's own keys; fp32 partial output).
-template <int MODE>
-struct EpiKeys {
-  static constexpr int kMax = MODE == 1 ? 16 : 15;  // P <= 16 passes; Bs <= 16
-};
+// The epilogue keys of a row (up to 15 branch passes, or Bs <= 16 block keys) join it
+// one at a time, so their number is not bounded by the kernel.
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     trunk_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                     const __grid_constant__ CUtensorMap map_v, const TrunkFwdArgs a) {
+                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
+                     const __grid_constant__ CUtensorMap map_ek, const __grid_constant__ CUtensorMap map_ev,
+                     const TrunkFwdArgs a) {
   using C = FwdCfg<D>;
-  constexpr int kMaxBranch = EpiKeys<MODE>::kMax;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
   const Geometry& g = a.g;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) TTT_CTA_MARK(0);
 
   // ---- work item: (query block jq, sequence n, KV head, pair of (pass, head) tiles),
   // largest jq first (longest causal rows first).
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                   : MODE == 1 ? *nkv_slot
                               : min(q0 + min(C::BM, len - q0) - 1 + g.limit_off, klen - 1) / C::BN + 1;
   const Watchdog wd{abort_flag, a.status, a.budget_ns};
+  if (threadIdx.x == 0) TTT_CTA_INFO(nkv);
 
   int p_of[2], h_of[2];
   for (int t = 0; t < 2; ++t) {
@@ -158,6 +160,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     p_of[t] = qh / gsz;
     h_of[t] = kvh * gsz + qh % gsz;
   }
+  // Epilogue keys whose k~ / V rows come as 128-row tiles into the ring stages once the
+  // trunk stream has released them (nothing reuses them afterwards): MODE 0 / 2 the
+  // branch passes 2 and 3 (key u = pass u+1 at the rows' own positions, the same for
+  // both query tiles), k~ in K stages nkv, nkv+1 and V in V stage nkv and K stage nkv+2;
+  // MODE 1 the tile's own block rows (k~ in K stage nkv, V in V stage nkv).  Further
+  // keys are read from global memory.
+  const int ne = MODE == 1   ? 1
+                 : MODE == 2 && g.ring != 2 ? 0
+                                            : min(max(p_of[0], nq_tiles > 1 ? p_of[1] : 0), kEpiTiles);
 
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
@@ -169,6 +180,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&map_q);
       tma_prefetch_desc(&map_k);
       tma_prefetch_desc(&map_v);
+      if (ne > 0) {
+        tma_prefetch_desc(&map_ek);
+        tma_prefetch_desc(&map_ev);
+      }
       mbar_arrive_expect_tx(q_full, nq_tiles * C::TILE);
       for (int t = 0; t < nq_tiles; ++t)
         for (int c = 0; c < C::KCH; ++c)
@@ -188,6 +203,34 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sV + vs * C::TILE + c * C::CHUNK, &map_v, v_full + vs, c * 64, kvh, krow);
       }
+      // the epilogue tiles, each into a stage whose last trunk reader has completed
+      const int erow = seq_start + q0;
+      auto k_stage_load = [&](int j, const CUtensorMap* map, bool is_v, int u) -> bool {
+        const int ks = j % C::KST;
+        if (j >= C::KST && !wait_bounded(k_empty + ks, ((j / C::KST) - 1) & 1, wd, kSiteFwdKvEmpty)) return false;
+        mbar_arrive_expect_tx(k_full + ks, C::TILE);
+        for (int c = 0; c < C::KCH; ++c) {
+          if (is_v)
+            tma_load_4d(sK + ks * C::TILE + c * C::CHUNK, map, k_full + ks, c * 64, kvh, erow, u + 1);
+          else
+            tma_load_3d(sK + ks * C::TILE + c * C::CHUNK, map, k_full + ks, c * 64, erow,
+                        MODE == 1 ? kvh : (u + 1) * g.Hkv + kvh);
+        }
+        return true;
+      };
+      bool eok = true;
+      for (int u = 0; eok && u < ne; ++u) eok = k_stage_load(nkv + u, &map_ek, false, u);
+      if (eok && ne > 0) {
+        const int vs = nkv % C::VST;
+        if (nkv < C::VST || wait_bounded(v_empty + vs, ((nkv / C::VST) - 1) & 1, wd, kSiteFwdKvEmpty)) {
+          mbar_arrive_expect_tx(v_full + vs, C::TILE);
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_4d(sV + vs * C::TILE + c * C::CHUNK, &map_ev, v_full + vs, c * 64, kvh, erow, MODE == 1 ? 0 : 1);
+        } else {
+          eok = false;
+        }
+      }
+      if (eok && ne > 1) k_stage_load(nkv + 2, &map_ev, true, 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -290,6 +333,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         break;
       }
       if (lane == 0 && wq == 0) TTT_TRACE(4 + t, j);
+      if (lane == 0 && wq == 0 && t == 0 && j == 0) TTT_CTA_MARK(1);
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
@@ -387,18 +431,32 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       }
       if (lane == 0 && wq == 0) TTT_TRACE(12 + t, j);
     }
-    if (ok && (nkv == 0 || wait_warp(o_final + t, 0, wd, kSiteFwdOFinal))) {
+    // the epilogue tiles this query tile reads (warp-agreed waits)
+    const int nkeys = MODE == 0 ? p_of[t] : MODE == 1 ? g.Bs : (g.ring == 2 ? p_of[t] : 0);  // epilogue keys
+    const int ne_t = MODE == 1 ? ne : min(nkeys, ne);
+    auto epi_tiles_ready = [&]() -> bool {
+      for (int u = 0; u < ne_t; ++u)
+        if (!wait_warp(k_full + (nkv + u) % C::KST, ((nkv + u) / C::KST) & 1, wd, kSiteFwdKvFull)) return false;
+      if (ne_t > 0 && !wait_warp(v_full + nkv % C::VST, (nkv / C::VST) & 1, wd, kSiteFwdKvFull)) return false;
+      if (ne_t > 1 && !wait_warp(k_full + (nkv + 2) % C::KST, ((nkv + 2) / C::KST) & 1, wd, kSiteFwdKvFull))
+        return false;
+      return true;
+    };
+    if (ok && (nkv == 0 || wait_warp(o_final + t, 0, wd, kSiteFwdOFinal)) && epi_tiles_ready()) {
       tc_fence_after();
-      // ---- epilogue: branch keys (a3) and the exact joint-LSE merge (a4).
+      if (lane == 0 && wq == 0 && t == 0) TTT_CTA_MARK(2);
+      // ---- epilogue: the epilogue keys (a3) and the exact joint-LSE merge (a4).
       // MODE 0: query (pass p, position qpos) also sees k~_j[tau], V_j[tau] of the branch
       // passes j = 1..p (0-based) at its own position.  MODE 1: a block token also sees
-      // the Bs keys of its own block (bidirectional).  Scores on the CUDA cores.  The
-      // trunk partial is (m_run, l_run, unnormalised O in TMEM), all in log2 units.
+      // the Bs keys of its own block (bidirectional).  MODE 2: the branch keys, in the step
+      // that meets the chunk's own keys only.  The trunk partial is (m_run, l_run,
+      // unnormalised O in TMEM), in log2 units; the keys join it one at a time by the
+      // same online rule (running max, rescaled sum and O), each key's k~ and V rows
+      // fetched in one round of loads, its score on the CUDA cores against q~ in smem.
       const bool valid = qpos < len;
       const int p = p_of[t], h = h_of[t];
       const int tau = seq_start + qpos;
       const int T = g.si.T;
-      const int nkeys = MODE == 0 ? p : MODE == 1 ? g.Bs : (g.ring == 2 ? p : 0);  // epilogue keys of this row
       const int bstart = MODE == 1 ? tau - qpos % g.Bs : 0;  // first row of the block
       // key u (0-based) of the epilogue: k~ row and V row
       auto krow_of = [&](int u) -> const uint4* {
@@ -406,96 +464,164 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                                     : static_cast<int64_t>(kvh) * T + bstart + u;
         return reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + r * D);
       };
-      auto vrow_of = [&](int u) -> const __nv_bfloat16* {
-        return MODE != 1 ? static_cast<const __nv_bfloat16*>(a.v) + (u + 1) * g.skv +
-                               (static_cast<int64_t>(tau) * g.Hkv + kvh) * D
-                         : static_cast<const __nv_bfloat16*>(a.v) +
-                               (static_cast<int64_t>(bstart + u) * g.Hkv + kvh) * D;
+      auto vrow_of = [&](int u) -> const uint4* {
+        return reinterpret_cast<const uint4*>(
+            MODE != 1 ? static_cast<const __nv_bfloat16*>(a.v) + (u + 1) * g.skv +
+                            (static_cast<int64_t>(tau) * g.Hkv + kvh) * D
+                      : static_cast<const __nv_bfloat16*>(a.v) + (static_cast<int64_t>(bstart + u) * g.Hkv + kvh) * D);
       };
-      float bs[kMaxBranch];
-      float m = m_run;
+      // this row of the Q tile (q~ in, the output row out: each thread touches only its
+      // own row, and every product that read the tile completed before o_final)
+      uint8_t* srow = sQ + t * C::TILE + row * 128;
+      auto unit = [&](int c8) -> uint8_t* { return srow + (c8 >> 3) * C::CHUNK + (((c8 & 7) ^ (row & 7)) << 4); };
+      // the warp's 32 rows all belong to the sequence: the output goes out by one tensor
+      // store per 64 columns
+      const bool warp_full = MODE != 2 && q0 + 32 * wq + 32 <= len;
+      float m = m_run, l = l_run;
+      bool o_live = nkv > 0;  // O in TMEM holds the trunk part (CTA-uniform)
+      // O <- alpha O + w V (V absent: w = 0), in TMEM for keys before the last, to the
+      // output (scaled by 1 / l) for the last
+      // 16-byte unit c8 of row rr of a 128-row tile in a ring stage (128-byte swizzle)
+      auto tile_unit = [&](const uint8_t* stage, int rr, int c8) -> const uint4* {
+        return reinterpret_cast<const uint4*>(stage + (c8 >> 3) * C::CHUNK + rr * 128 + (((c8 & 7) ^ (rr & 7)) << 4));
+      };
+      // V row: from a staged tile (vsm, row rr), else from global memory (vgl; none: w = 0)
+      auto fold = [&](float alpha, float w, const uint4* vgl, const uint8_t* vsm, int rr, bool last) {
+        const float inv_l = 1.f / l;
 #pragma unroll
-      for (int j = 1; j <= kMaxBranch; ++j) {
-        bs[j - 1] = -INFINITY;
-        if (j <= nkeys && valid) {
-          const uint4* kj = krow_of(j - 1);
-          const uint8_t* qrow = sQ + t * C::TILE + row * 128;
-          float acc = 0.f;
-#pragma unroll 4
-          for (int c8 = 0; c8 < D / 8; ++c8) {
-            const uint4 qv = *reinterpret_cast<const uint4*>(qrow + (c8 >> 3) * C::CHUNK + (((c8 & 7) ^ (row & 7)) << 4));
-            const uint4 kv = __ldg(kj + c8);
-            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qv);
-            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kv);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          if (o_live) {
+            tmem_ld32(lane_base + colO + 32 * c, o);
+            tmem_ld_wait();
+            reg_fence32(o);
+          } else {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 a2 = __bfloat1622float2(q2[u]);
-              const float2 b2 = __bfloat1622float2(k2[u]);
-              acc = fmaf(a2.x, b2.x, fmaf(a2.y, b2.y, acc));
-            }
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
           }
-          bs[j - 1] = acc * sl2;
-          m = fmaxf(m, bs[j - 1]);
-        }
-      }
-      const float scale_t = exp2_approx(m_run - m);
-      float l = l_run * scale_t;
-#pragma unroll
-      for (int j = 0; j < kMaxBranch; ++j) {
-        bs[j] = exp2_approx(bs[j] - m);  // branch weights (0 for absent passes)
-        l += bs[j];
-      }
-      const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + p * g.sq + (static_cast<int64_t>(tau) * g.H + h) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (nkv > 0) {  // CTA-uniform: no trunk key at all leaves O in TMEM unwritten
-          tmem_ld32(lane_base + colO + 32 * c, o);
-          tmem_ld_wait();
-          reg_fence32(o);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        if (valid) {
           float acc[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * scale_t;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 v4 = vsm   ? *tile_unit(vsm, rr, 4 * c + q4)
+                             : vgl ? __ldg(vgl + 4 * c + q4)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
 #pragma unroll
-          for (int j = 1; j <= kMaxBranch; ++j) {
-            if (j <= nkeys) {
-              const uint4* vj = reinterpret_cast<const uint4*>(vrow_of(j - 1) + 32 * c);
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                const uint4 vv = __ldg(vj + q4);
-                const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const float2 f2 = __bfloat1622float2(v2[u]);
-                  acc[8 * q4 + 2 * u] = fmaf(bs[j - 1], f2.x, acc[8 * q4 + 2 * u]);
-                  acc[8 * q4 + 2 * u + 1] = fmaf(bs[j - 1], f2.y, acc[8 * q4 + 2 * u + 1]);
-                }
-              }
+            for (int u = 0; u < 4; ++u) {
+              const float2 f2 = __bfloat1622float2(v2[u]);
+              acc[8 * q4 + 2 * u] = fmaf(w, f2.x, __uint_as_float(o[8 * q4 + 2 * u]) * alpha);
+              acc[8 * q4 + 2 * u + 1] = fmaf(w, f2.y, __uint_as_float(o[8 * q4 + 2 * u + 1]) * alpha);
             }
           }
-          if (MODE == 2) {
-            float4* dst = reinterpret_cast<float4*>(a.o_part + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D +
-                                                    32 * c);
+          if (!last) {
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              dst[q4] = make_float4(acc[4 * q4] * inv_l, acc[4 * q4 + 1] * inv_l, acc[4 * q4 + 2] * inv_l,
-                                    acc[4 * q4 + 3] * inv_l);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(acc[e]);
+            tmem_st32(lane_base + colO + 32 * c, o);
+          } else if (MODE == 2) {
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(a.o_part + ((static_cast<int64_t>(p) * T + tau) * g.H + h) * D +
+                                                      32 * c);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                dst[q4] = make_float4(acc[4 * q4] * inv_l, acc[4 * q4 + 1] * inv_l, acc[4 * q4 + 2] * inv_l,
+                                      acc[4 * q4 + 3] * inv_l);
+            }
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+            uint4 out[4];
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4)
-              dst[q4] = make_uint4(pack_bf16x2(acc[8 * q4] * inv_l, acc[8 * q4 + 1] * inv_l),
+              out[q4] = make_uint4(pack_bf16x2(acc[8 * q4] * inv_l, acc[8 * q4 + 1] * inv_l),
                                    pack_bf16x2(acc[8 * q4 + 2] * inv_l, acc[8 * q4 + 3] * inv_l),
                                    pack_bf16x2(acc[8 * q4 + 4] * inv_l, acc[8 * q4 + 5] * inv_l),
                                    pack_bf16x2(acc[8 * q4 + 6] * inv_l, acc[8 * q4 + 7] * inv_l));
+            if (warp_full) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) *reinterpret_cast<uint4*>(unit(4 * c + q4)) = out[q4];
+            } else if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + p * g.sq +
+                                                    (static_cast<int64_t>(tau) * g.H + h) * D + 32 * c);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) dst[q4] = out[q4];
+            }
           }
         }
+        if (!last) {
+          tmem_st_wait();
+          o_live = true;
+        }
+      };
+      for (int u = 0; u < nkeys; ++u) {
+        // key u from a staged tile when it is there: MODE 0 / 2 the first ne keys (row =
+        // this row), MODE 1 the block rows inside this tile
+        const uint8_t* ksm = nullptr;
+        const uint8_t* vsm = nullptr;
+        int rr = row;
+        if (MODE == 1) {
+          rr = row - qpos % g.Bs + u;
+          if (ne > 0 && rr >= 0 && rr < C::BM) {
+            ksm = sK + (nkv % C::KST) * C::TILE;
+            vsm = sV + (nkv % C::VST) * C::TILE;
+          }
+        } else if (u < ne) {
+          ksm = sK + ((nkv + u) % C::KST) * C::TILE;
+          vsm = u == 0 ? sV + (nkv % C::VST) * C::TILE : sK + ((nkv + 2) % C::KST) * C::TILE;
+        }
+        const uint4* vgl = nullptr;
+        float acc0 = 0.f, acc1 = 0.f;
+        auto dot_unit = [&](int c8, const uint4& kq) {
+          const uint4 qv = *reinterpret_cast<const uint4*>(unit(c8));
+          const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qv);
+          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kq);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 a2 = __bfloat1622float2(q2[e]);
+            const float2 b2 = __bfloat1622float2(k2[e]);
+            if (e & 1)
+              acc1 = fmaf(a2.x, b2.x, fmaf(a2.y, b2.y, acc1));
+            else
+              acc0 = fmaf(a2.x, b2.x, fmaf(a2.y, b2.y, acc0));
+          }
+        };
+        if (ksm) {
+#pragma unroll
+          for (int c8 = 0; c8 < D / 8; ++c8) dot_unit(c8, *tile_unit(ksm, rr, c8));
+        } else {
+          uint4 kv[D / 8];
+          if (valid) {
+            const uint4* kj = krow_of(u);
+            vgl = vrow_of(u);
+#pragma unroll
+            for (int c8 = 0; c8 < D / 8; ++c8) kv[c8] = __ldg(kj + c8);
+          } else {
+#pragma unroll
+            for (int c8 = 0; c8 < D / 8; ++c8) kv[c8] = make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < D / 8; ++c8) dot_unit(c8, kv[c8]);
+        }
+        const float s = valid ? (acc0 + acc1) * sl2 : -INFINITY;
+        const float m_new = fmaxf(m, s);
+        const float base = m_new == -INFINITY ? 0.f : m_new;  // a row that has seen no key yet
+        const float alpha = exp2_approx(m - base), w = exp2_approx(s - base);
+        l = l * alpha + w;
+        m = m_new;
+        fold(alpha, w, vgl, vsm, rr, u + 1 == nkeys);
+      }
+      if (nkeys == 0) fold(1.f, 0.f, nullptr, nullptr, row, true);
+      if (warp_full) {
+        // this warp's 32 output rows are in the tile's shared memory: one tensor store per
+        // 64 columns, issued once they are visible to the async proxy
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int cc = 0; cc < C::KCH; ++cc)
+            tma_store_4d(&map_o, sQ + t * C::TILE + cc * C::CHUNK + wq * 32 * 128, cc * 64, h, seq_start + q0 + 32 * wq,
+                         p);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        __syncwarp();
       }
       if (valid) a.lse[lse_index(g.si, g.H, p, h, n, tau, qpos)] = (m + __log2f(l)) * kLn2;
     }
@@ -504,12 +630,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) TTT_CTA_MARK(3);
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 template <int D, int MODE>
 cudaError_t launch(const TrunkFwdArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                   cudaStream_t stream) {
+                   const CUtensorMap& mo, const CUtensorMap& mek, const CUtensorMap& mev, cudaStream_t stream) {
   using C = FwdCfg<D>;
   cudaError_t e =
       cudaFuncSetAttribute(trunk_fwd_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -520,19 +647,24 @@ cudaError_t launch(const TrunkFwdArgs& a, const CUtensorMap& mq, const CUtensorM
   const long long blocks = static_cast<long long>(njq) * a.g.si.nseq * a.g.Hkv * npairs;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  trunk_fwd_kernel<D, MODE><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, a);
+  trunk_fwd_kernel<D, MODE><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mo, mek, mev, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
-                             const CUtensorMap& map_v, cudaStream_t stream) {
+                             const CUtensorMap& map_v, const CUtensorMap& map_o, const CUtensorMap& map_ek,
+                             const CUtensorMap& map_ev, cudaStream_t stream) {
+  const bool d128 = a.g.D == 128;
   if (a.g.ring > 0)
-    return a.g.D == 128 ? launch<128, 2>(a, map_q, map_k, map_v, stream) : launch<64, 2>(a, map_q, map_k, map_v, stream);
+    return d128 ? launch<128, 2>(a, map_q, map_k, map_v, map_o, map_ek, map_ev, stream)
+                : launch<64, 2>(a, map_q, map_k, map_v, map_o, map_ek, map_ev, stream);
   if (a.g.Bs > 0)
-    return a.g.D == 128 ? launch<128, 1>(a, map_q, map_k, map_v, stream) : launch<64, 1>(a, map_q, map_k, map_v, stream);
-  return a.g.D == 128 ? launch<128, 0>(a, map_q, map_k, map_v, stream) : launch<64, 0>(a, map_q, map_k, map_v, stream);
+    return d128 ? launch<128, 1>(a, map_q, map_k, map_v, map_o, map_ek, map_ev, stream)
+                : launch<64, 1>(a, map_q, map_k, map_v, map_o, map_ek, map_ev, stream);
+  return d128 ? launch<128, 0>(a, map_q, map_k, map_v, map_o, map_ek, map_ev, stream)
+              : launch<64, 0>(a, map_q, map_k, map_v, map_o, map_ek, map_ev, stream);
 }
 
 }  // namespace ttt

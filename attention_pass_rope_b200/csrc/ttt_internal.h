@@ -91,9 +91,15 @@ struct TrunkFwdArgs {
 };
 // a2+a3+a4: trunk causal attention on tcgen05 with the branch keys and the exact
 // joint-LSE merge in its epilogue.  Maps: q~ (3D {D, T, P*H}), k~_1 (3D {D, T, Hkv}),
-// V_1 (3D {D, Hkv, T}), all 64-element (128-byte) swizzled boxes.
+// V_1 (3D {D, Hkv, T}), all 64-element (128-byte) swizzled boxes; map_o is the bf16
+// output (4D {D, H, T, P}, passes g.sq apart, box {64, 1, 32, 1}) that full 32-row
+// warp slices are stored through (MODE 2 writes fp32 directly and ignores it).
+// map_ek / map_ev cover the epilogue keys' k~ and V (a.kr, a.v) as 128-row tiles:
+// MODE 0 / 2 k~ 3D {D, rows, P*Hkv} and V 4D {D, Hkv, rows, P} (passes g.skv apart);
+// MODE 1 k~ 3D {D, rows, Hkv} and V 4D {D, Hkv, rows, 1}.
 cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
-                             const CUtensorMap& map_v, cudaStream_t stream);
+                             const CUtensorMap& map_v, const CUtensorMap& map_o, const CUtensorMap& map_ek,
+                             const CUtensorMap& map_ev, cudaStream_t stream);
 
 // Row statistics of the backward, tile-aligned: for query head (p, h) and the 64-row
 // query tile j of sequence n, slot = start_n / 64 + n + j holds 64 values of
