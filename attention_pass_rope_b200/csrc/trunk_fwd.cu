@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   const int q0 = jq * C::BM;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;             // [KST]
+  uint64_t* q_full = bars + 0;             // [NQ]: one per query tile
+  uint64_t* k_full = bars + C::NQ;         // [KST]
   uint64_t* k_empty = k_full + C::KST;     // [KST]
   uint64_t* v_full = k_empty + C::KST;     // [VST]
   uint64_t* v_empty = v_full + C::VST;     // [VST]
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   int* nkv_slot = reinterpret_cast<int*>(abort_flag + 1);
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int t = 0; t < C::NQ; ++t) mbar_init(q_full + t, 1);
     for (int s = 0; s < C::KST; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
@@ -184,11 +184,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         tma_prefetch_desc(&map_ek);
         tma_prefetch_desc(&map_ev);
       }
-      mbar_arrive_expect_tx(q_full, nq_tiles * C::TILE);
-      for (int t = 0; t < nq_tiles; ++t)
+      // Q_0 first, then K_0, then Q_1: the first product S_0(0) needs only Q_0 and K_0
+      auto load_q = [&](int t) {
+        mbar_arrive_expect_tx(q_full + t, C::TILE);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &map_q, q_full, c * 64, seq_start + q0,
+          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &map_q, q_full + t, c * 64, seq_start + q0,
                       p_of[t] * g.H + h_of[t]);
+      };
+      load_q(0);
+      if (nkv == 0 && nq_tiles > 1) load_q(1);
       for (int j = 0; j < nkv; ++j) {
         const int krow = kstart + j * C::BN;
         const int ks = j % C::KST;
@@ -197,6 +201,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         mbar_arrive_expect_tx(k_full + ks, C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sK + ks * C::TILE + c * C::CHUNK, &map_k, k_full + ks, c * 64, krow, kvh);
+        if (j == 0 && nq_tiles > 1) load_q(1);
         const int vs = j % C::VST;
         if (j >= C::VST && !wait_bounded(v_empty + vs, ((j / C::VST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
         mbar_arrive_expect_tx(v_full + vs, C::TILE);
@@ -262,7 +267,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int kk = k0; kk < k1; ++kk)
           umma_ts_warp(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), idO, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_warp(q_full, 0, wd, kSiteFwdQ);
+      bool ok = true;
       // Order per KV tile j: for each query tile t, O_t += P_t(j-1) V_{j-1}, then
       // S_t(j) = Q_t K_j^T.  The in-order tensor pipe finishes reading P_t(j-1) (which
       // overlays S_t) before S_t(j) overwrites it.
@@ -292,6 +297,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (t == nq_tiles - 1) umma_commit_warp(v_empty + (j - 1) % C::VST);
           }
           if (j < nkv) {
+            if (j == 0 && !wait_warp(q_full + t, 0, wd, kSiteFwdQ)) {
+              ok = false;
+              break;
+            }
             if (t == 0 && !wait_warp(k_full + j % C::KST, (j / C::KST) & 1, wd, kSiteFwdKvFull)) {
               ok = false;
               break;
@@ -349,23 +358,25 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int e = 0; e < 32; ++e)
             if (k0 + 32 * c + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
       }
-      // row max: 8 independent chains, then a tree
+      // row max: 8 independent chains of three-input maxima, then a tree
       float mxv[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mxv[u] = fmaxf(__uint_as_float(sr[0][u]), __uint_as_float(sr[0][u + 8]));
+      for (int u = 0; u < 8; ++u)
+        mxv[u] = max3f(__uint_as_float(sr[0][u]), __uint_as_float(sr[0][u + 8]), __uint_as_float(sr[0][u + 16]));
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        mxv[u] = fmaxf(mxv[u], fmaxf(__uint_as_float(sr[0][u + 16]), __uint_as_float(sr[0][u + 24])));
-#pragma unroll
-        for (int c = 1; c < 4; ++c)
-          mxv[u] = fmaxf(fmaxf(mxv[u], __uint_as_float(sr[c][u])),
-                         fmaxf(fmaxf(__uint_as_float(sr[c][u + 8]), __uint_as_float(sr[c][u + 16])),
-                               __uint_as_float(sr[c][u + 24])));
+        mxv[u] = max3f(mxv[u], __uint_as_float(sr[0][u + 24]), __uint_as_float(sr[1][u]));
+        mxv[u] = max3f(mxv[u], __uint_as_float(sr[1][u + 8]), __uint_as_float(sr[1][u + 16]));
+        mxv[u] = max3f(mxv[u], __uint_as_float(sr[1][u + 24]), __uint_as_float(sr[2][u]));
+        mxv[u] = max3f(mxv[u], __uint_as_float(sr[2][u + 8]), __uint_as_float(sr[2][u + 16]));
+        mxv[u] = max3f(mxv[u], __uint_as_float(sr[2][u + 24]), __uint_as_float(sr[3][u]));
+        mxv[u] = max3f(mxv[u], __uint_as_float(sr[3][u + 8]), __uint_as_float(sr[3][u + 16]));
+        mxv[u] = fmaxf(mxv[u], __uint_as_float(sr[3][u + 24]));
       }
-#pragma unroll
-      for (int u = 4; u > 0; u >>= 1)
-#pragma unroll
-        for (int v = 0; v < u; ++v) mxv[v] = fmaxf(mxv[v], mxv[v + u]);
+      mxv[0] = max3f(mxv[0], mxv[1], mxv[2]);
+      mxv[3] = max3f(mxv[3], mxv[4], mxv[5]);
+      mxv[6] = fmaxf(mxv[6], mxv[7]);
+      mxv[0] = max3f(mxv[0], mxv[3], mxv[6]);
       const float m_new = fmaxf(m_run, mxv[0] * sl2);
       if (lane == 0 && wq == 0) TTT_TRACE(8 + t, j);
       const bool rescale = m_new > m_run + kRescaleThreshold;
@@ -378,7 +389,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       // a warp with a row whose O needs rescaling releases P only after the rescale (rare:
       // the running max grew by more than 2^8); the others release the first 64 keys early
       const bool warp_rescale = __any_sync(0xffffffffu, rescale && j > 0);
-      float rsv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // paired row-sum accumulators
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_run, -m_run);
       // P = 2^(s*scale*log2e - m), bf16 pairs into the first 64 columns of S_t; the first
       // 64 keys are released to the MMA warp before the last 64 are computed
 #pragma unroll
@@ -386,10 +398,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_run));
-          const float p1 = exp2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_run));
-          rsv[(2 * e) & 7] += p0;
-          rsv[(2 * e + 1) & 7] += p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sl2x2, negm2),
+                    x0, x1);
+          const float p0 = exp2_approx(x0);
+          const float p1 = exp2_approx(x1);
+          rs2[e & 3] = f2_add(rs2[e & 3], f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(lane_base + colS + 16 * c, pk);
@@ -400,11 +414,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           if (lane == 0) mbar_arrive(p_half + t);
         }
       }
-#pragma unroll
-      for (int u = 4; u > 0; u >>= 1)
-#pragma unroll
-        for (int v = 0; v < u; ++v) rsv[v] += rsv[v + u];
-      l_run += rsv[0];
+      rs2[0] = f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3]));
+      float rs_lo, rs_hi;
+      f2_unpack(rs2[0], rs_lo, rs_hi);
+      l_run += rs_lo + rs_hi;
       if (lane == 0 && wq == 0) TTT_TRACE(10 + t, j);
       if (warp_rescale) {
         // O of this row was complete up to tile j-1 when s_full fired (in-order MMAs), and
@@ -435,6 +448,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int nkeys = MODE == 0 ? p_of[t] : MODE == 1 ? g.Bs : (g.ring == 2 ? p_of[t] : 0);  // epilogue keys
     const int ne_t = MODE == 1 ? ne : min(nkeys, ne);
     auto epi_tiles_ready = [&]() -> bool {
+      // with no trunk key no product waited for the Q tile: the scores below read it
+      if (nkv == 0 && !wait_warp(q_full + t, 0, wd, kSiteFwdQ)) return false;
       for (int u = 0; u < ne_t; ++u)
         if (!wait_warp(k_full + (nkv + u) % C::KST, ((nkv + u) / C::KST) & 1, wd, kSiteFwdKvFull)) return false;
       if (ne_t > 0 && !wait_warp(v_full + nkv % C::VST, (nkv / C::VST) & 1, wd, kSiteFwdKvFull)) return false;
