@@ -372,6 +372,15 @@ ttt_status ttt_attn_fwd(const ttt_attn_desc* desc, const void* q, const void* k,
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_FWD, stream);
     TrunkFwdArgs a{g, nullptr, kr, v, o, lse, status, g_wait_budget_ns.load()};
+    // a workspace sized for the backward: its dq~ accumulator is zeroed here, by warps
+    // that the attention leaves idle, instead of in the backward's preprocess
+    Plan pb;
+    const bool zero_dq = make_plan(desc, 1, &pb) == TTT_OK && workspace_bytes >= pb.total;
+    if (zero_dq) {
+      a.zero_base = reinterpret_cast<float4*>(ws + pb.off[4]);
+      a.zero_n16 = static_cast<int64_t>(g.P) * g.H * static_cast<int64_t>(T) * static_cast<int64_t>(D) / 4;
+    }
+    a.dq_zeroed = reinterpret_cast<uint32_t*>(ws + kDqZeroedOffset);
     TTT_CHECK_CUDA(launch_trunk_fwd(a, mq, mk, mv, mo, mek, mev, stream));
   }
   return TTT_OK;
@@ -420,7 +429,11 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
-    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, nullptr, status, stream));
+    // a workspace untouched since the forward may hold an already zeroed dq~ accumulator
+    const uint32_t* dq_zeroed = (desc->flags & TTT_FLAG_ROTATED_IN_WORKSPACE)
+                                    ? reinterpret_cast<const uint32_t*>(ws + kDqZeroedOffset)
+                                    : nullptr;
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, nullptr, status, dq_zeroed, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);
@@ -431,6 +444,8 @@ ttt_status ttt_attn_bwd(const ttt_attn_desc* desc, const void* q, const void* k,
     EventScope es(desc->events, TTT_KERNEL_BRANCH_BWD, stream);
     TTT_CHECK_CUDA(launch_branch_bwd(g, qr, kr, v, dout, lse, ld, dq_acc, dq, dk, dv, stream));
   }
+  // the accumulator now holds this call's sums
+  TTT_CHECK_CUDA(cudaMemsetAsync(ws + kDqZeroedOffset, 0, sizeof(uint32_t), stream));
   return TTT_OK;
 }
 
@@ -543,7 +558,7 @@ ttt_status ttt_block_attn_bwd(const ttt_block_desc* desc, const void* k_ctx, con
   }
   {
     EventScope es(desc->events, TTT_KERNEL_BWD_PREPROCESS, stream);
-    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, qlim, status, stream));
+    TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, ld, dq_acc, tickets, qlim, status, nullptr, stream));
   }
   {
     EventScope es(desc->events, TTT_KERNEL_TRUNK_BWD, stream);

@@ -99,7 +99,8 @@ template <int D>
 __global__ void __launch_bounds__(kPreThreads)
     bwd_preprocess_kernel(Geometry g, const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                           const float* __restrict__ lse, float* __restrict__ ld, float* __restrict__ dq_acc,
-                          int* __restrict__ tickets, int ntile, int* __restrict__ qlim, uint32_t* status) {
+                          int* __restrict__ tickets, int ntile, int* __restrict__ qlim, uint32_t* status,
+                          const uint32_t* __restrict__ dq_zeroed) {
   constexpr int LPR = D / 8;                            // lanes per row
   constexpr int RPI = 32 / LPR;                         // rows per warp instruction
   constexpr int RPWARP = kPreRows / (kPreThreads / 32);  // rows per warp (8)
@@ -133,9 +134,12 @@ __global__ void __launch_bounds__(kPreThreads)
       b[u] = make_uint4(0, 0, 0, 0);
     }
   }
-  // zero this tile's dq~ accumulator rows (contiguous: nvalid rows of D floats)
-  float4* z = reinterpret_cast<float4*>(dq_acc + ((static_cast<int64_t>(p) * g.H + h) * T + start + pos0) * D);
-  for (int i = threadIdx.x; i < nvalid * D / 4; i += kPreThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // zero this tile's dq~ accumulator rows (contiguous: nvalid rows of D floats), unless
+  // the forward has zeroed the whole accumulator already
+  if (!dq_zeroed || *dq_zeroed != kDqZeroedMagic) {
+    float4* z = reinterpret_cast<float4*>(dq_acc + ((static_cast<int64_t>(p) * g.H + h) * T + start + pos0) * D);
+    for (int i = threadIdx.x; i < nvalid * D / 4; i += kPreThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
@@ -429,7 +433,8 @@ __global__ void watchdog_selftest_kernel(uint32_t* status, uint64_t budget_ns) {
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  float* dq_acc, int* tickets, int* qlim, uint32_t* status, cudaStream_t stream) {
+                                  float* dq_acc, int* tickets, int* qlim, uint32_t* status,
+                                  const uint32_t* dq_zeroed, cudaStream_t stream) {
   if (g.si.T == 0 || g.si.nseq == 0 || g.si.max_len == 0) return cudaSuccess;
   const int ntile = (g.si.max_len + kPreRows - 1) / kPreRows;
   const long long blocks = static_cast<long long>(g.P) * g.si.nseq * ntile * g.H;
@@ -437,11 +442,11 @@ cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* 
   auto* ob = static_cast<const __nv_bfloat16*>(o);
   auto* db = static_cast<const __nv_bfloat16*>(dout);
   if (g.D == 128)
-    bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
-                                                                                       tickets, ntile, qlim, status);
+    bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(
+        g, ob, db, lse, ld, dq_acc, tickets, ntile, qlim, status, dq_zeroed);
   else
-    bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(g, ob, db, lse, ld, dq_acc,
-                                                                                      tickets, ntile, qlim, status);
+    bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), kPreThreads, 0, stream>>>(
+        g, ob, db, lse, ld, dq_acc, tickets, ntile, qlim, status, dq_zeroed);
   return cudaGetLastError();
 }
 

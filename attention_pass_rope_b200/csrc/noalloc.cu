@@ -84,5 +84,6 @@ extern "C" ttt_status ttt_attn_fwd_noalloc(const ttt_attn_desc* desc, const void
   void* scratch = nullptr;
   const ttt_status st = scratch_on_current_device(&scratch);
   if (st != TTT_OK) return st;
-  return ttt_attn_fwd(desc, q, k, v, o, lse, scratch, kNoallocScratchBytes, stream);
+  // the forward's own size: a larger workspace would also get the backward's accumulator zeroed
+  return ttt_attn_fwd(desc, q, k, v, o, lse, scratch, need, stream);
 }

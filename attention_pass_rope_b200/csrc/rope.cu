@@ -9,8 +9,8 @@
 // g.sq and g.skv elements apart), writes the rotated
 // copies head-major (q~ [P][H][T][D], k~ [P][Hkv][T][D]) so that the attention
 // kernels fetch a (head, 128-token) tile as one contiguous block.  cos/sin depend
-// on (position, frequency) only: each CTA takes 8 tokens with all their passes, computes
-// cos/sin once per position it needs (8 + P - 1 of them) in double precision (argument
+// on (position, frequency) only: each CTA takes 4 tokens with all their passes, computes
+// cos/sin once per position it needs (4 + P - 1 of them) in double precision (argument
 // up to ~4e4 rad) and shares them across all heads.
 #include <cuda_bf16.h>
 
@@ -20,7 +20,7 @@ namespace ttt {
 
 namespace {
 
-constexpr int kRopeTok = 8;       // tokens per CTA
+constexpr int kRopeTok = 4;       // tokens per CTA
 constexpr int kRopeMaxP = 16;     // passes (positions i .. i+P-1 share one table)
 constexpr int kRopeThreads = 256;
 

@@ -8,9 +8,11 @@
 // for both.
 //
 // CTA = 12 warps:
-//   warp 0      TMA producer: two Q tiles once, then K/V tiles into a 2-stage ring
-//   warp 1      TMEM allocator and MMA issuer (one thread): S = Q K^T (SS form),
-//               O += P V (TS form, P read from TMEM)
+//   warp 0      TMA producer: Q_0, K_0, Q_1, then K/V tiles into 3- and 2-stage rings,
+//               then the epilogue keys' k~ / V tiles into the released stages
+//   warp 1      TMEM allocator and MMA issuer (the whole warp runs the loop, one lane
+//               issues): S = Q K^T (SS form), O += P V (TS form, P read from TMEM)
+//   warps 2-3   zero an optional region (the backward's dq~ accumulator) meanwhile
 //   warps 4-7   softmax for query tile 0 (one TMEM lane = one query row per thread)
 //   warps 8-11  softmax for query tile 1
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
@@ -18,7 +20,8 @@
 // The online softmax keeps a running max per row and rescales O (in TMEM) only when
 // the max grows by more than 2^8; the final normalisation uses the same max, so the
 // result is exact up to rounding.
-// Output: O_t (normalised, fp32, head-major) and lse_t (natural log) per row.
+// Output: O (bf16, public layout, full 32-row warp slices by TMA stores through the
+// Q tile's shared memory) and lse (natural log) per row; MODE 2 writes fp32 partials.
 #include "common.cuh"
 
 namespace ttt {
@@ -94,7 +97,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   int seq_start, len, kstart, klen;
   seq_bounds(g.si, n, seq_start, len);  // query rows
   seq_bounds(g.ksi, n, kstart, klen);   // key rows (the same tokens in MODE 0)
-  if (jq * C::BM >= len) return;  // the whole CTA leaves before touching TMEM
+  // this CTA's share of a.zero_base (see TrunkFwdArgs), by threads [first, first + nthr)
+  auto zero_share = [&](int first, int nthr) {
+    if (a.dq_zeroed && blockIdx.x == 0 && static_cast<int>(threadIdx.x) == first)
+      *a.dq_zeroed = a.zero_n16 > 0 ? kDqZeroedMagic : 0u;  // read by a later kernel only
+    if (a.zero_n16 <= 0) return;
+    const int64_t per = (a.zero_n16 + gridDim.x - 1) / gridDim.x;
+    const int64_t lo = static_cast<int64_t>(blockIdx.x) * per;
+    const int64_t hi = min(lo + per, a.zero_n16);
+    for (int64_t i = lo + (static_cast<int>(threadIdx.x) - first); i < hi; i += nthr)
+      a.zero_base[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  if (jq * C::BM >= len) {  // the whole CTA leaves before touching TMEM
+    zero_share(0, C::THREADS);
+    return;
+  }
   const int nq_tiles = (2 * pair + 1 < G) ? 2 : 1;
   const int q0 = jq * C::BM;
 
@@ -319,6 +336,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       wait_drain(drain, 0, wd, kSiteFwdDrain);
     }
     __syncwarp();
+  } else if (warp == 2 || warp == 3) {
+    zero_share(64, 64);
   } else if (warp >= 4 && warp < 4 + 4 * nq_tiles) {
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;

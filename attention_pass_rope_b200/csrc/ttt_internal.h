@@ -88,7 +88,18 @@ struct TrunkFwdArgs {
   float* lse;      // fp32 merged lse, public layout
   uint32_t* status;
   uint64_t budget_ns;
+  // optional: a region that the otherwise idle warps zero while the attention runs (the
+  // backward's dq~ accumulator, when the workspace is the backward's); 16-byte units
+  float4* zero_base;
+  int64_t zero_n16;
+  uint32_t* dq_zeroed;  // optional marker word: set to kDqZeroedMagic when zero_n16 > 0, else to 0
 };
+
+// Workspace word next to the status word: the forward has zeroed the backward's dq~
+// accumulator in this workspace (a backward told that the workspace is untouched since
+// the forward then skips that zeroing, and clears the word).
+constexpr uint32_t kDqZeroedMagic = 0x01010101u;  // every byte 1 (a byte-wise memset)
+constexpr size_t kDqZeroedOffset = 4;
 // a2+a3+a4: trunk causal attention on tcgen05 with the branch keys and the exact
 // joint-LSE merge in its epilogue.  Maps: q~ (3D {D, T, P*H}), k~_1 (3D {D, T, Hkv}),
 // V_1 (3D {D, Hkv, T}), all 64-element (128-byte) swizzled boxes; map_o is the bf16
@@ -109,11 +120,13 @@ cudaError_t launch_trunk_fwd(const TrunkFwdArgs& a, const CUtensorMap& map_q, co
 __host__ __device__ inline int ld_slots(const SeqInfo& si) { return si.T / 64 + si.nseq + 1; }
 
 // a5: delta = rowsum(dO * O); writes the tile-aligned (-lse*log2e, delta) rows and
-// zeroes the fp32 dq~ accumulator [P][H][T][D] and the per-slot order tickets.
+// zeroes the fp32 dq~ accumulator [P][H][T][D] (unless dq_zeroed is given and holds
+// kDqZeroedMagic) and the per-slot order tickets.
 // Block-draft geometry (g.Bs > 0): also writes qlim (the trunk-key limit of every query
 // row) and records kStatusBadAnchors in *status if a sequence's anchors decrease.
 cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* dout, const float* lse, float* ld,
-                                  float* dq_acc, int* tickets, int* qlim, uint32_t* status, cudaStream_t stream);
+                                  float* dq_acc, int* tickets, int* qlim, uint32_t* status,
+                                  const uint32_t* dq_zeroed, cudaStream_t stream);
 
 struct TrunkBwdArgs {
   Geometry g;

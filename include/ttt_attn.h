@@ -124,7 +124,11 @@ typedef enum {
    * the backward uses them instead of rotating q and k again.  The backward's
    * workspace layout starts with the forward's (ttt_attn_workspace_layout), so a
    * workspace sized for the backward and passed to both calls qualifies.  If the
-   * promise is broken the gradients are wrong; nothing is read out of bounds. */
+   * promise is broken the gradients are wrong; nothing is read out of bounds.
+   * A forward given a workspace of at least the backward's size also zeroes the
+   * backward's dq~ accumulator in it (on warps the attention leaves idle) and marks
+   * that in the word after the status word; a backward with this flag then skips
+   * its own zeroing, and every backward clears the mark. */
   TTT_FLAG_ROTATED_IN_WORKSPACE = 1,
   /* ttt_attn_bwd: bitwise reproducible dq.  The trunk backward adds the fp32
    * partial dq~ of the key tiles of a query tile in key-tile order (each waits,
@@ -328,7 +332,8 @@ ttt_status ttt_attn_device_status(void* workspace, void* stream, uint32_t* detai
 
 /* Workspace sub-buffers (byte offsets from the workspace base), for inspection of
  * the intermediate results by tests:
- *   fwd: [0] status word, [1] q~ bf16 [P][H][Tt][D], [2] k~ bf16 [P][Hkv][Tt][D];
+ *   fwd: [0] status word (bytes 0-3; bytes 4-7: the "dq~ accumulator zeroed" mark),
+ *        [1] q~ bf16 [P][H][Tt][D], [2] k~ bf16 [P][Hkv][Tt][D];
  *   bwd: [0] status, [1] q~, [2] k~, [3] row statistics fp32: for query head (p, h)
  *        and the 64-row query tile j of sequence n, 128 floats at slot
  *        start_n/64 + n + j of row p*H + h (-lse * log2(e) of the 64 rows, then their

@@ -298,6 +298,45 @@ def test_backward_reusing_forward_rotation(name):
 
 
 @needs_cuda
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_forward_zeroes_backward_accumulator(name):
+    """A forward given a backward-sized workspace zeroes the dq~ accumulator there and
+    sets the mark after the status word; the backward that reuses the workspace skips
+    its own zeroing and clears the mark, so a second backward on the same workspace
+    zeroes again: same dk/dv bit for bit and the same dq up to the order of the fp32
+    additions.  A forward-sized workspace gets no mark."""
+    from attention_pass_rope_b200 import ops, ttt_attn_bwd, ttt_attn_fwd
+    w = ttt_inputs.workloads()["tiny"] if name == "tiny" else \
+        ttt_inputs.thd("ragged", [300, 128, 17, 1], 4, 8, 2, 128, 1e4)
+    inp = ttt_inputs.make_inputs(w)
+    q, k, v, do, cu = parity.gpu_shapes(w, inp)
+    kw = dict(theta=w.theta, cu_seqlens=cu, max_seqlen=None if w.dense else w.max_seqlen)
+    lay = ops._layout(q, k, v, cu, kw["max_seqlen"])
+    mark = lambda ws: int(ws[4:8].view(torch.int32).item())  # noqa: E731
+    ws = ops.alloc_workspace(ops.workspace_bytes(lay, w.theta, for_backward=True), q.device)
+    ws.fill_(0xAB)  # the accumulator starts as garbage
+    o, lse = ttt_attn_fwd(q, k, v, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    assert mark(ws) == 0x01010101
+    g1 = ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, rotated_in_workspace=True, **kw)
+    torch.cuda.synchronize()
+    assert mark(ws) == 0
+    g2 = ttt_attn_bwd(q, k, v, o, lse, do, workspace=ws, rotated_in_workspace=True, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+    rel = float((g1[0].float() - g2[0].float()).norm() / g1[0].float().norm())
+    assert rel < 1e-3, rel
+    m = parity.compare_full(w, inp, {"o": parity.flat(o, w), "lse": lse, "dq": parity.flat(g1[0], w),
+                                     "dk": parity.flat(g1[1], w), "dv": parity.flat(g1[2], w)})
+    parity.assert_within(m)
+    wsf = ops.alloc_workspace(ops.workspace_bytes(lay, w.theta, for_backward=False), q.device)
+    wsf.fill_(0xAB)
+    ttt_attn_fwd(q, k, v, workspace=wsf, **kw)
+    torch.cuda.synchronize()
+    assert mark(wsf) == 0
+
+
+@needs_cuda
 @pytest.mark.parametrize("keep_rotated", [False, True])
 def test_autograd_function(keep_rotated):
     """ttt_attention under torch.autograd (both settings of keep_rotated) against the oracle."""
