@@ -176,22 +176,24 @@ __global__ void __launch_bounds__(kPreThreads)
 }
 
 // ---------------------------------------------------------------------------
-// a7 + a8: branch backward and finalisation.  One warp per (token, KV head) item:
-//   for every pass p and group head h:
+// a7 + a8: branch backward and finalisation.  One warp per token at a time, for each of
+// its KV heads and every pass p and group head h:
 //     dq~ = dq_acc (trunk part) + sum_j dS_j k~_j        (j = passes 1..p, 0-based)
 //     dS_j = P_j (dO . V_j - delta),  P_j = exp(sigma q~ . k~_j - lse)
 //     dk~_j += dS_j q~,  dV_j += P_j dO                   (accumulated over p >= j, h)
 //     dQ_p = R(i+p)^T (sigma dq~)
 //   dK_j = R(i+j)^T (sigma dk~_j) and dV_j for the branch passes j >= 1 (dK_1 and dV_1
 //   are written by the trunk backward).
-// The kernel is bound by memory latency, so what counts is the bytes each warp keeps in
-// flight.  A warp works through (item, pass) units -- the unit's dq~ rows, q~ rows, dO
-// rows, lse and delta of the group's heads and the branch keys / values it needs -- and
+// A warp works through (KV head, pass) units -- the unit's dq~ rows, q~ rows, dO rows,
+// lse and delta of the group's heads and the branch keys / values it needs -- and
 // fetches the next unit into the other half of a two-stage shared-memory buffer with
-// cp.async while it computes the current one (no registers hold data in flight).  Each
-// warp takes items w, w + W, ... (W = warps in the grid) so that neighbouring warps read
-// neighbouring rows.  Shared memory: the block's inverse frequencies (double), then per
-// warp the cos/sin of positions i..i+P-1, the branch-pass accumulators and the stages.
+// cp.async while it computes the current one (no registers hold data in flight).  The
+// cos / sin of the token's positions i..i+P-1 are formed once and serve all its KV
+// heads.  Each warp takes tokens w, w + W, ... (W = warps in the grid).  The kernel is
+// bound by instruction issue (ncu: issue slots ~64 % busy with 4 warps per scheduler),
+// then by memory latency.  Shared memory: the block's inverse frequencies (double),
+// then per warp the cos/sin of positions i..i+P-1, the branch-pass accumulators and the
+// stages.
 // ---------------------------------------------------------------------------
 struct BranchLayout {
   int cs, acc, stage, dqa, q, o, kj, vj, lse, dl, stage_bytes, warp_bytes;
@@ -216,7 +218,7 @@ __host__ __device__ inline BranchLayout branch_layout(int D, int gsz, int P) {
   return L;
 }
 
-constexpr int kBranchItemsPerWarp = 8;
+constexpr int kBranchTokensPerWarp = 1;
 constexpr int kBranchFreqBytes = 512;  // inverse frequencies (double [D/2]), padded
 
 template <int D>
@@ -244,14 +246,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   float* acc = reinterpret_cast<float*>(wsm + Lo.acc);
   auto stage = [&](int st) { return wsm + Lo.stage + st * Lo.stage_bytes; };
   const int T = g.si.T;
-  const int64_t nitems = static_cast<int64_t>(T) * g.Hkv;
   const int64_t W = static_cast<int64_t>(gridDim.x) * warps_per_block;
   const int64_t dl_base = static_cast<int64_t>(ld_slots(g.si)) * 128;
 
-  // queue the copies of unit (item, p) into stage st (one commit group per unit)
-  auto issue = [&](int64_t item, int p, int st) {
-    const int tau = static_cast<int>(item / g.Hkv);
-    const int kvh = static_cast<int>(item % g.Hkv);
+  // queue the copies of unit (token tau, KV head kvh, pass p) into stage st (one commit
+  // group per unit)
+  auto issue = [&](int tau, int kvh, int p, int st) {
     unsigned char* sb = stage(st);
     constexpr int RC32 = D / 4;  // 16-byte chunks of an fp32 row
     constexpr int RC16 = D / 8;  // 16-byte chunks of a bf16 row
@@ -286,40 +286,49 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     cp_async_commit();
   };
 
-  int64_t item = static_cast<int64_t>(blockIdx.x) * warps_per_block + wib;
-  if (item >= nitems) return;
+  // one token per warp at a time, all its KV heads and passes: the token's cos / sin
+  // serve all of them
+  int tau = static_cast<int>(static_cast<int64_t>(blockIdx.x) * warps_per_block + wib);
+  if (tau >= T) return;
   int st = 0;
-  issue(item, 0, 0);
+  issue(tau, 0, 0, 0);
   while (true) {
-    const int tau = static_cast<int>(item / g.Hkv);
-    const int kvh = static_cast<int>(item % g.Hkv);
     int n, pos;
     token_position(g.si, tau, n, pos);
-    // cos / sin of this token's positions, zeroed branch accumulators
+    // cos / sin of this token's positions
     for (int p = 0; p < g.P; ++p)
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const int d = LaneMap<D>::d(lane, 0, e);
         angle_cos_sin(pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
       }
-    for (int j = 0; j < NB; ++j)
+    const int64_t next_tau = tau + W;
+    for (int kvh = 0; kvh < g.Hkv; ++kvh) {
+      // zeroed branch accumulators of this KV head
+      for (int j = 0; j < NB; ++j)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
+        for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-          acc[(j * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
-          acc[(j * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
+          for (int e = 0; e < E; ++e) {
+            acc[(j * 2 + 0) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
+            acc[(j * 2 + 1) * D + LaneMap<D>::d(lane, hh, e)] = 0.f;
+          }
+      for (int p = 0; p < g.P; ++p) {
+        // fetch the next unit while this one is computed
+        int nt = tau, nk = kvh, np = p + 1;
+        if (np == g.P) {
+          np = 0;
+          if (++nk == g.Hkv) {
+            nk = 0;
+            nt = next_tau < T ? static_cast<int>(next_tau) : -1;
+          }
         }
-    const int64_t next_item = item + W;
-    for (int p = 0; p < g.P; ++p) {
-      // fetch the next unit while this one is computed
-      const bool more = p + 1 < g.P || next_item < nitems;
-      if (more) {
-        issue(p + 1 < g.P ? item : next_item, p + 1 < g.P ? p + 1 : 0, st ^ 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
+        if (nt >= 0) {
+          issue(nt, nk, np, st ^ 1);
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
+        }
       __syncwarp();
       const unsigned char* sb = stage(st);
       const float* sdqa = reinterpret_cast<const float*>(sb + Lo.dqa);
@@ -405,9 +414,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       store_bf16_row<D>(dk + krow, lane, kx);
       store_bf16_row<D>(dv + krow, lane, vx);
     }
-    __syncwarp();  // cos / sin and the accumulators are rewritten for the next item
-    item = next_item;
-    if (item >= nitems) break;
+    __syncwarp();  // the accumulators are rewritten for the next KV head
+    }
+    __syncwarp();  // cos / sin are rewritten for the next token
+    if (next_tau >= T) break;
+    tau = static_cast<int>(next_tau);
   }
 }
 
@@ -453,14 +464,14 @@ cudaError_t launch_bwd_preprocess(const Geometry& g, const void* o, const void* 
 cudaError_t launch_branch_bwd(const Geometry& g, const void* qr, const void* kr, const void* v, const void* dout,
                               const float* lse, const float* ld, const float* dq_acc, void* dq, void* dk, void* dv,
                               cudaStream_t stream) {
-  const int64_t items = static_cast<int64_t>(g.si.T) * g.Hkv;
+  const int64_t items = g.si.T;  // tokens
   if (items == 0) return cudaSuccess;
   const BranchLayout Lo = branch_layout(g.D, g.H / g.Hkv, g.P);
   // as many warps per block as 227 KB of shared memory holds (at most kWarpsPerBlock)
   const int wpb = static_cast<int>(std::min<int64_t>(kWarpsPerBlock, (227 * 1024 - kBranchFreqBytes) / Lo.warp_bytes));
   if (wpb < 1) return cudaErrorInvalidConfiguration;
   const size_t smem = kBranchFreqBytes + static_cast<size_t>(wpb) * Lo.warp_bytes;
-  const int64_t per_block = static_cast<int64_t>(wpb) * kBranchItemsPerWarp;
+  const int64_t per_block = static_cast<int64_t>(wpb) * kBranchTokensPerWarp;
   const int64_t blocks = (items + per_block - 1) / per_block;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   auto* qb = static_cast<const __nv_bfloat16*>(qr);
