@@ -344,6 +344,77 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         c[e] = cs[p * D + LaneMap<D>::d(lane, 0, e)];
         sn[e] = cs[p * D + D / 2 + LaneMap<D>::d(lane, 0, e)];
       }
+      if (p > 0 && p <= 2) {
+        // up to two branch keys (P <= 3): their k~ / V rows are read once for the group's
+        // heads, and the heads' dk~ / dV contributions are summed in registers before
+        // they join the accumulators
+        float kjr[2][2][E], vjr[2][2][E], akr[2][2][E], avr[2][2][E];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          if (jj < p) {
+            load_bf16_row<D>(skj + jj * D, lane, kjr[jj]);
+            load_bf16_row<D>(svj + jj * D, lane, vjr[jj]);
+          }
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int e = 0; e < E; ++e) akr[jj][x][e] = avr[jj][x][e] = 0.f;
+        }
+        for (int hh = 0; hh < gsz; ++hh) {
+          float dqv[2][E], q[2][E], dO[2][E];
+          load_f32_row<D>(sdqa + hh * D, lane, dqv);
+          load_bf16_row<D>(sq + hh * D, lane, q);
+          load_bf16_row<D>(so + hh * D, lane, dO);
+          const float lse_v = slse[hh], dl = sdl[hh];
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            if (jj >= p) continue;
+            float sdot = 0.f, tdot = 0.f;
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+              for (int e = 0; e < E; ++e) {
+                sdot = fmaf(q[x][e], kjr[jj][x][e], sdot);
+                tdot = fmaf(dO[x][e], vjr[jj][x][e], tdot);
+              }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+              tdot += __shfl_xor_sync(0xffffffffu, tdot, o);
+            }
+            const float pj = __expf(sdot * g.scale - lse_v);
+            const float dsj = pj * (tdot - dl);
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+              for (int e = 0; e < E; ++e) {
+                dqv[x][e] = fmaf(dsj, kjr[jj][x][e], dqv[x][e]);
+                akr[jj][x][e] = fmaf(dsj, q[x][e], akr[jj][x][e]);
+                avr[jj][x][e] = fmaf(pj, dO[x][e], avr[jj][x][e]);
+              }
+          }
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int e = 0; e < E; ++e) dqv[x][e] *= g.scale;
+          rotate_back<D>(dqv, c, sn);
+          store_bf16_row<D>(dq + p * g.sq + (static_cast<int64_t>(tau) * g.H + kvh * gsz + hh) * D, lane, dqv);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          if (jj >= p) continue;
+          float* akp = acc + (jj * 2 + 0) * D;
+          float* avp = acc + (jj * 2 + 1) * D;
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              const int d = LaneMap<D>::d(lane, x, e);
+              akp[d] += akr[jj][x][e];
+              avp[d] += avr[jj][x][e];
+            }
+        }
+      } else
       for (int hh = 0; hh < gsz; ++hh) {
         float dqv[2][E], q[2][E], dO[2][E];
         load_f32_row<D>(sdqa + hh * D, lane, dqv);
