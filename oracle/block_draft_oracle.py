@@ -24,6 +24,11 @@ The page gives the pattern in one line.  Readings where it is silent:
 * RoPE is rotate-half at the token's position (trunk key t at t, block token j
   at a+j), the same frequencies as the TTT attention; the softmax scale is
   1/sqrt(D) unless given; query head h reads KV head h // (H // Hkv).
+* Sliding-window block layers (item 4 of the same list names them) see only the
+  last ``window`` context positions of their trunk: t in [max(0, a - window + 1), a].
+  The page names the layers and nothing more; the window reading here is the plainest
+  one that keeps the anchor as the trunk's end.  ``window=None`` (or 0) is the full
+  trunk 0..a.
 * ``rope_round="bf16"`` rounds the rotated queries and keys to bf16 (round to
   nearest even) before the dot products, the library's defined semantics for
   this attention as for the TTT attention (bf16 operands into the tensor cores);
@@ -72,19 +77,26 @@ def _rotate(k_ctx, anchors, qb, kb, theta, pos_offset=0, rope_round=None):
     return kt, qr, kr
 
 
-def block_mask(L, anchors, Bs):
-    """[nb*Bs, L + nb*Bs] visibility: block query (b, j) sees trunk t <= anchor_b and the
-    Bs keys of block b."""
+def trunk_start(a, window):
+    """First trunk key of a block anchored at a: 0, or a - window + 1 (at least 0) for a
+    sliding-window layer."""
+    return 0 if not window else max(0, a - int(window) + 1)
+
+
+def block_mask(L, anchors, Bs, window=None):
+    """[nb*Bs, L + nb*Bs] visibility: block query (b, j) sees trunk t in
+    [trunk_start(anchor_b), anchor_b] and the Bs keys of block b."""
     nb = len(anchors)
     m = np.zeros((nb * Bs, L + nb * Bs), dtype=bool)
     for b, a in enumerate(anchors):
         rows = slice(b * Bs, (b + 1) * Bs)
-        m[rows, : a + 1] = True
+        m[rows, trunk_start(a, window): a + 1] = True
         m[rows, L + b * Bs: L + (b + 1) * Bs] = True
     return m
 
 
-def forward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_offset=0, rope_round=None):
+def forward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_offset=0, rope_round=None,
+                       window=None):
     L, Hkv, D = k_ctx.shape
     nb, Bs, H, _ = qb.shape
     g = H // Hkv
@@ -93,7 +105,7 @@ def forward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos
     K = np.concatenate([kt, kr.reshape(nb * Bs, Hkv, D)])      # [L + nb*Bs, Hkv, D]
     V = np.concatenate([v_ctx, vb.reshape(nb * Bs, Hkv, D)])
     Q = qr.reshape(nb * Bs, H, D)
-    m = block_mask(L, anchors, Bs)
+    m = block_mask(L, anchors, Bs, window)
     O = np.zeros((nb * Bs, H, D))
     lse = np.zeros((H, nb * Bs))
     for h in range(H):
@@ -108,7 +120,7 @@ def forward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos
 
 
 def backward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, do, theta, scale=None, pos_offset=0,
-                        rope_round=None):
+                        rope_round=None, window=None):
     """Gradients with respect to the pre-RoPE inputs: (dqb, dk_ctx, dv_ctx, dkb, dvb)."""
     L, Hkv, D = k_ctx.shape
     nb, Bs, H, _ = qb.shape
@@ -119,7 +131,7 @@ def backward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, do, theta, scale=None
     V = np.concatenate([v_ctx, vb.reshape(nb * Bs, Hkv, D)])
     Q = qr.reshape(nb * Bs, H, D)
     dO = do.reshape(nb * Bs, H, D)
-    m = block_mask(L, anchors, Bs)
+    m = block_mask(L, anchors, Bs, window)
     dQ = np.zeros_like(Q)
     dK = np.zeros_like(K)
     dV = np.zeros_like(V)
@@ -142,8 +154,9 @@ def backward_bruteforce(k_ctx, v_ctx, anchors, qb, kb, vb, do, theta, scale=None
 
 
 def forward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_offset=0, return_parts=False,
-                    rope_round=None):
-    """Per block: trunk softmax over t <= anchor, block softmax over its Bs keys, merged."""
+                    rope_round=None, window=None):
+    """Per block: trunk softmax over its trunk keys (t <= anchor, from trunk_start), block
+    softmax over its Bs keys, merged."""
     L, Hkv, D = k_ctx.shape
     nb, Bs, H, _ = qb.shape
     g = H // Hkv
@@ -153,13 +166,14 @@ def forward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_of
     lse = np.zeros((nb, H, Bs))
     parts = []
     for b, a in enumerate(anchors):
+        t0 = trunk_start(a, window)
         for h in range(H):
             kv = h // g
-            St = sc * (qr[b, :, h] @ kt[: a + 1, kv].T)        # [Bs, a+1]
+            St = sc * (qr[b, :, h] @ kt[t0: a + 1, kv].T)      # [Bs, a+1-t0]
             mt = St.max(axis=1, keepdims=True)
             Et = np.exp(St - mt)
             lt = mt[:, 0] + np.log(Et.sum(axis=1))
-            Ot = (Et @ v_ctx[: a + 1, kv]) / Et.sum(axis=1, keepdims=True)
+            Ot = (Et @ v_ctx[t0: a + 1, kv]) / Et.sum(axis=1, keepdims=True)
             Sb = sc * (qr[b, :, h] @ kr[b, :, kv].T)           # [Bs, Bs], bidirectional
             mb = Sb.max(axis=1, keepdims=True)
             Eb = np.exp(Sb - mb)
@@ -173,7 +187,7 @@ def forward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, theta, scale=None, pos_of
 
 
 def backward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, do, O, lse, theta, scale=None, pos_offset=0,
-                     rope_round=None):
+                     rope_round=None, window=None):
     """Gradients from the merged lse: P = exp(s - lse) for both parts,
     delta = rowsum(dO * O), dS = P (dP - delta)."""
     L, Hkv, D = k_ctx.shape
@@ -187,17 +201,18 @@ def backward_twopart(k_ctx, v_ctx, anchors, qb, kb, vb, do, O, lse, theta, scale
     dkr = np.zeros_like(kr)
     dvb = np.zeros_like(vb)
     for b, a in enumerate(anchors):
+        t0 = trunk_start(a, window)
         for h in range(H):
             kv = h // g
             l = lse[b, h][:, None]
             delta = np.sum(do[b, :, h] * O[b, :, h], axis=1, keepdims=True)
-            Pt = np.exp(sc * (qr[b, :, h] @ kt[: a + 1, kv].T) - l)
-            dSt = Pt * (do[b, :, h] @ v_ctx[: a + 1, kv].T - delta)
+            Pt = np.exp(sc * (qr[b, :, h] @ kt[t0: a + 1, kv].T) - l)
+            dSt = Pt * (do[b, :, h] @ v_ctx[t0: a + 1, kv].T - delta)
             Pb = np.exp(sc * (qr[b, :, h] @ kr[b, :, kv].T) - l)
             dSb = Pb * (do[b, :, h] @ vb[b, :, kv].T - delta)
-            dqr[b, :, h] = sc * (dSt @ kt[: a + 1, kv] + dSb @ kr[b, :, kv])
-            dkt[: a + 1, kv] += sc * dSt.T @ qr[b, :, h]
-            dvt[: a + 1, kv] += Pt.T @ do[b, :, h]
+            dqr[b, :, h] = sc * (dSt @ kt[t0: a + 1, kv] + dSb @ kr[b, :, kv])
+            dkt[t0: a + 1, kv] += sc * dSt.T @ qr[b, :, h]
+            dvt[t0: a + 1, kv] += Pt.T @ do[b, :, h]
             dkr[b, :, kv] += sc * dSb.T @ qr[b, :, h]
             dvb[b, :, kv] += Pb.T @ do[b, :, h]
     pos_b = (np.asarray(anchors)[:, None] + np.arange(Bs)[None, :] + pos_offset).reshape(-1)

@@ -188,3 +188,85 @@ def test_oracle_matches_its_fixture():
     assert set(ref) == set(got)
     for name in ref:
         np.testing.assert_allclose(got[name], ref[name], rtol=0, atol=1e-13, err_msg=name)
+
+
+# ----------------------------------------------------------------------------- sliding-window trunk
+@pytest.mark.parametrize("window", [1, 3, 6])
+def test_window_equals_masked_sdpa(window):
+    """A sliding-window layer is one masked softmax too: torch SDPA (fp64) with the trunk
+    part of the mask written out here as a - window < t <= a, outputs and autograd
+    gradients against both oracle forms."""
+    L, Bs, H, Hkv, D, theta = 11, 3, 4, 2, 8, 1e4
+    anchors = [0, 2, 7, 10]
+    c = case(L=L, Bs=Bs, H=H, Hkv=Hkv, D=D, anchors=anchors)
+    nb = len(anchors)
+    O, lse = bd.forward_twopart(theta=theta, window=window, **c)
+    Ob, lb = bd.forward_bruteforce(theta=theta, window=window, **c)
+    np.testing.assert_allclose(Ob, O, atol=1e-13)
+    np.testing.assert_allclose(lb, lse, atol=1e-13)
+    do = rnd(*O.shape)
+    grads = bd.backward_twopart(theta=theta, do=do, O=O, lse=lse, window=window, **c)
+    grads_b = bd.backward_bruteforce(theta=theta, do=do, window=window, **c)
+    t = {n: torch.tensor(c[n], requires_grad=True) for n in ("k_ctx", "v_ctx", "qb", "kb", "vb")}
+    pos_b = [a + j for a in anchors for j in range(Bs)]
+    q = torch_rope(t["qb"].reshape(nb * Bs, H, D), pos_b, theta)
+    k = torch.cat([torch_rope(t["k_ctx"], list(range(L)), theta),
+                   torch_rope(t["kb"].reshape(nb * Bs, Hkv, D), pos_b, theta)])
+    v = torch.cat([t["v_ctx"], t["vb"].reshape(nb * Bs, Hkv, D)])
+    mask = torch.zeros(nb * Bs, L + nb * Bs, dtype=torch.bool)
+    for b, a in enumerate(anchors):
+        for j in range(Bs):
+            for tt in range(L):
+                mask[b * Bs + j, tt] = a - window < tt <= a
+            mask[b * Bs + j, L + b * Bs: L + (b + 1) * Bs] = True
+    g = H // Hkv
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q.transpose(0, 1)[None], k.transpose(0, 1).repeat_interleave(g, 0)[None],
+        v.transpose(0, 1).repeat_interleave(g, 0)[None], attn_mask=mask)[0].transpose(0, 1)
+    np.testing.assert_allclose(O.reshape(nb * Bs, H, D), out.detach().numpy(), atol=1e-12)
+    (out * torch.tensor(do.reshape(nb * Bs, H, D))).sum().backward()
+    for got, got_b, name in zip(grads, grads_b, ("qb", "k_ctx", "v_ctx", "kb", "vb")):
+        np.testing.assert_allclose(got, t[name].grad.numpy(), atol=1e-11, err_msg=name)
+        np.testing.assert_allclose(got_b, t[name].grad.numpy(), atol=1e-11, err_msg=name)
+
+
+def test_window_covering_the_trunk_is_the_full_layer():
+    """A window of at least anchor + 1 keys changes nothing (bit for bit), and so does 0."""
+    c = case(L=9, anchors=[0, 4, 8], Bs=2)
+    O, lse = bd.forward_twopart(theta=1e4, **c)
+    for w in (0, 9, 50):
+        O2, l2 = bd.forward_twopart(theta=1e4, window=w, **c)
+        np.testing.assert_array_equal(O2, O)
+        np.testing.assert_array_equal(l2, lse)
+
+
+def test_window_uniform_scores_closed_form():
+    """q = 0: O is the mean of the min(window, a + 1) trunk values in the window and the
+    Bs block values, lse the log of their count."""
+    c = case(L=12, anchors=[1, 5, 11], Bs=2, H=2, Hkv=1)
+    c["qb"] = np.zeros_like(c["qb"])
+    w = 4
+    O, lse = bd.forward_twopart(theta=1e4, window=w, **c)
+    for b, a in enumerate(c["anchors"]):
+        t0 = max(0, a - w + 1)
+        vis = np.concatenate([c["v_ctx"][t0: a + 1, 0], c["vb"][b, :, 0]])
+        for j in range(2):
+            for h in range(2):
+                np.testing.assert_allclose(O[b, j, h], vis.mean(axis=0), atol=1e-14)
+                assert abs(lse[b, h, j] - np.log(a + 1 - t0 + 2)) < 1e-14
+
+
+def test_window_one_sees_the_anchor_key_only():
+    """window = 1: the trunk part is the anchor's key alone, so its lse is that one score
+    and keys before the anchor do not matter."""
+    c = case(L=10, anchors=[3, 9], Bs=2, H=2, Hkv=1, D=8)
+    O, lse, parts = bd.forward_twopart(theta=1e4, window=1, return_parts=True, **c)
+    kt, qr, _ = bd._rotate(c["k_ctx"], c["anchors"], c["qb"], c["kb"], 1e4)
+    sc = 1.0 / np.sqrt(8)
+    for b, h, lt, _ in parts:
+        a = c["anchors"][b]
+        np.testing.assert_allclose(lt, sc * qr[b, :, h] @ kt[a, h // 2], atol=1e-13)
+    before = dict(c, k_ctx=c["k_ctx"].copy(), v_ctx=c["v_ctx"].copy())
+    before["k_ctx"][:3] += 5.0
+    before["v_ctx"][4:9] -= 2.0
+    np.testing.assert_array_equal(bd.forward_twopart(theta=1e4, window=1, **before)[0], O)
