@@ -72,6 +72,7 @@ class TTTBlockDesc(ctypes.Structure):
         ("max_blocks", ctypes.c_int),
         ("events", ctypes.c_void_p),
         ("flags", ctypes.c_int),
+        ("window", ctypes.c_int),
     ]
 
 

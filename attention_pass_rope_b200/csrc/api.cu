@@ -128,6 +128,7 @@ ttt_status make_block_plan(const ttt_block_desc* d, int for_backward, Plan* out)
   if (d->H < 1 || d->Hkv < 1 || d->D < 1 || d->Bs < 1) return TTT_ERR_INVALID_ARG;
   if (d->H % d->Hkv != 0) return TTT_ERR_INVALID_ARG;
   if (d->Bs > 16) return TTT_ERR_UNSUPPORTED;
+  if (d->window < 0) return TTT_ERR_INVALID_ARG;
   if (d->D != 64 && d->D != 128) return TTT_ERR_UNSUPPORTED;
   if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return TTT_ERR_INVALID_ARG;
   if (!(d->softmax_scale >= 0.f) || !std::isfinite(d->softmax_scale)) return TTT_ERR_INVALID_ARG;
@@ -141,6 +142,7 @@ ttt_status make_block_plan(const ttt_block_desc* d, int for_backward, Plan* out)
   g.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt(static_cast<float>(d->D));
   g.Bs = d->Bs;
   g.anchors = d->anchors;
+  g.window = d->window;
   g.ring = 0;
   g.limit_off = 0;
   g.pos0 = 0;

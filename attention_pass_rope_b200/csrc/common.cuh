@@ -608,6 +608,12 @@ __device__ __forceinline__ int block_row_limit(const Geometry& g, int qstart, in
   return min(max(a, 0), klen - 1);
 }
 
+// First trunk key of a block-draft row whose last trunk key is lim: 0, or for a
+// sliding-window layer lim - window + 1 (at least 0).
+__device__ __forceinline__ int block_row_start(const Geometry& g, int lim) {
+  return g.window > 0 ? max(0, lim - g.window + 1) : 0;
+}
+
 // RoPE position of that row: the clamped anchor (0 for an empty context) plus the
 // row's index in its block.
 __device__ __forceinline__ int block_row_position(const Geometry& g, int qstart, int r, int klen) {

@@ -103,6 +103,21 @@ __device__ int first_tile_seeing(const Geometry& g, const int* qlim, int qstart,
   return lo;
 }
 
+// Last 64-row query tile of a block-draft sequence whose first row still sees a key of
+// [k0, k1] (for a sliding-window layer the first key of a row is block_row_start of its
+// limit, non-decreasing too, so the tiles that see the key tile are a range).
+__device__ int last_tile_seeing(const Geometry& g, const int* qlim, int qstart, int qlen, int k1) {
+  int lo = -1, hi = (qlen + 63) / 64 - 1;  // answer in [lo, hi]; -1 = no tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (block_row_start(g, __ldg(qlim + qstart + mid * 64)) <= k1)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
 // dK of the trunk keys, finalised: sigma * R(pos)^T dk~ in bf16, for one key row held
 // by the calling thread as 32-column chunks (c, c + D/2 pair the RoPE dimensions).
 template <int D>
@@ -177,7 +192,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int gsz = g.H / g.Hkv;
   const int G = g.P * gsz;
   const int jq0 = MODE == 0 ? k0 / C::BQ : first_tile_seeing(g, a.qlim, seq_start, len, k0);
-  const int nqt = (len + C::BQ - 1) / C::BQ - jq0;
+  const int jq1 = MODE == 1 && g.window > 0 ? last_tile_seeing(g, a.qlim, seq_start, len, k0 + C::BK - 1)
+                                            : (len + C::BQ - 1) / C::BQ - 1;
+  const int nqt = max(jq1 - jq0 + 1, 0);
   const int NIT = G * nqt;
   if (threadIdx.x == 0) TTT_CTA_INFO(NIT);
   if (NIT <= 0) {
@@ -419,7 +436,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int qlo = ii.q0 + 32 * hf;
       const bool interior =
           (qlo + 32 <= len) && (k0 + C::BK <= klen) &&
-          (MODE == 0 ? qlo >= k0 + C::BK - 1 : __ldg(a.qlim + seq_start + qlo) >= k0 + C::BK - 1);
+          (MODE == 0 ? qlo >= k0 + C::BK - 1
+                     : __ldg(a.qlim + seq_start + qlo) >= k0 + C::BK - 1 &&
+                           block_row_start(g, __ldg(a.qlim + seq_start + qlo + 31)) <= k0);
       // P = 2^(s*scale*log2e - lse*log2e), dS = P (dP - delta), two columns per
       // instruction; the bf16 pairs are packed straight from the results
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -443,13 +462,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
           if (!interior) {
             // padding rows of the statistics are never written: select, do not multiply
-            int lim0 = qlo + c, lim1 = qlo + c + 1;
+            int lim0 = qlo + c, lim1 = qlo + c + 1, st0 = 0, st1 = 0;
             if (MODE == 1) {
               lim0 = qlo + c < len ? __ldg(a.qlim + seq_start + qlo + c) : -1;
               lim1 = qlo + c + 1 < len ? __ldg(a.qlim + seq_start + qlo + c + 1) : -1;
+              st0 = block_row_start(g, lim0);
+              st1 = block_row_start(g, lim1);
             }
-            const bool v0 = kvalid && qlo + c < len && kpos <= lim0;
-            const bool v1 = kvalid && qlo + c + 1 < len && kpos <= lim1;
+            const bool v0 = kvalid && qlo + c < len && kpos <= lim0 && kpos >= st0;
+            const bool v1 = kvalid && qlo + c + 1 < len && kpos <= lim1 && kpos >= st1;
             p0 = v0 ? p0 : 0.f;
             d0 = v0 ? d0 : 0.f;
             p1 = v1 ? p1 : 0.f;

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   uint32_t* abort_flag = tmem_slot + 1;
   int* nkv_slot = reinterpret_cast<int*>(abort_flag + 1);
+  int* jlo_slot = nkv_slot + 1;  // MODE 1: first key tile streamed
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < C::NQ; ++t) mbar_init(q_full + t, 1);
@@ -152,14 +153,26 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
   if (MODE == 1 && warp == 2) {
-    // key tiles to stream: up to the largest anchor among this tile's rows
-    // (none for an empty context: the rows see their block's keys only)
+    // key tiles to stream: up to the largest anchor among this tile's rows, from the
+    // smallest first key (0, or a sliding window's start); none for an empty context
+    // (the rows see their block's keys only).  One row per block suffices.
     const int rows = min(C::BM, len - q0);
-    int mx = -1;
-    for (int r = lane * g.Bs; r < rows; r += 32 * g.Bs) mx = max(mx, block_row_limit(g, seq_start, q0 + r, klen));
+    int mx = -1, mn = 0x7fffffff;
+    for (int r = lane * g.Bs; r < rows; r += 32 * g.Bs) {
+      const int lim = block_row_limit(g, seq_start, q0 + r, klen);
+      mx = max(mx, lim);
+      mn = min(mn, block_row_start(g, lim));
+    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) *nkv_slot = (mx + C::BN) / C::BN;
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    if (lane == 0) {
+      const int jlo = mx < 0 ? 0 : mn / C::BN;
+      *jlo_slot = jlo;
+      *nkv_slot = (mx + C::BN) / C::BN - jlo;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -168,6 +181,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   const int nkv = MODE == 0 ? jq + 1
                   : MODE == 1 ? *nkv_slot
                               : min(q0 + min(C::BM, len - q0) - 1 + g.limit_off, klen - 1) / C::BN + 1;
+  const int jlo = MODE == 1 ? *jlo_slot : 0;  // key tile j of the stream is tile jlo + j
   const Watchdog wd{abort_flag, a.status, a.budget_ns};
   if (threadIdx.x == 0) TTT_CTA_INFO(nkv);
 
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       load_q(0);
       if (nkv == 0 && nq_tiles > 1) load_q(1);
       for (int j = 0; j < nkv; ++j) {
-        const int krow = kstart + j * C::BN;
+        const int krow = kstart + (jlo + j) * C::BN;
         const int ks = j % C::KST;
         if (j >= C::KST && !wait_bounded(k_empty + ks, ((j / C::KST) - 1) & 1, wd, kSiteFwdKvEmpty)) break;
         TTT_TRACE(14, j);
@@ -352,6 +366,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int lim = MODE == 0   ? qpos
                     : MODE == 1 ? (qpos < len ? block_row_limit(g, seq_start, qpos, klen) : 0)
                                 : min(qpos + g.limit_off, klen - 1);
+    const int lo = MODE == 1 ? block_row_start(g, lim) : 0;  // first visible key of this row
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
@@ -369,13 +384,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
-      const int k0 = j * C::BN;
-      if (k0 + C::BN - 1 > lim) {
+      const int k0 = (jlo + j) * C::BN;
+      if (k0 + C::BN - 1 > lim || k0 < lo) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (k0 + 32 * c + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
+            if (k0 + 32 * c + e > lim || k0 + 32 * c + e < lo) sr[c][e] = __float_as_uint(-INFINITY);
       }
       // row max: 8 independent chains of three-input maxima, then a tree
       float mxv[8];
@@ -409,7 +424,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       // the running max grew by more than 2^8); the others release the first 64 keys early
       const bool warp_rescale = __any_sync(0xffffffffu, rescale && j > 0);
       uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // paired row-sum accumulators
-      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_run, -m_run);
+      // a row that has seen no key yet (a sliding window's leading tiles) exponentiates
+      // against 0: its scores are all -inf, so its P is 0
+      const float mneg = m_run == -INFINITY ? 0.f : -m_run;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(mneg, mneg);
       // P = 2^(s*scale*log2e - m), bf16 pairs into the first 64 columns of S_t; the first
       // 64 keys are released to the MMA warp before the last 64 are computed
 #pragma unroll

@@ -49,7 +49,8 @@ struct SeqInfo {
 // of each per batch entry.  For the TTT attention they are the same tokens.  For the
 // block-draft attention (Bs > 0) query row r of sequence n is token r % Bs of block
 // (start_n + r) / Bs, and the keys are the context tokens: the row sees the context
-// keys 0..anchor of its block (qlim) and the Bs keys of its own block.
+// keys 0..anchor of its block (qlim; a sliding-window layer only the last `window` of
+// them) and the Bs keys of its own block.
 struct Geometry {
   SeqInfo si;   // query rows (TTT: tokens; block draft: block rows)
   SeqInfo ksi;  // key rows (TTT: = si; block draft: context tokens)
@@ -60,6 +61,7 @@ struct Geometry {
   int64_t skv;  // elements between passes of the public k, v, dk, dv
   int Bs;                    // block-draft: tokens per block (0: TTT attention)
   const int32_t* anchors;    // block-draft: device int32, anchor position of every block
+  int window;                // block-draft: trunk keys a - window + 1 .. a of anchor a (0: all)
   // context-parallel ring step (ring > 0): the queries are one chunk of a sequence, the
   // keys another chunk of the same sequence; query row r sees key row t iff
   // t <= r + limit_off (global positions: limit_off = q_start - kv_start >= 0)

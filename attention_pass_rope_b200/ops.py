@@ -338,7 +338,7 @@ def _block_layout(k_ctx, v_ctx, qb, kb, vb, anchors, cu_ctx, cu_blocks, max_ctx,
 
 
 def make_block_desc(lay: BlockLayout, anchors, theta: float, scale: Optional[float], events=None,
-                    flags: int = 0) -> _lib.TTTBlockDesc:
+                    flags: int = 0, window: int = 0) -> _lib.TTTBlockDesc:
     d = _lib.TTTBlockDesc()
     d.layout = _lib.TTT_LAYOUT_BSHD if lay.dense else _lib.TTT_LAYOUT_THD
     d.B, d.S, d.nblk = lay.B, lay.S, lay.nblk
@@ -352,6 +352,7 @@ def make_block_desc(lay: BlockLayout, anchors, theta: float, scale: Optional[flo
         d.max_ctx, d.max_blocks = lay.max_ctx, lay.max_blocks
     d.events = ctypes.addressof(events) if events is not None else None
     d.flags = int(flags)
+    d.window = int(window or 0)
     return d
 
 
@@ -365,15 +366,16 @@ def block_workspace_bytes(lay: BlockLayout, anchors, theta: float, scale=None, f
 
 def block_attn_fwd(k_ctx, v_ctx, qb, kb, vb, anchors, *, theta: float, scale: Optional[float] = None, cu_ctx=None,
                    cu_blocks=None, max_ctx=None, max_blocks=None, workspace: Optional[torch.Tensor] = None, out=None,
-                   events=None):
-    """Block-draft forward: returns (o, lse)."""
+                   events=None, window: int = 0):
+    """Block-draft forward: returns (o, lse).  ``window`` > 0: a sliding-window layer,
+    each block sees the context keys anchor - window + 1 .. anchor."""
     lay = _block_layout(k_ctx, v_ctx, qb, kb, vb, anchors, cu_ctx, cu_blocks, max_ctx, max_blocks)
     if out is None:
         o = torch.empty_like(qb)
         lse = torch.empty(lay.lse_shape, dtype=torch.float32, device=qb.device)
     else:
         o, lse = out
-    desc = make_block_desc(lay, anchors, theta, scale, events)
+    desc = make_block_desc(lay, anchors, theta, scale, events, window=window)
     L = _lib.lib()
     if workspace is None:
         workspace = alloc_workspace(L.ttt_block_workspace_size(ctypes.byref(desc), 0), qb.device)
@@ -386,9 +388,9 @@ def block_attn_fwd(k_ctx, v_ctx, qb, kb, vb, anchors, *, theta: float, scale: Op
 def block_attn_bwd(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse, dout, *, theta: float, scale: Optional[float] = None,
                    cu_ctx=None, cu_blocks=None, max_ctx=None, max_blocks=None,
                    workspace: Optional[torch.Tensor] = None, out=None, events=None, rotated_in_workspace=False,
-                   deterministic=False):
+                   deterministic=False, window: int = 0):
     """Block-draft backward: returns (dk_ctx, dv_ctx, dqb, dkb, dvb) with respect to the
-    pre-RoPE inputs."""
+    pre-RoPE inputs (``window`` as in block_attn_fwd)."""
     if rotated_in_workspace and workspace is None:
         raise ValueError("rotated_in_workspace needs the forward's workspace")
     lay = _block_layout(k_ctx, v_ctx, qb, kb, vb, anchors, cu_ctx, cu_blocks, max_ctx, max_blocks)
@@ -401,7 +403,7 @@ def block_attn_bwd(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse, dout, *, theta: fl
         out = tuple(torch.empty_like(t) for t in (k_ctx, v_ctx, qb, kb, vb))
     flags = (_lib.TTT_FLAG_ROTATED_IN_WORKSPACE if rotated_in_workspace else 0) | \
         (_lib.TTT_FLAG_DETERMINISTIC_DQ if deterministic else 0)
-    desc = make_block_desc(lay, anchors, theta, scale, events, flags)
+    desc = make_block_desc(lay, anchors, theta, scale, events, flags, window)
     L = _lib.lib()
     if workspace is None:
         workspace = alloc_workspace(L.ttt_block_workspace_size(ctypes.byref(desc), 1), qb.device)
@@ -415,12 +417,12 @@ def block_attn_bwd(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse, dout, *, theta: fl
 
 class _BlockAttention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, k_ctx, v_ctx, qb, kb, vb, anchors, theta, scale, cu_ctx, cu_blocks, max_ctx, max_blocks):
+    def forward(ctx, k_ctx, v_ctx, qb, kb, vb, anchors, theta, scale, cu_ctx, cu_blocks, max_ctx, max_blocks, window):
         o, lse = block_attn_fwd(k_ctx, v_ctx, qb, kb, vb, anchors, theta=theta, scale=scale, cu_ctx=cu_ctx,
-                                cu_blocks=cu_blocks, max_ctx=max_ctx, max_blocks=max_blocks)
+                                cu_blocks=cu_blocks, max_ctx=max_ctx, max_blocks=max_blocks, window=window)
         ctx.save_for_backward(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse,
                               *(t for t in (cu_ctx, cu_blocks) if t is not None))
-        ctx.kw = dict(theta=theta, scale=scale, max_ctx=max_ctx, max_blocks=max_blocks)
+        ctx.kw = dict(theta=theta, scale=scale, max_ctx=max_ctx, max_blocks=max_blocks, window=window)
         ctx.packed = cu_ctx is not None
         return o
 
@@ -430,11 +432,11 @@ class _BlockAttention(torch.autograd.Function):
         k_ctx, v_ctx, qb, kb, vb, anchors, o, lse = saved[:8]
         cu = dict(cu_ctx=saved[8], cu_blocks=saved[9]) if ctx.packed else {}
         grads = block_attn_bwd(k_ctx, v_ctx, qb, kb, vb, anchors, o, lse, do.contiguous(), **cu, **ctx.kw)
-        return (*grads, None, None, None, None, None, None, None)
+        return (*grads, None, None, None, None, None, None, None, None)
 
 
 def block_attention(k_ctx, v_ctx, qb, kb, vb, anchors, *, theta: float, scale: Optional[float] = None, cu_ctx=None,
-                    cu_blocks=None, max_ctx=None, max_blocks=None):
+                    cu_blocks=None, max_ctx=None, max_blocks=None, window: int = 0):
     """Differentiable block-draft attention (autograd over the C ABI); returns o."""
     return _BlockAttention.apply(k_ctx, v_ctx, qb, kb, vb, anchors, theta, scale, cu_ctx, cu_blocks, max_ctx,
-                                 max_blocks)
+                                 max_blocks, window)

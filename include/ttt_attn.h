@@ -199,10 +199,11 @@ ttt_status ttt_attn_noalloc_watchdog_selftest(uint64_t budget_ns, void* stream);
  *   A block b of Bs tokens starts at the anchor position a_b of its sequence; its
  *   token j sits at position a_b + j and has its own q, k, v.  With kv(h) = h / (H/Hkv):
  *     q~ = R(a_b + j) q,  k~ = R(a_b + j) k (block tokens),  k~_ctx[t] = R(t) k_ctx[t]
- *     trunk keys: k~_ctx[t], v_ctx[t] for t = 0..a_b            (truncated at the anchor)
+ *     trunk keys: k~_ctx[t], v_ctx[t] for t = s_b..a_b          (truncated at the anchor;
+ *                 s_b = 0, or max(0, a_b - window + 1) for a sliding-window layer)
  *     block keys: k~, v of the Bs tokens of block b             (bidirectional)
  *     lse = logaddexp(lse_trunk, lse_block), O = the exact merge of the two partial
- *     softmaxes, i.e. one softmax over the (a_b + 1) + Bs visible keys.
+ *     softmaxes, i.e. one softmax over the (a_b - s_b + 1) + Bs visible keys.
  *   Rotated q~ / k~ are rounded to bf16 before the dot products, as in the TTT call.
  *
  * Layouts (row-major, contiguous; NB = total blocks, Tc = total context tokens):
@@ -240,6 +241,11 @@ typedef struct {
   const ttt_attn_events* events; /* optional: TTT_KERNEL_ROPE_FWD, _TRUNK_FWD, _ROPE_BWD,
                                     _BWD_PREPROCESS, _TRUNK_BWD, _BRANCH_BWD (block part) */
   int flags;                 /* TTT_FLAG_* bits */
+  /* Sliding-window block layers ("DFlash/DSpark and EAGLE-3 TTT draft co-training",
+   * NeMo-RL issue 3698, "What I'm working on", item 4): a block anchored at a sees only
+   * the context keys a - window + 1 .. a (from 0 when that is negative); 0 = the whole
+   * trunk 0..a.  >= 0. */
+  int window;
 } ttt_block_desc;
 
 /* Workspace bytes of ttt_block_attn_fwd (for_backward = 0) or ttt_block_attn_bwd (1); 0

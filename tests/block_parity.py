@@ -29,7 +29,7 @@ def gpu_tensors(w: ttt_inputs.BlockWorkload, inp: ttt_inputs.BlockInputs, device
     return {n: x.contiguous() for n, x in t.items()}, kw
 
 
-def run_gpu(w, inp, with_grad=True, scale=None, reuse_rotation=False, deterministic=False):
+def run_gpu(w, inp, with_grad=True, scale=None, reuse_rotation=False, deterministic=False, window=0):
     from attention_pass_rope_b200 import ops
     t, kw = gpu_tensors(w, inp)
     args = (t["k_ctx"], t["v_ctx"], t["qb"], t["kb"], t["vb"], t["anchors"])
@@ -39,11 +39,12 @@ def run_gpu(w, inp, with_grad=True, scale=None, reuse_rotation=False, determinis
                                 kw.get("max_blocks"))
         ws = ops.alloc_workspace(ops.block_workspace_bytes(lay, t["anchors"], w.theta, scale, for_backward=True),
                                  t["qb"].device)
-    o, lse = ops.block_attn_fwd(*args, theta=w.theta, scale=scale, workspace=ws, **kw)
+    o, lse = ops.block_attn_fwd(*args, theta=w.theta, scale=scale, workspace=ws, window=window, **kw)
     out = {"o": o.reshape(w.NB, w.Bs, w.H, w.D), "lse": lse}
     if with_grad:
         g = ops.block_attn_bwd(*args, o, lse, t["do"], theta=w.theta, scale=scale, workspace=ws,
-                               rotated_in_workspace=reuse_rotation, deterministic=deterministic, **kw)
+                               rotated_in_workspace=reuse_rotation, deterministic=deterministic, window=window,
+                               **kw)
         out.update(dk_ctx=g[0].reshape(w.Tc, w.Hkv, w.D), dv_ctx=g[1].reshape(w.Tc, w.Hkv, w.D),
                    dqb=g[2].reshape(w.NB, w.Bs, w.H, w.D), dkb=g[3].reshape(w.NB, w.Bs, w.Hkv, w.D),
                    dvb=g[4].reshape(w.NB, w.Bs, w.Hkv, w.D))
@@ -59,7 +60,7 @@ def gpu_lse_rows(w, lse, n, h):
     return lse[h, b0 * w.Bs: b1 * w.Bs]
 
 
-def compare(w, inp, gpu, with_grad=True, kv_heads=None, seqs=None, scale=None):
+def compare(w, inp, gpu, with_grad=True, kv_heads=None, seqs=None, scale=None, window=0):
     """Oracle (rope_round="bf16") per sequence and KV-head group; element-wise metrics."""
     g = w.H // w.Hkv
     kv_heads = range(w.Hkv) if kv_heads is None else kv_heads
@@ -78,14 +79,14 @@ def compare(w, inp, gpu, with_grad=True, kv_heads=None, seqs=None, scale=None):
             ks = slice(kv, kv + 1)
             c = dict(k_ctx=f64(inp.k_ctx[c0:c1, ks]), v_ctx=f64(inp.v_ctx[c0:c1, ks]), anchors=anchors,
                      qb=f64(inp.qb[b0:b1, :, hs]), kb=f64(inp.kb[b0:b1, :, ks]), vb=f64(inp.vb[b0:b1, :, ks]))
-            O, lse = bd.forward_twopart(theta=w.theta, scale=scale, rope_round="bf16", **c)
+            O, lse = bd.forward_twopart(theta=w.theta, scale=scale, rope_round="bf16", window=window, **c)
             o_err = max(o_err, float(np.max(np.abs(to64(gpu["o"][b0:b1, :, hs]) - O))))
             for hh in range(g):
                 got = to64(gpu_lse_rows(w, gpu["lse"], n, kv * g + hh))
                 l_err = max(l_err, float(np.max(np.abs(got - lse[:, hh].reshape(-1)))))
             if with_grad:
                 ref = bd.backward_twopart(do=f64(inp.do[b0:b1, :, hs]), O=O, lse=lse, theta=w.theta, scale=scale,
-                                          rope_round="bf16", **c)
+                                          rope_round="bf16", window=window, **c)
                 got = (gpu["dqb"][b0:b1, :, hs], gpu["dk_ctx"][c0:c1, ks], gpu["dv_ctx"][c0:c1, ks],
                        gpu["dkb"][b0:b1, :, ks], gpu["dvb"][b0:b1, :, ks])
                 for name, r_, g_ in zip(("dqb", "dk_ctx", "dv_ctx", "dkb", "dvb"), ref, got):

@@ -181,3 +181,26 @@ def test_forward_layout_is_a_prefix_of_backward(L, kw):
     assert nf == 3 and nb == 6
     assert list(f[:nf]) == list(b[:nf])
     assert L.ttt_attn_workspace_size(ctypes.byref(d), 1) >= L.ttt_attn_workspace_size(ctypes.byref(d), 0) > 0
+
+
+def block_desc(**kw):
+    d = _lib.TTTBlockDesc()
+    d.layout, d.B, d.S, d.nblk, d.H, d.Hkv, d.D, d.Bs = 0, 2, 4096, 256, 32, 8, 128, 16
+    d.rope_theta, d.softmax_scale = 1e6, 0.0
+    d.anchors = 0x1000  # only checked for NULL by the sizing call, never read on the host
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_block_window_validation(L):
+    """Sliding-window block layers: window >= 0 (0 = the whole trunk) sizes the same
+    workspace; a negative window is rejected before any CUDA call."""
+    L.ttt_block_workspace_size.restype = ctypes.c_size_t
+    L.ttt_block_workspace_size.argtypes = [ctypes.POINTER(_lib.TTTBlockDesc), ctypes.c_int]
+    full = L.ttt_block_workspace_size(ctypes.byref(block_desc()), 1)
+    assert full > 0
+    for w in (1, 1024, 10 ** 6):
+        assert L.ttt_block_workspace_size(ctypes.byref(block_desc(window=w)), 1) == full
+    assert L.ttt_block_workspace_size(ctypes.byref(block_desc(window=-1)), 1) == 0
+    assert ctypes.sizeof(_lib.TTTBlockDesc) % 8 == 0

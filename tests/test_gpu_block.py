@@ -14,10 +14,10 @@ pytestmark = pytest.mark.gpu
 needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 
 
-def _check(w, scale=None, **kw):
+def _check(w, scale=None, window=0, **kw):
     inp = ttt_inputs.make_block_inputs(w)
-    gpu = bp.run_gpu(w, inp, scale=scale)
-    m = bp.compare(w, inp, gpu, scale=scale, **kw)
+    gpu = bp.run_gpu(w, inp, scale=scale, window=window)
+    m = bp.compare(w, inp, gpu, scale=scale, window=window, **kw)
     print(w.name, m)
     bp.assert_within(m)
     return m
@@ -127,3 +127,47 @@ def test_block_unsorted_anchors_reported():
     ops.block_attn_bwd(*args, o, lse, t["do"], theta=w.theta, workspace=ws, **kw)
     st, word = ops.device_status(ws)
     assert st == _lib.TTT_ERR_INVALID_ARG and word == 0x72000001
+
+
+# ----------------------------------------------------------------------------- sliding-window layers
+def _ragged_anchors(ctx, nblk, seed):
+    import random
+    rng = random.Random(seed)
+    anchors = []
+    for L, nb in zip(ctx, nblk):
+        a = sorted([0, L - 1] + [rng.randrange(L) for _ in range(max(nb - 2, 0))])[:nb] if nb else []
+        if nb == 1:
+            a = [L - 1]
+        anchors += a
+    return anchors
+
+
+@needs_cuda
+@pytest.mark.parametrize("window", [1, 50, 129, 1000])
+def test_block_window_ragged_thd(window):
+    """Sliding-window layers on the packed batch of test_block_ragged_thd (Bs = 16,
+    D = 128): a window of 1 (the anchor's key alone), 50 and 129 (trunk ranges that start
+    inside a key tile and cross tile edges), and 1000 (longer than every context: the
+    full layer)."""
+    ctx = [1, 130, 300, 64, 257]
+    nblk = [1, 9, 17, 0, 5]
+    w = ttt_inputs.block_thd(f"block_window{window}", ctx, nblk, 16, 8, 2, 128, 1e4,
+                             anchors=_ragged_anchors(ctx, nblk, 7))
+    _check(w, window=window)
+
+
+@needs_cuda
+@pytest.mark.parametrize("window", [128, 200])
+def test_block_window_dense_edges(window):
+    """Dense, anchors at 0, at the tile edges 127 / 128 and at the last position, with
+    windows of exactly one key tile and of a tile and a half (D = 64, Bs = 5)."""
+    anchors = [0, 0, 127, 128, 255, 299] * 3
+    w = ttt_inputs.block_dense(f"block_window_edges{window}", 3, 300, 6, 5, 4, 4, 64, 1e6, anchors=anchors)
+    _check(w, window=window)
+
+
+@needs_cuda
+def test_block_window_4k_sampled_group():
+    """The 4K block workload as a sliding-window layer of 1024 keys: sequence 0, KV head
+    3 against the oracle."""
+    _check(ttt_inputs.block_workloads()["block_draft_4k"], window=1024, kv_heads=[3], seqs=[0])
