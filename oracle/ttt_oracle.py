@@ -615,3 +615,69 @@ def chunk_partial(qc, kt, vt, theta, q_start, kv_start, branch_k=None, branch_v=
             O[p0, :, h] = out
             lse[p0, h] = np.where(has, m[:, 0] + np.log(np.where(z > 0, z, 1.0)), -np.inf)
     return O, lse
+
+
+def chunk_backward_partial(qc, kt, vt, doc, lse_c, delta_c, theta, q_start, kv_start, branch_k=None,
+                           branch_v=None, scale=None, rope_round="bf16"):
+    """Backward contribution of one (query chunk, trunk-key chunk) pair of the context-
+    parallel ring (NeMo-RL issue 3698, "What I'm working on", item 4), given the query
+    rows' FINAL lse and delta = rowsum(dO * O) over the whole sequence.
+
+    Plain definition over the pair's visible entries (kv_start + t <= q_start + i):
+    P = exp(sigma q~.k~ - lse), dS = P (dO.V - delta), dq~ = sigma dS k~,
+    dk~ = sigma dS^T q~ (summed over every pass and query head of the group),
+    dV = P^T dO; the gradients are returned in the pre-RoPE frame (R^T at each row's
+    position).  With branch_k / branch_v ([P, Lq, Hkv, D], the chunk's own keys and
+    values of every pass) the branch keys of passes 2..p at the row's own position add
+    their part to dq and give dk_b, dv_b (the chunk's branch-pass gradients; pass 1
+    zero).  Summed over the ring's pairs these give the whole sequence's gradients.
+
+    qc [P, Lq, H, D], doc [P, Lq, H, D]; kt, vt [Lk, Hkv, D]; lse_c, delta_c [P, H, Lq].
+    Returns (dq [P, Lq, H, D], dk [Lk, Hkv, D], dv [Lk, Hkv, D], dk_b, dv_b or None)."""
+    P, Lq, H, D = qc.shape
+    Lk, Hkv = kt.shape[0], kt.shape[1]
+    g = H // Hkv
+    sc = _scale(D, scale)
+    ktr = rope_rotate(kt.astype(np.float64), np.arange(Lk) + kv_start, theta)
+    qr = np.stack([rope_rotate(qc[p0].astype(np.float64), np.arange(Lq) + q_start + p0, theta) for p0 in range(P)])
+    kbr = None
+    if branch_k is not None:
+        kbr = np.stack([rope_rotate(branch_k[j].astype(np.float64), np.arange(Lq) + q_start + j, theta)
+                        for j in range(P)])
+    if rope_round == "bf16":
+        ktr, qr = bf16_round(ktr), bf16_round(qr)
+        if kbr is not None:
+            kbr = bf16_round(kbr)
+    visible = (kv_start + np.arange(Lk))[None, :] <= (q_start + np.arange(Lq))[:, None]
+    vt64 = vt.astype(np.float64)
+    dqr = np.zeros((P, Lq, H, D))
+    dkr = np.zeros((Lk, Hkv, D))
+    dv = np.zeros((Lk, Hkv, D))
+    dkbr = np.zeros((P, Lq, Hkv, D)) if kbr is not None else None
+    dvb = np.zeros((P, Lq, Hkv, D)) if kbr is not None else None
+    for h in range(H):
+        kv = h // g
+        for p0 in range(P):
+            l = lse_c[p0, h][:, None]
+            dl = delta_c[p0, h][:, None]
+            do = doc[p0, :, h].astype(np.float64)
+            s = np.where(visible, sc * (qr[p0, :, h] @ ktr[:, kv].T), -np.inf)
+            Pm = np.exp(s - l)
+            dS = Pm * (do @ vt64[:, kv].T - dl)
+            dqr[p0, :, h] += sc * dS @ ktr[:, kv]
+            dkr[:, kv] += sc * dS.T @ qr[p0, :, h]
+            dv[:, kv] += Pm.T @ do
+            if kbr is not None:
+                for j in range(1, p0 + 1):
+                    sb = sc * np.sum(qr[p0, :, h] * kbr[j, :, kv], axis=1, keepdims=True)
+                    pb = np.exp(sb - l)
+                    dsb = pb * (np.sum(do * branch_v[j, :, kv].astype(np.float64), axis=1, keepdims=True) - dl)
+                    dqr[p0, :, h] += sc * dsb * kbr[j, :, kv]
+                    dkbr[j, :, kv] += sc * dsb * qr[p0, :, h]
+                    dvb[j, :, kv] += pb * do
+    dq = np.stack([rope_rotate(dqr[p0], np.arange(Lq) + q_start + p0, theta, inverse=True) for p0 in range(P)])
+    dk = rope_rotate(dkr, np.arange(Lk) + kv_start, theta, inverse=True)
+    if kbr is not None:
+        dkb = np.stack([rope_rotate(dkbr[j], np.arange(Lq) + q_start + j, theta, inverse=True) for j in range(P)])
+        return dq, dk, dv, dkb, dvb
+    return dq, dk, dv, None, None

@@ -369,3 +369,35 @@ def test_oracle_matches_its_fixture():
     assert set(ref) == set(got)
     for name in ref:
         np.testing.assert_allclose(got[name], ref[name], rtol=0, atol=1e-13, err_msg=name)
+
+
+def test_chunk_backward_partials_sum_to_the_whole_backward():
+    """The ring's backward contributions over every (query chunk, earlier-or-same key
+    chunk) pair, with the whole sequence's lse and delta, sum to backward_twopart on the
+    whole sequence (a chunk split the plain definition does not know about)."""
+    rng = np.random.default_rng(77)
+    P, L, H, Hkv, D, theta = 3, 11, 4, 2, 8, 1e4
+    q, k, v, do = (rng.standard_normal(s) for s in ((P, L, H, D), (P, L, Hkv, D), (P, L, Hkv, D), (P, L, H, D)))
+    O, lse = orc.forward_twopart(q, k, v, theta)
+    dq, dk, dv = orc.backward_twopart(q, k, v, do, lse, theta)
+    delta = np.einsum("plhd,plhd->phl", do, O)
+    cuts = [(0, 3), (3, 4), (7, 4)]
+    gq, gk, gv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for a, n in cuts:
+        for b, m in cuts:
+            if b > a:
+                continue
+            own = a == b
+            r = orc.chunk_backward_partial(q[:, a:a + n], k[0, b:b + m], v[0, b:b + m], do[:, a:a + n],
+                                           lse[:, :, a:a + n], delta[:, :, a:a + n], theta, a, b,
+                                           branch_k=k[:, a:a + n] if own else None,
+                                           branch_v=v[:, a:a + n] if own else None)
+            gq[:, a:a + n] += r[0]
+            gk[0, b:b + m] += r[1]
+            gv[0, b:b + m] += r[2]
+            if own:
+                gk[1:, a:a + n] += r[3][1:]
+                gv[1:, a:a + n] += r[4][1:]
+    np.testing.assert_allclose(gq, dq, atol=1e-11)
+    np.testing.assert_allclose(gk, dk, atol=1e-11)
+    np.testing.assert_allclose(gv, dv, atol=1e-11)
