@@ -159,6 +159,16 @@ def lib() -> ctypes.CDLL:
     L.ttt_ring_merge.restype = ctypes.c_int
     L.ttt_ring_finish.argtypes = [RD, vp, vp, vp]
     L.ttt_ring_finish.restype = ctypes.c_int
+    L.ttt_ring_bwd_workspace_size.argtypes = [RD]
+    L.ttt_ring_bwd_workspace_size.restype = ctypes.c_size_t
+    L.ttt_ring_bwd_prepare.argtypes = [RD, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.ttt_ring_bwd_prepare.restype = ctypes.c_int
+    L.ttt_ring_bwd_step.argtypes = [RD, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.ttt_ring_bwd_step.restype = ctypes.c_int
+    L.ttt_ring_bwd_finish.argtypes = [RD, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.ttt_ring_bwd_finish.restype = ctypes.c_int
+    L.ttt_ring_dkv_finish.argtypes = [RD, vp, vp, vp, vp, vp]
+    L.ttt_ring_dkv_finish.restype = ctypes.c_int
     L.ttt_status_string.argtypes = [ctypes.c_int]
     L.ttt_status_string.restype = ctypes.c_char_p
     L.ttt_attn_version.argtypes = []

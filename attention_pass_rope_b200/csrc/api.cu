@@ -657,6 +657,120 @@ ttt_status ttt_ring_finish(const ttt_ring_desc* desc, const float* o_acc, void* 
   return TTT_OK;
 }
 
+// ---- ring backward
+namespace {
+struct RingBwdPlan {
+  size_t off[4];  // status, row statistics, dq~ accumulator, order tickets
+  size_t total;
+};
+RingBwdPlan ring_bwd_plan(const Geometry& g) {
+  RingBwdPlan pl{};
+  const size_t T = static_cast<size_t>(g.si.T), P = g.P, H = g.H, D = g.D;
+  const size_t slots = static_cast<size_t>(ld_slots(g.si));
+  size_t o = 0;
+  pl.off[0] = 0;
+  o = align_up(256);
+  pl.off[1] = o;
+  o = align_up(o + P * H * slots * 128 * 4);
+  pl.off[2] = o;
+  o = align_up(o + P * H * T * D * 4);
+  pl.off[3] = o;
+  o = align_up(o + P * H * slots * 4);
+  pl.total = o;
+  return pl;
+}
+}  // namespace
+
+size_t ttt_ring_bwd_workspace_size(const ttt_ring_desc* desc) {
+  Geometry g;
+  if (make_ring_geometry(desc, &g) != TTT_OK) return 0;
+  return ring_bwd_plan(g).total;
+}
+
+ttt_status ttt_ring_bwd_prepare(const ttt_ring_desc* desc, const void* o, const float* lse, const void* dout,
+                                void* workspace, size_t workspace_bytes, void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0) return TTT_OK;
+  const RingBwdPlan pl = ring_bwd_plan(g);
+  if (!o || !lse || !dout || !ptr_aligned(o, 16) || !ptr_aligned(dout, 16) || !ptr_aligned(lse, 4))
+    return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  clear_stale_error();
+  TTT_CHECK_CUDA(cudaMemsetAsync(ws, 0, sizeof(uint32_t), stream));
+  TTT_CHECK_CUDA(launch_bwd_preprocess(g, o, dout, lse, reinterpret_cast<float*>(ws + pl.off[1]),
+                                       reinterpret_cast<float*>(ws + pl.off[2]), reinterpret_cast<int*>(ws + pl.off[3]),
+                                       nullptr, reinterpret_cast<uint32_t*>(ws), nullptr, stream));
+  return TTT_OK;
+}
+
+ttt_status ttt_ring_bwd_step(const ttt_ring_desc* desc, const void* qr, const void* dout, const void* kr_visit,
+                             const void* v_visit, float* dk_acc, float* dv_acc, void* workspace, size_t workspace_bytes,
+                             void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0 || desc->kv_len == 0) return TTT_OK;
+  if (desc->kv_start > desc->q_start) return TTT_ERR_INVALID_ARG;  // no visible key
+  const RingBwdPlan pl = ring_bwd_plan(g);
+  if (!qr || !dout || !kr_visit || !v_visit || !dk_acc || !dv_acc) return TTT_ERR_INVALID_ARG;
+  if (!ptr_aligned(qr, 16) || !ptr_aligned(dout, 16) || !ptr_aligned(kr_visit, 16) || !ptr_aligned(v_visit, 16) ||
+      !ptr_aligned(dk_acc, 16) || !ptr_aligned(dv_acc, 16))
+    return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const uint64_t Lq = desc->q_len, Lk = desc->kv_len, D = g.D, P = g.P, H = g.H, Hkv = g.Hkv;
+  clear_stale_error();
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, qr, D, Lq, P * H, D * 2, Lq * D * 2, 64, 1) ||
+      !make_map(&mk, kr_visit, D, Lk, Hkv, D * 2, Lk * D * 2, 128, 1) ||
+      !make_map(&mv, v_visit, D, Hkv, Lk, D * 2, Hkv * D * 2, 1, 128) ||
+      !make_map4(&mdo, dout, {D, H, Lq, P}, {D * 2, H * D * 2, static_cast<uint64_t>(g.sq) * 2}, {1, 64, 1}))
+    return TTT_ERR_CUDA;
+  TrunkBwdArgs a{g, reinterpret_cast<const float*>(ws + pl.off[1]), reinterpret_cast<float*>(ws + pl.off[2]),
+                 nullptr, nullptr, nullptr, nullptr, reinterpret_cast<uint32_t*>(ws), g_wait_budget_ns.load(),
+                 dk_acc, dv_acc};
+  TTT_CHECK_CUDA(launch_trunk_bwd(a, mq, mk, mv, mdo, stream));
+  return TTT_OK;
+}
+
+ttt_status ttt_ring_bwd_finish(const ttt_ring_desc* desc, const void* qr, const void* kr_local, const void* v_local,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                               size_t workspace_bytes, void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0) return TTT_OK;
+  const RingBwdPlan pl = ring_bwd_plan(g);
+  if (!qr || !kr_local || !v_local || !dout || !lse || !dq || !dk || !dv) return TTT_ERR_INVALID_ARG;
+  for (const void* p : {qr, kr_local, v_local, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                        static_cast<const void*>(dv)})
+    if (!ptr_aligned(p, 16)) return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || !ptr_aligned(workspace, 256)) return TTT_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  clear_stale_error();
+  TTT_CHECK_CUDA(launch_branch_bwd(g, qr, kr_local, v_local, dout, lse, reinterpret_cast<const float*>(ws + pl.off[1]),
+                                   reinterpret_cast<const float*>(ws + pl.off[2]), dq, dk, dv,
+                                   static_cast<cudaStream_t>(stream_)));
+  return TTT_OK;
+}
+
+ttt_status ttt_ring_dkv_finish(const ttt_ring_desc* desc, const float* dk_acc, const float* dv_acc, void* dk,
+                               void* dv, void* stream_) {
+  Geometry g;
+  const ttt_status st = make_ring_geometry(desc, &g);
+  if (st != TTT_OK) return st;
+  if (desc->q_len == 0) return TTT_OK;
+  if (!dk_acc || !dv_acc || !dk || !dv || !ptr_aligned(dk, 16) || !ptr_aligned(dv, 16)) return TTT_ERR_INVALID_ARG;
+  clear_stale_error();
+  TTT_CHECK_CUDA(launch_ring_dkv_finish(g, desc->q_len, dk_acc, dv_acc, dk, dv, static_cast<cudaStream_t>(stream_)));
+  return TTT_OK;
+}
+
 ttt_status ttt_attn_device_status(void* workspace, void* stream_, uint32_t* detail) {
   if (!workspace) return TTT_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);

@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const int d = LaneMap<D>::d(lane, 0, e);
-        angle_cos_sin(pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
+        angle_cos_sin(g.pos0 + pos + p, inv_freq[d], cs[p * D + d], cs[p * D + D / 2 + d]);
       }
     const int64_t next_tau = tau + W;
     for (int kvh = 0; kvh < g.Hkv; ++kvh) {

@@ -70,7 +70,44 @@ __global__ void __launch_bounds__(256) ring_finish_kernel(int64_t n, const float
   *reinterpret_cast<uint2*>(o + i) = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
 }
 
+// Trunk dK / dV of a chunk from the accumulators that travelled around the ring and came
+// home: dK_1[t] = sigma * R(pos0 + t)^T dk~[t] and dV_1[t], bf16 into the pass-1 rows of
+// the chunk's public dk, dv.  One warp per (token, KV head); lane l takes the rotation
+// pairs (d, d + D/2) for d = l, l + 32, ... < D/2.
+__global__ void __launch_bounds__(256) ring_dkv_finish_kernel(Geometry g, int n, const float* __restrict__ dk_acc,
+                                                              const float* __restrict__ dv_acc,
+                                                              __nv_bfloat16* __restrict__ dk,
+                                                              __nv_bfloat16* __restrict__ dv) {
+  const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (item >= static_cast<int64_t>(n) * g.Hkv) return;
+  const int lane = threadIdx.x & 31;
+  const int t = static_cast<int>(item / g.Hkv), kvh = static_cast<int>(item % g.Hkv);
+  const int D = g.D, half = D / 2;
+  const float* ka = dk_acc + (static_cast<int64_t>(kvh) * n + t) * D;
+  const float* va = dv_acc + (static_cast<int64_t>(kvh) * n + t) * D;
+  __nv_bfloat16* kd = dk + (static_cast<int64_t>(t) * g.Hkv + kvh) * D;  // pass 1 of the public layout
+  __nv_bfloat16* vd = dv + (static_cast<int64_t>(t) * g.Hkv + kvh) * D;
+  for (int d = lane; d < half; d += 32) {
+    float c, s;
+    angle_cos_sin(g.pos0 + t, pow(static_cast<double>(g.theta), -2.0 * d / D), c, s);
+    const float x1 = ka[d] * g.scale, x2 = ka[d + half] * g.scale;
+    kd[d] = __float2bfloat16_rn(fmaf(x1, c, x2 * s));
+    kd[d + half] = __float2bfloat16_rn(fmaf(x2, c, -x1 * s));
+    vd[d] = __float2bfloat16_rn(va[d]);
+    vd[d + half] = __float2bfloat16_rn(va[d + half]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_ring_dkv_finish(const Geometry& g, int n, const float* dk_acc, const float* dv_acc, void* dk,
+                                   void* dv, cudaStream_t stream) {
+  const int64_t items = static_cast<int64_t>(n) * g.Hkv;
+  if (items <= 0) return cudaSuccess;
+  ring_dkv_finish_kernel<<<static_cast<unsigned>((items + 7) / 8), 256, 0, stream>>>(
+      g, n, dk_acc, dv_acc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_ring_merge(int rows, int D, int H, int Lq, float* o_acc, float* lse_acc, const float* o_part,
                               const float* lse_part, bool first, cudaStream_t stream) {

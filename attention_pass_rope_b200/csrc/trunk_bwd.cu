@@ -153,7 +153,10 @@ __device__ __forceinline__ void store_dk_row(__nv_bfloat16* dst, int pos, float 
 
 // MODE 0: TTT trunk (queries and keys are the same tokens, causal).  MODE 1: block-draft
 // trunk (queries are block rows, keys the context; a query row sees the keys up to its
-// block's anchor, a.qlim).
+// block's anchor, a.qlim).  MODE 2: one step of the context-parallel ring (queries are a
+// chunk of the sequence, keys a visiting chunk; row r sees key t iff t <= r +
+// g.limit_off); the keys' dk~ and dV are added to fp32 accumulators that travel with the
+// chunk, the dq~ of the rows as in MODE 0.
 template <int D, int MODE>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     trunk_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -191,13 +194,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   if (k0 >= klen) return;
   const int gsz = g.H / g.Hkv;
   const int G = g.P * gsz;
-  const int jq0 = MODE == 0 ? k0 / C::BQ : first_tile_seeing(g, a.qlim, seq_start, len, k0);
+  const int off = MODE == 2 ? g.limit_off : 0;  // row r sees key t iff t <= r + off (MODE 0, 2)
+  const int jq0 = MODE == 1 ? first_tile_seeing(g, a.qlim, seq_start, len, k0) : max(k0 - off, 0) / C::BQ;
   const int jq1 = MODE == 1 && g.window > 0 ? last_tile_seeing(g, a.qlim, seq_start, len, k0 + C::BK - 1)
                                             : (len + C::BQ - 1) / C::BQ - 1;
   const int nqt = max(jq1 - jq0 + 1, 0);
   const int NIT = G * nqt;
   if (threadIdx.x == 0) TTT_CTA_INFO(NIT);
   if (NIT <= 0) {
+    if (MODE == 2) return;  // the accumulators keep what other steps added
     // block-draft keys that no query row sees: zero gradients
     for (int i = threadIdx.x; i < C::BK * (D / 8); i += blockDim.x) {
       const int r = i / (D / 8), c8 = i % (D / 8);
@@ -434,11 +439,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const float* ldp = sLD + s * 2 * C::BQ + 32 * hf;
       // interior tile: every (key, query) pair of this half is visible
       const int qlo = ii.q0 + 32 * hf;
-      const bool interior =
-          (qlo + 32 <= len) && (k0 + C::BK <= klen) &&
-          (MODE == 0 ? qlo >= k0 + C::BK - 1
-                     : __ldg(a.qlim + seq_start + qlo) >= k0 + C::BK - 1 &&
-                           block_row_start(g, __ldg(a.qlim + seq_start + qlo + 31)) <= k0);
+      bool interior = false;
+      if (qlo + 32 <= len && k0 + C::BK <= klen) {
+        if (MODE != 1) {
+          interior = qlo + off >= k0 + C::BK - 1;
+        } else {
+          // the first row has the smallest limit, the last the largest window start; both
+          // loads are issued before either is compared (no dependent round trip)
+          const int l_first = __ldg(a.qlim + seq_start + qlo);
+          const int l_last = g.window > 0 ? __ldg(a.qlim + seq_start + qlo + 31) : 0;
+          interior = l_first >= k0 + C::BK - 1 && block_row_start(g, l_last) <= k0;
+        }
+      }
       // P = 2^(s*scale*log2e - lse*log2e), dS = P (dP - delta), two columns per
       // instruction; the bf16 pairs are packed straight from the results
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -462,7 +474,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
           if (!interior) {
             // padding rows of the statistics are never written: select, do not multiply
-            int lim0 = qlo + c, lim1 = qlo + c + 1, st0 = 0, st1 = 0;
+            int lim0 = qlo + c + off, lim1 = qlo + c + 1 + off, st0 = 0, st1 = 0;
             if (MODE == 1) {
               lim0 = qlo + c < len ? __ldg(a.qlim + seq_start + qlo + c) : -1;
               lim1 = qlo + c + 1 < len ? __ldg(a.qlim + seq_start + qlo + c + 1) : -1;
@@ -511,7 +523,28 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_after();
       if (lane == 0 && warp == 4) TTT_CTA_MARK(2);
       const int64_t tau = kstart + kpos;
-      if (hf == 0) {
+      if (MODE == 2) {
+        // ring step: add this CTA's raw dV / dk~ rows to the travelling accumulators
+        float* acc = (hf == 0 ? a.dv_acc : a.dk_acc) + (static_cast<int64_t>(kvh) * klen + kpos) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + (hf == 0 ? C::COL_DV : C::COL_DK) + 32 * c, v);
+          tmem_ld_wait();
+          reg_fence32(v);
+          if (!kvalid) continue;
+          float4* dst = reinterpret_cast<float4*>(acc + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float4 x = dst[e];
+            x.x += __uint_as_float(v[4 * e]);
+            x.y += __uint_as_float(v[4 * e + 1]);
+            x.z += __uint_as_float(v[4 * e + 2]);
+            x.w += __uint_as_float(v[4 * e + 3]);
+            dst[e] = x;
+          }
+        }
+      } else if (hf == 0) {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -641,6 +674,9 @@ cudaError_t launch(const TrunkBwdArgs& a, const CUtensorMap& mq, const CUtensorM
 
 cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, const CUtensorMap& map_k,
                              const CUtensorMap& map_v, const CUtensorMap& map_do, cudaStream_t stream) {
+  if (a.g.ring > 0)
+    return a.g.D == 128 ? launch<128, 2>(a, map_q, map_k, map_v, map_do, stream)
+                        : launch<64, 2>(a, map_q, map_k, map_v, map_do, stream);
   if (a.g.Bs > 0)
     return a.g.D == 128 ? launch<128, 1>(a, map_q, map_k, map_v, map_do, stream)
                         : launch<64, 1>(a, map_q, map_k, map_v, map_do, stream);

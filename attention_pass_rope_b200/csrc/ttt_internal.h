@@ -140,6 +140,10 @@ struct TrunkBwdArgs {
   const int* qlim;     // block-draft: trunk-key limit of every query row; nullptr otherwise
   uint32_t* status;
   uint64_t budget_ns;
+  // ring step (g.ring > 0): the visiting chunk's dk~ (before sigma and the inverse
+  // rotation) and dV as fp32 [Hkv][klen][D], added to (dk / dv are not written)
+  float* dk_acc;
+  float* dv_acc;
 };
 // a6: trunk backward on tcgen05; maps: q~ (box 64 rows), k~_1 (box 128 rows),
 // V_1 (box 128 rows), dO (4D {D, H, T, P}, pass stride g.sq, box 64 rows).
@@ -166,6 +170,10 @@ cudaError_t launch_block_bwd(const Geometry& g, const void* qr, const void* kr, 
 
 // Ring: running merge of partial results (acc <- acc (+) part by log-sum-exp; `first`
 // copies), and the final bf16 output.  O rows are [P][Lq][H][D] fp32, lse [P][H][Lq].
+// Ring backward: a chunk's trunk dK / dV from its returned fp32 accumulators
+// ([Hkv][n][D], dk~ before sigma and the inverse rotation), bf16 into the pass-1 rows.
+cudaError_t launch_ring_dkv_finish(const Geometry& g, int n, const float* dk_acc, const float* dv_acc, void* dk,
+                                   void* dv, cudaStream_t stream);
 cudaError_t launch_ring_merge(int rows, int D, int H, int Lq, float* o_acc, float* lse_acc, const float* o_part,
                               const float* lse_part, bool first, cudaStream_t stream);
 cudaError_t launch_ring_finish(int64_t n, const float* o_acc, void* o, cudaStream_t stream);

@@ -65,6 +65,9 @@ class TrunkChunk:
     start: int                 # global position of its first token
     kr: torch.Tensor           # rotated pass-1 keys [Hkv, len, D]
     v: torch.Tensor            # pass-1 values [len, Hkv, D]
+    # backward only: the chunk's dk~ / dV accumulators [Hkv, len, D], which travel with it
+    dk_acc: Optional[torch.Tensor] = None
+    dv_acc: Optional[torch.Tensor] = None
 
 
 class P2PExchange:
@@ -101,9 +104,14 @@ class P2PExchange:
         for c, (start, n), like in zip(chunks, meta_in.tolist(), recv_like):
             r = TrunkChunk(int(start), like.kr.new_empty((like.kr.shape[0], int(n), like.kr.shape[2])),
                            like.v.new_empty((int(n), *like.v.shape[1:])))
+            pairs = [(c.kr, r.kr), (c.v, r.v)]
+            if c.dk_acc is not None:
+                r.dk_acc = c.dk_acc.new_empty((c.dk_acc.shape[0], int(n), c.dk_acc.shape[2]))
+                r.dv_acc = c.dv_acc.new_empty((c.dv_acc.shape[0], int(n), c.dv_acc.shape[2]))
+                pairs += [(c.dk_acc, r.dk_acc), (c.dv_acc, r.dv_acc)]
             out.append(r)
-            ops += [dist.P2POp(dist.isend, c.kr, nxt, self.group), dist.P2POp(dist.irecv, r.kr, prv, self.group),
-                    dist.P2POp(dist.isend, c.v, nxt, self.group), dist.P2POp(dist.irecv, r.v, prv, self.group)]
+            for snd, rcv in pairs:
+                ops += [dist.P2POp(dist.isend, snd, nxt, self.group), dist.P2POp(dist.irecv, rcv, prv, self.group)]
         self._wait(dist.batch_isend_irecv(ops))
         return out
 
@@ -130,6 +138,40 @@ def ring_forward(local: Sequence[dict], step: Callable, merge: Callable, finish:
                 part = step(qc, tc, include_branch=(tc.start == qc["start"]))
                 acc[i] = merge(acc[i], part)
     return [finish(qc, a) for qc, a in zip(local, acc)]
+
+
+def ring_backward(local: Sequence[dict], prepare: Callable, step: Callable, finish: Callable,
+                  finish_trunk: Callable, exchange, world: int, trunk: Sequence[TrunkChunk], zeros: Callable):
+    """The ring's backward on one rank, after ring_forward.
+
+    local: this rank's query chunks (with whatever the functions need: the final o and
+      lse, dout); trunk: its own trunk chunks.
+    prepare(q_chunk): delta and the chunk's zeroed dq~ accumulator.
+    step(q_chunk, trunk_chunk, include_branch): the pair's contribution -- dq~ into the
+      query chunk's accumulator, dk~ / dV into the trunk chunk's travelling accumulators.
+    finish(q_chunk) -> the query chunk's dq and branch-pass dK / dV.
+    finish_trunk(trunk_chunk) -> its pass-1 dK / dV from its accumulators, home again.
+    zeros(trunk_chunk) -> (dk_acc, dv_acc) zeroed.
+    The trunk chunks travel as in the forward, each with its accumulators; after the
+    ring one more shift brings every accumulator back to its owner.
+    Returns ([finish(q) for q in local], [finish_trunk(t) for t in this rank's own])."""
+    for qc in local:
+        prepare(qc)
+    held = []
+    for tc in trunk:
+        dk_acc, dv_acc = zeros(tc)
+        held.append(dataclasses.replace(tc, dk_acc=dk_acc, dv_acc=dv_acc))
+    for s in range(world):
+        if s > 0:
+            held = exchange.shift(held, trunk)
+        for qc in local:
+            for tc in held:
+                if tc.start > qc["start"]:
+                    continue  # a chunk that starts later holds no key this chunk sees
+                step(qc, tc, include_branch=(tc.start == qc["start"]))
+    if world > 1:
+        held = exchange.shift(held, trunk)  # the accumulators come home
+    return [finish(qc) for qc in local], [finish_trunk(tc) for tc in held]
 
 
 # ----------------------------------------------------------------------------- CUDA implementation
@@ -204,3 +246,53 @@ def gpu_ops():
         return o, la
 
     return step, merge, finish
+
+
+def gpu_bwd_ops(theta: float, scale=None):
+    """(prepare, step, finish, finish_trunk, zeros) of the ring's backward on the GPU
+    through the C ABI (theta, scale as in the forward).  A query chunk dict needs, besides what rotate_chunk gives, "o" and
+    "lse" (the forward's final result) and "do"; prepare adds its workspace."""
+    L = _lib.lib()
+
+    def desc_of(qc, tc=None):
+        return _desc(qc["P"], qc["H"], qc["Hkv"], qc["D"], qc["theta"], qc["scale"], qc["len"], qc["start"],
+                     0 if tc is None else tc.kr.shape[1], 0 if tc is None else tc.start)
+
+    def prepare(qc):
+        d = desc_of(qc)
+        ws = torch.empty(L.ttt_ring_bwd_workspace_size(ctypes.byref(d)), dtype=torch.uint8, device=qc["qr"].device)
+        qc["bwd_ws"] = ws
+        _lib.check(L.ttt_ring_bwd_prepare(ctypes.byref(d), _p(qc["o"]), _p(qc["lse"]), _p(qc["do"]), _p(ws),
+                                          ws.numel(), _s()), "ttt_ring_bwd_prepare")
+
+    def step(qc, tc: TrunkChunk, include_branch: bool):
+        d = desc_of(qc, tc)
+        ws = qc["bwd_ws"]
+        _lib.check(L.ttt_ring_bwd_step(ctypes.byref(d), _p(qc["qr"]), _p(qc["do"]), _p(tc.kr), _p(tc.v),
+                                       _p(tc.dk_acc), _p(tc.dv_acc), _p(ws), ws.numel(), _s()), "ttt_ring_bwd_step")
+
+    def finish(qc):
+        d = desc_of(qc)
+        ws = qc["bwd_ws"]
+        dq = torch.empty_like(qc["do"])
+        dk = torch.zeros(qc["P"], qc["len"], qc["Hkv"], qc["D"], dtype=torch.bfloat16, device=dq.device)
+        dv = torch.zeros_like(dk)
+        _lib.check(L.ttt_ring_bwd_finish(ctypes.byref(d), _p(qc["qr"]), _p(qc["kr"]), _p(qc["v"]), _p(qc["do"]),
+                                         _p(qc["lse"]), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _s()),
+                   "ttt_ring_bwd_finish")
+        return dq, dk, dv
+
+    def finish_trunk(tc: TrunkChunk):
+        n, Hkv, D = tc.kr.shape[1], tc.kr.shape[0], tc.kr.shape[2]
+        d = _desc(1, Hkv, Hkv, D, theta, scale, n, tc.start)
+        dk = torch.empty(n, Hkv, D, dtype=torch.bfloat16, device=tc.kr.device)
+        dv = torch.empty_like(dk)
+        _lib.check(L.ttt_ring_dkv_finish(ctypes.byref(d), _p(tc.dk_acc), _p(tc.dv_acc), _p(dk), _p(dv), _s()),
+                   "ttt_ring_dkv_finish")
+        return tc.start, dk, dv
+
+    def zeros(tc: TrunkChunk):
+        z = torch.zeros(tc.kr.shape, dtype=torch.float32, device=tc.kr.device)
+        return z, torch.zeros_like(z)
+
+    return prepare, step, finish, finish_trunk, zeros

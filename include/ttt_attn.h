@@ -321,6 +321,36 @@ ttt_status ttt_ring_merge(const ttt_ring_desc* desc, float* o_acc, float* lse_ac
 /* o (bf16 [P][q_len][H][D]) <- o_acc; the lse is lse_acc itself. */
 ttt_status ttt_ring_finish(const ttt_ring_desc* desc, const float* o_acc, void* o, void* stream);
 
+/* Ring backward (same page and item).  With the final o, lse of a local chunk and its
+ * dout:
+ *   1. ttt_ring_bwd_prepare: delta = rowsum(dout * o) and the row statistics into the
+ *      chunk's workspace, its fp32 dq~ accumulator zeroed (the workspace's first word
+ *      is the status word of the bounded waits: ttt_attn_device_status);
+ *   2. ttt_ring_bwd_step, once per visiting chunk the forward met (kv_start <= q_start):
+ *      adds the chunk's trunk dq~ to the accumulator, and the visiting keys' dk~ (before
+ *      sigma and the inverse rotation) and dV to dk_acc, dv_acc (fp32 [Hkv][kv_len][D]);
+ *      these accumulators travel with the visiting chunk and come home after the ring
+ *      (moving them is the caller's, as in the forward);
+ *   3. ttt_ring_bwd_finish: the branch keys' part, dq (every pass) and the dK / dV of
+ *      the branch passes (p >= 2) of the local chunk, bf16 in the public layout;
+ *   4. ttt_ring_dkv_finish on a chunk's returned accumulators (desc describing that
+ *      chunk: q_len, q_start): the pass-1 rows of its dk, dv.
+ * After all of it the gradients equal ttt_attn_bwd's on the whole sequence (up to
+ * rounding and the order of the fp32 additions).  Layouts as in the forward; dq, dout
+ * [P][q_len][H][D], dk, dv [P][q_len][Hkv][D].  The calls read and write this GPU's
+ * memory only. */
+size_t ttt_ring_bwd_workspace_size(const ttt_ring_desc* desc);
+ttt_status ttt_ring_bwd_prepare(const ttt_ring_desc* desc, const void* o, const float* lse, const void* dout,
+                                void* workspace, size_t workspace_bytes, void* stream);
+ttt_status ttt_ring_bwd_step(const ttt_ring_desc* desc, const void* qr, const void* dout, const void* kr_visit,
+                             const void* v_visit, float* dk_acc, float* dv_acc, void* workspace,
+                             size_t workspace_bytes, void* stream);
+ttt_status ttt_ring_bwd_finish(const ttt_ring_desc* desc, const void* qr, const void* kr_local, const void* v_local,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                               size_t workspace_bytes, void* stream);
+ttt_status ttt_ring_dkv_finish(const ttt_ring_desc* desc, const float* dk_acc, const float* dv_acc, void* dk,
+                               void* dv, void* stream);
+
 /* The error behind the most recent TTT_ERR_CUDA returned by any call in this
  * process: a cudaError_t value, or 100000 + the CUresult when encoding a TMA tensor
  * map failed; 0 if there was none.  Not reset by later successful calls. */

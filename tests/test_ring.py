@@ -50,14 +50,14 @@ def _merge_np(acc, part):
     return wa * oa + wb * ob, l
 
 
-def _cpu_rank(rank, world, port, out, L, drop_rank, delay_rank, timeout_s):
+def _cpu_rank(rank, world, port, out, L, drop_rank, delay_rank, timeout_s, with_bwd=False):
     sys.path.insert(0, ROOT)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
                                          timeout=datetime.timedelta(seconds=60))
     try:
         w = ttt_inputs.thd("ring", [L], 3, 4, 2, 16, 1e4)
-        inp = ttt_inputs.make_inputs(w, with_grad=False)
+        inp = ttt_inputs.make_inputs(w, with_grad=with_bwd)
         q, k, v = (t.double().numpy() for t in (inp.q, inp.k, inp.v))
         chunks = ring.zigzag_chunks(L, world)
         local, trunk = [], []
@@ -84,9 +84,38 @@ def _cpu_rank(rank, world, port, out, L, drop_rank, delay_rank, timeout_s):
                     time.sleep(timeout_s / 4)
                 return super().shift(held, like)
 
-        res = ring.ring_forward(local, step, _merge_np, lambda qc, acc: acc, Ex(rank, world, timeout_s), world,
-                                trunk)
-        out[rank] = ("ok", [(qc["start"], o, l) for qc, (o, l) in zip(local, res)])
+        ex = Ex(rank, world, timeout_s)
+        res = ring.ring_forward(local, step, _merge_np, lambda qc, acc: acc, ex, world, trunk)
+        if not with_bwd:
+            out[rank] = ("ok", [(qc["start"], o, l) for qc, (o, l) in zip(local, res)])
+            return
+        # backward: the forward's final (o, lse) per chunk, dO, the oracle's pair
+        # contributions as the step; the trunk chunks' accumulators travel with them
+        dO = inp.do.double().numpy()
+        for qc, (o, l) in zip(local, res):
+            a, n = qc["start"], qc["q"].shape[1]
+            qc.update(o=o, lse=l, do=dO[:, a:a + n], delta=np.einsum("plhd,plhd->phl", dO[:, a:a + n], o))
+
+        def prepare(qc):
+            qc["dq"] = np.zeros_like(qc["q"])
+
+        def bstep(qc, tc, include_branch):
+            r = orc.chunk_backward_partial(qc["q"], tc.kr.transpose(0, 1).numpy(), tc.v.numpy(), qc["do"],
+                                           qc["lse"], qc["delta"], 1e4, qc["start"], tc.start,
+                                           branch_k=qc["k"] if include_branch else None,
+                                           branch_v=qc["v"] if include_branch else None)
+            qc["dq"] += r[0]
+            tc.dk_acc += torch.from_numpy(r[1].transpose(1, 0, 2).copy())
+            tc.dv_acc += torch.from_numpy(r[2].transpose(1, 0, 2).copy())
+            if include_branch:
+                qc["dkb"], qc["dvb"] = r[3], r[4]
+
+        zeros = lambda tc: (torch.zeros_like(tc.kr), torch.zeros_like(tc.kr))  # both [Hkv, len, D]  # noqa: E731
+        grads, trunk_g = ring.ring_backward(local, prepare, bstep,
+                                            lambda qc: (qc["start"], qc["dq"], qc["dkb"], qc["dvb"]),
+                                            lambda tc: (tc.start, tc.dk_acc.numpy(), tc.dv_acc.numpy()),
+                                            ex, world, trunk, zeros)
+        out[rank] = ("ok", grads, trunk_g)
     except ring.RingTimeout as e:
         out[rank] = ("timeout", str(e))
     except RuntimeError as e:
@@ -95,14 +124,14 @@ def _cpu_rank(rank, world, port, out, L, drop_rank, delay_rank, timeout_s):
         os._exit(0)  # a rank whose peer vanished must not wait in the group's teardown
 
 
-def _run_ring(world, L=37, drop_rank=-1, delay_rank=-1, timeout_s=4.0):
+def _run_ring(world, L=37, drop_rank=-1, delay_rank=-1, timeout_s=4.0, with_bwd=False):
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
         out = m.dict()
-        ps = [ctx.Process(target=_cpu_rank, args=(r, world, port, out, L, drop_rank, delay_rank, timeout_s))
+        ps = [ctx.Process(target=_cpu_rank, args=(r, world, port, out, L, drop_rank, delay_rank, timeout_s, with_bwd))
               for r in range(world)]
         for p in ps:
             p.start()
@@ -129,6 +158,36 @@ def test_ring_over_gloo_ranks_equals_the_oracle(world):
             np.testing.assert_allclose(l, lse[:, :, a:a + n], atol=1e-12)
             seen += n
     assert seen == L
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ring_backward_over_gloo_ranks_equals_the_oracle(world):
+    """The ring's backward: each rank adds its query chunks' contributions (the oracle's
+    pair contributions, from the forward's final lse) while the trunk chunks travel with
+    their dk / dV accumulators, which one more shift brings home; gathered, dq, dk and
+    dv equal the oracle's backward on the whole sequence."""
+    L = 37
+    res = _run_ring(world, L, with_bwd=True)
+    w = ttt_inputs.thd("ring", [L], 3, 4, 2, 16, 1e4)
+    inp = ttt_inputs.make_inputs(w)
+    q, k, v, do = (t.double().numpy() for t in (inp.q, inp.k, inp.v, inp.do))
+    O, lse = orc.forward_twopart(q, k, v, 1e4)
+    dq, dk, dv = orc.backward_twopart(q, k, v, do, lse, 1e4)
+    gq, gk, gv = np.full_like(dq, np.nan), np.full_like(dk, np.nan), np.full_like(dv, np.nan)
+    for r in range(world):
+        assert res[r][0] == "ok", res[r]
+        for a, dqc, dkb, dvb in res[r][1]:
+            n = dqc.shape[1]
+            gq[:, a:a + n] = dqc
+            gk[1:, a:a + n] = dkb[1:]
+            gv[1:, a:a + n] = dvb[1:]
+        for a, dka, dva in res[r][2]:
+            n = dva.shape[1]
+            gk[0, a:a + n] = dka.transpose(1, 0, 2)
+            gv[0, a:a + n] = dva.transpose(1, 0, 2)
+    np.testing.assert_allclose(gq, dq, atol=1e-11)
+    np.testing.assert_allclose(gk, dk, atol=1e-11)
+    np.testing.assert_allclose(gv, dv, atol=1e-11)
 
 
 def test_ring_late_peer_inside_the_limit():
@@ -195,4 +254,74 @@ def test_ring_cuda_steps_emulated_on_one_device(world, L, P, H, Hkv, D):
     kv = [Hkv - 1] if H > 8 else None
     m = parity.compare_full(w, inp, {"o": o, "lse": lse}, with_grad=False, kv_heads=kv)
     print("ring", world, L, m)
+    parity.assert_within(m)
+
+
+@pytest.mark.gpu
+@needs_cuda
+@pytest.mark.parametrize("world,L,P,H,Hkv,D", [(2, 1000, 3, 8, 2, 128), (4, 4096, 3, 32, 8, 128),
+                                               (3, 777, 5, 4, 1, 64)])
+def test_ring_backward_cuda_emulated_on_one_device(world, L, P, H, Hkv, D):
+    """The ring's CUDA backward: every rank's prepare (delta, statistics, zeroed dq~),
+    its steps against the trunk chunks it would hold (dq~ into the query chunk's
+    accumulator, dk~ / dV into the trunk chunk's fp32 accumulators, which in a real ring
+    travel with it and come home), the branch part and dq finish, and the trunk chunks'
+    dK / dV finish; the ranks one after another on one device, after the CUDA forward
+    ring.  Against the oracle's backward on the whole sequence: dq, dk, dv relative L2 <=
+    1e-2 (per pass too)."""
+    from tests import parity
+    w = ttt_inputs.thd("ring_gpu", [L], P, H, Hkv, D, 1e6)
+    inp = ttt_inputs.make_inputs(w)
+    q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.do))
+    chunks = ring.zigzag_chunks(L, world)
+    local = {}
+    for r in range(world):
+        local[r] = []
+        for c in ring.rank_chunks(r, world):
+            a, n = chunks[c]
+            qc = ring.rotate_chunk(q[:, a:a + n].contiguous(), k[:, a:a + n].contiguous(), v[:, a:a + n].contiguous(),
+                                   a, w.theta)
+            qc["do"] = do[:, a:a + n].contiguous()
+            local[r].append(qc)
+    trunks = {r: [ring.trunk_of(c) for c in local[r]] for r in range(world)}
+    step, merge, finish = ring.gpu_ops()
+    o = torch.full((P, L, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((P, H, L), float("nan"), device="cuda")
+    for r in range(world):
+        res = ring.ring_forward(local[r], step, merge, finish, _EmulatedExchange(r, world, trunks), world, trunks[r])
+        for qc, (oc, lc) in zip(local[r], res):
+            qc["o"], qc["lse"] = oc, lc.contiguous()
+            o[:, qc["start"]:qc["start"] + qc["len"]] = oc
+            lse[:, :, qc["start"]:qc["start"] + qc["len"]] = lc
+    prepare, bstep, bfinish, finish_trunk, zeros = ring.gpu_bwd_ops(w.theta)
+    # every trunk chunk's accumulators, shared by the emulated ranks
+    for r in range(world):
+        trunks[r] = [ring.TrunkChunk(tc.start, tc.kr, tc.v, *zeros(tc)) for tc in trunks[r]]
+    for r in range(world):
+        for qc in local[r]:
+            prepare(qc)
+    for r in range(world):
+        for s in range(world):
+            for qc in local[r]:
+                for tc in trunks[(r - s) % world]:
+                    if tc.start <= qc["start"]:
+                        bstep(qc, tc, tc.start == qc["start"])
+    dq = torch.full((P, L, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dk = torch.full((P, L, Hkv, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dv = torch.full_like(dk, float("nan"))
+    for r in range(world):
+        for qc in local[r]:
+            a, n = qc["start"], qc["len"]
+            dqc, dkc, dvc = bfinish(qc)
+            dq[:, a:a + n] = dqc
+            dk[1:, a:a + n] = dkc[1:]
+            dv[1:, a:a + n] = dvc[1:]
+        for tc in trunks[r]:
+            a, dkt, dvt = finish_trunk(tc)
+            dk[0, a:a + dkt.shape[0]] = dkt
+            dv[0, a:a + dvt.shape[0]] = dvt
+    torch.cuda.synchronize()
+    kv = [Hkv - 1] if H > 8 else None
+    m = parity.compare_full(w, inp, {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}, kv_heads=kv)
+    print("ring bwd", world, L, m)
     parity.assert_within(m)
