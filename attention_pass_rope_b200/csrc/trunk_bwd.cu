@@ -156,13 +156,17 @@ __device__ __forceinline__ void store_dk_row(__nv_bfloat16* dst, int pos, float 
 // block's anchor, a.qlim).  MODE 2: one step of the context-parallel ring (queries are a
 // chunk of the sequence, keys a visiting chunk; row r sees key t iff t <= r +
 // g.limit_off); the keys' dk~ and dV are added to fp32 accumulators that travel with the
-// chunk, the dq~ of the rows as in MODE 0.
+// chunk, the dq~ of the rows as in MODE 0.  MODE 3: MODE 1 for a sliding-window layer (a
+// row sees the keys from block_row_start of its limit up to the limit); a mode of its own
+// so that the window's bounds cost nothing in the plain block-draft kernel.
 template <int D, int MODE>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     trunk_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
                      const TrunkBwdArgs a) {
   using C = BwdCfg<D>;
+  constexpr bool BLOCK = MODE == 1 || MODE == 3;
+  constexpr bool WIN = MODE == 3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
@@ -195,9 +199,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int gsz = g.H / g.Hkv;
   const int G = g.P * gsz;
   const int off = MODE == 2 ? g.limit_off : 0;  // row r sees key t iff t <= r + off (MODE 0, 2)
-  const int jq0 = MODE == 1 ? first_tile_seeing(g, a.qlim, seq_start, len, k0) : max(k0 - off, 0) / C::BQ;
-  const int jq1 = MODE == 1 && g.window > 0 ? last_tile_seeing(g, a.qlim, seq_start, len, k0 + C::BK - 1)
-                                            : (len + C::BQ - 1) / C::BQ - 1;
+  const int jq0 = BLOCK ? first_tile_seeing(g, a.qlim, seq_start, len, k0) : max(k0 - off, 0) / C::BQ;
+  const int jq1 = WIN ? last_tile_seeing(g, a.qlim, seq_start, len, k0 + C::BK - 1) : (len + C::BQ - 1) / C::BQ - 1;
   const int nqt = max(jq1 - jq0 + 1, 0);
   const int NIT = G * nqt;
   if (threadIdx.x == 0) TTT_CTA_INFO(NIT);
@@ -441,13 +444,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int qlo = ii.q0 + 32 * hf;
       bool interior = false;
       if (qlo + 32 <= len && k0 + C::BK <= klen) {
-        if (MODE != 1) {
+        if (!BLOCK) {
           interior = qlo + off >= k0 + C::BK - 1;
+        } else if (!WIN) {
+          interior = __ldg(a.qlim + seq_start + qlo) >= k0 + C::BK - 1;
         } else {
           // the first row has the smallest limit, the last the largest window start; both
           // loads are issued before either is compared (no dependent round trip)
           const int l_first = __ldg(a.qlim + seq_start + qlo);
-          const int l_last = g.window > 0 ? __ldg(a.qlim + seq_start + qlo + 31) : 0;
+          const int l_last = __ldg(a.qlim + seq_start + qlo + 31);
           interior = l_first >= k0 + C::BK - 1 && block_row_start(g, l_last) <= k0;
         }
       }
@@ -474,15 +479,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
           if (!interior) {
             // padding rows of the statistics are never written: select, do not multiply
-            int lim0 = qlo + c + off, lim1 = qlo + c + 1 + off, st0 = 0, st1 = 0;
-            if (MODE == 1) {
+            int lim0 = qlo + c + off, lim1 = qlo + c + 1 + off;
+            if (BLOCK) {
               lim0 = qlo + c < len ? __ldg(a.qlim + seq_start + qlo + c) : -1;
               lim1 = qlo + c + 1 < len ? __ldg(a.qlim + seq_start + qlo + c + 1) : -1;
-              st0 = block_row_start(g, lim0);
-              st1 = block_row_start(g, lim1);
             }
-            const bool v0 = kvalid && qlo + c < len && kpos <= lim0 && kpos >= st0;
-            const bool v1 = kvalid && qlo + c + 1 < len && kpos <= lim1 && kpos >= st1;
+            bool v0 = kvalid && qlo + c < len && kpos <= lim0;
+            bool v1 = kvalid && qlo + c + 1 < len && kpos <= lim1;
+            if (WIN) {
+              v0 = v0 && kpos >= block_row_start(g, lim0);
+              v1 = v1 && kpos >= block_row_start(g, lim1);
+            }
             p0 = v0 ? p0 : 0.f;
             d0 = v0 ? d0 : 0.f;
             p1 = v1 ? p1 : 0.f;
@@ -677,6 +684,9 @@ cudaError_t launch_trunk_bwd(const TrunkBwdArgs& a, const CUtensorMap& map_q, co
   if (a.g.ring > 0)
     return a.g.D == 128 ? launch<128, 2>(a, map_q, map_k, map_v, map_do, stream)
                         : launch<64, 2>(a, map_q, map_k, map_v, map_do, stream);
+  if (a.g.Bs > 0 && a.g.window > 0)
+    return a.g.D == 128 ? launch<128, 3>(a, map_q, map_k, map_v, map_do, stream)
+                        : launch<64, 3>(a, map_q, map_k, map_v, map_do, stream);
   if (a.g.Bs > 0)
     return a.g.D == 128 ? launch<128, 1>(a, map_q, map_k, map_v, map_do, stream)
                         : launch<64, 1>(a, map_q, map_k, map_v, map_do, stream);
