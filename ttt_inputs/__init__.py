@@ -1,9 +1,10 @@
-"""Seeded synthetic inputs for the multi-pass TTT trunk+branch attention.
+"""Seeded synthetic inputs for the multi-pass TTT trunk+branch attention, the block-draft
+attention and the draft's soft cross-entropy distillation loss.
 
 This module is the only code shared by the fp64 oracle (``oracle/``) and the
 CUDA path (``attention_pass_rope_b200``).  It draws random numbers and packs
-them into tensors; it holds none of the attention arithmetic (no RoPE, no
-softmax, no masking).
+them into tensors; it holds none of the method's arithmetic (no RoPE, no
+softmax, no masking, no teacher alignment).
 
 Recipe (the same for every workload):
 
@@ -256,3 +257,68 @@ def make_block_inputs(w: BlockWorkload) -> BlockInputs:
     vb = draw(w.NB, w.Bs, w.Hkv, w.D)
     do = draw(w.NB, w.Bs, w.H, w.D)
     return BlockInputs(k_ctx, v_ctx, qb, kb, vb, do, anchors)
+
+
+@dataclasses.dataclass(frozen=True)
+class SoftCEWorkload:
+    """Shape of one distillation-loss call: P draft passes over the tokens of ``lengths``
+    (sequences packed back to back), hidden size d, vocabulary V."""
+
+    name: str
+    P: int
+    lengths: tuple
+    d: int
+    V: int
+    seed: int = 0
+    mask_keep: float = 0.9   # probability that a teacher position is counted
+
+    @property
+    def T(self) -> int:
+        return int(sum(self.lengths))
+
+    @property
+    def cu_seqlens(self) -> list:
+        out = [0]
+        for n in self.lengths:
+            out.append(out[-1] + int(n))
+        return out
+
+    def flops_fwd(self) -> float:
+        """The logits GEMM of every (pass, token) row: 2 * d * V per row."""
+        return 2.0 * self.P * self.T * self.d * self.V
+
+    def flops_fwd_bwd(self, with_dw: bool = True) -> float:
+        """Forward logits, recomputed logits, dh and (optionally) dW: 2 * d * V each per row."""
+        return self.flops_fwd() * (4.0 if with_dw else 3.0)
+
+
+def softce_workloads() -> dict:
+    """Distillation-loss workloads with the Qwen3-8B head (d = 4096, V = 151936)."""
+    return {
+        "softce_tiny": SoftCEWorkload("softce_tiny", P=3, lengths=(70, 129, 1, 56), d=128, V=1000),
+        "softce_mid": SoftCEWorkload("softce_mid", P=3, lengths=(700, 333, 1011), d=512, V=32771),
+        "softce_qwen3_8b_4k": SoftCEWorkload("softce_qwen3_8b_4k", P=3, lengths=(4096, 4096), d=4096, V=151936),
+    }
+
+
+@dataclasses.dataclass
+class SoftCEInputs:
+    """bf16 tensors on the CPU and the uint8 loss mask."""
+
+    h: torch.Tensor      # [P, T, d] draft hidden states
+    W: torch.Tensor      # [V, d] vocabulary head
+    y: torch.Tensor      # [T, V] teacher logits
+    mask: torch.Tensor   # [T] uint8, 1 = teacher position counted
+
+
+def make_softce_inputs(w: SoftCEWorkload) -> SoftCEInputs:
+    """One generator seeded with ``w.seed``, drawn in this order: h (N(0, 1), the scale
+    of a normalised hidden state), W (N(0, 1) / sqrt(d), so that a logit has unit scale
+    times 2), y (N(0, 1) times 3: a teacher sharper than the draft) and the mask
+    (Bernoulli(mask_keep)); the floating tensors are rounded to bf16."""
+    g = torch.Generator().manual_seed(w.seed)
+    h = torch.randn(w.P, w.T, w.d, generator=g).to(torch.bfloat16)
+    W = (torch.randn(w.V, w.d, generator=g) * (2.0 / w.d ** 0.5)).to(torch.bfloat16)
+    y = (torch.randn(w.T, w.V, generator=g) * 3.0).to(torch.bfloat16)
+    mask = (torch.rand(w.T, generator=g) < w.mask_keep).to(torch.uint8)
+    return SoftCEInputs(h, W, y, mask)
