@@ -92,6 +92,22 @@ class TTTRingDesc(ctypes.Structure):
     ]
 
 
+class TTTSoftceDesc(ctypes.Structure):
+    _fields_ = [
+        ("P", ctypes.c_int),
+        ("T", ctypes.c_int),
+        ("d", ctypes.c_int),
+        ("V", ctypes.c_int),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("nseq", ctypes.c_int),
+        ("loss_mask", ctypes.c_void_p),
+        ("pass_weight", ctypes.c_void_p),
+        ("pass_count", ctypes.c_void_p),
+        ("token_chunk_size", ctypes.c_int),
+        ("events", ctypes.c_void_p),
+    ]
+
+
 class TTTError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -169,6 +185,13 @@ def lib() -> ctypes.CDLL:
     L.ttt_ring_bwd_finish.restype = ctypes.c_int
     L.ttt_ring_dkv_finish.argtypes = [RD, vp, vp, vp, vp, vp]
     L.ttt_ring_dkv_finish.restype = ctypes.c_int
+    CD = P(TTTSoftceDesc)
+    L.ttt_softce_workspace_size.argtypes = [CD, ctypes.c_int]
+    L.ttt_softce_workspace_size.restype = sz
+    L.ttt_softce_fwd.argtypes = [CD, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.ttt_softce_fwd.restype = ctypes.c_int
+    L.ttt_softce_bwd.argtypes = [CD, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
+    L.ttt_softce_bwd.restype = ctypes.c_int
     L.ttt_status_string.argtypes = [ctypes.c_int]
     L.ttt_status_string.restype = ctypes.c_char_p
     L.ttt_attn_version.argtypes = []

@@ -315,6 +315,27 @@ struct EventScope {
 inline void clear_stale_error() { (void)cudaGetLastError(); }
 
 }  // namespace
+
+bool encode_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                   uint64_t s1_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    g_last_cuda_error.store(static_cast<int>(cudaErrorSymbolNotFound));
+    return false;
+  }
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {s1_bytes};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_cuda_error.store(kEncodeErrorBase + static_cast<int>(r));
+  return r == CUDA_SUCCESS;
+}
+
+uint64_t wait_budget_ns() { return g_wait_budget_ns.load(); }
+
+void record_cuda_error(int code) { g_last_cuda_error.store(code); }
 }  // namespace ttt
 
 using namespace ttt;

@@ -32,6 +32,11 @@ enum WaitSite : uint32_t {
   kSiteBwdDrain = 0x29,
   kSiteBwdSdpFree = 0x2a,
   kSiteBwdTicket = 0x2b,
+  kSiteCeFull = 0x40,
+  kSiteCeEmpty = 0x41,
+  kSiteCeAccFull = 0x42,
+  kSiteCeAccEmpty = 0x43,
+  kSiteCeDrain = 0x44,
 };
 
 // Where the sequences are: dense batches (cu_seqlens == nullptr) hold nseq = B
@@ -179,5 +184,28 @@ cudaError_t launch_ring_merge(int rows, int D, int H, int Lq, float* o_acc, floa
 cudaError_t launch_ring_finish(int64_t n, const float* o_acc, void* o, cudaStream_t stream);
 
 cudaError_t launch_watchdog_selftest(uint32_t* status, uint64_t budget_ns, cudaStream_t stream);
+
+// Arguments of the soft cross-entropy GEMM kernel (softce.cu).  Output tile rows are
+// draft rows row0 + m (STATS, DZ) or the GEMM's own rows (BF16, ACC).
+struct SoftceGemmArgs {
+  int M, N, K;              // output rows, output columns, reduction depth
+  int row0;                 // STATS / DZ: first draft row of this launch
+  int R;                    // draft rows in all (the stride of stats and lse)
+  int V;                    // vocabulary (teacher row length)
+  const int32_t* tidx;      // [R] teacher row of every draft row, -1 = invalid
+  const void* y;            // bf16 teacher logits [T][V]
+  float* stats;             // STATS: [ceil(V/256)][5][R] per-tile softmax statistics
+  const float* lse;         // DZ: [2][R] logsumexp of the draft and of the teacher row
+  const float* coef;        // DZ: [R] gradient coefficient g * w_p / N_p (0 = invalid)
+  uint32_t* status;
+  uint64_t budget_ns;
+};
+
+// Helpers of api.cu that the other host entry points share.
+// 2-D tensor map (dims and strides innermost first), box {b0, b1}.
+bool encode_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                   uint64_t s1_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw);
+uint64_t wait_budget_ns();
+void record_cuda_error(int code);
 
 }  // namespace ttt

@@ -260,6 +260,44 @@ def block_job(args, w, device, rank):
                unit_note="tokens = block tokens", name=w.name)
 
 
+SOFTCE_METRIC = "TTT draft soft cross-entropy loss fwd+bwd TFLOP/s at 1 B200; % of bf16 tensor peak"
+SOFTCE_KERNELS = {0: "rows_fwd", 1: "logits", 2: "reduce", 4: "dz", 5: "dh", 6: "dw"}
+
+
+def softce_job(args, w, device, rank):
+    from attention_pass_rope_b200 import softce as ce
+    inp = ttt_inputs.make_softce_inputs(dataclasses.replace(w, seed=w.seed + rank))
+    h, W, y, m = (t.to(device).contiguous() for t in (inp.h, inp.W, inp.y, inp.mask))
+    cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device=device)
+    chunk = args.chunk or 4096
+    R = w.P * w.T
+    nch = (R + chunk - 1) // chunk
+    need = max(ce.workspace_bytes(ce.make_desc(h, W, y, cu, m), False),
+               ce.workspace_bytes(ce.make_desc(h, W, y, cu, m, token_chunk_size=chunk), True))
+    ws = torch.empty(need, dtype=torch.uint8, device=device)
+    loss = torch.empty(w.P + 1, dtype=torch.float32, device=device)
+    rows = torch.empty(w.P, w.T, dtype=torch.float32, device=device)
+    lse = torch.empty(2, w.P, w.T, dtype=torch.float32, device=device)
+    dh = torch.empty_like(h)
+    dW = torch.zeros(w.V, w.d, dtype=torch.float32, device=device)
+
+    def step(events=None):
+        # the gradient of the head is accumulated across steps, as over micro-batches
+        ce.softce_fwd(h, W, y, cu_seqlens=cu, loss_mask=m, workspace=ws, events=events, out=(loss, rows, lse))
+        ce.softce_bwd(h, W, y, lse, cu_seqlens=cu, loss_mask=m, token_chunk_size=chunk, dW=dW, dh=dh,
+                      workspace=ws, events=events)
+
+    desc = (f"{w.name}: P={w.P} passes x T={w.T} tokens ({len(w.lengths)} sequences of {w.lengths[0]}), "
+            f"d={w.d}, V={w.V}, backward chunks of {chunk} rows ({nch} chunks), loss mask keep {w.mask_keep}")
+    return Job(step=step, ws=ws, host_src=(inp.h, inp.W, inp.y, inp.mask), dev_in=(h, W, y, m),
+               outputs=(loss, rows, lse, dh, dW), flops=w.flops_fwd_bwd(), tokens=w.T, desc=desc,
+               launches=4 + 1 + 3 * nch, unit_note="tokens = positions, each carrying P draft rows", name=w.name,
+               metric=SOFTCE_METRIC, kernel_names=SOFTCE_KERNELS, status=ce.device_status,
+               # dominant kernel: the dW GEMM (the largest share of the step); its per-launch
+               # work is one chunk's 2 * rows * V * d, timed at the first chunk
+               dom_kernel="dw", dom_flops=2.0 * min(chunk, R) * w.V * w.d)
+
+
 def run_ours(args, rank, world, local):
     from attention_pass_rope_b200 import _lib, ops
 
@@ -271,29 +309,34 @@ def run_ours(args, rank, world, local):
                                              device_id=device)
     if args.workload in ttt_inputs.block_workloads():
         job = block_job(args, ttt_inputs.block_workloads()[args.workload], device, rank)
+    elif args.workload in ttt_inputs.softce_workloads():
+        job = softce_job(args, ttt_inputs.softce_workloads()[args.workload], device, rank)
     else:
         job = ttt_job(args, workload(args), device, rank)
     step, ws = job.step, job.ws
+    names = getattr(job, "kernel_names", None) or {i: n for i, n in enumerate(_lib.KERNELS)
+                                                    if not n.startswith("unused")}
+    status = getattr(job, "status", None) or ops.device_status
 
     # per-kernel CUDA events, recorded by the library on the launching stream
     K = args.steps
     evs = [_lib.TTTEvents() for _ in range(K)]
     ev_objs = []
     for e in evs:
-        objs = []
-        for kk in range(len(_lib.KERNELS)):
+        objs = {}
+        for kk in names:
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()  # torch creates the CUDA event on first use; the library re-records it
             b.record()
             e.start[kk] = a.cuda_event
             e.stop[kk] = b.cuda_event
-            objs.append((a, b))
+            objs[kk] = (a, b)
         ev_objs.append(objs)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    st, word = ops.device_status(ws)
+    st, word = status(ws)
     if st != _lib.TTT_OK:
         raise RuntimeError(f"device status after warm-up: {st} {word:#x}")
 
@@ -316,11 +359,9 @@ def run_ours(args, rank, world, local):
     clocks = sampler.stop()
     ms = t0.elapsed_time(t1)
     per_kernel = {}
-    for kk, name in enumerate(_lib.KERNELS):
-        if name.startswith("unused"):
-            continue
+    for kk, name in names.items():
         per_kernel[name] = sum(ev_objs[i][kk][0].elapsed_time(ev_objs[i][kk][1]) for i in range(K)) / K
-    st, word = ops.device_status(ws)
+    st, word = status(ws)
     if st != _lib.TTT_OK:
         raise RuntimeError(f"device status after timing: {st} {word:#x}")
 
@@ -358,13 +399,14 @@ def run_ours(args, rank, world, local):
     tflops = whole_job_tflops(flops, world, ms_step)
     peaks, peak_src = load_peaks()
     peak, peak_kind = applicable_peak(peaks, peak_src, ms * 1e-3)
-    # dominant kernel: the trunk backward (tensor bound); its algorithmic flops per launch
-    # are 10*D per visible trunk pair per query head (and pass)
-    bwd_ms = per_kernel["trunk_bwd"]
-    achieved = job.trunk_bwd_flops / (bwd_ms * 1e-3) / 1e12
-    traffic = read_traffic("trunk_bwd", job.name)
+    # dominant kernel (tensor bound) and its algorithmic flops per launch: the trunk
+    # backward's 10*D per visible trunk pair per query head (and pass), or the job's own
+    dom = getattr(job, "dom_kernel", "trunk_bwd")
+    dom_flops = getattr(job, "dom_flops", None) or job.trunk_bwd_flops
+    achieved = dom_flops / (per_kernel[dom] * 1e-3) / 1e12
+    traffic = read_traffic(dom, job.name)
     line = {
-        "metric": METRIC,
+        "metric": getattr(job, "metric", METRIC),
         "value": round(tflops, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -384,7 +426,7 @@ def run_ours(args, rank, world, local):
         "peak": {"tflops": peak, "source": peak_kind, "pct_of_burst": round(100.0 * tflops / world / peaks["bf16_tflops"], 2),
                  "pct_of_sustained": round(100.0 * tflops / world / peaks["bf16_tflops_sustained"], 2)},
         "kernel_ms": {k_: round(v_, 4) for k_, v_ in per_kernel.items()},
-        "roofline": {"kernel": "trunk_bwd", "bound": "tensor", "achieved": round(achieved, 2),
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": peak_kind,
                      "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
@@ -398,6 +440,8 @@ def run_ours(args, rank, world, local):
     if rank == 0 and not args.no_cpu_baseline:
         if args.workload in ttt_inputs.block_workloads():
             line["cpu_baseline"] = block_cpu_baseline(ttt_inputs.block_workloads()[args.workload])
+        elif args.workload in ttt_inputs.softce_workloads():
+            line["cpu_baseline"] = softce_cpu_baseline(ttt_inputs.softce_workloads()[args.workload])
         else:
             line["cpu_baseline"] = cpu_baseline(workload(args), budget_s=args.cpu_budget)
     if world > 1:
@@ -499,14 +543,44 @@ def block_cpu_baseline(w):
                       f"workload, {dt:.1f} s", "seconds": round(dt, 2)}
 
 
+def softce_cpu_baseline(w, n_rows=8):
+    """The fp64 soft-CE oracle on n_rows draft rows of the workload (pass 0, the first valid
+    rows): their losses and dh, i.e. three 2*V*d passes per row (logits, logits again, dz W)."""
+    from oracle import softce_oracle as sco
+    inp = ttt_inputs.make_softce_inputs(w)
+    m = inp.mask.numpy().astype(bool)
+    idx = sco.teacher_index(w.cu_seqlens[:2], 1, m[:w.cu_seqlens[1]])
+    ts = [t for t in range(idx.shape[1]) if idx[0, t] >= 0][:n_rows]
+    hr = inp.h[0, ts]
+    yr = inp.y[[int(idx[0, t]) for t in ts]]
+    t0 = time.perf_counter()
+    sco.rows_forward(hr, inp.W, yr)
+    sco.rows_dh(hr, inp.W, yr, [1.0] * len(ts))
+    dt = time.perf_counter() - t0
+    fl = 3 * 2.0 * len(ts) * w.V * w.d
+    cores = blas_threads() or len(os.sched_getaffinity(0))
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 soft-CE oracle, loss and dh of {len(ts)} draft rows (of {w.P * w.T}), {dt:.1f} s",
+            "seconds": round(dt, 2)}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
+    metric = METRIC
+    sample = f"sequence 0, KV head 0 of {args.workload} per step"
     if args.workload in ttt_inputs.block_workloads():
         wb = ttt_inputs.block_workloads()[args.workload]
         runs = [block_cpu_baseline(wb) for _ in range(args.steps)]
         dt = sum(r["seconds"] for r in runs) / len(runs)
         value = sum(r["value"] for r in runs) / len(runs)
+    elif args.workload in ttt_inputs.softce_workloads():
+        ws_ = ttt_inputs.softce_workloads()[args.workload]
+        runs = [softce_cpu_baseline(ws_) for _ in range(args.steps)]
+        dt = sum(r["seconds"] for r in runs) / len(runs)
+        value = sum(r["value"] for r in runs) / len(runs)
+        metric = SOFTCE_METRIC
+        sample = runs[0]["sample"] + " per step"
     else:
         w = workload(args)
         # the oracle has no warm-up state; one untimed sample warms the BLAS pool
@@ -520,7 +594,7 @@ def run_reference(args, rank, world):
     cores = blas_threads() or len(os.sched_getaffinity(0))
     line = {
         "impl": "reference",
-        "metric": METRIC,
+        "metric": metric,
         "value": round(value, 6),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -534,7 +608,7 @@ def run_reference(args, rank, world):
         "data": "synthetic",
         "config": {"workload": args.workload, "parallelism": "cpu oracle, rank 0 only"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"sequence 0, KV head 0 of {args.workload} per step"},
+                         "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -547,7 +621,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(ttt_inputs.workloads()) + sorted(ttt_inputs.block_workloads()))
+                    choices=sorted(ttt_inputs.workloads()) + sorted(ttt_inputs.block_workloads()) +
+                    sorted(ttt_inputs.softce_workloads()))
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="soft-CE backward: draft rows per chunk (0: the pages' default, 4096)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=30.0)
     ap.add_argument("--batch", type=int, default=0, help="override B of a dense workload (profiling)")

@@ -351,6 +351,78 @@ ttt_status ttt_ring_bwd_finish(const ttt_ring_desc* desc, const void* qr, const 
 ttt_status ttt_ring_dkv_finish(const ttt_ring_desc* desc, const float* dk_acc, const float* dv_acc, void* dk,
                                void* dv, void* stream);
 
+/* ------------------------------------------------------------------------------
+ * Soft cross-entropy distillation loss of the draft passes.  Source: "DFlash/DSpark
+ * and EAGLE-3 TTT draft co-training ..." (NeMo-RL issue 3698), "What I'm working on",
+ * item 3 (the draft learns the target's distribution through a soft cross-entropy,
+ * computed in token chunks and split over the vocabulary, normalised per pass over
+ * the global batch) and item 2 (the draft rides the target's vocabulary head); the
+ * loss's token_chunk_size, default 4096 tokens: "bounded multi-pass EAGLE-3 TTT
+ * provider" (NeMo-RL PR 3725), merge note 3.
+ *
+ *   Draft row r = p*T + t (pass p = 0..P-1, token t of the packed tokens) has logits
+ *   z_r = W h_r (fp32 sums of bf16 products).  Its teacher position u = t + p must lie
+ *   in t's sequence and have loss_mask[u] != 0, else the row is invalid:
+ *     l_r = logsumexp(z_r) - sum_v softmax(y_u)_v z_r,v   (0 for an invalid row),
+ *     N_p = pass_count[p] if given, else the number of valid rows of pass p,
+ *     L_p = w_p / N_p * sum_t l_{p,t}  (0 if N_p = 0),   L = sum_p L_p.
+ *   Backward of grad * L: dz_r = grad * w_p / N_p * (softmax(z_r) - softmax(y_u)),
+ *   rounded to bf16; dh_r = W^T dz_r; dW += sum_r dz_r h_r^T.  The teacher y is not
+ *   differentiated.
+ *
+ * Layouts (device memory, row-major, 16-byte aligned): h bf16 [P][T][d], W bf16 [V][d],
+ * y bf16 [T][V], dh bf16 [P][T][d], dW fp32 [V][d].  Supported: d and V multiples of
+ * 8, P*T < 2^31.  Sequences: cu_seqlens (device int32[nseq+1]), or, when it is NULL,
+ * nseq equal sequences of T / nseq tokens (nseq = 0 or 1: one sequence).
+ * Ownership, asynchrony and errors are those of the attention calls: the caller owns
+ * every buffer, the calls enqueue on `stream` and return at once, the workspace's
+ * first word is the status word of the bounded in-kernel waits
+ * (ttt_attn_device_status).
+ * ------------------------------------------------------------------------------ */
+typedef struct {
+  int P;                         /* draft passes */
+  int T;                         /* tokens, all sequences back to back */
+  int d;                         /* hidden size */
+  int V;                         /* vocabulary */
+  const int32_t* cu_seqlens;     /* device int32[nseq+1], or NULL (see above) */
+  int nseq;
+  const uint8_t* loss_mask;      /* device uint8[T] over teacher positions; NULL: all counted */
+  const float* pass_weight;      /* device float[P]: w_p; NULL: all 1 */
+  const float* pass_count;       /* device float[P]: N_p (e.g. summed over ranks); NULL: counted here */
+  int token_chunk_size;          /* backward: draft rows per chunk of dz; 0 selects 4096 */
+  const ttt_attn_events* events; /* optional, indices TTT_SOFTCE_KERNEL_* */
+} ttt_softce_desc;
+
+/* Kernel indices of the soft-CE calls in ttt_attn_events (the backward's chunked
+ * kernels are timed at their first chunk). */
+enum {
+  TTT_SOFTCE_KERNEL_ROWS = 0,    /* teacher rows, pass counts (and coefficients) */
+  TTT_SOFTCE_KERNEL_LOGITS = 1,  /* forward logits GEMM with the softmax statistics */
+  TTT_SOFTCE_KERNEL_REDUCE = 2,  /* merge of the statistics, per-pass sums */
+  TTT_SOFTCE_KERNEL_DZ = 4,      /* backward: logits recomputed, dz */
+  TTT_SOFTCE_KERNEL_DH = 5,      /* dh = dz W */
+  TTT_SOFTCE_KERNEL_DW = 6       /* dW += dz^T h */
+};
+
+/* Bytes of workspace for ttt_softce_fwd (for_backward = 0) or ttt_softce_bwd (1); 0 if
+ * the descriptor is invalid.  256-byte aligned.  Forward: about 20 * P*T * ceil(V/256)
+ * bytes (the per-tile statistics); backward: about 2 * chunk * V bytes (one chunk of
+ * dz). */
+size_t ttt_softce_workspace_size(const ttt_softce_desc* desc, int for_backward);
+
+/* Forward.  Writes row_loss float[P*T] (l_r), lse float[2][P*T] (logsumexp of z_r,
+ * then of the teacher row y_u; 0 for an invalid row; the backward reads it) and loss
+ * float[P+1] (L_0 .. L_{P-1}, then L). */
+ttt_status ttt_softce_fwd(const ttt_softce_desc* desc, const void* h, const void* W, const void* y,
+                          float* row_loss, float* lse, float* loss, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Backward of grad * L, given the forward's lse.  Writes dh; adds to dW unless dW is
+ * NULL (then dW is not computed).  Visits the rows token_chunk_size at a time. */
+ttt_status ttt_softce_bwd(const ttt_softce_desc* desc, const void* h, const void* W, const void* y,
+                          const float* lse, float grad, void* dh, float* dW, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
 /* The error behind the most recent TTT_ERR_CUDA returned by any call in this
  * process: a cudaError_t value, or 100000 + the CUresult when encoding a TMA tensor
  * map failed; 0 if there was none.  Not reset by later successful calls. */

@@ -134,7 +134,7 @@ def backward(h, W, y, cu_seqlens, loss_mask=None, pass_weight=None, counts=None,
     dz = logit_grad(h, W, y, cu_seqlens, loss_mask, pass_weight, counts, grad)
     h, W = _f64(h), _f64(W)
     dh = dz @ W
-    dW = np.einsum("ptv,ptd->vd", dz, h)
+    dW = dz.reshape(-1, dz.shape[-1]).T @ h.reshape(-1, h.shape[-1])
     return dh, dW
 
 
@@ -149,3 +149,36 @@ def row_dh(h_row, W, y_row, coef):
     W = _f64(W)
     z = W @ _f64(h_row)
     return coef * ((_softmax(z) - _softmax(_f64(y_row))) @ W)
+
+
+def rows_logits(h_rows, W, slice_rows=16384):
+    """z [n, V] of a few draft rows h_rows [n, d] (fp64).  W is converted to fp64 a slice
+    of vocabulary rows at a time, so that a full-size head is never held in fp64; each
+    logit is the same dot product as in :func:`forward`."""
+    H = _f64(h_rows)
+    V = W.shape[0]
+    z = np.empty((H.shape[0], V))
+    for v0 in range(0, V, slice_rows):
+        Ws = _f64(W[v0:v0 + slice_rows])
+        z[:, v0:v0 + Ws.shape[0]] = H @ Ws.T
+    return z
+
+
+def rows_forward(h_rows, W, y_rows):
+    """(loss [n], lse [n]) of n valid pairs from their hidden states and teacher rows."""
+    z = rows_logits(h_rows, W)
+    y = _f64(y_rows)
+    loss = np.array([pair_loss(z[i], y[i]) for i in range(z.shape[0])])
+    return loss, _logsumexp(z)
+
+
+def rows_dh(h_rows, W, y_rows, coef, slice_rows=16384):
+    """dh [n, d] of n valid pairs with gradient coefficients coef [n] (grad * w_p / N_p)."""
+    z = rows_logits(h_rows, W, slice_rows)
+    dz = np.asarray(coef, dtype=np.float64)[:, None] * (_softmax(z) - _softmax(_f64(y_rows)))
+    V = W.shape[0]
+    dh = np.zeros((z.shape[0], W.shape[1]))
+    for v0 in range(0, V, slice_rows):
+        Ws = _f64(W[v0:v0 + slice_rows])
+        dh += dz[:, v0:v0 + Ws.shape[0]] @ Ws
+    return dh

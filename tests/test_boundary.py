@@ -204,3 +204,56 @@ def test_block_window_validation(L):
         assert L.ttt_block_workspace_size(ctypes.byref(block_desc(window=w)), 1) == full
     assert L.ttt_block_workspace_size(ctypes.byref(block_desc(window=-1)), 1) == 0
     assert ctypes.sizeof(_lib.TTTBlockDesc) % 8 == 0
+
+
+def softce_desc(**kw):
+    d = _lib.TTTSoftceDesc()
+    d.P, d.T, d.d, d.V = 3, 8192, 4096, 151936
+    d.nseq = 1
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_softce_workspace_sizes(L):
+    """Forward: status block, teacher rows, counts, then 5 floats per (row, 256-column
+    vocabulary tile); backward: rows, counts, coefficients and one chunk of bf16 dz
+    (4096 rows by default) at a row stride of V rounded up to 64."""
+    d = softce_desc()
+    R, ntn = 3 * 8192, (151936 + 255) // 256
+    fwd = L.ttt_softce_workspace_size(ctypes.byref(d), 0)
+    bwd = L.ttt_softce_workspace_size(ctypes.byref(d), 1)
+    assert fwd >= ntn * 5 * R * 4 and fwd - ntn * 5 * R * 4 < R * 4 + 4096
+    assert bwd >= 4096 * 151936 * 2 and bwd - 4096 * 151936 * 2 < 2 * R * 4 + 4096
+    d2 = softce_desc(token_chunk_size=100)
+    assert L.ttt_softce_workspace_size(ctypes.byref(d2), 1) < bwd
+
+
+def test_softce_rejects_bad_arguments(L):
+    """Every rejection happens before any CUDA call (this machine has no GPU)."""
+    ok = softce_desc()
+    assert L.ttt_softce_workspace_size(None, 0) == 0
+    for bad in (dict(P=0), dict(T=-1), dict(d=4), dict(V=0), dict(token_chunk_size=-1), dict(nseq=-1)):
+        assert L.ttt_softce_workspace_size(ctypes.byref(softce_desc(**bad)), 0) == 0, bad
+    # d or V not a multiple of 8: unsupported
+    for bad in (dict(d=4100), dict(V=151937)):
+        assert L.ttt_softce_workspace_size(ctypes.byref(softce_desc(**bad)), 1) == 0, bad
+    fake = ctypes.c_void_p(1 << 20)
+    vp = ctypes.c_void_p
+    # missing loss pointer, missing inputs, unaligned input, missing workspace
+    assert L.ttt_softce_fwd(ctypes.byref(ok), fake, fake, fake, fake, fake, None, fake, 1 << 40, None) == \
+        _lib.TTT_ERR_INVALID_ARG
+    assert L.ttt_softce_fwd(ctypes.byref(ok), None, fake, fake, fake, fake, fake, fake, 1 << 40, None) == \
+        _lib.TTT_ERR_INVALID_ARG
+    assert L.ttt_softce_fwd(ctypes.byref(ok), vp((1 << 20) + 2), fake, fake, fake, fake, fake, fake, 1 << 40,
+                            None) == _lib.TTT_ERR_INVALID_ARG
+    assert L.ttt_softce_fwd(ctypes.byref(ok), fake, fake, fake, fake, fake, fake, None, 1 << 40, None) == \
+        _lib.TTT_ERR_WORKSPACE
+    assert L.ttt_softce_fwd(ctypes.byref(ok), fake, fake, fake, fake, fake, fake, fake, 1024, None) == \
+        _lib.TTT_ERR_WORKSPACE
+    assert L.ttt_softce_bwd(ctypes.byref(ok), fake, fake, fake, fake, ctypes.c_float(float("nan")), fake, None,
+                            fake, 1 << 40, None) == _lib.TTT_ERR_INVALID_ARG
+    assert L.ttt_softce_bwd(ctypes.byref(ok), fake, fake, fake, None, ctypes.c_float(1.0), fake, None, fake,
+                            1 << 40, None) == _lib.TTT_ERR_INVALID_ARG
+    # a dense descriptor whose T is not a multiple of nseq
+    assert L.ttt_softce_workspace_size(ctypes.byref(softce_desc(nseq=3, T=8192)), 0) == 0

@@ -1,0 +1,186 @@
+"""GPU parity of the soft cross-entropy distillation loss (the library's kernels through
+the C ABI) against the fp64 oracle, on the same seeded inputs.
+
+Tolerances, from the arithmetic: the logits are fp32 sums of exact bf16 products and the
+softmax statistics fp32, so a row's loss and logsumexp are good to ~1e-5 in practice;
+LOSS_ATOL allows 1e-3.  The backward rounds dz to bf16 (relative 2^-9 per element)
+before the dh and dW GEMMs, so gradients are compared by relative L2 at 1e-2, overall
+and per pass."""
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import ttt_inputs as ti
+from attention_pass_rope_b200 import softce as ce
+from oracle import softce_oracle as sco
+
+pytestmark = pytest.mark.gpu
+
+LOSS_ATOL = 1e-3
+PASS_RTOL = 1e-4
+GRAD_RL2 = 1e-2
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def _cuda_opt(x, dtype):
+    return None if x is None else torch.tensor(x, dtype=dtype, device="cuda")
+
+
+def run_gpu(inp, cu, *, pass_weight=None, pass_count=None, grad=1.0, chunk=0, mask=True):
+    h, W, y = inp.h.cuda(), inp.W.cuda(), inp.y.cuda()
+    m = inp.mask.cuda() if mask else None
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    pw = _cuda_opt(pass_weight, torch.float32)
+    pc = _cuda_opt(pass_count, torch.float32)
+    loss, rows, lse = ce.softce_fwd(h, W, y, cu_seqlens=cu_t, loss_mask=m, pass_weight=pw, pass_count=pc)
+    dh, dW = ce.softce_bwd(h, W, y, lse, grad=grad, cu_seqlens=cu_t, loss_mask=m, pass_weight=pw, pass_count=pc,
+                           token_chunk_size=chunk)
+    torch.cuda.synchronize()
+    return loss.cpu().numpy(), rows.cpu().numpy(), lse.cpu().numpy(), dh.float().cpu().numpy(), dW.cpu().numpy()
+
+
+def compare(inp, cu, out, *, pass_weight=None, pass_count=None, grad=1.0, mask=True):
+    loss, rows, lse, dh, dW = out
+    P = inp.h.shape[0]
+    m = inp.mask.numpy().astype(bool) if mask else None
+    ref = sco.forward(inp.h, inp.W, inp.y, cu, m, pass_weight, pass_count)
+    idx = sco.teacher_index(cu, P, m)
+    valid = idx >= 0
+    if valid.any():
+        assert np.abs(rows[valid] - ref["rows"][valid]).max() <= LOSS_ATOL
+        assert np.abs(lse[0][valid] - ref["lse_z"][valid]).max() <= LOSS_ATOL
+        y64 = inp.y.double().numpy()
+        lse_y = scipy.special.logsumexp(y64[idx[valid]], axis=1)
+        assert np.abs(lse[1][valid] - lse_y).max() <= LOSS_ATOL
+    assert np.all(rows[~valid] == 0) and np.all(lse[:, ~valid] == 0)
+    np.testing.assert_allclose(loss[:P], ref["pass_loss"], rtol=PASS_RTOL, atol=1e-6)
+    assert loss[P] == pytest.approx(ref["loss"], rel=PASS_RTOL, abs=1e-6)
+    dh_ref, dW_ref = sco.backward(inp.h, inp.W, inp.y, cu, m, pass_weight, pass_count, grad)
+    if np.linalg.norm(dh_ref) == 0:
+        assert np.all(dh == 0) and np.all(dW == 0)
+        return
+    assert rel_l2(dh, dh_ref) <= GRAD_RL2
+    for p in range(P):
+        if np.linalg.norm(dh_ref[p]) > 0:
+            assert rel_l2(dh[p], dh_ref[p]) <= GRAD_RL2, p
+        else:
+            assert np.all(dh[p] == 0), p
+    assert rel_l2(dW, dW_ref) <= GRAD_RL2
+
+
+def test_softce_tiny():
+    w = ti.softce_workloads()["softce_tiny"]
+    inp = ti.make_softce_inputs(w)
+    compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens))
+
+
+def test_softce_tiny_chunks_weights_counts():
+    """Ragged backward chunks (100 rows: 7 full chunks and one of 68), pass weights, given
+    global counts and an upstream gradient."""
+    w = ti.softce_workloads()["softce_tiny"]
+    inp = ti.make_softce_inputs(w)
+    kw = dict(pass_weight=[1.0, 0.8, 0.64], pass_count=[500.0, 400.0, 300.0], grad=0.5)
+    compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens, chunk=100, **kw), **kw)
+
+
+def test_softce_mid():
+    """Several 128 x 256 tiles in every GEMM, a ragged last vocabulary tile (8200 =
+    32 * 256 + 8), eight K slices in the logits GEMM."""
+    w = ti.softce_workloads()["softce_mid"]
+    inp = ti.make_softce_inputs(w)
+    compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens, chunk=1000))
+
+
+def test_softce_dh_chunk_invariant_and_dw_accumulates():
+    w = ti.softce_workloads()["softce_tiny"]
+    inp = ti.make_softce_inputs(w)
+    h, W, y, m = inp.h.cuda(), inp.W.cuda(), inp.y.cuda(), inp.mask.cuda()
+    cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device="cuda")
+    _, _, lse = ce.softce_fwd(h, W, y, cu_seqlens=cu, loss_mask=m)
+    dh0, dW0 = ce.softce_bwd(h, W, y, lse, cu_seqlens=cu, loss_mask=m)
+    dh1, dW1 = ce.softce_bwd(h, W, y, lse, cu_seqlens=cu, loss_mask=m, token_chunk_size=37)
+    torch.cuda.synchronize()
+    # a row's dh depends on its own dz row only, reduced in the same order
+    assert torch.equal(dh0, dh1)
+    assert rel_l2(dW1.cpu().numpy(), dW0.cpu().numpy()) < 1e-5
+    # dW is added to
+    ce.softce_bwd(h, W, y, lse, cu_seqlens=cu, loss_mask=m, dW=dW1)
+    torch.cuda.synchronize()
+    assert rel_l2(dW1.cpu().numpy(), 2 * dW0.cpu().numpy()) < 1e-5
+    _, none = ce.softce_bwd(h, W, y, lse, cu_seqlens=cu, loss_mask=m, with_dw=False)
+    assert none is None
+
+
+def test_softce_degenerate_cases():
+    w = ti.softce_workloads()["softce_tiny"]
+    inp = ti.make_softce_inputs(w)
+    # every teacher position masked: no valid row, zero losses and gradients
+    inp0 = ti.SoftCEInputs(inp.h, inp.W, inp.y, torch.zeros_like(inp.mask))
+    out = run_gpu(inp0, w.cu_seqlens)
+    assert np.all(out[0] == 0) and np.all(out[1] == 0) and np.all(out[3] == 0) and np.all(out[4] == 0)
+    # one-token sequences: only pass 1 has valid rows
+    lengths = (1, 1, 1, 1, 1)
+    w1 = ti.SoftCEWorkload("one_token", P=3, lengths=lengths, d=64, V=264, seed=3)
+    inp1 = ti.make_softce_inputs(w1)
+    out1 = run_gpu(inp1, w1.cu_seqlens, mask=False)
+    assert out1[0][1] == 0 and out1[0][2] == 0
+    compare(inp1, w1.cu_seqlens, out1, mask=False)
+    # no tokens at all
+    h = torch.zeros(3, 0, 64, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(264, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(0, 264, dtype=torch.bfloat16, device="cuda")
+    loss, rows, lse = ce.softce_fwd(h, W, y)
+    dh, dW = ce.softce_bwd(h, W, y, lse)
+    torch.cuda.synchronize()
+    assert loss.abs().sum().item() == 0 and dh.numel() == 0 and dW.abs().sum().item() == 0
+
+
+@pytest.mark.slow
+def test_softce_qwen3_8b_4k_sampled_rows():
+    """The full-size workload (P = 3 over 2 x 4096 tokens, d = 4096, V = 151936) in the
+    launch configuration that the bench times (backward chunks of 4096 rows): sampled
+    rows' losses, logsumexps and dh against the oracle's few-rows forms, and properties
+    that hold at any size for the rest."""
+    w = ti.softce_workloads()["softce_qwen3_8b_4k"]
+    inp = ti.make_softce_inputs(w)
+    cu = w.cu_seqlens
+    loss, rows, lse, dh, dW = run_gpu(inp, cu, chunk=4096)
+    P, T = w.P, w.T
+    m = inp.mask.numpy().astype(bool)
+    idx = sco.teacher_index(cu, P, m)
+    counts = (idx >= 0).sum(axis=1)
+    # rows at tile edges (127/128 of a 128-row tile), chunk edges (4095/4096) and the ends
+    cand = [(0, 0), (0, 127), (0, 128), (1, 4095), (1, 4096), (2, 4094), (2, 8190), (0, 8191), (1, 3000),
+            (2, 5000), (0, 6143), (1, 6144)]
+    pairs = [(p, t) for p, t in cand if idx[p, t] >= 0]
+    assert len(pairs) >= 8
+    hr = torch.stack([inp.h[p, t] for p, t in pairs])
+    yr = torch.stack([inp.y[idx[p, t]] for p, t in pairs])
+    ref_loss, ref_lse = sco.rows_forward(hr, inp.W, yr)
+    got_loss = np.array([rows[p, t] for p, t in pairs])
+    got_lse = np.array([lse[0, p, t] for p, t in pairs])
+    assert np.abs(got_loss - ref_loss).max() <= LOSS_ATOL
+    assert np.abs(got_lse - ref_lse).max() <= LOSS_ATOL
+    coef = np.array([1.0 / counts[p] for p, t in pairs])
+    ref_dh = sco.rows_dh(hr, inp.W, yr, coef)
+    got_dh = np.stack([dh[p, t] for p, t in pairs])
+    assert rel_l2(got_dh, ref_dh) <= GRAD_RL2
+    for i in range(len(pairs)):
+        assert rel_l2(got_dh[i], ref_dh[i]) <= 2 * GRAD_RL2, pairs[i]
+    # invalid rows are zero; the pass losses are the normalised sums of the row losses
+    assert np.all(rows[idx < 0] == 0) and np.all(dh[idx < 0] == 0)
+    for p in range(P):
+        assert loss[p] == pytest.approx(rows[p].astype(np.float64).sum() / counts[p], rel=1e-5)
+    assert loss[P] == pytest.approx(loss[:P].sum(), rel=1e-6)
+    # dz rows sum to zero over the vocabulary up to their bf16 rounding: so do dW's columns
+    assert np.all(np.isfinite(dW))
+    col_sum = np.abs(dW.astype(np.float64).sum(axis=0))
+    col_abs = np.abs(dW.astype(np.float64)).sum(axis=0)
+    assert np.all(col_sum <= 1e-2 * col_abs + 1e-12)

@@ -204,3 +204,23 @@ def test_row_forms_match_the_full_forms():
         assert lse == pytest.approx(out["lse_z"][p, t], rel=1e-13)
         coef = 0.9 * [1.0, 0.5, 2.0][p] / n[p]
         assert np.allclose(sco.row_dh(h[p, t], W, y[u], coef), dh[p, t], rtol=1e-12, atol=1e-15)
+
+
+def test_sliced_row_forms_match_the_full_forms():
+    """The few-rows forms used at full size (vocabulary in slices) agree with the full
+    forms, with a slice size that leaves a ragged last slice."""
+    h, W, y, cu = _inputs(V=37, seed=19)
+    w = [1.0, 0.5, 2.0]
+    out = sco.forward(h, W, y, cu, pass_weight=w)
+    dh, _ = sco.backward(h, W, y, cu, pass_weight=w, grad=1.1)
+    idx = sco.teacher_index(cu, 3)
+    pairs = [(0, 2), (1, 7), (2, 15), (0, 18)]
+    hr = np.stack([h[p, t] for p, t in pairs])
+    yr = np.stack([y[idx[p, t]] for p, t in pairs])
+    coef = np.array([1.1 * w[p] / out["counts"][p] for p, t in pairs])
+    loss, lse = sco.rows_forward(hr, W, yr)
+    assert np.allclose(loss, [out["rows"][p, t] for p, t in pairs], rtol=1e-13)
+    assert np.allclose(lse, [out["lse_z"][p, t] for p, t in pairs], rtol=1e-13)
+    assert np.allclose(sco.rows_logits(hr, W, slice_rows=10), hr @ W.T, rtol=1e-14)
+    assert np.allclose(sco.rows_dh(hr, W, yr, coef, slice_rows=10), [dh[p, t] for p, t in pairs],
+                       rtol=1e-12, atol=1e-15)

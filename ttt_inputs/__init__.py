@@ -296,7 +296,7 @@ def softce_workloads() -> dict:
     """Distillation-loss workloads with the Qwen3-8B head (d = 4096, V = 151936)."""
     return {
         "softce_tiny": SoftCEWorkload("softce_tiny", P=3, lengths=(70, 129, 1, 56), d=128, V=1000),
-        "softce_mid": SoftCEWorkload("softce_mid", P=3, lengths=(700, 333, 1011), d=512, V=32771),
+        "softce_mid": SoftCEWorkload("softce_mid", P=3, lengths=(300, 129, 571), d=512, V=8200),
         "softce_qwen3_8b_4k": SoftCEWorkload("softce_qwen3_8b_4k", P=3, lengths=(4096, 4096), d=4096, V=151936),
     }
 
