@@ -298,6 +298,9 @@ def softce_workloads() -> dict:
         "softce_tiny": SoftCEWorkload("softce_tiny", P=3, lengths=(70, 129, 1, 56), d=128, V=1000),
         "softce_mid": SoftCEWorkload("softce_mid", P=3, lengths=(300, 129, 571), d=512, V=8200),
         "softce_qwen3_8b_4k": SoftCEWorkload("softce_qwen3_8b_4k", P=3, lengths=(4096, 4096), d=4096, V=151936),
+        # a 32K draft vocabulary (EAGLE-3 drafters may predict a reduced vocabulary): the
+        # profiling case of the same kernels, a few GB on the device
+        "softce_qwen3_8b_v32k": SoftCEWorkload("softce_qwen3_8b_v32k", P=3, lengths=(2048, 2048), d=4096, V=32768),
     }
 
 
