@@ -192,6 +192,8 @@ def lib() -> ctypes.CDLL:
     L.ttt_softce_fwd.restype = ctypes.c_int
     L.ttt_softce_bwd.argtypes = [CD, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
     L.ttt_softce_bwd.restype = ctypes.c_int
+    L.ttt_softce_fwd_bwd.argtypes = [CD, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.ttt_softce_fwd_bwd.restype = ctypes.c_int
     L.ttt_status_string.argtypes = [ctypes.c_int]
     L.ttt_status_string.restype = ctypes.c_char_p
     L.ttt_attn_version.argtypes = []

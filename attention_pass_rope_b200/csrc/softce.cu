@@ -15,9 +15,15 @@
 //   DZ     the same logits recomputed in the backward: dz = c_r (softmax(z) - q),
 //          rounded to bf16 and stored (one token chunk of rows at a time);
 //   BF16   dh = dz W (W as an MN-major operand), stored as bf16;
-//   ACC    dW += dz^T h (both operands MN-major), fp32 reduce-add by TMA.
+//   ACC    dW += dz^T h (both operands MN-major), fp32 reduce-add by TMA;
+//   STATSZ the forward's statistics, and the chunk's fp32 logits stored as well.
 // Small kernels finish the job: teacher rows and pass counts, the merge of the tile
-// statistics into lse and l, and the per-pass sums.
+// statistics into lse and l, the per-pass sums, and (fused call) dz from stored logits.
+//
+// The fused call (ttt_softce_fwd_bwd) takes the loss's upstream gradient up front: per
+// chunk of rows it runs the STATSZ GEMM, merges the statistics, turns the stored logits
+// into dz with one memory pass, then dh and dW.  That is three GEMM passes where separate
+// forward and backward calls need four (the backward recomputes the logits).
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -44,7 +50,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
-enum Epi { EPI_STATS = 0, EPI_DZ = 1, EPI_BF16 = 2, EPI_ACC = 3 };
+enum Epi { EPI_STATS = 0, EPI_DZ = 1, EPI_BF16 = 2, EPI_ACC = 3, EPI_STATSZ = 4 };
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
   asm volatile(
@@ -92,6 +98,47 @@ __device__ __forceinline__ void load_y8(const __nv_bfloat16* yrow, int col, int 
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = -INFINITY;
   }
+}
+
+// One 32-column slice of a row's logits v (fp32 bits) and of its teacher row: updates the
+// running maxima (log2 units) and sums of the draft and teacher softmaxes and sum e^(y-m) z.
+__device__ __forceinline__ void stats_update(const uint32_t (&v)[32], int col0, int V, const __nv_bfloat16* yrow,
+                                             float& mz, float& sz, float& my, float& sy, float& ac) {
+  float zl[32], yl[32];
+#pragma unroll
+  for (int g8 = 0; g8 < 4; ++g8) {
+    float y8[8];
+    load_y8(yrow, col0 + 8 * g8, V, y8);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * g8 + i;
+      zl[j] = col0 + j < V ? __uint_as_float(v[j]) * kLog2e : -INFINITY;
+      yl[j] = y8[i] * kLog2e;
+    }
+  }
+  float cz = zl[0], cy = yl[0];
+#pragma unroll
+  for (int j = 1; j < 31; j += 2) {
+    cz = max3f(cz, zl[j], zl[j + 1]);
+    cy = max3f(cy, yl[j], yl[j + 1]);
+  }
+  cz = fmaxf(cz, zl[31]);
+  cy = fmaxf(cy, yl[31]);
+  const float nz = fmaxf(mz, cz), ny = fmaxf(my, cy);
+  float ssz = 0.f, ssy = 0.f, sac = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    ssz += exp2_approx(zl[j] - nz);
+    const float e = exp2_approx(yl[j] - ny);
+    ssy += e;
+    sac = fmaf(e, col0 + j < V ? __uint_as_float(v[j]) : 0.f, sac);
+  }
+  const float fz = exp2_approx(mz - nz), fy = exp2_approx(my - ny);
+  sz = fmaf(sz, fz, ssz);
+  sy = fmaf(sy, fy, ssy);
+  ac = fmaf(ac, fy, sac);
+  mz = nz;
+  my = ny;
 }
 
 template <int EPI>
@@ -163,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(sa, &map_a, full + s, m0, k0);
             tma_load_2d(sa + kATile / 2, &map_a, full + s, m0 + 64, k0);
           } else {
-            tma_load_2d(sa, &map_a, full + s, k0, (EPI <= EPI_DZ ? a.row0 : 0) + m0);
+            tma_load_2d(sa, &map_a, full + s, k0, (EPI <= EPI_DZ || EPI == EPI_STATSZ ? a.row0 : 0) + m0);
           }
           if (B_MN) {
 #pragma unroll
@@ -230,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tacc = tmem + (static_cast<uint32_t>(32 * q) << 16) + b * kBN;
       const int r = m0 + row;  // output row of this thread
 
-      if (EPI == EPI_STATS) {
+      if (EPI == EPI_STATS || EPI == EPI_STATSZ) {
         const int u = r < a.M ? __ldg(a.tidx + a.row0 + r) : -1;
         const __nv_bfloat16* yrow = static_cast<const __nv_bfloat16*>(a.y) + static_cast<int64_t>(u < 0 ? 0 : u) * a.V;
         float mz = -INFINITY, sz = 0.f, my = -INFINITY, sy = 0.f, ac = 0.f;
@@ -242,44 +289,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tacc + 32 * c, v);
           tmem_ld_wait();
           reg_fence32(v);
-          if (u >= 0) {
-          float zl[32], yl[32];
+          if (EPI == EPI_STATSZ) {
+            // the fp32 logits of this row out through a swizzled slab and a TMA store
+            uint8_t* slab = slabs + (nslab & 1) * kSlab;
+            if (lane == 0) bulk_wait_read1();
+            __syncwarp();
+            uint8_t* rowp = slab + lane * 128;
 #pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) {
-            float y8[8];
-            load_y8(yrow, col0 + 8 * g8, a.V, y8);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int j = 8 * g8 + i;
-              const bool in = col0 + j < a.V;
-              zl[j] = in ? __uint_as_float(v[j]) * kLog2e : -INFINITY;
-              yl[j] = y8[i] * kLog2e;
+            for (int k = 0; k < 8; ++k)
+              *reinterpret_cast<uint4*>(rowp + ((k ^ (lane & 7)) << 4)) =
+                  make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&map_out, slab, col0, m0 + 32 * q);
+              bulk_commit();
             }
+            ++nslab;
           }
-          float cz = zl[0], cy = yl[0];
-#pragma unroll
-          for (int j = 1; j < 31; j += 2) {
-            cz = max3f(cz, zl[j], zl[j + 1]);
-            cy = max3f(cy, yl[j], yl[j + 1]);
-          }
-          cz = fmaxf(cz, zl[31]);
-          cy = fmaxf(cy, yl[31]);
-          const float nz = fmaxf(mz, cz), ny = fmaxf(my, cy);
-          float ssz = 0.f, ssy = 0.f, sac = 0.f;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            ssz += exp2_approx(zl[j] - nz);
-            const float e = exp2_approx(yl[j] - ny);
-            ssy += e;
-            sac = fmaf(e, col0 + j < a.V ? __uint_as_float(v[j]) : 0.f, sac);
-          }
-          const float fz = exp2_approx(mz - nz), fy = exp2_approx(my - ny);
-          sz = fmaf(sz, fz, ssz);
-          sy = fmaf(sy, fy, ssy);
-          ac = fmaf(ac, fy, sac);
-          mz = nz;
-          my = ny;
-          }
+          if (u >= 0) stats_update(v, col0, a.V, yrow, mz, sz, my, sy, ac);
         }
         tc_fence_before();
         __syncwarp();
@@ -458,36 +486,100 @@ __global__ void __launch_bounds__(1024) softce_rows_kernel(int P, int T, const i
 
 // Merge of the per-tile statistics of every row: lse of the draft logits and of the
 // teacher row, and the loss l = lse_z - (sum_v e^(y_v - M) z_v) / (sum_v e^(y_v - M)).
-__global__ void __launch_bounds__(256) softce_combine_kernel(int R, int ntn, const int32_t* tidx,
-                                                             const float* stats, float* row_loss, float* lse) {
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= R) return;
-  if (tidx[r] < 0) {
-    row_loss[r] = 0.f;
-    lse[r] = 0.f;
-    lse[static_cast<int64_t>(R) + r] = 0.f;
-    return;
-  }
-  float Mz = -INFINITY, Sz = 0.f, My = -INFINITY, Sy = 0.f, A = 0.f;
-  for (int n = 0; n < ntn; ++n) {
-    const float* st = stats + static_cast<int64_t>(n) * 5 * R + r;
-    const float mz = st[0], sz = st[R], my = st[2 * static_cast<int64_t>(R)];
-    const float sy = st[3 * static_cast<int64_t>(R)], ac = st[4 * static_cast<int64_t>(R)];
-    const float nz = fmaxf(Mz, mz);
+// A block takes 32 rows (threadIdx.x, so that every tile's 32 values are one coalesced
+// load) and kCombineSlices threads per row that merge interleaved tiles, then one
+// thread per row merges their results.
+constexpr int kCombineSlices = 16;
+
+__device__ __forceinline__ void merge_stats(float& Mz, float& Sz, float& My, float& Sy, float& A, float mz, float sz,
+                                            float my, float sy, float ac) {
+  const float nz = fmaxf(Mz, mz);
+  if (nz != -INFINITY) {
     Sz = Sz * exp2f(Mz - nz) + sz * exp2f(mz - nz);
     Mz = nz;
-    const float ny = fmaxf(My, my);
+  }
+  const float ny = fmaxf(My, my);
+  if (ny != -INFINITY) {
     const float f0 = exp2f(My - ny), f1 = exp2f(my - ny);
     Sy = Sy * f0 + sy * f1;
     A = A * f0 + ac * f1;
     My = ny;
   }
+}
+
+__global__ void __launch_bounds__(32 * kCombineSlices) softce_combine_kernel(int R, int ntn, int r0, int nrows,
+                                                                             const int32_t* tidx, const float* stats,
+                                                                             float* row_loss, float* lse) {
+  __shared__ float part[5][kCombineSlices][33];
+  const int i = blockIdx.x * 32 + threadIdx.x;
+  const int r = r0 + i;
+  const bool live = i < nrows && tidx[r] >= 0;
+  float Mz = -INFINITY, Sz = 0.f, My = -INFINITY, Sy = 0.f, A = 0.f;
+  if (live) {
+    for (int n = threadIdx.y; n < ntn; n += kCombineSlices) {
+      const float* st = stats + static_cast<int64_t>(n) * 5 * R + r;
+      merge_stats(Mz, Sz, My, Sy, A, st[0], st[R], st[2 * static_cast<int64_t>(R)], st[3 * static_cast<int64_t>(R)],
+                  st[4 * static_cast<int64_t>(R)]);
+    }
+  }
+  part[0][threadIdx.y][threadIdx.x] = Mz;
+  part[1][threadIdx.y][threadIdx.x] = Sz;
+  part[2][threadIdx.y][threadIdx.x] = My;
+  part[3][threadIdx.y][threadIdx.x] = Sy;
+  part[4][threadIdx.y][threadIdx.x] = A;
+  __syncthreads();
+  if (threadIdx.y != 0 || i >= nrows) return;
+  if (!live) {
+    row_loss[r] = 0.f;
+    lse[r] = 0.f;
+    lse[static_cast<int64_t>(R) + r] = 0.f;
+    return;
+  }
+  for (int k = 1; k < kCombineSlices; ++k)
+    merge_stats(Mz, Sz, My, Sy, A, part[0][k][threadIdx.x], part[1][k][threadIdx.x], part[2][k][threadIdx.x],
+                part[3][k][threadIdx.x], part[4][k][threadIdx.x]);
   constexpr float kLn2 = 0.6931471805599453f;
   const float lz = (Mz + log2f(Sz)) * kLn2;
   const float ly = (My + log2f(Sy)) * kLn2;
   row_loss[r] = lz - A / Sy;
   lse[r] = lz;
   lse[static_cast<int64_t>(R) + r] = ly;
+}
+
+// dz of rows r0 .. r0+nrows from their stored fp32 logits (fused call): one warp per row,
+// four columns per lane and step; dz = c_r (2^(z log2e - lse_z log2e) - 2^(y log2e -
+// lse_y log2e)) rounded to bf16, the same expression as the DZ epilogue (0 for a row with
+// c_r = 0).  z and dz rows are ldz elements apart.
+__global__ void __launch_bounds__(256) softce_dz_kernel(int R, int V, int ldz, int r0, int nrows,
+                                                        const int32_t* tidx, const float* coef, const float* lse,
+                                                        const __nv_bfloat16* y, const float* z, __nv_bfloat16* dz) {
+  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= nrows) return;
+  const int r = r0 + i;
+  const int u = tidx[r];
+  const float cf = u >= 0 ? coef[r] : 0.f;
+  uint2* out = reinterpret_cast<uint2*>(dz + static_cast<int64_t>(i) * ldz);
+  if (cf == 0.f) {
+    for (int c4 = lane; c4 < V / 4; c4 += 32) out[c4] = make_uint2(0u, 0u);
+    return;
+  }
+  const float lz = lse[r] * kLog2e, ly = lse[static_cast<int64_t>(R) + r] * kLog2e;
+  const float4* zr = reinterpret_cast<const float4*>(z + static_cast<int64_t>(i) * ldz);
+  const uint2* yr = reinterpret_cast<const uint2*>(y + static_cast<int64_t>(u) * V);
+#pragma unroll 4
+  for (int c4 = lane; c4 < V / 4; c4 += 32) {
+    const float4 zz = __ldcs(zr + c4);
+    const uint2 yy = __ldg(yr + c4);
+    const float zs[4] = {zz.x, zz.y, zz.z, zz.w};
+    const float ys[4] = {__uint_as_float(yy.x << 16), __uint_as_float(yy.x & 0xFFFF0000u),
+                         __uint_as_float(yy.y << 16), __uint_as_float(yy.y & 0xFFFF0000u)};
+    float d[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      d[k] = cf * (exp2_approx(fmaf(zs[k], kLog2e, -lz)) - exp2_approx(fmaf(ys[k], kLog2e, -ly)));
+    out[c4] = make_uint2(pack_bf16x2(d[0], d[1]), pack_bf16x2(d[2], d[3]));
+  }
 }
 
 // Per-pass sums in a fixed order: L_p = w_p / N_p * sum_t l_{p,t}, then L.
@@ -542,14 +634,15 @@ cudaError_t launch_gemm(const SoftceGemmArgs& a, const CUtensorMap& ma, const CU
 
 struct CePlan {
   int P, T, d, V, R, ntn, C, Vp;
-  size_t off_tidx, off_counts, off_coef, off_stats, off_dz, total;
+  size_t off_tidx, off_counts, off_coef, off_stats, off_z, off_dz, total;
 };
 
 constexpr size_t kCeAlign = 1024;
 inline size_t ce_align(size_t x) { return (x + kCeAlign - 1) / kCeAlign * kCeAlign; }
 
-ttt_status ce_plan(const ttt_softce_desc* d, int for_backward, CePlan* out) {
-  if (!d) return TTT_ERR_INVALID_ARG;
+// mode 0: forward, 1: backward, 2: the fused forward + backward
+ttt_status ce_plan(const ttt_softce_desc* d, int mode, CePlan* out) {
+  if (!d || mode < 0 || mode > 2) return TTT_ERR_INVALID_ARG;
   if (d->P < 1 || d->T < 0 || d->d < 8 || d->V < 8) return TTT_ERR_INVALID_ARG;
   if (d->d % 8 != 0 || d->V % 8 != 0) return TTT_ERR_UNSUPPORTED;
   if (d->token_chunk_size < 0 || d->nseq < 0) return TTT_ERR_INVALID_ARG;
@@ -570,12 +663,19 @@ ttt_status ce_plan(const ttt_softce_desc* d, int for_backward, CePlan* out) {
   pl.off_tidx = kCeAlign;  // the status word lives in the first block
   pl.off_counts = ce_align(pl.off_tidx + static_cast<size_t>(pl.R) * 4);
   const size_t after_counts = ce_align(pl.off_counts + static_cast<size_t>(pl.P) * 4);
-  if (!for_backward) {
+  const size_t stats_bytes = static_cast<size_t>(pl.ntn) * 5 * pl.R * 4;
+  if (mode == 0) {
     pl.off_stats = after_counts;
-    pl.total = pl.off_stats + static_cast<size_t>(pl.ntn) * 5 * pl.R * 4;
-  } else {
+    pl.total = pl.off_stats + stats_bytes;
+  } else if (mode == 1) {
     pl.off_coef = after_counts;
     pl.off_dz = ce_align(pl.off_coef + static_cast<size_t>(pl.R) * 4);
+    pl.total = pl.off_dz + static_cast<size_t>(pl.C) * pl.Vp * 2;
+  } else {
+    pl.off_coef = after_counts;
+    pl.off_stats = ce_align(pl.off_coef + static_cast<size_t>(pl.R) * 4);
+    pl.off_z = ce_align(pl.off_stats + stats_bytes);
+    pl.off_dz = ce_align(pl.off_z + static_cast<size_t>(pl.C) * pl.Vp * 4);
     pl.total = pl.off_dz + static_cast<size_t>(pl.C) * pl.Vp * 2;
   }
   *out = pl;
@@ -672,7 +772,8 @@ ttt_status ttt_softce_fwd(const ttt_softce_desc* desc, const void* h, const void
   }
   {
     CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_REDUCE, stream);
-    softce_combine_kernel<<<(pl.R + 255) / 256, 256, 0, stream>>>(pl.R, pl.ntn, tidx, stats, row_loss, lse);
+    softce_combine_kernel<<<(pl.R + 31) / 32, dim3(32, kCombineSlices), 0, stream>>>(pl.R, pl.ntn, 0, pl.R, tidx,
+                                                                                      stats, row_loss, lse);
     CE_CHECK(cudaGetLastError());
     softce_finalize_kernel<<<1, 1024, 0, stream>>>(pl.P, pl.T, row_loss, counts, desc->pass_weight, loss);
     CE_CHECK(cudaGetLastError());
@@ -763,6 +864,113 @@ ttt_status ttt_softce_bwd(const ttt_softce_desc* desc, const void* h, const void
       CE_CHECK(launch_gemm<EPI_ACC>(a, mz_mn, mh_mn, mdw, stream));
     }
   }
+  return TTT_OK;
+}
+
+ttt_status ttt_softce_fwd_bwd(const ttt_softce_desc* desc, const void* h, const void* W, const void* y, float grad,
+                              float* row_loss, float* lse, float* loss, void* dh, float* dW, void* workspace,
+                              size_t workspace_bytes, void* stream_) {
+  CePlan pl;
+  const ttt_status st = ce_plan(desc, 2, &pl);
+  if (st != TTT_OK) return st;
+  if (!loss) return TTT_ERR_INVALID_ARG;
+  if (pl.R > 0 && (!h || !W || !y || !row_loss || !lse || !dh)) return TTT_ERR_INVALID_ARG;
+  if (pl.R > 0 && (!aligned16(h) || !aligned16(W) || !aligned16(y) || !aligned16(dh) || (dW && !aligned16(dW))))
+    return TTT_ERR_INVALID_ARG;
+  if (!std::isfinite(grad)) return TTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return TTT_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  CE_CHECK(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  if (pl.R == 0) {
+    CE_CHECK(cudaMemsetAsync(loss, 0, sizeof(float) * (pl.P + 1), stream));
+    return TTT_OK;
+  }
+  int32_t* tidx = reinterpret_cast<int32_t*>(ws + pl.off_tidx);
+  float* counts = reinterpret_cast<float*>(ws + pl.off_counts);
+  float* coef = reinterpret_cast<float*>(ws + pl.off_coef);
+  float* stats = reinterpret_cast<float*>(ws + pl.off_stats);
+  float* zbuf = reinterpret_cast<float*>(ws + pl.off_z);
+  uint8_t* dz = ws + pl.off_dz;
+  {
+    CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_ROWS, stream);
+    softce_rows_kernel<<<pl.P, 1024, 0, stream>>>(pl.P, pl.T, desc->cu_seqlens, desc->nseq, desc->loss_mask,
+                                                 desc->pass_weight, desc->pass_count, grad, tidx, counts, coef);
+    CE_CHECK(cudaGetLastError());
+  }
+  const uint64_t hrow = static_cast<uint64_t>(pl.d) * 2, zrow = static_cast<uint64_t>(pl.Vp) * 2;
+  CUtensorMap mh, mw_k, mw_mn, mdw;
+  if (!encode_map_2d(&mh, kBf16, h, pl.d, pl.R, hrow, 64, 128, kSw128) ||
+      !encode_map_2d(&mw_k, kBf16, W, pl.d, pl.V, hrow, 64, 256, kSw128) ||
+      !encode_map_2d(&mw_mn, kBf16, W, pl.d, pl.V, hrow, 64, 64, kSw128))
+    return TTT_ERR_CUDA;
+  if (dW && !encode_map_2d(&mdw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, pl.d, pl.V, static_cast<uint64_t>(pl.d) * 4,
+                           32, 32, kSw128))
+    return TTT_ERR_CUDA;
+  SoftceGemmArgs base{};
+  base.R = pl.R;
+  base.V = pl.V;
+  base.tidx = tidx;
+  base.y = y;
+  base.stats = stats;
+  base.status = status;
+  base.budget_ns = wait_budget_ns();
+  for (int r0 = 0; r0 < pl.R; r0 += pl.C) {
+    const int c = pl.R - r0 < pl.C ? pl.R - r0 : pl.C;
+    const bool first = r0 == 0;
+    const uint8_t* hc = static_cast<const uint8_t*>(h) + static_cast<size_t>(r0) * hrow;
+    uint8_t* dhc = static_cast<uint8_t*>(dh) + static_cast<size_t>(r0) * hrow;
+    CUtensorMap mz_out, mz_k, mz_mn, mdh, mh_mn;
+    if (!encode_map_2d(&mz_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, zbuf, pl.V, c, static_cast<uint64_t>(pl.Vp) * 4, 32,
+                       32, kSw128) ||
+        !encode_map_2d(&mz_k, kBf16, dz, pl.V, c, zrow, 64, 128, kSw128) ||
+        !encode_map_2d(&mz_mn, kBf16, dz, pl.V, c, zrow, 64, 64, kSw128) ||
+        !encode_map_2d(&mdh, kBf16, dhc, pl.d, c, hrow, 64, 32, kSw128) ||
+        !encode_map_2d(&mh_mn, kBf16, hc, pl.d, c, hrow, 64, 64, kSw128))
+      return TTT_ERR_CUDA;
+    {
+      CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_LOGITS, stream, first);
+      SoftceGemmArgs a = base;
+      a.M = c;
+      a.N = pl.V;
+      a.K = pl.d;
+      a.row0 = r0;
+      CE_CHECK(launch_gemm<EPI_STATSZ>(a, mh, mw_k, mz_out, stream));
+    }
+    {
+      CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_REDUCE, stream, first);
+      softce_combine_kernel<<<(c + 31) / 32, dim3(32, kCombineSlices), 0, stream>>>(pl.R, pl.ntn, r0, c, tidx, stats,
+                                                                                   row_loss, lse);
+      CE_CHECK(cudaGetLastError());
+    }
+    {
+      CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_DZ, stream, first);
+      softce_dz_kernel<<<(c + 7) / 8, 256, 0, stream>>>(pl.R, pl.V, pl.Vp, r0, c, tidx, coef, lse,
+                                                        static_cast<const __nv_bfloat16*>(y), zbuf,
+                                                        reinterpret_cast<__nv_bfloat16*>(dz));
+      CE_CHECK(cudaGetLastError());
+    }
+    {
+      CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_DH, stream, first);
+      SoftceGemmArgs a = base;
+      a.M = c;
+      a.N = pl.d;
+      a.K = pl.V;
+      CE_CHECK(launch_gemm<EPI_BF16>(a, mz_k, mw_mn, mdh, stream));
+    }
+    if (dW) {
+      CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_DW, stream, first);
+      SoftceGemmArgs a = base;
+      a.M = pl.V;
+      a.N = pl.d;
+      a.K = c;
+      CE_CHECK(launch_gemm<EPI_ACC>(a, mz_mn, mh_mn, mdw, stream));
+    }
+  }
+  softce_finalize_kernel<<<1, 1024, 0, stream>>>(pl.P, pl.T, row_loss, counts, desc->pass_weight, loss);
+  CE_CHECK(cudaGetLastError());
   return TTT_OK;
 }
 

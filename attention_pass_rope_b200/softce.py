@@ -65,7 +65,8 @@ def make_desc(h, W, y, cu_seqlens=None, loss_mask=None, pass_weight=None, pass_c
     return desc
 
 
-def workspace_bytes(desc: _lib.TTTSoftceDesc, for_backward: bool) -> int:
+def workspace_bytes(desc: _lib.TTTSoftceDesc, for_backward) -> int:
+    """Workspace of the forward (0 / False), the backward (1 / True) or the fused call (2)."""
     n = _lib.lib().ttt_softce_workspace_size(ctypes.byref(desc), int(for_backward))
     if n == 0:
         raise _lib.TTTError(_lib.TTT_ERR_INVALID_ARG, "ttt_softce_workspace_size")
@@ -125,6 +126,42 @@ def softce_bwd(h, W, y, lse, *, grad: float = 1.0, cu_seqlens=None, loss_mask=No
                                          workspace.numel(), _stream()),
                "ttt_softce_bwd")
     return dh, dW
+
+
+def softce_fwd_bwd(h, W, y, *, grad: float = 1.0, cu_seqlens=None, loss_mask=None, pass_weight=None,
+                   pass_count=None, token_chunk_size: int = 0, with_dw: bool = True, dW=None, dh=None, out=None,
+                   workspace: Optional[torch.Tensor] = None, events=None):
+    """Forward and backward of grad * L in one sweep (the logits GEMM runs once): returns
+    (loss, row_loss, lse, dh, dW), the outputs of :func:`softce_fwd` and :func:`softce_bwd`."""
+    desc = make_desc(h, W, y, cu_seqlens, loss_mask, pass_weight, pass_count, token_chunk_size, events)
+    P, T = desc.P, desc.T
+    dev = h.device
+    if out is None:
+        loss = torch.empty(P + 1, dtype=torch.float32, device=dev)
+        row_loss = torch.empty(P, T, dtype=torch.float32, device=dev)
+        lse = torch.empty(2, P, T, dtype=torch.float32, device=dev)
+    else:
+        loss, row_loss, lse = out
+        for t, shape in ((loss, (P + 1,)), (row_loss, (P, T)), (lse, (2, P, T))):
+            if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"out tensors must be contiguous float32 of shapes {(P + 1,)}, {(P, T)}, {(2, P, T)}")
+    if dh is None:
+        dh = torch.empty_like(h)
+    elif dh.dtype != torch.bfloat16 or dh.shape != h.shape or not dh.is_contiguous():
+        raise ValueError("dh must be a contiguous bf16 tensor shaped like h")
+    if with_dw and dW is None:
+        dW = torch.zeros(desc.V, desc.d, dtype=torch.float32, device=dev)
+    if dW is not None and (dW.dtype != torch.float32 or tuple(dW.shape) != (desc.V, desc.d)
+                           or not dW.is_contiguous()):
+        raise ValueError("dW must be a contiguous float32 [V, d]")
+    need = workspace_bytes(desc, 2)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _lib.check(_lib.lib().ttt_softce_fwd_bwd(ctypes.byref(desc), _ptr(h), _ptr(W), _ptr(y), ctypes.c_float(grad),
+                                             _ptr(row_loss), _ptr(lse), _ptr(loss), _ptr(dh), _ptr(dW),
+                                             _ptr(workspace), workspace.numel(), _stream()),
+               "ttt_softce_fwd_bwd")
+    return loss, row_loss, lse, dh, dW
 
 
 def device_status(workspace: torch.Tensor) -> tuple:

@@ -261,7 +261,7 @@ def block_job(args, w, device, rank):
 
 
 SOFTCE_METRIC = "TTT draft soft cross-entropy loss fwd+bwd TFLOP/s at 1 B200; % of bf16 tensor peak"
-SOFTCE_KERNELS = {0: "rows_fwd", 1: "logits", 2: "reduce", 4: "dz", 5: "dh", 6: "dw"}
+SOFTCE_KERNELS = {0: "rows", 1: "logits", 2: "combine", 4: "dz", 5: "dh", 6: "dw"}
 
 
 def softce_job(args, w, device, rank):
@@ -272,8 +272,7 @@ def softce_job(args, w, device, rank):
     chunk = args.chunk or 4096
     R = w.P * w.T
     nch = (R + chunk - 1) // chunk
-    need = max(ce.workspace_bytes(ce.make_desc(h, W, y, cu, m), False),
-               ce.workspace_bytes(ce.make_desc(h, W, y, cu, m, token_chunk_size=chunk), True))
+    need = ce.workspace_bytes(ce.make_desc(h, W, y, cu, m, token_chunk_size=chunk), 2)
     ws = torch.empty(need, dtype=torch.uint8, device=device)
     loss = torch.empty(w.P + 1, dtype=torch.float32, device=device)
     rows = torch.empty(w.P, w.T, dtype=torch.float32, device=device)
@@ -282,16 +281,17 @@ def softce_job(args, w, device, rank):
     dW = torch.zeros(w.V, w.d, dtype=torch.float32, device=device)
 
     def step(events=None):
-        # the gradient of the head is accumulated across steps, as over micro-batches
-        ce.softce_fwd(h, W, y, cu_seqlens=cu, loss_mask=m, workspace=ws, events=events, out=(loss, rows, lse))
-        ce.softce_bwd(h, W, y, lse, cu_seqlens=cu, loss_mask=m, token_chunk_size=chunk, dW=dW, dh=dh,
-                      workspace=ws, events=events)
+        # the loss's forward and backward in one sweep (upstream gradient 1); the gradient of
+        # the head is accumulated across steps, as over micro-batches
+        ce.softce_fwd_bwd(h, W, y, cu_seqlens=cu, loss_mask=m, token_chunk_size=chunk, dW=dW, dh=dh,
+                          out=(loss, rows, lse), workspace=ws, events=events)
 
     desc = (f"{w.name}: P={w.P} passes x T={w.T} tokens ({len(w.lengths)} sequences of {w.lengths[0]}), "
-            f"d={w.d}, V={w.V}, backward chunks of {chunk} rows ({nch} chunks), loss mask keep {w.mask_keep}")
+            f"d={w.d}, V={w.V}, fused forward + backward in chunks of {chunk} rows ({nch} chunks), "
+            f"loss mask keep {w.mask_keep}; work = logits, dh and dW GEMMs")
     return Job(step=step, ws=ws, host_src=(inp.h, inp.W, inp.y, inp.mask), dev_in=(h, W, y, m),
                outputs=(loss, rows, lse, dh, dW), flops=w.flops_fwd_bwd(), tokens=w.T, desc=desc,
-               launches=4 + 1 + 3 * nch, unit_note="tokens = positions, each carrying P draft rows", name=w.name,
+               launches=2 + 5 * nch, unit_note="tokens = positions, each carrying P draft rows", name=w.name,
                metric=SOFTCE_METRIC, kernel_names=SOFTCE_KERNELS, status=ce.device_status,
                # dominant kernel: the dW GEMM (the largest share of the step); its per-launch
                # work is one chunk's 2 * rows * V * d, timed at the first chunk

@@ -397,17 +397,18 @@ typedef struct {
  * kernels are timed at their first chunk). */
 enum {
   TTT_SOFTCE_KERNEL_ROWS = 0,    /* teacher rows, pass counts (and coefficients) */
-  TTT_SOFTCE_KERNEL_LOGITS = 1,  /* forward logits GEMM with the softmax statistics */
-  TTT_SOFTCE_KERNEL_REDUCE = 2,  /* merge of the statistics, per-pass sums */
-  TTT_SOFTCE_KERNEL_DZ = 4,      /* backward: logits recomputed, dz */
+  TTT_SOFTCE_KERNEL_LOGITS = 1,  /* forward logits GEMM with the softmax statistics (fused: and the logits) */
+  TTT_SOFTCE_KERNEL_REDUCE = 2,  /* merge of the statistics, per-pass sums (fused: the merge) */
+  TTT_SOFTCE_KERNEL_DZ = 4,      /* backward: logits recomputed, dz (fused: dz from the stored logits) */
   TTT_SOFTCE_KERNEL_DH = 5,      /* dh = dz W */
   TTT_SOFTCE_KERNEL_DW = 6       /* dW += dz^T h */
 };
 
-/* Bytes of workspace for ttt_softce_fwd (for_backward = 0) or ttt_softce_bwd (1); 0 if
- * the descriptor is invalid.  256-byte aligned.  Forward: about 20 * P*T * ceil(V/256)
- * bytes (the per-tile statistics); backward: about 2 * chunk * V bytes (one chunk of
- * dz). */
+/* Bytes of workspace for ttt_softce_fwd (for_backward = 0), ttt_softce_bwd (1) or
+ * ttt_softce_fwd_bwd (2); 0 if the descriptor is invalid.  256-byte aligned.  Forward:
+ * about 20 * P*T * ceil(V/256) bytes (the per-tile statistics); backward: about
+ * 2 * chunk * V bytes (one chunk of dz); fused: both, plus 4 * chunk * V bytes (one chunk
+ * of fp32 logits). */
 size_t ttt_softce_workspace_size(const ttt_softce_desc* desc, int for_backward);
 
 /* Forward.  Writes row_loss float[P*T] (l_r), lse float[2][P*T] (logsumexp of z_r,
@@ -422,6 +423,15 @@ ttt_status ttt_softce_fwd(const ttt_softce_desc* desc, const void* h, const void
 ttt_status ttt_softce_bwd(const ttt_softce_desc* desc, const void* h, const void* W, const void* y,
                           const float* lse, float grad, void* dh, float* dW, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/* Forward and backward in one sweep, for a caller that knows the loss's upstream gradient
+ * `grad` before the forward (a loss's is usually 1).  Same outputs as ttt_softce_fwd
+ * followed by ttt_softce_bwd with that grad, bit for bit.  Per chunk of token_chunk_size
+ * rows it keeps the chunk's fp32 logits in the workspace and derives dz from them, so the
+ * logits GEMM runs once instead of twice. */
+ttt_status ttt_softce_fwd_bwd(const ttt_softce_desc* desc, const void* h, const void* W, const void* y, float grad,
+                              float* row_loss, float* lse, float* loss, void* dh, float* dW, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /* The error behind the most recent TTT_ERR_CUDA returned by any call in this
  * process: a cudaError_t value, or 100000 + the CUresult when encoding a TMA tensor

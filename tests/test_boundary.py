@@ -227,6 +227,11 @@ def test_softce_workspace_sizes(L):
     assert bwd >= 4096 * 151936 * 2 and bwd - 4096 * 151936 * 2 < 2 * R * 4 + 4096
     d2 = softce_desc(token_chunk_size=100)
     assert L.ttt_softce_workspace_size(ctypes.byref(d2), 1) < bwd
+    # fused: statistics, coefficients, one chunk of fp32 logits and one of bf16 dz
+    fused = L.ttt_softce_workspace_size(ctypes.byref(d), 2)
+    assert fused >= ntn * 5 * R * 4 + 4096 * 151936 * 6
+    assert fused - (ntn * 5 * R * 4 + 4096 * 151936 * 6) < 2 * R * 4 + 8192
+    assert L.ttt_softce_workspace_size(ctypes.byref(d), 3) == 0
 
 
 def test_softce_rejects_bad_arguments(L):
@@ -255,5 +260,9 @@ def test_softce_rejects_bad_arguments(L):
                             fake, 1 << 40, None) == _lib.TTT_ERR_INVALID_ARG
     assert L.ttt_softce_bwd(ctypes.byref(ok), fake, fake, fake, None, ctypes.c_float(1.0), fake, None, fake,
                             1 << 40, None) == _lib.TTT_ERR_INVALID_ARG
+    assert L.ttt_softce_fwd_bwd(ctypes.byref(ok), fake, fake, fake, ctypes.c_float(1.0), fake, fake, None, fake,
+                                None, fake, 1 << 40, None) == _lib.TTT_ERR_INVALID_ARG
+    assert L.ttt_softce_fwd_bwd(ctypes.byref(ok), fake, fake, fake, ctypes.c_float(1.0), fake, fake, fake, fake,
+                                None, fake, 1024, None) == _lib.TTT_ERR_WORKSPACE
     # a dense descriptor whose T is not a multiple of nseq
     assert L.ttt_softce_workspace_size(ctypes.byref(softce_desc(nseq=3, T=8192)), 0) == 0

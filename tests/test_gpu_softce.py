@@ -33,15 +33,18 @@ def _cuda_opt(x, dtype):
     return None if x is None else torch.tensor(x, dtype=dtype, device="cuda")
 
 
-def run_gpu(inp, cu, *, pass_weight=None, pass_count=None, grad=1.0, chunk=0, mask=True):
+def run_gpu(inp, cu, *, pass_weight=None, pass_count=None, grad=1.0, chunk=0, mask=True, fused=False):
     h, W, y = inp.h.cuda(), inp.W.cuda(), inp.y.cuda()
     m = inp.mask.cuda() if mask else None
     cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
     pw = _cuda_opt(pass_weight, torch.float32)
     pc = _cuda_opt(pass_count, torch.float32)
-    loss, rows, lse = ce.softce_fwd(h, W, y, cu_seqlens=cu_t, loss_mask=m, pass_weight=pw, pass_count=pc)
-    dh, dW = ce.softce_bwd(h, W, y, lse, grad=grad, cu_seqlens=cu_t, loss_mask=m, pass_weight=pw, pass_count=pc,
-                           token_chunk_size=chunk)
+    kw = dict(cu_seqlens=cu_t, loss_mask=m, pass_weight=pw, pass_count=pc)
+    if fused:
+        loss, rows, lse, dh, dW = ce.softce_fwd_bwd(h, W, y, grad=grad, token_chunk_size=chunk, **kw)
+    else:
+        loss, rows, lse = ce.softce_fwd(h, W, y, **kw)
+        dh, dW = ce.softce_bwd(h, W, y, lse, grad=grad, token_chunk_size=chunk, **kw)
     torch.cuda.synchronize()
     return loss.cpu().numpy(), rows.cpu().numpy(), lse.cpu().numpy(), dh.float().cpu().numpy(), dW.cpu().numpy()
 
@@ -98,6 +101,25 @@ def test_softce_mid():
     compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens, chunk=1000))
 
 
+def test_softce_fused_equals_separate_calls():
+    """The fused call gives the separate calls' outputs bit for bit (the same logits, the
+    same dz expression, the same GEMMs), and the oracle's values."""
+    w = ti.softce_workloads()["softce_tiny"]
+    inp = ti.make_softce_inputs(w)
+    kw = dict(pass_weight=[1.0, 0.8, 0.64], pass_count=[500.0, 400.0, 300.0], grad=0.5)
+    sep = run_gpu(inp, w.cu_seqlens, chunk=100, **kw)
+    fus = run_gpu(inp, w.cu_seqlens, chunk=100, fused=True, **kw)
+    for a, b in zip(sep, fus):
+        assert np.array_equal(a, b)
+    compare(inp, w.cu_seqlens, fus, **kw)
+
+
+def test_softce_fused_mid():
+    w = ti.softce_workloads()["softce_mid"]
+    inp = ti.make_softce_inputs(w)
+    compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens, chunk=1000, fused=True))
+
+
 def test_softce_dh_chunk_invariant_and_dw_accumulates():
     w = ti.softce_workloads()["softce_tiny"]
     inp = ti.make_softce_inputs(w)
@@ -138,20 +160,25 @@ def test_softce_degenerate_cases():
     y = torch.zeros(0, 264, dtype=torch.bfloat16, device="cuda")
     loss, rows, lse = ce.softce_fwd(h, W, y)
     dh, dW = ce.softce_bwd(h, W, y, lse)
+    loss2, _, _, dh2, dW2 = ce.softce_fwd_bwd(h, W, y)
     torch.cuda.synchronize()
     assert loss.abs().sum().item() == 0 and dh.numel() == 0 and dW.abs().sum().item() == 0
+    assert loss2.abs().sum().item() == 0 and dW2.abs().sum().item() == 0
+    # fused, every position masked
+    out0 = run_gpu(inp0, w.cu_seqlens, fused=True)
+    assert all(np.all(x == 0) for x in (out0[0], out0[1], out0[3], out0[4]))
 
 
 @pytest.mark.slow
 def test_softce_qwen3_8b_4k_sampled_rows():
     """The full-size workload (P = 3 over 2 x 4096 tokens, d = 4096, V = 151936) in the
-    launch configuration that the bench times (backward chunks of 4096 rows): sampled
+    launch configuration that the bench times (the fused call, chunks of 4096 rows): sampled
     rows' losses, logsumexps and dh against the oracle's few-rows forms, and properties
     that hold at any size for the rest."""
     w = ti.softce_workloads()["softce_qwen3_8b_4k"]
     inp = ti.make_softce_inputs(w)
     cu = w.cu_seqlens
-    loss, rows, lse, dh, dW = run_gpu(inp, cu, chunk=4096)
+    loss, rows, lse, dh, dW = run_gpu(inp, cu, chunk=4096, fused=True)
     P, T = w.P, w.T
     m = inp.mask.numpy().astype(bool)
     idx = sco.teacher_index(cu, P, m)

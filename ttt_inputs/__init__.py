@@ -288,8 +288,9 @@ class SoftCEWorkload:
         return 2.0 * self.P * self.T * self.d * self.V
 
     def flops_fwd_bwd(self, with_dw: bool = True) -> float:
-        """Forward logits, recomputed logits, dh and (optionally) dW: 2 * d * V each per row."""
-        return self.flops_fwd() * (4.0 if with_dw else 3.0)
+        """The algorithmic work of forward and backward: the logits, dh and (optionally) dW,
+        2 * d * V each per row (a recomputation of the logits is not counted)."""
+        return self.flops_fwd() * (3.0 if with_dw else 2.0)
 
 
 def softce_workloads() -> dict:
