@@ -221,7 +221,8 @@ def ttt_job(args, w, device, rank):
             if w.dense else
             f"{w.name}: THD nseq={w.nseq} T={w.T} P={w.P} H={w.H}/{w.Hkv} D={w.D} theta={w.theta:g}")
     return Job(step=step, ws=ws, host_src=(inp.q, inp.k, inp.v, inp.do), dev_in=(q, k, v, do),
-               outputs=(o, lse, dq, dk, dv), flops=w.flops_fwd_bwd(),
+               outputs=(o, lse, dq, dk, dv), flops=w.flops_fwd_bwd(), flops_12d=w.flops_fwd_bwd(per_pair=12),
+               query_tokens=w.P * w.T,
                trunk_bwd_flops=10 * w.D * w.trunk_pairs * w.H * w.P, tokens=w.T, desc=desc,
                launches=5, unit_note="tokens = B*S (or T) positions, each carrying P passes", name=w.name)
 
@@ -256,6 +257,7 @@ def block_job(args, w, device, rank):
             f"theta={w.theta:g}, anchors sorted uniform")
     return Job(step=step, ws=ws, host_src=(inp.k_ctx, inp.v_ctx, inp.qb, inp.kb, inp.vb, inp.do),
                dev_in=(k_ctx, v_ctx, qb, kb, vb, do), outputs=(o, lse) + grads, flops=w.flops_fwd_bwd(a),
+               flops_12d=w.flops_fwd_bwd(a, per_pair=12),
                trunk_bwd_flops=10 * w.D * trunk_pairs * w.H, tokens=w.NB * w.Bs, desc=desc, launches=6,
                unit_note="tokens = block tokens", name=w.name)
 
@@ -422,6 +424,12 @@ def run_ours(args, rank, world, local):
                    "flops_per_step": flops, "parallelism": f"replicas{world}",
                    "l2": "inputs per step (%.0f MB) exceed L2 (126 MB)" % (h2d / 1e6)},
         "tokens_per_s": round(job.tokens * world / (ms_step * 1e-3), 1),
+        # the stricter count without the backward's recomputed Q K^T (12*D per pair), and
+        # P*B*S query-tokens/s (every position carries P passes)
+        **({"tflops_12d": round(whole_job_tflops(job.flops_12d, world, ms_step), 2)}
+           if getattr(job, "flops_12d", None) else {}),
+        **({"query_tokens_per_s": round(job.query_tokens * world / (ms_step * 1e-3), 1)}
+           if getattr(job, "query_tokens", None) else {}),
         "pct_of_peak": round(100.0 * tflops / world / peak, 2),
         "peak": {"tflops": peak, "source": peak_kind, "pct_of_burst": round(100.0 * tflops / world / peaks["bf16_tflops"], 2),
                  "pct_of_sustained": round(100.0 * tflops / world / peaks["bf16_tflops_sustained"], 2)},

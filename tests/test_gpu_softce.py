@@ -169,6 +169,45 @@ def test_softce_degenerate_cases():
     assert all(np.all(x == 0) for x in (out0[0], out0[1], out0[3], out0[4]))
 
 
+def test_softce_ragged_hidden_size():
+    """d = 72: a partial last K slice in the logits GEMM (64 + 8), a partial column tile in
+    dh and dW, and a partial 32-column slice at the end of the vocabulary (V = 264)."""
+    w = ti.SoftCEWorkload("d72", P=2, lengths=(40, 97), d=72, V=264, seed=5)
+    inp = ti.make_softce_inputs(w)
+    compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens, chunk=50))
+    compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens, chunk=50, fused=True))
+
+
+def test_softce_dense_sequences_without_cu_seqlens():
+    """A dense batch described by nseq equal sequences (no cu_seqlens): the same results as
+    the packed description of the same tokens."""
+    import ctypes
+    from attention_pass_rope_b200 import _lib
+    w = ti.SoftCEWorkload("dense3", P=3, lengths=(60, 60, 60), d=64, V=512, seed=9)
+    inp = ti.make_softce_inputs(w)
+    h, W, y, m = inp.h.cuda(), inp.W.cuda(), inp.y.cuda(), inp.mask.cuda()
+    desc = ce.make_desc(h, W, y, None, m)
+    desc.nseq = 3
+    P, T = w.P, w.T
+    loss = torch.empty(P + 1, device="cuda")
+    rows = torch.empty(P, T, device="cuda")
+    lse = torch.empty(2, P, T, device="cuda")
+    dh = torch.empty_like(h)
+    dW = torch.zeros(w.V, w.d, device="cuda")
+    ws = torch.empty(ce.workspace_bytes(desc, 2), dtype=torch.uint8, device="cuda")
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    _lib.check(_lib.lib().ttt_softce_fwd_bwd(ctypes.byref(desc), ptr(h), ptr(W), ptr(y), ctypes.c_float(1.0),
+                                             ptr(rows), ptr(lse), ptr(loss), ptr(dh), ptr(dW), ptr(ws), ws.numel(),
+                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)),
+               "ttt_softce_fwd_bwd")
+    torch.cuda.synchronize()
+    out = (loss.cpu().numpy(), rows.cpu().numpy(), lse.cpu().numpy(), dh.float().cpu().numpy(), dW.cpu().numpy())
+    compare(inp, w.cu_seqlens, out)
+    packed = run_gpu(inp, w.cu_seqlens, fused=True)
+    for a, b in zip(out, packed):
+        assert np.array_equal(a, b)
+
+
 @pytest.mark.slow
 def test_softce_qwen3_8b_4k_sampled_rows():
     """The full-size workload (P = 3 over 2 x 4096 tokens, d = 4096, V = 151936) in the
