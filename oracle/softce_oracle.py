@@ -36,9 +36,16 @@ The pages name the loss and nothing of its formula.  Readings where they are sil
 * The token chunk size changes only the order in which an implementation visits the
   pairs, not the values; the oracle takes all pairs at once.
 
+* Per-slot normalisation (same item): block drafters normalise per slot of a block
+  instead of per pass.  The general form takes, for every draft row, its teacher
+  position (or -1) and its normalisation group: L_g = w_g / N_g * sum over the valid
+  rows of group g, L = sum_g L_g.  The TTT passes are the case group = pass, teacher =
+  t + p - 1 (:func:`ttt_mapping`).
+
 Array conventions: h [P, T, d] (pass-major, tokens of all sequences concatenated,
 ``cu_seqlens`` their boundaries); W [V, d]; y [T, V]; loss_mask [T] (teacher
-positions), 1 = counted.  Inputs are taken as given (bf16 values in fp64).
+positions), 1 = counted.  The general form: draft rows h [R, d], y [Ty, V], loss_mask
+[Ty], teacher [R], group [R].  Inputs are taken as given (bf16 values in fp64).
 """
 
 from __future__ import annotations
@@ -182,3 +189,52 @@ def rows_dh(h_rows, W, y_rows, coef, slice_rows=16384):
         Ws = _f64(W[v0:v0 + slice_rows])
         dh += dz[:, v0:v0 + Ws.shape[0]] @ Ws
     return dh
+
+
+def ttt_mapping(cu_seqlens, P):
+    """(teacher [P*T], group [P*T]) of the TTT passes in the general form: row p*T + t
+    learns position t + p of its sequence (or nothing), in group p."""
+    idx = teacher_index(cu_seqlens, P)
+    T = idx.shape[1]
+    return idx.reshape(-1), np.repeat(np.arange(P), T)
+
+
+def forward_mapped(h_rows, W, y, teacher, group, ngroups, loss_mask=None, group_weight=None, counts=None):
+    """The loss with an explicit teacher position and normalisation group per draft row.
+    Returns a dict: ``rows`` [R], ``lse_z`` [R], ``group_loss`` [G], ``loss``, ``counts`` [G]."""
+    h, W, y = _f64(h_rows), _f64(W), _f64(y)
+    teacher = np.asarray(teacher, dtype=np.int64)
+    group = np.asarray(group, dtype=np.int64)
+    Ty = y.shape[0]
+    valid = (teacher >= 0) & (teacher < Ty)
+    if loss_mask is not None:
+        m = np.asarray(loss_mask).astype(bool)
+        valid &= np.array([bool(m[u]) if 0 <= u < Ty else False for u in teacher])
+    z = h @ W.T
+    lse_z = _logsumexp(z)
+    rows = np.zeros(h.shape[0])
+    for r in np.nonzero(valid)[0]:
+        rows[r] = pair_loss(z[r], y[teacher[r]])
+    w = np.ones(ngroups) if group_weight is None else np.asarray(group_weight, dtype=np.float64)
+    n = (np.array([np.sum(valid & (group == g)) for g in range(ngroups)], dtype=np.float64)
+         if counts is None else np.asarray(counts, dtype=np.float64))
+    gl = np.array([w[g] / n[g] * rows[group == g].sum() if n[g] > 0 else 0.0 for g in range(ngroups)])
+    return {"rows": rows, "lse_z": lse_z, "group_loss": gl, "loss": float(gl.sum()), "counts": n, "valid": valid}
+
+
+def backward_mapped(h_rows, W, y, teacher, group, ngroups, loss_mask=None, group_weight=None, counts=None,
+                    grad=1.0):
+    """(dh [R, d], dW [V, d]) of grad * L in the general form."""
+    out = forward_mapped(h_rows, W, y, teacher, group, ngroups, loss_mask, group_weight, counts)
+    h, W, y = _f64(h_rows), _f64(W), _f64(y)
+    teacher = np.asarray(teacher, dtype=np.int64)
+    group = np.asarray(group, dtype=np.int64)
+    w = np.ones(ngroups) if group_weight is None else np.asarray(group_weight, dtype=np.float64)
+    n = out["counts"]
+    z = h @ W.T
+    dz = np.zeros_like(z)
+    for r in np.nonzero(out["valid"])[0]:
+        g = group[r]
+        if n[g] > 0:
+            dz[r] = grad * w[g] / n[g] * (_softmax(z[r]) - _softmax(y[teacher[r]]))
+    return dz @ W, dz.T @ h

@@ -224,3 +224,79 @@ def test_sliced_row_forms_match_the_full_forms():
     assert np.allclose(sco.rows_logits(hr, W, slice_rows=10), hr @ W.T, rtol=1e-14)
     assert np.allclose(sco.rows_dh(hr, W, yr, coef, slice_rows=10), [dh[p, t] for p, t in pairs],
                        rtol=1e-12, atol=1e-15)
+
+
+def test_general_form_reduces_to_the_pass_form():
+    """The TTT passes written as explicit teacher positions and groups give the pass form's
+    values, forward and backward."""
+    h, W, y, cu = _inputs(seed=23)
+    P, T, d = h.shape
+    mask = np.random.default_rng(24).random(T) < 0.8
+    w = [1.0, 0.6, 0.3]
+    teacher, group = sco.ttt_mapping(cu, P)
+    ref = sco.forward(h, W, y, cu, mask, w)
+    got = sco.forward_mapped(h.reshape(P * T, d), W, y, teacher, group, P, mask, w)
+    assert np.allclose(got["rows"], ref["rows"].reshape(-1), rtol=1e-13, atol=1e-15)
+    assert np.allclose(got["group_loss"], ref["pass_loss"], rtol=1e-13)
+    dh_ref, dW_ref = sco.backward(h, W, y, cu, mask, w, grad=0.7)
+    dh, dW = sco.backward_mapped(h.reshape(P * T, d), W, y, teacher, group, P, mask, w, grad=0.7)
+    assert np.allclose(dh, dh_ref.reshape(P * T, d), rtol=1e-12, atol=1e-15)
+    assert np.allclose(dW, dW_ref, rtol=1e-12, atol=1e-15)
+
+
+def test_per_slot_groups_closed_form_and_independence():
+    """Block slots as groups: with W = 0 every valid row costs log V, so L_g = w_g log V for
+    any slot with a valid row; a row's teacher outside [0, Ty) or masked is invalid; moving a
+    row to another group changes only those two groups' losses."""
+    g = np.random.default_rng(29)
+    nb, Bs, d, V, Ty = 5, 4, 8, 13, 30
+    R = nb * Bs
+    h = g.standard_normal((R, d))
+    y = g.standard_normal((Ty, V))
+    anchors = np.array([0, 6, 11, 20, 28])
+    teacher = np.array([a + j for a in anchors for j in range(Bs)])      # last block runs past Ty
+    group = np.tile(np.arange(Bs), nb)
+    mask = np.ones(Ty, dtype=bool)
+    mask[7] = False
+    out0 = sco.forward_mapped(h, np.zeros((V, d)), y, teacher, group, Bs, mask, [1.0, 2.0, 0.5, 0.25])
+    valid = out0["valid"]
+    assert not valid[teacher >= Ty].any() and not valid[teacher == 7].any()
+    for s_ in range(Bs):
+        if valid[group == s_].any():
+            assert out0["group_loss"][s_] == pytest.approx([1.0, 2.0, 0.5, 0.25][s_] * math.log(V), rel=1e-13)
+    W = g.standard_normal((V, d))
+    base = sco.forward_mapped(h, W, y, teacher, group, Bs)
+    g2 = group.copy()
+    g2[5] = 3                                                            # row 5 (slot 1) moves to slot 3
+    moved = sco.forward_mapped(h, W, y, teacher, g2, Bs)
+    assert np.allclose(moved["group_loss"][[0, 2]], base["group_loss"][[0, 2]], rtol=1e-14)
+    assert not np.isclose(moved["group_loss"][1], base["group_loss"][1])
+    assert np.allclose(moved["rows"], base["rows"], rtol=1e-14)
+
+
+def test_general_form_gradients_match_central_differences():
+    g = np.random.default_rng(31)
+    R, d, V, Ty, G = 7, 4, 6, 5, 3
+    h = g.standard_normal((R, d))
+    W = g.standard_normal((V, d))
+    y = g.standard_normal((Ty, V))
+    teacher = np.array([0, 1, 4, -1, 2, 9, 3])
+    group = np.array([0, 1, 2, 0, 1, 2, 2])
+    wts = [0.5, 1.5, 1.0]
+    dh, dW = sco.backward_mapped(h, W, y, teacher, group, G, None, wts, grad=1.2)
+
+    def L(hh, WW):
+        return 1.2 * sco.forward_mapped(hh, WW, y, teacher, group, G, None, wts)["loss"]
+
+    eps = 1e-6
+    for (r, j) in [(0, 0), (2, 3), (4, 1), (6, 2)]:
+        hp, hm = h.copy(), h.copy()
+        hp[r, j] += eps
+        hm[r, j] -= eps
+        assert dh[r, j] == pytest.approx((L(hp, W) - L(hm, W)) / (2 * eps), rel=1e-6, abs=1e-9)
+    for (v, j) in [(0, 0), (5, 3), (2, 1)]:
+        Wp, Wm = W.copy(), W.copy()
+        Wp[v, j] += eps
+        Wm[v, j] -= eps
+        assert dW[v, j] == pytest.approx((L(h, Wp) - L(h, Wm)) / (2 * eps), rel=1e-6, abs=1e-9)
+    assert np.all(dh[3] == 0) and np.all(dh[5] == 0)                    # teacher -1 and past Ty
