@@ -105,6 +105,10 @@ class TTTSoftceDesc(ctypes.Structure):
         ("pass_count", ctypes.c_void_p),
         ("token_chunk_size", ctypes.c_int),
         ("events", ctypes.c_void_p),
+        ("row_teacher", ctypes.c_void_p),
+        ("row_group", ctypes.c_void_p),
+        ("ngroups", ctypes.c_int),
+        ("teacher_rows", ctypes.c_int),
     ]
 
 

@@ -484,6 +484,38 @@ __global__ void __launch_bounds__(1024) softce_rows_kernel(int P, int T, const i
   }
 }
 
+// General form, step 1: the teacher position of every draft row (or -1) and the valid
+// rows per group (int atomics: exact and order-free).
+__global__ void __launch_bounds__(256) softce_rows_general_kernel(int R, int Ty, int G, const int32_t* row_teacher,
+                                                                  const int32_t* row_group, const uint8_t* mask,
+                                                                  int32_t* tidx, int* icount) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= R) return;
+  const int u = row_teacher[r];
+  const int g = row_group ? row_group[r] : 0;
+  const bool valid = u >= 0 && u < Ty && g >= 0 && g < G && (!mask || __ldg(mask + u) != 0);
+  tidx[r] = valid ? u : -1;
+  if (valid) atomicAdd(icount + g, 1);
+}
+
+// General form, step 2: N_g (given or counted) and each row's coefficient g * w_g / N_g.
+__global__ void __launch_bounds__(256) softce_coef_general_kernel(int R, int G, const int32_t* row_group,
+                                                                  const int32_t* tidx, const int* icount,
+                                                                  const float* weight, const float* given,
+                                                                  float grad, float* counts, float* coef) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r < G) counts[r] = given ? given[r] : static_cast<float>(icount[r]);
+  if (!coef || r >= R) return;
+  if (tidx[r] < 0) {
+    coef[r] = 0.f;
+    return;
+  }
+  const int g = row_group ? row_group[r] : 0;
+  const float n = given ? given[g] : static_cast<float>(icount[g]);
+  const float w = weight ? weight[g] : 1.f;
+  coef[r] = n > 0.f ? grad * w / n : 0.f;
+}
+
 // Merge of the per-tile statistics of every row: lse of the draft logits and of the
 // teacher row, and the loss l = lse_z - (sum_v e^(y_v - M) z_v) / (sum_v e^(y_v - M)).
 // A block takes 32 rows (threadIdx.x, so that every tile's 32 values are one coalesced
@@ -582,15 +614,24 @@ __global__ void __launch_bounds__(256) softce_dz_kernel(int R, int V, int ldz, i
   }
 }
 
-// Per-pass sums in a fixed order: L_p = w_p / N_p * sum_t l_{p,t}, then L.
+// Per-group sums in a fixed order: L_g = w_g / N_g * sum of the group's row losses, then
+// L.  The TTT passes are the groups of T consecutive rows; in the general form (group
+// array given, or `general` with every row in group 0) the rows of a group are gathered
+// by a filtered pass over all R rows.
 __global__ void __launch_bounds__(1024) softce_finalize_kernel(int P, int T, const float* row_loss,
                                                                const float* counts, const float* pass_weight,
-                                                               float* loss) {
+                                                               float* loss, int R = 0, bool general = false,
+                                                               const int32_t* row_group = nullptr) {
   __shared__ double part[32];
   double total = 0.0;
   for (int p = 0; p < P; ++p) {
     double s = 0.0;
-    for (int t = threadIdx.x; t < T; t += blockDim.x) s += row_loss[static_cast<int64_t>(p) * T + t];
+    if (!general) {
+      for (int t = threadIdx.x; t < T; t += blockDim.x) s += row_loss[static_cast<int64_t>(p) * T + t];
+    } else {
+      for (int r = threadIdx.x; r < R; r += blockDim.x)
+        if ((row_group ? row_group[r] : 0) == p) s += row_loss[r];
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
@@ -634,6 +675,8 @@ cudaError_t launch_gemm(const SoftceGemmArgs& a, const CUtensorMap& ma, const CU
 
 struct CePlan {
   int P, T, d, V, R, ntn, C, Vp;
+  bool general;  // explicit teacher positions and groups (row_teacher)
+  int G, Ty;     // normalisation groups, teacher rows
   size_t off_tidx, off_counts, off_coef, off_stats, off_z, off_dz, total;
 };
 
@@ -645,9 +688,16 @@ ttt_status ce_plan(const ttt_softce_desc* d, int mode, CePlan* out) {
   if (!d || mode < 0 || mode > 2) return TTT_ERR_INVALID_ARG;
   if (d->P < 1 || d->T < 0 || d->d < 8 || d->V < 8) return TTT_ERR_INVALID_ARG;
   if (d->d % 8 != 0 || d->V % 8 != 0) return TTT_ERR_UNSUPPORTED;
-  if (d->token_chunk_size < 0 || d->nseq < 0) return TTT_ERR_INVALID_ARG;
-  if (d->cu_seqlens && d->nseq < 1) return TTT_ERR_INVALID_ARG;
-  if (!d->cu_seqlens && d->nseq > 1 && d->T % d->nseq != 0) return TTT_ERR_INVALID_ARG;
+  if (d->token_chunk_size < 0) return TTT_ERR_INVALID_ARG;
+  const bool general = d->row_teacher != nullptr;
+  if (general) {
+    if (d->ngroups < 1 || d->teacher_rows < 0) return TTT_ERR_INVALID_ARG;
+    if (d->ngroups > 1 && !d->row_group) return TTT_ERR_INVALID_ARG;
+  } else {
+    if (d->nseq < 0) return TTT_ERR_INVALID_ARG;
+    if (d->cu_seqlens && d->nseq < 1) return TTT_ERR_INVALID_ARG;
+    if (!d->cu_seqlens && d->nseq > 1 && d->T % d->nseq != 0) return TTT_ERR_INVALID_ARG;
+  }
   const long long R = static_cast<long long>(d->P) * d->T;
   if (R >= (1LL << 31)) return TTT_ERR_UNSUPPORTED;
   CePlan pl{};
@@ -656,13 +706,17 @@ ttt_status ce_plan(const ttt_softce_desc* d, int mode, CePlan* out) {
   pl.d = d->d;
   pl.V = d->V;
   pl.R = static_cast<int>(R);
+  pl.general = general;
+  pl.G = general ? d->ngroups : d->P;
+  pl.Ty = general ? d->teacher_rows : d->T;
   pl.ntn = (d->V + kBN - 1) / kBN;
   const int chunk = d->token_chunk_size > 0 ? d->token_chunk_size : 4096;
   pl.C = static_cast<int>(R < chunk ? (R > 0 ? R : 1) : chunk);
   pl.Vp = (d->V + 63) / 64 * 64;
   pl.off_tidx = kCeAlign;  // the status word lives in the first block
   pl.off_counts = ce_align(pl.off_tidx + static_cast<size_t>(pl.R) * 4);
-  const size_t after_counts = ce_align(pl.off_counts + static_cast<size_t>(pl.P) * 4);
+  // N_g as floats, then the int counts of the general form
+  const size_t after_counts = ce_align(pl.off_counts + static_cast<size_t>(pl.G) * 8);
   const size_t stats_bytes = static_cast<size_t>(pl.ntn) * 5 * pl.R * 4;
   if (mode == 0) {
     pl.off_stats = after_counts;
@@ -709,6 +763,29 @@ struct CeEvents {
 constexpr CUtensorMapDataType kBf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 constexpr CUtensorMapSwizzle kSw128 = CU_TENSOR_MAP_SWIZZLE_128B;
 
+// Teacher rows, N_g and (coef non-NULL) the rows' gradient coefficients, for either form.
+ttt_status launch_rows(const ttt_softce_desc* d, const CePlan& pl, float grad, uint8_t* ws, int32_t* tidx,
+                       float* counts, float* coef, cudaStream_t stream) {
+  CeEvents ev(d->events, TTT_SOFTCE_KERNEL_ROWS, stream);
+  if (!pl.general) {
+    softce_rows_kernel<<<pl.P, 1024, 0, stream>>>(pl.P, pl.T, d->cu_seqlens, d->nseq, d->loss_mask, d->pass_weight,
+                                                 d->pass_count, grad, tidx, counts, coef);
+    CE_CHECK(cudaGetLastError());
+    return TTT_OK;
+  }
+  int* icount = reinterpret_cast<int*>(counts + pl.G);
+  CE_CHECK(cudaMemsetAsync(icount, 0, sizeof(int) * pl.G, stream));
+  softce_rows_general_kernel<<<(pl.R + 255) / 256, 256, 0, stream>>>(pl.R, pl.Ty, pl.G, d->row_teacher, d->row_group,
+                                                                      d->loss_mask, tidx, icount);
+  CE_CHECK(cudaGetLastError());
+  const int n = pl.R > pl.G ? pl.R : pl.G;
+  softce_coef_general_kernel<<<(n + 255) / 256, 256, 0, stream>>>(pl.R, pl.G, d->row_group, tidx, icount,
+                                                                  d->pass_weight, d->pass_count, grad, counts, coef);
+  CE_CHECK(cudaGetLastError());
+  (void)ws;
+  return TTT_OK;
+}
+
 }  // namespace
 }  // namespace ttt
 
@@ -738,17 +815,15 @@ ttt_status ttt_softce_fwd(const ttt_softce_desc* desc, const void* h, const void
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   CE_CHECK(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   if (pl.R == 0) {
-    CE_CHECK(cudaMemsetAsync(loss, 0, sizeof(float) * (pl.P + 1), stream));
+    CE_CHECK(cudaMemsetAsync(loss, 0, sizeof(float) * (pl.G + 1), stream));
     return TTT_OK;
   }
   int32_t* tidx = reinterpret_cast<int32_t*>(ws + pl.off_tidx);
   float* counts = reinterpret_cast<float*>(ws + pl.off_counts);
   float* stats = reinterpret_cast<float*>(ws + pl.off_stats);
   {
-    CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_ROWS, stream);
-    softce_rows_kernel<<<pl.P, 1024, 0, stream>>>(pl.P, pl.T, desc->cu_seqlens, desc->nseq, desc->loss_mask,
-                                                 desc->pass_weight, desc->pass_count, 1.f, tidx, counts, nullptr);
-    CE_CHECK(cudaGetLastError());
+    const ttt_status sr = launch_rows(desc, pl, 1.f, ws, tidx, counts, nullptr, stream);
+    if (sr != TTT_OK) return sr;
   }
   CUtensorMap mh, mw;
   if (!encode_map_2d(&mh, kBf16, h, pl.d, pl.R, static_cast<uint64_t>(pl.d) * 2, 64, 128, kSw128) ||
@@ -775,7 +850,8 @@ ttt_status ttt_softce_fwd(const ttt_softce_desc* desc, const void* h, const void
     softce_combine_kernel<<<(pl.R + 31) / 32, dim3(32, kCombineSlices), 0, stream>>>(pl.R, pl.ntn, 0, pl.R, tidx,
                                                                                       stats, row_loss, lse);
     CE_CHECK(cudaGetLastError());
-    softce_finalize_kernel<<<1, 1024, 0, stream>>>(pl.P, pl.T, row_loss, counts, desc->pass_weight, loss);
+    softce_finalize_kernel<<<1, 1024, 0, stream>>>(pl.G, pl.T, row_loss, counts, desc->pass_weight, loss, pl.R,
+                                                   pl.general, desc->row_group);
     CE_CHECK(cudaGetLastError());
   }
   return TTT_OK;
@@ -803,10 +879,8 @@ ttt_status ttt_softce_bwd(const ttt_softce_desc* desc, const void* h, const void
   float* coef = reinterpret_cast<float*>(ws + pl.off_coef);
   uint8_t* dz = ws + pl.off_dz;
   {
-    CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_ROWS, stream);
-    softce_rows_kernel<<<pl.P, 1024, 0, stream>>>(pl.P, pl.T, desc->cu_seqlens, desc->nseq, desc->loss_mask,
-                                                 desc->pass_weight, desc->pass_count, grad, tidx, counts, coef);
-    CE_CHECK(cudaGetLastError());
+    const ttt_status sr = launch_rows(desc, pl, grad, ws, tidx, counts, coef, stream);
+    if (sr != TTT_OK) return sr;
   }
   const uint64_t hrow = static_cast<uint64_t>(pl.d) * 2, zrow = static_cast<uint64_t>(pl.Vp) * 2;
   CUtensorMap mh, mw_k, mw_mn, mdw;
@@ -885,7 +959,7 @@ ttt_status ttt_softce_fwd_bwd(const ttt_softce_desc* desc, const void* h, const 
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   CE_CHECK(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   if (pl.R == 0) {
-    CE_CHECK(cudaMemsetAsync(loss, 0, sizeof(float) * (pl.P + 1), stream));
+    CE_CHECK(cudaMemsetAsync(loss, 0, sizeof(float) * (pl.G + 1), stream));
     return TTT_OK;
   }
   int32_t* tidx = reinterpret_cast<int32_t*>(ws + pl.off_tidx);
@@ -895,10 +969,8 @@ ttt_status ttt_softce_fwd_bwd(const ttt_softce_desc* desc, const void* h, const 
   float* zbuf = reinterpret_cast<float*>(ws + pl.off_z);
   uint8_t* dz = ws + pl.off_dz;
   {
-    CeEvents ev(desc->events, TTT_SOFTCE_KERNEL_ROWS, stream);
-    softce_rows_kernel<<<pl.P, 1024, 0, stream>>>(pl.P, pl.T, desc->cu_seqlens, desc->nseq, desc->loss_mask,
-                                                 desc->pass_weight, desc->pass_count, grad, tidx, counts, coef);
-    CE_CHECK(cudaGetLastError());
+    const ttt_status sr = launch_rows(desc, pl, grad, ws, tidx, counts, coef, stream);
+    if (sr != TTT_OK) return sr;
   }
   const uint64_t hrow = static_cast<uint64_t>(pl.d) * 2, zrow = static_cast<uint64_t>(pl.Vp) * 2;
   CUtensorMap mh, mw_k, mw_mn, mdw;
@@ -969,7 +1041,8 @@ ttt_status ttt_softce_fwd_bwd(const ttt_softce_desc* desc, const void* h, const 
       CE_CHECK(launch_gemm<EPI_ACC>(a, mz_mn, mh_mn, mdw, stream));
     }
   }
-  softce_finalize_kernel<<<1, 1024, 0, stream>>>(pl.P, pl.T, row_loss, counts, desc->pass_weight, loss);
+  softce_finalize_kernel<<<1, 1024, 0, stream>>>(pl.G, pl.T, row_loss, counts, desc->pass_weight, loss, pl.R,
+                                                 pl.general, desc->row_group);
   CE_CHECK(cudaGetLastError());
   return TTT_OK;
 }

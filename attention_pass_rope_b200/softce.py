@@ -10,6 +10,11 @@ bf16 (the vocabulary head), y [T, V] bf16 (the teacher's logits), loss_mask [T] 
 (teacher positions counted), cu_seqlens int32 [nseq + 1] or None (one sequence),
 pass_weight / pass_count float32 [P] or None.  Pass p at token t learns the teacher
 row t + p of its own sequence.
+
+General form (``row_teacher`` given: e.g. the slots of block drafters, normalised per
+slot): row r of h viewed as [P*T, d] learns teacher row row_teacher[r] (int32, -1 =
+none) of y [Ty, V] and is normalised in group row_group[r] (int32, None = group 0) of
+``ngroups``; loss_mask is [Ty], pass_weight / pass_count [ngroups], the loss [ngroups + 1].
 """
 
 from __future__ import annotations
@@ -31,13 +36,16 @@ def _stream():
 
 
 def make_desc(h, W, y, cu_seqlens=None, loss_mask=None, pass_weight=None, pass_count=None,
-              token_chunk_size: int = 0, events=None) -> _lib.TTTSoftceDesc:
+              token_chunk_size: int = 0, events=None, row_teacher=None, row_group=None,
+              ngroups: int = 1) -> _lib.TTTSoftceDesc:
     if h.dim() != 3 or W.dim() != 2 or y.dim() != 2:
-        raise ValueError("h must be [P, T, d], W [V, d], y [T, V]")
+        raise ValueError("h must be [P, T, d], W [V, d], y [T, V] (or [Ty, V] with row_teacher)")
     P, T, d = h.shape
     V = W.shape[0]
-    if W.shape[1] != d or tuple(y.shape) != (T, V):
+    Ty = y.shape[0] if row_teacher is not None else T
+    if W.shape[1] != d or tuple(y.shape) != (Ty, V):
         raise ValueError(f"shape mismatch: h {tuple(h.shape)}, W {tuple(W.shape)}, y {tuple(y.shape)}")
+    G = int(ngroups) if row_teacher is not None else int(P)
     for name, t in (("h", h), ("W", W), ("y", y)):
         if t.dtype != torch.bfloat16 or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous bf16 tensor")
@@ -52,17 +60,30 @@ def make_desc(h, W, y, cu_seqlens=None, loss_mask=None, pass_weight=None, pass_c
         desc.cu_seqlens = None
         desc.nseq = 1
     if loss_mask is not None:
-        if loss_mask.dtype != torch.uint8 or tuple(loss_mask.shape) != (T,):
-            raise ValueError("loss_mask must be uint8 [T]")
+        if loss_mask.dtype != torch.uint8 or tuple(loss_mask.shape) != (Ty,):
+            raise ValueError("loss_mask must be uint8 [T] ([Ty] with row_teacher)")
         desc.loss_mask = loss_mask.data_ptr()
     for name, t in (("pass_weight", pass_weight), ("pass_count", pass_count)):
         if t is not None:
-            if t.dtype != torch.float32 or tuple(t.shape) != (P,):
-                raise ValueError(f"{name} must be float32 [P]")
+            if t.dtype != torch.float32 or tuple(t.shape) != (G,):
+                raise ValueError(f"{name} must be float32 [P] ([ngroups] with row_teacher)")
             setattr(desc, name, t.data_ptr())
     desc.token_chunk_size = int(token_chunk_size)
     desc.events = ctypes.addressof(events) if events is not None else None
+    if row_teacher is not None:
+        for name, t in (("row_teacher", row_teacher), ("row_group", row_group)):
+            if t is not None and (t.dtype != torch.int32 or tuple(t.shape) != (P * T,) or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous int32 [P*T]")
+        desc.row_teacher = row_teacher.data_ptr()
+        desc.row_group = None if row_group is None else row_group.data_ptr()
+        desc.ngroups = G
+        desc.teacher_rows = int(Ty)
     return desc
+
+
+def ngroups_of(desc: _lib.TTTSoftceDesc) -> int:
+    """Normalisation groups of a descriptor: the passes, or ngroups in the general form."""
+    return int(desc.ngroups) if desc.row_teacher else int(desc.P)
 
 
 def workspace_bytes(desc: _lib.TTTSoftceDesc, for_backward) -> int:
@@ -74,22 +95,24 @@ def workspace_bytes(desc: _lib.TTTSoftceDesc, for_backward) -> int:
 
 
 def softce_fwd(h, W, y, *, cu_seqlens=None, loss_mask=None, pass_weight=None, pass_count=None,
-               workspace: Optional[torch.Tensor] = None, events=None, out=None):
-    """Forward: returns (loss [P + 1] = per-pass losses then their sum, row_loss [P, T],
-    lse [2, P, T] = logsumexp of each row's logits and of its teacher row).  ``out`` =
-    (loss, row_loss, lse) writes into given float32 tensors of those shapes."""
-    desc = make_desc(h, W, y, cu_seqlens, loss_mask, pass_weight, pass_count, 0, events)
-    P, T = desc.P, desc.T
+               workspace: Optional[torch.Tensor] = None, events=None, out=None, row_teacher=None, row_group=None,
+               ngroups: int = 1):
+    """Forward: returns (loss [G + 1] = per-pass (per-group) losses then their sum,
+    row_loss [P, T], lse [2, P, T] = logsumexp of each row's logits and of its teacher
+    row).  ``out`` = (loss, row_loss, lse) writes into given float32 tensors."""
+    desc = make_desc(h, W, y, cu_seqlens, loss_mask, pass_weight, pass_count, 0, events, row_teacher, row_group,
+                     ngroups)
+    P, T, G = desc.P, desc.T, ngroups_of(desc)
     dev = h.device
     if out is None:
-        loss = torch.empty(P + 1, dtype=torch.float32, device=dev)
+        loss = torch.empty(G + 1, dtype=torch.float32, device=dev)
         row_loss = torch.empty(P, T, dtype=torch.float32, device=dev)
         lse = torch.empty(2, P, T, dtype=torch.float32, device=dev)
     else:
         loss, row_loss, lse = out
-        for t, shape in ((loss, (P + 1,)), (row_loss, (P, T)), (lse, (2, P, T))):
+        for t, shape in ((loss, (G + 1,)), (row_loss, (P, T)), (lse, (2, P, T))):
             if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous():
-                raise ValueError(f"out tensors must be contiguous float32 of shapes {(P + 1,)}, {(P, T)}, {(2, P, T)}")
+                raise ValueError(f"out tensors must be contiguous float32 of shapes {(G + 1,)}, {(P, T)}, {(2, P, T)}")
     need = workspace_bytes(desc, False)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -101,11 +124,13 @@ def softce_fwd(h, W, y, *, cu_seqlens=None, loss_mask=None, pass_weight=None, pa
 
 def softce_bwd(h, W, y, lse, *, grad: float = 1.0, cu_seqlens=None, loss_mask=None, pass_weight=None,
                pass_count=None, token_chunk_size: int = 0, with_dw: bool = True, dW=None, dh=None,
-               workspace: Optional[torch.Tensor] = None, events=None):
+               workspace: Optional[torch.Tensor] = None, events=None, row_teacher=None, row_group=None,
+               ngroups: int = 1):
     """Backward of grad * L: returns (dh [P, T, d] bf16, dW [V, d] fp32 or None).  A given
     ``dW`` (fp32 [V, d]) is added to; otherwise a zeroed one is allocated.  A given ``dh``
     (bf16 like h) is written."""
-    desc = make_desc(h, W, y, cu_seqlens, loss_mask, pass_weight, pass_count, token_chunk_size, events)
+    desc = make_desc(h, W, y, cu_seqlens, loss_mask, pass_weight, pass_count, token_chunk_size, events,
+                     row_teacher, row_group, ngroups)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (2, desc.P, desc.T) or not lse.is_contiguous():
         raise ValueError("lse must be the forward's float32 [2, P, T]")
     dev = h.device
@@ -130,21 +155,23 @@ def softce_bwd(h, W, y, lse, *, grad: float = 1.0, cu_seqlens=None, loss_mask=No
 
 def softce_fwd_bwd(h, W, y, *, grad: float = 1.0, cu_seqlens=None, loss_mask=None, pass_weight=None,
                    pass_count=None, token_chunk_size: int = 0, with_dw: bool = True, dW=None, dh=None, out=None,
-                   workspace: Optional[torch.Tensor] = None, events=None):
+                   workspace: Optional[torch.Tensor] = None, events=None, row_teacher=None, row_group=None,
+                   ngroups: int = 1):
     """Forward and backward of grad * L in one sweep (the logits GEMM runs once): returns
     (loss, row_loss, lse, dh, dW), the outputs of :func:`softce_fwd` and :func:`softce_bwd`."""
-    desc = make_desc(h, W, y, cu_seqlens, loss_mask, pass_weight, pass_count, token_chunk_size, events)
-    P, T = desc.P, desc.T
+    desc = make_desc(h, W, y, cu_seqlens, loss_mask, pass_weight, pass_count, token_chunk_size, events,
+                     row_teacher, row_group, ngroups)
+    P, T, G = desc.P, desc.T, ngroups_of(desc)
     dev = h.device
     if out is None:
-        loss = torch.empty(P + 1, dtype=torch.float32, device=dev)
+        loss = torch.empty(G + 1, dtype=torch.float32, device=dev)
         row_loss = torch.empty(P, T, dtype=torch.float32, device=dev)
         lse = torch.empty(2, P, T, dtype=torch.float32, device=dev)
     else:
         loss, row_loss, lse = out
-        for t, shape in ((loss, (P + 1,)), (row_loss, (P, T)), (lse, (2, P, T))):
+        for t, shape in ((loss, (G + 1,)), (row_loss, (P, T)), (lse, (2, P, T))):
             if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous():
-                raise ValueError(f"out tensors must be contiguous float32 of shapes {(P + 1,)}, {(P, T)}, {(2, P, T)}")
+                raise ValueError(f"out tensors must be contiguous float32 of shapes {(G + 1,)}, {(P, T)}, {(2, P, T)}")
     if dh is None:
         dh = torch.empty_like(h)
     elif dh.dtype != torch.bfloat16 or dh.shape != h.shape or not dh.is_contiguous():

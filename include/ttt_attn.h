@@ -391,6 +391,18 @@ typedef struct {
   const float* pass_count;       /* device float[P]: N_p (e.g. summed over ranks); NULL: counted here */
   int token_chunk_size;          /* backward: draft rows per chunk of dz; 0 selects 4096 */
   const ttt_attn_events* events; /* optional, indices TTT_SOFTCE_KERNEL_* */
+  /* General form, for normalisation groups other than the passes (e.g. the slots of a
+   * block drafter, issue 3698 item 3's per-slot normalisation).  When row_teacher is
+   * non-NULL, draft row r (of P*T) learns teacher position row_teacher[r] and belongs to
+   * normalisation group row_group[r] (NULL: every row in group 0); a row whose teacher
+   * position lies outside [0, teacher_rows), whose group lies outside [0, ngroups) or
+   * whose position is masked is invalid.  y then has teacher_rows rows, loss_mask
+   * teacher_rows entries, pass_weight / pass_count ngroups entries, the loss ngroups + 1
+   * values; cu_seqlens and nseq are not read. */
+  const int32_t* row_teacher;    /* device int32[P*T], or NULL for the TTT passes */
+  const int32_t* row_group;      /* device int32[P*T], or NULL */
+  int ngroups;                   /* >= 1 with row_teacher; groups > 1 need row_group */
+  int teacher_rows;              /* rows of y with row_teacher */
 } ttt_softce_desc;
 
 /* Kernel indices of the soft-CE calls in ttt_attn_events (the backward's chunked
@@ -413,7 +425,7 @@ size_t ttt_softce_workspace_size(const ttt_softce_desc* desc, int for_backward);
 
 /* Forward.  Writes row_loss float[P*T] (l_r), lse float[2][P*T] (logsumexp of z_r,
  * then of the teacher row y_u; 0 for an invalid row; the backward reads it) and loss
- * float[P+1] (L_0 .. L_{P-1}, then L). */
+ * float[G+1] (L_0 .. L_{G-1}, then L), G = P (or ngroups in the general form). */
 ttt_status ttt_softce_fwd(const ttt_softce_desc* desc, const void* h, const void* W, const void* y,
                           float* row_loss, float* lse, float* loss, void* workspace, size_t workspace_bytes,
                           void* stream);

@@ -264,5 +264,14 @@ def test_softce_rejects_bad_arguments(L):
                                 None, fake, 1 << 40, None) == _lib.TTT_ERR_INVALID_ARG
     assert L.ttt_softce_fwd_bwd(ctypes.byref(ok), fake, fake, fake, ctypes.c_float(1.0), fake, fake, fake, fake,
                                 None, fake, 1024, None) == _lib.TTT_ERR_WORKSPACE
+    # general form: groups >= 1, and several groups need the group array
+    d_g = softce_desc(row_teacher=fake.value, ngroups=0, teacher_rows=10)
+    assert L.ttt_softce_workspace_size(ctypes.byref(d_g), 0) == 0
+    d_g = softce_desc(row_teacher=fake.value, ngroups=4, teacher_rows=10)
+    assert L.ttt_softce_workspace_size(ctypes.byref(d_g), 0) == 0
+    d_g = softce_desc(row_teacher=fake.value, row_group=fake.value, ngroups=4, teacher_rows=10)
+    assert L.ttt_softce_workspace_size(ctypes.byref(d_g), 0) > 0
+    d_g = softce_desc(row_teacher=fake.value, ngroups=1, teacher_rows=-1)
+    assert L.ttt_softce_workspace_size(ctypes.byref(d_g), 0) == 0
     # a dense descriptor whose T is not a multiple of nseq
     assert L.ttt_softce_workspace_size(ctypes.byref(softce_desc(nseq=3, T=8192)), 0) == 0

@@ -208,6 +208,71 @@ def test_softce_dense_sequences_without_cu_seqlens():
         assert np.array_equal(a, b)
 
 
+def test_softce_general_form_equals_pass_form():
+    """The TTT passes given as explicit teacher positions and groups: the same rows, lse,
+    dh and dW bit for bit as the pass form, and the same per-pass losses (summed in
+    another order)."""
+    w = ti.softce_workloads()["softce_tiny"]
+    inp = ti.make_softce_inputs(w)
+    h, W, y, m = inp.h.cuda(), inp.W.cuda(), inp.y.cuda(), inp.mask.cuda()
+    cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device="cuda")
+    teacher, group = sco.ttt_mapping(w.cu_seqlens, w.P)
+    rt = torch.tensor(teacher, dtype=torch.int32, device="cuda")
+    rg = torch.tensor(group, dtype=torch.int32, device="cuda")
+    pw = torch.tensor([1.0, 0.7, 0.4], device="cuda")
+    a = ce.softce_fwd_bwd(h, W, y, cu_seqlens=cu, loss_mask=m, pass_weight=pw, token_chunk_size=100)
+    b = ce.softce_fwd_bwd(h, W, y, loss_mask=m, pass_weight=pw, token_chunk_size=100, row_teacher=rt, row_group=rg,
+                          ngroups=w.P)
+    c_loss, c_rows, c_lse = ce.softce_fwd(h, W, y, loss_mask=m, pass_weight=pw, row_teacher=rt, row_group=rg,
+                                          ngroups=w.P)
+    c_dh, c_dW = ce.softce_bwd(h, W, y, c_lse, loss_mask=m, pass_weight=pw, token_chunk_size=100, row_teacher=rt,
+                               row_group=rg, ngroups=w.P)
+    torch.cuda.synchronize()
+    for x, z in zip(a[1:], b[1:]):
+        assert torch.equal(x, z)
+    assert torch.equal(c_rows, b[1]) and torch.equal(c_lse, b[2]) and torch.equal(c_dh, b[3])
+    assert torch.equal(c_dW, b[4])
+    assert torch.allclose(a[0], b[0], rtol=1e-6, atol=0) and torch.equal(c_loss, b[0])
+
+
+def test_softce_block_slots():
+    """Block drafters normalised per slot: 40 blocks of 16 slots at sorted anchors over 300
+    teacher positions (the last blocks run past them), slot weights, a mask; forward, the
+    separate backward and the fused call against the oracle's general form."""
+    g = torch.Generator().manual_seed(11)
+    nb, Bs, d, V, Ty = 40, 16, 128, 1000, 300
+    hq = torch.randn(1, nb * Bs, d, generator=g).to(torch.bfloat16)
+    Wq = (torch.randn(V, d, generator=g) * (2.0 / d ** 0.5)).to(torch.bfloat16)
+    yq = (torch.randn(Ty, V, generator=g) * 3.0).to(torch.bfloat16)
+    mq = (torch.rand(Ty, generator=g) < 0.9).to(torch.uint8)
+    anchors = torch.sort(torch.randint(0, Ty, (nb,), generator=g)).values
+    teacher = (anchors[:, None] + torch.arange(Bs)[None, :]).reshape(-1).to(torch.int32)
+    group = torch.arange(Bs).repeat(nb).to(torch.int32)
+    wts = [1.0 / (1 + j) for j in range(Bs)]
+    h, W, y, m = hq.cuda(), Wq.cuda(), yq.cuda(), mq.cuda()
+    rt, rg = teacher.cuda(), group.cuda()
+    pw = torch.tensor(wts, device="cuda")
+    kw = dict(loss_mask=m, pass_weight=pw, row_teacher=rt, row_group=rg, ngroups=Bs)
+    loss, rows, lse = ce.softce_fwd(h, W, y, **kw)
+    dh, dW = ce.softce_bwd(h, W, y, lse, grad=0.8, token_chunk_size=200, **kw)
+    f = ce.softce_fwd_bwd(h, W, y, grad=0.8, token_chunk_size=200, **kw)
+    torch.cuda.synchronize()
+    ref = sco.forward_mapped(hq[0], Wq, yq, teacher.numpy(), group.numpy(), Bs, mq.numpy(), wts)
+    dh_ref, dW_ref = sco.backward_mapped(hq[0], Wq, yq, teacher.numpy(), group.numpy(), Bs, mq.numpy(), wts,
+                                         grad=0.8)
+    valid = ref["valid"]
+    assert valid.sum() > 0 and (~valid).sum() > 0
+    got_rows = rows.cpu().numpy()[0]
+    assert np.abs(got_rows[valid] - ref["rows"][valid]).max() <= LOSS_ATOL
+    assert np.all(got_rows[~valid] == 0)
+    np.testing.assert_allclose(loss.cpu().numpy()[:Bs], ref["group_loss"], rtol=PASS_RTOL, atol=1e-6)
+    assert loss.cpu().numpy()[Bs] == pytest.approx(ref["loss"], rel=PASS_RTOL)
+    assert rel_l2(dh.float().cpu().numpy()[0], dh_ref) <= GRAD_RL2
+    assert rel_l2(dW.cpu().numpy(), dW_ref) <= GRAD_RL2
+    for x, z in zip((loss, rows, lse, dh, dW), f):
+        assert torch.equal(x, z)
+
+
 @pytest.mark.slow
 def test_softce_qwen3_8b_4k_sampled_rows():
     """The full-size workload (P = 3 over 2 x 4096 tokens, d = 4096, V = 151936) in the
