@@ -687,7 +687,8 @@ inline size_t ce_align(size_t x) { return (x + kCeAlign - 1) / kCeAlign * kCeAli
 ttt_status ce_plan(const ttt_softce_desc* d, int mode, CePlan* out) {
   if (!d || mode < 0 || mode > 2) return TTT_ERR_INVALID_ARG;
   if (d->P < 1 || d->T < 0 || d->d < 8 || d->V < 8) return TTT_ERR_INVALID_ARG;
-  if (d->d % 8 != 0 || d->V % 8 != 0) return TTT_ERR_UNSUPPORTED;
+  // the TMA boxes are 64 hidden columns and 256 vocabulary rows: smaller tensors are not taken
+  if (d->d % 8 != 0 || d->V % 8 != 0 || d->d < 64 || d->V < 256) return TTT_ERR_UNSUPPORTED;
   if (d->token_chunk_size < 0) return TTT_ERR_INVALID_ARG;
   const bool general = d->row_teacher != nullptr;
   if (general) {

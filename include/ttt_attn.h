@@ -372,7 +372,7 @@ ttt_status ttt_ring_dkv_finish(const ttt_ring_desc* desc, const float* dk_acc, c
  *
  * Layouts (device memory, row-major, 16-byte aligned): h bf16 [P][T][d], W bf16 [V][d],
  * y bf16 [T][V], dh bf16 [P][T][d], dW fp32 [V][d].  Supported: d and V multiples of
- * 8, P*T < 2^31.  Sequences: cu_seqlens (device int32[nseq+1]), or, when it is NULL,
+ * 8, d >= 64, V >= 256, P*T < 2^31.  Sequences: cu_seqlens (device int32[nseq+1]), or, when it is NULL,
  * nseq equal sequences of T / nseq tokens (nseq = 0 or 1: one sequence).
  * Ownership, asynchrony and errors are those of the attention calls: the caller owns
  * every buffer, the calls enqueue on `stream` and return at once, the workspace's

@@ -240,8 +240,8 @@ def test_softce_rejects_bad_arguments(L):
     assert L.ttt_softce_workspace_size(None, 0) == 0
     for bad in (dict(P=0), dict(T=-1), dict(d=4), dict(V=0), dict(token_chunk_size=-1), dict(nseq=-1)):
         assert L.ttt_softce_workspace_size(ctypes.byref(softce_desc(**bad)), 0) == 0, bad
-    # d or V not a multiple of 8: unsupported
-    for bad in (dict(d=4100), dict(V=151937)):
+    # d or V not a multiple of 8, or smaller than one TMA box: unsupported
+    for bad in (dict(d=4100), dict(V=151937), dict(d=32), dict(V=128)):
         assert L.ttt_softce_workspace_size(ctypes.byref(softce_desc(**bad)), 1) == 0, bad
     fake = ctypes.c_void_p(1 << 20)
     vp = ctypes.c_void_p
