@@ -300,3 +300,22 @@ def test_general_form_gradients_match_central_differences():
         Wm[v, j] -= eps
         assert dW[v, j] == pytest.approx((L(h, Wp) - L(h, Wm)) / (2 * eps), rel=1e-6, abs=1e-9)
     assert np.all(dh[3] == 0) and np.all(dh[5] == 0)                    # teacher -1 and past Ty
+
+
+def test_oracle_matches_its_fixture():
+    """The soft-CE oracle reproduces tests/golden/softce_fixture.txt (written by the
+    committed tests/golden/make_softce_fixture.py, which calls the oracle only): any later
+    change to the oracle's arithmetic shows up here.  The fixture's invalid rows (a masked
+    teacher position, positions past a sequence's end or past the teacher rows) are 0."""
+    import os
+    import sys
+    golden = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    sys.path.insert(0, golden)
+    import make_softce_fixture as mk
+    ref = mk.read(os.path.join(golden, "softce_fixture.txt"))
+    got = mk.compute()
+    assert set(ref) == set(got)
+    for name in ref:
+        np.testing.assert_allclose(np.asarray(got[name]), ref[name], rtol=0, atol=1e-13, err_msg=name)
+    assert ref["rows"][0, 3] == 0 and ref["rows"][1, 2] == 0 and ref["rows"][1, 4] == 0
+    assert ref["g_rows"][3] == 0 and ref["g_rows"][5] == 0
