@@ -45,6 +45,30 @@ def test_packed_ragged(P, H, Hkv, D, lengths):
     _check(ttt_inputs.thd("ragged", lengths, P, H, Hkv, D, 1e4))
 
 
+def _random_config(seed):
+    """A seeded random packed configuration: 1-6 sequences of 0-400 tokens, P in 1..5,
+    D in {64, 128}, GQA groups of 1-4 with 1-3 KV heads, theta in {1e4, 1e6}."""
+    rng = np.random.default_rng(seed)
+    nseq = int(rng.integers(1, 7))
+    lengths = [int(x) for x in rng.integers(0, 401, nseq)]
+    if sum(lengths) == 0:
+        lengths[0] = 1
+    Hkv = int(rng.integers(1, 4))
+    H = Hkv * int(rng.integers(1, 5))
+    return dict(lengths=lengths, P=int(rng.integers(1, 6)), H=H, Hkv=Hkv, D=int(rng.choice([64, 128])),
+                theta=float(rng.choice([1e4, 1e6])))
+
+
+@needs_cuda
+@pytest.mark.parametrize("seed", range(8))
+def test_random_configurations(seed):
+    """Seeded random combinations of the packed layout's parameters, every element against
+    the oracle (the explicit cases above pin the individual edges; this covers their
+    combinations)."""
+    c = _random_config(1000 + seed)
+    _check(ttt_inputs.thd(f"random{seed}", c["lengths"], c["P"], c["H"], c["Hkv"], c["D"], c["theta"]))
+
+
 @needs_cuda
 @pytest.mark.parametrize("B,S,P,H,Hkv,D", [(2, 200, 3, 4, 4, 128), (3, 64, 5, 2, 1, 64), (1, 384, 2, 8, 2, 128)])
 def test_dense_tails(B, S, P, H, Hkv, D):
