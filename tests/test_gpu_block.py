@@ -3,6 +3,7 @@ the CUDA path through the C ABI against the fp64 block-draft oracle on the same 
 inputs.  Tolerances as for the TTT attention: O max-abs <= 2e-2, lse max-abs <= 1e-3,
 gradient relative L2 <= 1e-2 (each of dqb, dk_ctx, dv_ctx, dkb, dvb on its own)."""
 
+import numpy as np
 import pytest
 import torch
 
@@ -171,3 +172,35 @@ def test_block_window_4k_sampled_group():
     """The 4K block workload as a sliding-window layer of 1024 keys: sequence 0, KV head
     3 against the oracle."""
     _check(ttt_inputs.block_workloads()["block_draft_4k"], window=1024, kv_heads=[3], seqs=[0])
+
+
+def _random_block_config(seed):
+    """A seeded random packed block-draft configuration: 1-4 sequences with contexts of
+    1-300 tokens and 0-12 blocks each at sorted random anchors (repeats allowed), Bs in
+    1..16, D in {64, 128}, 1-2 KV heads with groups of 1-4, and a sliding window (0 = the
+    full layer) half of the time."""
+    rng = np.random.default_rng(seed)
+    nseq = int(rng.integers(1, 5))
+    ctx = [int(x) for x in rng.integers(1, 301, nseq)]
+    nblk = [int(x) for x in rng.integers(0, 13, nseq)]
+    if sum(nblk) == 0:
+        nblk[0] = 1
+    anchors = []
+    for L, nb in zip(ctx, nblk):
+        anchors += sorted(int(a) for a in rng.integers(0, L, nb))
+    Hkv = int(rng.integers(1, 3))
+    H = Hkv * int(rng.integers(1, 5))
+    window = int(rng.integers(1, 200)) if rng.random() < 0.5 else 0
+    return dict(ctx=ctx, nblk=nblk, anchors=anchors, Bs=int(rng.integers(1, 17)), H=H, Hkv=Hkv,
+                D=int(rng.choice([64, 128])), window=window)
+
+
+@needs_cuda
+@pytest.mark.parametrize("seed", range(6))
+def test_block_random_configurations(seed):
+    """Seeded random combinations of the block-draft parameters, every element against the
+    oracle."""
+    c = _random_block_config(2000 + seed)
+    w = ttt_inputs.block_thd(f"block_random{seed}", c["ctx"], c["nblk"], c["Bs"], c["H"], c["Hkv"], c["D"], 1e4,
+                             anchors=c["anchors"])
+    _check(w, window=c["window"])
