@@ -273,6 +273,30 @@ def test_softce_block_slots():
         assert torch.equal(x, z)
 
 
+def _random_softce_config(seed):
+    """A seeded random soft-CE configuration: 1-4 sequences of 1-300 tokens, P in 1..4, d a
+    multiple of 8 in [64, 320], V a multiple of 8 in [256, 3000], a random chunk size, pass
+    weights and upstream gradient, the fused call half of the time."""
+    rng = np.random.default_rng(seed)
+    nseq = int(rng.integers(1, 5))
+    lengths = tuple(int(x) for x in rng.integers(1, 301, nseq))
+    P = int(rng.integers(1, 5))
+    d = 8 * int(rng.integers(8, 41))
+    V = 8 * int(rng.integers(32, 376))
+    return dict(w=ti.SoftCEWorkload(f"rnd{seed}", P=P, lengths=lengths, d=d, V=V, seed=seed),
+                chunk=int(rng.integers(1, 600)), weights=[float(x) for x in rng.uniform(0.2, 2.0, P)],
+                grad=float(rng.uniform(0.5, 2.0)), fused=bool(rng.random() < 0.5))
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_softce_random_configurations(seed):
+    c = _random_softce_config(3000 + seed)
+    w = c["w"]
+    inp = ti.make_softce_inputs(w)
+    kw = dict(pass_weight=c["weights"], grad=c["grad"])
+    compare(inp, w.cu_seqlens, run_gpu(inp, w.cu_seqlens, chunk=c["chunk"], fused=c["fused"], **kw), **kw)
+
+
 @pytest.mark.slow
 def test_softce_qwen3_8b_4k_sampled_rows():
     """The full-size workload (P = 3 over 2 x 4096 tokens, d = 4096, V = 151936) in the
