@@ -222,7 +222,11 @@ class _EmulatedExchange:
 @pytest.mark.gpu
 @needs_cuda
 @pytest.mark.parametrize("world,L,P,H,Hkv,D", [(2, 1000, 3, 8, 2, 128), (4, 4096, 3, 32, 8, 128),
-                                               (3, 777, 5, 4, 1, 64)])
+                                               (3, 777, 5, 4, 1, 64),
+                                               # chunks shorter than a tile, no branch keys (P = 1),
+                                               # a group of 3, four passes over uneven chunks
+                                               (2, 129, 2, 2, 1, 64), (4, 333, 1, 6, 2, 128),
+                                               (3, 2500, 4, 8, 4, 128)])
 def test_ring_cuda_steps_emulated_on_one_device(world, L, P, H, Hkv, D):
     """The zigzag ring's CUDA steps (rotation at global positions, partial attention of a
     query chunk against a visiting trunk chunk, log-sum-exp merge, bf16 finish), all
@@ -260,7 +264,11 @@ def test_ring_cuda_steps_emulated_on_one_device(world, L, P, H, Hkv, D):
 @pytest.mark.gpu
 @needs_cuda
 @pytest.mark.parametrize("world,L,P,H,Hkv,D", [(2, 1000, 3, 8, 2, 128), (4, 4096, 3, 32, 8, 128),
-                                               (3, 777, 5, 4, 1, 64)])
+                                               (3, 777, 5, 4, 1, 64),
+                                               # chunks shorter than a tile, no branch keys (P = 1),
+                                               # a group of 3, four passes over uneven chunks
+                                               (2, 129, 2, 2, 1, 64), (4, 333, 1, 6, 2, 128),
+                                               (3, 2500, 4, 8, 4, 128)])
 def test_ring_backward_cuda_emulated_on_one_device(world, L, P, H, Hkv, D):
     """The ring's CUDA backward: every rank's prepare (delta, statistics, zeroed dq~),
     its steps against the trunk chunks it would hold (dq~ into the query chunk's
