@@ -135,12 +135,12 @@ __device__ __forceinline__ void fma4(float (&acc)[4], float a, const float4& b) 
 __device__ __forceinline__ float dot4(const float4& a, const float4& b, float acc) {
   return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
 }
-__device__ __forceinline__ float4 bf4(const __nv_bfloat16* p) {  // 4 bf16 -> float4 (8-byte aligned)
-  const uint2 u = *reinterpret_cast<const uint2*>(p);
+__device__ __forceinline__ float4 bf4u(const uint2 u) {  // 4 bf16 (as loaded) -> float4
   const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
   const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
   return make_float4(a.x, a.y, b.x, b.y);
 }
+constexpr int kLoadBatch = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kBlockThreads)
@@ -182,15 +182,27 @@ __global__ void __launch_bounds__(kBlockThreads)
   const int tid = threadIdx.x;
 
   // block keys / values (rows >= Bs zero), cos / sin of the block's positions
-  for (int e = tid; e < BP * (D / 4); e += blockDim.x) {
-    const int j = e / (D / 4), d = 4 * (e % (D / 4));
-    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), v4 = k4;
-    if (j < Bs) {
-      k4 = bf4(kr + (static_cast<int64_t>(kvh) * T + row0 + j) * D + d);
-      v4 = bf4(vb + (static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D + d);
+  {
+    constexpr int kIt = (BP * (D / 4) + kBlockThreads - 1) / kBlockThreads;
+    uint2 ka[kIt], va[kIt];
+#pragma unroll
+    for (int u = 0; u < kIt; ++u) {
+      const int e = tid + u * kBlockThreads;
+      const int j = e / (D / 4), d = 4 * (e % (D / 4));
+      ka[u] = va[u] = make_uint2(0u, 0u);
+      if (e < BP * (D / 4) && j < Bs) {
+        ka[u] = *reinterpret_cast<const uint2*>(kr + (static_cast<int64_t>(kvh) * T + row0 + j) * D + d);
+        va[u] = *reinterpret_cast<const uint2*>(vb + (static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D + d);
+      }
     }
-    *reinterpret_cast<float4*>(sK + j * LD + d) = k4;
-    *reinterpret_cast<float4*>(sV + j * LD + d) = v4;
+#pragma unroll
+    for (int u = 0; u < kIt; ++u) {
+      const int e = tid + u * kBlockThreads;
+      if (e >= BP * (D / 4)) break;
+      const int j = e / (D / 4), d = 4 * (e % (D / 4));
+      *reinterpret_cast<float4*>(sK + j * LD + d) = bf4u(ka[u]);
+      *reinterpret_cast<float4*>(sV + j * LD + d) = bf4u(va[u]);
+    }
   }
   for (int d = tid; d < HALF; d += blockDim.x) sF[d] = pow(static_cast<double>(g.theta), -2.0 * d / D);
   __syncthreads();
@@ -214,16 +226,29 @@ __global__ void __launch_bounds__(kBlockThreads)
     const int R = nh * Bs;
     const int RP = (R + 3) & ~3;
     __syncthreads();  // the previous pass's readers of sQ / sO / sP / sD are done
-    for (int e = tid; e < RP * (D / 4); e += blockDim.x) {
-      const int r = e / (D / 4), d = 4 * (e % (D / 4));
-      float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), o4 = q4;
-      if (r < R) {
-        const int h = kvh * gsz + h0 + r / Bs, i = r % Bs;
-        q4 = bf4(qr + (static_cast<int64_t>(h) * T + row0 + i) * D + d);
-        o4 = bf4(dout + (static_cast<int64_t>(row0 + i) * g.H + h) * D + d);
+    // kLoadBatch iterations' loads are issued before any of them is converted and stored,
+    // so that a thread waits for one round trip per batch rather than per element group
+    for (int e0 = tid; e0 < RP * (D / 4); e0 += kLoadBatch * kBlockThreads) {
+      uint2 qa[kLoadBatch], oa[kLoadBatch];
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) {
+        const int e = e0 + u * kBlockThreads;
+        const int r = e / (D / 4), d = 4 * (e % (D / 4));
+        qa[u] = oa[u] = make_uint2(0u, 0u);
+        if (e < RP * (D / 4) && r < R) {
+          const int h = kvh * gsz + h0 + r / Bs, i = r % Bs;
+          qa[u] = *reinterpret_cast<const uint2*>(qr + (static_cast<int64_t>(h) * T + row0 + i) * D + d);
+          oa[u] = *reinterpret_cast<const uint2*>(dout + (static_cast<int64_t>(row0 + i) * g.H + h) * D + d);
+        }
       }
-      *reinterpret_cast<float4*>(sQ + r * LD + d) = q4;
-      *reinterpret_cast<float4*>(sO + r * LD + d) = o4;
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) {
+        const int e = e0 + u * kBlockThreads;
+        if (e >= RP * (D / 4)) break;
+        const int r = e / (D / 4), d = 4 * (e % (D / 4));
+        *reinterpret_cast<float4*>(sQ + r * LD + d) = bf4u(qa[u]);
+        *reinterpret_cast<float4*>(sO + r * LD + d) = bf4u(oa[u]);
+      }
     }
     for (int r = tid; r < RP; r += blockDim.x) {
       float l = 0.f, dl = 0.f;
