@@ -116,11 +116,14 @@ constexpr int kBlockRows = 64;  // stacked query rows per pass over the group's 
 
 template <int D>
 struct BlockSmem {
-  static constexpr int LD = D + 4;  // row stride (floats): 16-byte aligned rows, staggered banks
-  static constexpr int BP = 16;     // block keys, padded
-  // Q, dO [64][LD]; K, V [16][LD]; P, dS [64][16]; cos, sin [16][D/2]; lse, delta [64];
-  // then the inverse frequencies (double [D/2])
-  static constexpr size_t kFloats = 2 * kBlockRows * LD + 2 * BP * LD + 2 * kBlockRows * BP + 2 * BP * (D / 2) +
+  static constexpr int LD = D + 4;   // fp32 row stride (floats): 16-byte aligned rows, staggered banks
+  static constexpr int LDH = D + 8;  // bf16 row stride (elements): 16-byte aligned rows, staggered banks
+  static constexpr int BP = 16;      // block keys, padded
+  // Q, dO bf16 [64][LDH] (at the end: dk~ / dV fp32 [16][LD] over them); K, V [16][LD];
+  // P, dS [64][16]; cos, sin [16][D/2]; lse, delta [64]; then the inverse frequencies
+  // (double [D/2]).  bf16 staging of Q and dO keeps three CTAs on an SM.
+  static_assert(kBlockRows * LDH * 2 >= 16 * LD * 4, "dk~ / dV fit over the staged rows");
+  static constexpr size_t kFloats = kBlockRows * LDH + 2 * BP * LD + 2 * kBlockRows * BP + 2 * BP * (D / 2) +
                                     2 * kBlockRows;
   static constexpr size_t bytes = kFloats * sizeof(float) + (D / 2) * sizeof(double);
 };
@@ -150,12 +153,13 @@ __global__ void __launch_bounds__(kBlockThreads)
                      __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
   using SM = BlockSmem<D>;
   constexpr int LD = SM::LD;
+  constexpr int LDH = SM::LDH;
   constexpr int BP = SM::BP;
   constexpr int HALF = D / 2;
   extern __shared__ __align__(16) float blk_smem[];
-  float* sQ = blk_smem;                  // [64][LD]
-  float* sO = sQ + kBlockRows * LD;      // [64][LD] dO
-  float* sK = sO + kBlockRows * LD;      // [16][LD]
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(blk_smem);  // [64][LDH]
+  __nv_bfloat16* sO = sQ + kBlockRows * LDH;                        // [64][LDH] dO
+  float* sK = reinterpret_cast<float*>(sO + kBlockRows * LDH);      // [16][LD]
   float* sV = sK + BP * LD;              // [16][LD]
   float* sP = sV + BP * LD;              // [64][16] scores, then P
   float* sD = sP + kBlockRows * BP;      // [64][16] dP, then dS
@@ -246,8 +250,8 @@ __global__ void __launch_bounds__(kBlockThreads)
         const int e = e0 + u * kBlockThreads;
         if (e >= RP * (D / 4)) break;
         const int r = e / (D / 4), d = 4 * (e % (D / 4));
-        *reinterpret_cast<float4*>(sQ + r * LD + d) = bf4u(qa[u]);
-        *reinterpret_cast<float4*>(sO + r * LD + d) = bf4u(oa[u]);
+        *reinterpret_cast<uint2*>(sQ + r * LDH + d) = qa[u];
+        *reinterpret_cast<uint2*>(sO + r * LDH + d) = oa[u];
       }
     }
     for (int r = tid; r < RP; r += blockDim.x) {
@@ -266,14 +270,14 @@ __global__ void __launch_bounds__(kBlockThreads)
       const int blk = tid & 63;
       const int rb = blk / (BP / 4), cb = blk % (BP / 4);
       if (4 * rb < RP) {
-        const float* A = tid < 64 ? sQ : sO;
+        const __nv_bfloat16* A = tid < 64 ? sQ : sO;
         const float* Bm = tid < 64 ? sK : sV;
         float s[4][4] = {};
 #pragma unroll 4
         for (int d = 0; d < D; d += 4) {
           float4 a[4], bb[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) a[u] = ld4(A + (4 * rb + u) * LD + d);
+          for (int u = 0; u < 4; ++u) a[u] = bf4u(*reinterpret_cast<const uint2*>(A + (4 * rb + u) * LDH + d));
 #pragma unroll
           for (int v = 0; v < 4; ++v) bb[v] = ld4(Bm + (4 * cb + v) * LD + d);
 #pragma unroll
@@ -350,10 +354,11 @@ __global__ void __launch_bounds__(kBlockThreads)
     // dk~ (sum of dS q~) and dV (sum of P dO) over this pass's rows
     if (acc_on) {
       const float* W = acc_v ? sP : sD;  // P for dV, dS for dk~
-      const float* X = acc_v ? sO : sQ;
+      const __nv_bfloat16* X = acc_v ? sO : sQ;
       for (int r = 0; r < R; ++r) {
         const float4 w4 = ld4(W + r * BP + 4 * akb);
-        const float4 x0 = ld4(X + r * LD + acol), x1 = ld4(X + r * LD + acol + 4);
+        const uint4 xr = *reinterpret_cast<const uint4*>(X + r * LDH + acol);
+        const float4 x0 = bf4u(make_uint2(xr.x, xr.y)), x1 = bf4u(make_uint2(xr.z, xr.w));
         const float w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -367,8 +372,10 @@ __global__ void __launch_bounds__(kBlockThreads)
   }
   // dk~ and dV to shared memory (over sQ / sO), then dK = sigma R^T dk~ and dV in bf16
   __syncthreads();
+  float* fQ = reinterpret_cast<float*>(sQ);  // dk~ [16][LD] over the staged rows
+  float* fO = reinterpret_cast<float*>(sO);  // dV [16][LD]
   if (acc_on) {
-    float* dst = acc_v ? sO : sQ;
+    float* dst = acc_v ? fO : fQ;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       *reinterpret_cast<float4*>(dst + (4 * akb + v) * LD + acol) =
@@ -380,14 +387,14 @@ __global__ void __launch_bounds__(kBlockThreads)
   __syncthreads();
   for (int e = tid; e < Bs * HALF; e += blockDim.x) {
     const int j = e / HALF, d = e % HALF;
-    const float x1 = sQ[j * LD + d] * g.scale, x2 = sQ[j * LD + d + HALF] * g.scale;
+    const float x1 = fQ[j * LD + d] * g.scale, x2 = fQ[j * LD + d + HALF] * g.scale;
     const float c = sC[j * HALF + d], s = sN[j * HALF + d];
     __nv_bfloat16* ok = dk + (static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D;
     ok[d] = __float2bfloat16_rn(fmaf(x1, c, x2 * s));
     ok[d + HALF] = __float2bfloat16_rn(fmaf(x2, c, -x1 * s));
     __nv_bfloat16* ov = dv + (static_cast<int64_t>(row0 + j) * g.Hkv + kvh) * D;
-    ov[d] = __float2bfloat16_rn(sO[j * LD + d]);
-    ov[d + HALF] = __float2bfloat16_rn(sO[j * LD + d + HALF]);
+    ov[d] = __float2bfloat16_rn(fO[j * LD + d]);
+    ov[d + HALF] = __float2bfloat16_rn(fO[j * LD + d + HALF]);
   }
 }
 
